@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of NSA selected-block attention (forward + backward) on B200.
+
+One step = the whole path on one batch: forward (index inversion, tensor-core tile
+kernel, log-sum-exp merge) then backward (inversion, D = rowsum(dO * O), tile
+kernel, dQ merge, dK/dV reduction) of the headline workload: one sequence of
+T = 65536 tokens, 16 query heads over 4 KV heads (group 4), head_dim 128,
+block 64, top-16 blocks per (token, KV head), bf16 inputs ~ N(0, 1).
+
+`value` is useful TFLOP/s: 4 * d * (keys attended after the causal mask) per query
+head per token for the forward, 2.5x that for the backward, summed over all ranks
+and divided by the device time of K steps (CUDA events, max over ranks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own independent problem (weak scaling, no data
+collective).  `--impl reference` times the fp64 CPU oracle on a bounded sample of
+the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nsa_inputs as ni  # noqa: E402
+
+METRIC = "selected-attn fwd/bwd TFLOP/s and ms at T=64k; % of B200 bf16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- work
+
+def attended_keys(cu_seqlens, block_idx, block_size):
+    """Keys each (token, KV head) row attends after the causal mask (counting only)."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, hkv, topk = block_idx.shape
+    out = np.zeros((T, hkv), dtype=np.int64)
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        if b == a:
+            continue
+        i = np.arange(b - a, dtype=np.int64)
+        qb = (i // block_size)[:, None, None]
+        x = block_idx[a:b].astype(np.int64)
+        x = np.sort(np.where((x >= 0) & (x <= qb), x, -1), axis=2)
+        first = np.ones_like(x, dtype=bool)
+        first[:, :, 1:] = x[:, :, 1:] != x[:, :, :-1]
+        keep = first & (x >= 0)
+        full = (keep & (x < qb)).sum(axis=2)
+        diag = (keep & (x == qb)).sum(axis=2)
+        out[a:b] = full * block_size + diag * ((i % block_size) + 1)[:, None]
+    return out
+
+
+def useful_flops(p: ni.Problem):
+    keys = attended_keys(p.cu_seqlens, p.block_idx, p.block_size)
+    G = p.hq // p.hkv
+    fwd = 4.0 * p.head_dim * float(keys.sum()) * G
+    return fwd, 2.5 * fwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_selected_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, launch_units: float):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    if not k:
+        return None
+    # stored per unit of work (useful FLOP) so that a smaller capture scales
+    return float(k["dram_bytes_per_useful_flop"]) * launch_units
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="nsa_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        loaded = [s for s, r in zip(sm, rows) if num(r[3]) and num(r[3]) > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank, dist):
+    import torch
+    import block_sparse_attention_selected_b200 as nsa
+    from block_sparse_attention_selected_b200 import build as nsa_build
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    nsa_build.build()
+    lib = nsa.load_library()
+
+    spec = dict(ni.WORKLOADS[args.workload])
+    spec["seed"] = spec["seed"] + 1000 * rank
+    p = ni.make_problem(name=args.workload, head_dim=128, with_dout=True, **spec)
+    fwd_flops, bwd_flops = useful_flops(p)
+    step_flops = fwd_flops + bwd_flops
+    T, hq, hkv, d, topk, bs, nseq = p.T, p.hq, p.hkv, 128, p.topk, p.block_size, p.nseq
+
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).pin_memory()
+    h_q, h_k, h_v, h_do = bf(p.q), bf(p.k), bf(p.v), bf(p.dout)
+    h_cu = torch.from_numpy(p.cu_seqlens).pin_memory()
+    h_bi = torch.from_numpy(np.ascontiguousarray(p.block_idx)).pin_memory()
+    q, k, v, do = (x.to(dev) for x in (h_q, h_k, h_v, h_do))
+    cu, bi = h_cu.to(dev), h_bi.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = nsa.nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, bs, True)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes_ptr = nsa._ptr
+    scale = p.scale
+    import ctypes
+    n_fwd = ctypes.c_int(0)
+    n_bwd = ctypes.c_int(0)
+
+    def ev_array(evs):
+        arr = (ctypes.c_void_p * len(evs))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+        return arr
+
+    def step(fwd_ev=None, bwd_ev=None, q_=q, k_=k, v_=v, do_=do, cu_=cu, bi_=bi):
+        rc = lib.nsa_sel_attn_fwd_profiled(
+            sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
+            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream),
+            fwd_ev, 4 if fwd_ev is not None else 0, ctypes.byref(n_fwd))
+        if rc:
+            raise RuntimeError(f"forward failed: {rc}")
+        rc = lib.nsa_sel_attn_bwd_profiled(
+            sp(q_), sp(k_), sp(v_), sp(out), sp(lse), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
+            sp(bi_), topk, bs, scale, sp(dq), sp(dk), sp(dv), sp(ws), ws_bytes,
+            ctypes.c_void_p(stream.cuda_stream), bwd_ev, 6 if bwd_ev is not None else 0,
+            ctypes.byref(n_bwd))
+        if rc:
+            raise RuntimeError(f"backward failed: {rc}")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = nsa.nsa_sel_check_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {st}")
+
+    K = args.steps
+    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    farr = [ev_array(e) for e in fevs]
+    barr = [ev_array(e) for e in bevs]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        step(farr[i], barr[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1))
+    if nsa.nsa_sel_check_status(ws) != 0:
+        raise RuntimeError("device status error in the timed region")
+    ms_step = elapsed_ms / K
+    value = world * step_flops * K / (elapsed_ms * 1e-3) / 1e12
+
+    def avg(evs, a, b):
+        return statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+
+    phase = {
+        "fwd_ms": avg(fevs, 0, 3), "fwd_invert_ms": avg(fevs, 0, 1),
+        "fwd_tiles_ms": avg(fevs, 1, 2), "fwd_merge_ms": avg(fevs, 2, 3),
+        "bwd_ms": avg(bevs, 0, 5), "bwd_invert_ms": avg(bevs, 0, 1),
+        "bwd_delta_ms": avg(bevs, 1, 2), "bwd_tiles_ms": avg(bevs, 2, 3),
+        "bwd_dq_merge_ms": avg(bevs, 3, 4), "bwd_dkdv_reduce_ms": avg(bevs, 4, 5),
+    }
+    peaks, peak_src = load_peaks()
+    tc_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if phase["bwd_tiles_ms"] >= phase["fwd_tiles_ms"]:
+        dom, dom_ms, dom_flops = "k_bwd_tiles", phase["bwd_tiles_ms"], bwd_flops
+    else:
+        dom, dom_ms, dom_flops = "k_fwd_tiles", phase["fwd_tiles_ms"], fwd_flops
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
+                "peak": tc_peak, "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4),
+                "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                "traffic": profiled_traffic(dom, dom_flops)}
+    fwd_tiles_tflops = fwd_flops / (phase["fwd_tiles_ms"] * 1e-3) / 1e12
+    bwd_tiles_tflops = bwd_flops / (phase["bwd_tiles_ms"] * 1e-3) / 1e12
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    # end to end through the C ABI with host buffers: H2D inputs, fwd+bwd, D2H outputs
+    e2e = None
+    if not args.no_e2e:
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h_dq = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+        h_dk = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
+        h_dv = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+        d_in = [torch.empty_like(x) for x in (q, k, v, do, cu, bi)]
+        h_in = [h_q, h_k, h_v, h_do, h_cu, h_bi]
+        h2d = sum(x.numel() * x.element_size() for x in h_in)
+        d2h = sum(x.numel() * x.element_size() for x in (h_out, h_lse, h_dq, h_dk, h_dv))
+        Ke = max(2, min(K, 5))
+
+        def e2e_step():
+            for dst, src in zip(d_in, h_in):
+                dst.copy_(src, non_blocking=True)
+            step(None, None, *d_in)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+            h_dq.copy_(dq, non_blocking=True)
+            h_dk.copy_(dk, non_blocking=True)
+            h_dv.copy_(dv, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b))
+        e2e = {"value": round(world * step_flops * Ke / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, tokens=args.cpu_tokens)
+
+    launches = K * (n_fwd.value + n_bwd.value)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO; index rule init+local+random earlier)",
+        "config": {"workload": args.workload, "total_tokens": T, "num_seqs": nseq, "hq": hq,
+                   "hkv": hkv, "group": hq // hkv, "head_dim": d, "block_size": bs, "topk": topk,
+                   "parallelism": f"independent problem per rank x{world}",
+                   "l2": "inputs larger than L2 (Q 268 MB, partials 4.3 GB); no flush"},
+        "fwd_ms": round(phase["fwd_ms"], 4), "bwd_ms": round(phase["bwd_ms"], 4),
+        "fwd_tflops": round(fwd_flops / (phase["fwd_ms"] * 1e-3) / 1e12, 2),
+        "bwd_tflops": round(bwd_flops / (phase["bwd_ms"] * 1e-3) / 1e12, 2),
+        "fwd_pct_of_bf16_peak": round(100 * fwd_flops / (phase["fwd_ms"] * 1e-3) / 1e12 / burst, 2),
+        "fwd_tiles_tflops": round(fwd_tiles_tflops, 2),
+        "bwd_tiles_tflops": round(bwd_tiles_tflops, 2),
+        "phases_ms": {k2: round(v2, 4) for k2, v2 in phase.items()},
+        "useful_tflop_per_step": round(step_flops / 1e12, 4),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return line
+
+
+# ----------------------------------------------------------------- oracle baselines
+
+def oracle_sample(workload: str, tokens: int):
+    spec = dict(ni.WORKLOADS[workload])
+    spec["lengths"] = [min(tokens, sum(spec["lengths"]))]
+    return ni.make_problem(name=workload + f"_prefix{tokens}", head_dim=128, **spec)
+
+
+def time_oracle_step(p, nthreads):
+    import oracle
+    t = time.perf_counter()
+    oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale, nthreads=nthreads)
+    oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+               nthreads=nthreads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(workload: str, tokens: int):
+    cores = len(os.sched_getaffinity(0))
+    p = oracle_sample(workload, tokens)
+    f, b = useful_flops(p)
+    dt = time_oracle_step(p, cores)
+    return {"value": round((f + b) / dt / 1e12, 6), "unit": UNIT, "cores": cores,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"first {p.T} tokens (all {p.hq} heads) of the workload, forward + full "
+                      f"backward in fp64; useful FLOPs by the same formula"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cores = len(os.sched_getaffinity(0))
+    p = oracle_sample(args.workload, args.ref_tokens)
+    f, b = useful_flops(p)
+    for _ in range(args.warmup):
+        time_oracle_step(p, cores)
+    times = [time_oracle_step(p, cores) for _ in range(args.steps)]
+    total = sum(times)
+    value = (f + b) * len(times) / total / 1e12
+    sample = (f"first {p.T} tokens (all {p.hq} heads) of the workload per step, forward + full "
+              f"backward in fp64")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * total / len(times), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_tokens": p.T},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
+                             "value": round(value, 6), "unit": UNIT},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return line
+
+
+# ---------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=ni.HEADLINE, choices=sorted(ni.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=2048)
+    ap.add_argument("--ref-tokens", type=int, default=1024)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

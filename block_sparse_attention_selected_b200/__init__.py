@@ -1,0 +1,256 @@
+"""NSA selected-block attention on B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/nsa_sel.h`` (``libnsa_sel.so``,
+built in this directory by ``build.py``).  Functions carry the C names and only
+marshal arguments: every step of the computation runs in the CUDA library.  There
+is no fallback: if the library or a CUDA device is missing, calls raise.
+
+Tensors: q [T, hq, 128], k/v [T, hkv, 128] bf16 CUDA; cu_seqlens int32 [nseq+1];
+block_idx int32 [T, hkv, topk] (block numbers local to each sequence, -1 pads).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnsa_sel.so")
+
+NSA_OK = 0
+STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
+                3: "NSA_ERR_WORKSPACE", 4: "NSA_ERR_CUDA", 5: "NSA_ERR_TIMEOUT",
+                6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
+EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
+            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_invert_index", "nsa_sel_validate_indices", "nsa_sel_check_status",
+            "nsa_sel_status_string"]
+
+_lib = None
+_lock = threading.Lock()
+
+
+class NsaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn}: {STATUS_NAMES.get(code, code)} ({_status_string(code)})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads the CUDA library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with "
+                                   "`python -m block_sparse_attention_selected_b200.build`")
+            lib = ctypes.CDLL(path)
+            P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            lib.nsa_sel_attn_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+            lib.nsa_sel_attn_workspace_size.restype = Z
+            lib.nsa_sel_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, P, I, I, F, P, P, P, Z, P]
+            lib.nsa_sel_attn_fwd.restype = I
+            lib.nsa_sel_attn_bwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, I, I, F,
+                                             P, P, P, P, Z, P]
+            lib.nsa_sel_attn_bwd.restype = I
+            lib.nsa_sel_attn_fwd_profiled.argtypes = lib.nsa_sel_attn_fwd.argtypes + [P, I, P]
+            lib.nsa_sel_attn_fwd_profiled.restype = I
+            lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, P]
+            lib.nsa_sel_attn_bwd_profiled.restype = I
+            lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
+            lib.nsa_sel_invert_index.restype = I
+            lib.nsa_sel_validate_indices.argtypes = [P, I, I, I, P, I, I, P, P, P, Z, P]
+            lib.nsa_sel_validate_indices.restype = I
+            lib.nsa_sel_check_status.argtypes = [P, P]
+            lib.nsa_sel_check_status.restype = I
+            lib.nsa_sel_status_string.argtypes = [I]
+            lib.nsa_sel_status_string.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return load_library().nsa_sel_status_string(code).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(fn: str, code: int):
+    if code != NSA_OK:
+        raise NsaError(fn, code)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype, ndim=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_ws_cache: dict = {}
+
+
+def nsa_sel_attn_workspace_size(total_tokens, num_seqs, hq, hkv, head_dim, topk, block_size,
+                                for_bwd=False) -> int:
+    n = load_library().nsa_sel_attn_workspace_size(total_tokens, num_seqs, hq, hkv, head_dim,
+                                                   topk, block_size, int(bool(for_bwd)))
+    if n == 0:
+        raise NsaError("nsa_sel_attn_workspace_size", 2)
+    return int(n)
+
+
+def get_workspace(nbytes: int, device) -> torch.Tensor:
+    """A cached uint8 device buffer of at least nbytes (grown on demand)."""
+    dev = torch.device(device)
+    ws = _ws_cache.get(dev)
+    if ws is None or ws.numel() < nbytes:
+        _ws_cache.pop(dev, None)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        _ws_cache[dev] = ws
+    return ws
+
+
+def release_workspaces():
+    _ws_cache.clear()
+
+
+def _shapes(q, k, cu_seqlens, block_idx):
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    topk = block_idx.shape[2]
+    return T, hq, hkv, d, topk, cu_seqlens.numel() - 1
+
+
+def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out=None, lse=None,
+                     workspace=None):
+    """Forward selected attention; returns (out bf16 [T,hq,d], lse fp32 [hq,T])."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(k, "k", torch.bfloat16, 3, dev)
+    _need(v, "v", torch.bfloat16, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(block_idx, "block_idx", torch.int32, 3, dev)
+    T, hq, hkv, d, topk, nseq = _shapes(q, k, cu_seqlens, block_idx)
+    if k.shape != (T, hkv, d) or v.shape != (T, hkv, d) or block_idx.shape[:2] != (T, hkv):
+        raise ValueError("inconsistent shapes")
+    scale = float(d ** -0.5 if scale is None else scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.bfloat16, 3, dev)
+    _need(lse, "lse", torch.float32, 2, dev)
+    nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, False)
+    ws = workspace if workspace is not None else get_workspace(nbytes, dev)
+    _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, _ptr(block_idx), topk,
+        block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
+    return out, lse
+
+
+def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size, scale=None,
+                     dq=None, dk=None, dv=None, workspace=None):
+    """Backward; returns (dq, dk, dv) bf16."""
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 3, dev)
+    _need(lse, "lse", torch.float32, 2, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(block_idx, "block_idx", torch.int32, 3, dev)
+    T, hq, hkv, d, topk, nseq = _shapes(q, k, cu_seqlens, block_idx)
+    scale = float(d ** -0.5 if scale is None else scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, True)
+    ws = workspace if workspace is not None else get_workspace(nbytes, dev)
+    _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
+        hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(ws), ws.numel(), _stream(dev)))
+    return dq, dk, dv
+
+
+def nsa_sel_invert_index(cu_seqlens, block_idx, block_size, workspace=None):
+    """The block-index inversion; returns (offsets int32 [hkv*NB+1], entries int32 [n])."""
+    dev = block_idx.device
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(block_idx, "block_idx", torch.int32, 3, dev)
+    T, hkv, topk = block_idx.shape
+    nseq = cu_seqlens.numel() - 1
+    nbytes = nsa_sel_attn_workspace_size(T, nseq, hkv, hkv, 128, topk, block_size, False)
+    ws = workspace if workspace is not None else get_workspace(nbytes, dev)
+    offsets = torch.empty(hkv * (T // block_size + nseq) + 1, dtype=torch.int32, device=dev)
+    entries = torch.empty(max(T * hkv * topk, 1), dtype=torch.int32, device=dev)
+    counts = torch.zeros(2, dtype=torch.int32, device=dev)
+    _check("nsa_sel_invert_index", load_library().nsa_sel_invert_index(
+        _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
+        _ptr(entries), _ptr(counts), _ptr(ws), ws.numel(), _stream(dev)))
+    nb, n = (int(x) for x in counts.tolist())
+    return offsets[:hkv * nb + 1], entries[:n]
+
+
+def nsa_sel_validate_indices(cu_seqlens, block_idx, block_size, workspace=None):
+    """(n_out_of_range, n_duplicates); synchronous."""
+    dev = block_idx.device
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(block_idx, "block_idx", torch.int32, 3, dev)
+    T, hkv, topk = block_idx.shape
+    ws = workspace if workspace is not None else get_workspace(256, dev)
+    a, b = ctypes.c_longlong(0), ctypes.c_longlong(0)
+    code = load_library().nsa_sel_validate_indices(
+        _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, _ptr(block_idx), topk, block_size,
+        ctypes.byref(a), ctypes.byref(b), _ptr(ws), ws.numel(), _stream(dev))
+    if code not in (0, 6):
+        raise NsaError("nsa_sel_validate_indices", code)
+    return int(a.value), int(b.value)
+
+
+def nsa_sel_check_status(workspace=None, device=None) -> int:
+    """Device-side status of the last call that used this workspace (synchronises)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    ws = workspace if workspace is not None else _ws_cache.get(dev)
+    if ws is None:
+        return NSA_OK
+    return int(load_library().nsa_sel_check_status(_ptr(ws), _stream(ws.device)))
+
+
+class SelectedAttention(torch.autograd.Function):
+    """Autograd wrapper: forward saves LSE, backward returns dQ, dK, dV."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, cu_seqlens, block_idx, block_size, scale):
+        out, lse = nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale)
+        ctx.save_for_backward(q, k, v, out, lse, cu_seqlens, block_idx)
+        ctx.block_size, ctx.scale = block_size, scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse, cu, bi = ctx.saved_tensors
+        dq, dk, dv = nsa_sel_attn_bwd(q, k, v, out, lse, dout.contiguous(), cu, bi,
+                                      ctx.block_size, ctx.scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def selected_attention(q, k, v, cu_seqlens, block_idx, block_size=64, scale=None):
+    return SelectedAttention.apply(q, k, v, cu_seqlens, block_idx, block_size,
+                                   float(q.shape[-1] ** -0.5 if scale is None else scale))

@@ -1,0 +1,509 @@
+// api.cu -- the C ABI declared in include/nsa_sel.h.
+//
+// Host side only: argument checks (before any launch), the workspace layout, the
+// TMA tensor maps for K and V, and the launch sequences of the forward and backward
+// passes.  All work is enqueued on the caller's stream; nothing is allocated.
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "nsa_common.cuh"
+#include "nsa_kernels.h"
+
+using namespace nsa;
+
+namespace {
+
+constexpr int kChunkTiles = 32;   // tiles per backward work unit
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Dims {
+    int T, nseq, hq, hkv, d, topk, bs, G;
+    long long nent;
+    int nbk_cap;
+    int key_bits;
+    int sort_tiles;
+    long long tiles_cap, units_cap;
+};
+
+struct Layout {
+    size_t status, blkoff, keys0, keys1, vals0, vals1, hist, offsets, tile_off, chunk_off;
+    size_t part_o, part_lse, delta, part_dkdv;
+    size_t total;
+};
+
+nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int bs, Dims* D) {
+    if (T < 0 || nseq < 1 || hq < 1 || hkv < 1 || d < 1 || topk < 1 || bs < 1)
+        return NSA_ERR_INVALID_ARG;
+    if (hq % hkv != 0) return NSA_ERR_INVALID_ARG;
+    if (d != kHeadDim || (bs != 64 && bs != 128) || topk > kMaxTopk) return NSA_ERR_UNSUPPORTED;
+    const int G = hq / hkv;
+    if (G > kMaxGroup || kTileRows % G != 0) return NSA_ERR_UNSUPPORTED;
+    if (T >= (1 << 25)) return NSA_ERR_UNSUPPORTED;
+    const long long nent = (long long)T * hkv * topk;
+    if (nent >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;
+    const long long nbk_cap = (long long)hkv * ((long long)T / bs + nseq);
+    if (nbk_cap >= (1ll << 30)) return NSA_ERR_UNSUPPORTED;
+    D->T = T; D->nseq = nseq; D->hq = hq; D->hkv = hkv; D->d = d; D->topk = topk; D->bs = bs;
+    D->G = G;
+    D->nent = nent;
+    D->nbk_cap = (int)nbk_cap;
+    int bits = 1;
+    while ((1ll << bits) <= nbk_cap) ++bits;   // 2^bits > nbk_cap
+    D->key_bits = bits;
+    D->sort_tiles = (int)((nent + kSortTile - 1) / kSortTile);
+    const int tpt = kTileRows / G;
+    D->tiles_cap = (nent + tpt - 1) / tpt + nbk_cap;
+    D->units_cap = (D->tiles_cap + kChunkTiles - 1) / kChunkTiles + nbk_cap;
+    return NSA_OK;
+}
+
+Layout make_layout(const Dims& D, bool bwd) {
+    Layout L{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+    L.status = take(sizeof(DevStatus));
+    L.blkoff = take(sizeof(int32_t) * (D.nseq + 1));
+    L.keys0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
+    L.keys1 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
+    L.vals0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
+    L.vals1 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
+    L.hist = take(sizeof(uint32_t) * 256 * (size_t)std::max(D.sort_tiles, 1));
+    L.offsets = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
+    L.tile_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
+    L.chunk_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
+    const size_t rows = (size_t)D.T * D.hq * D.topk;
+    L.part_o = take(rows * kHeadDim * 2);   // bf16 partial O (forward) / dQ (backward)
+    L.part_lse = take(rows * sizeof(float));
+    if (bwd) {
+        L.delta = take(sizeof(float) * (size_t)D.hq * D.T);
+        L.part_dkdv = take(sizeof(float) * 2 * (size_t)D.bs * kHeadDim * (size_t)D.units_cap);
+    }
+    L.total = o;
+    return L;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+nsa_status_t check_device(int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_NO_DEVICE;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return NSA_ERR_NO_DEVICE;
+    if (major != 10 || minor != 0) return NSA_ERR_NO_DEVICE;
+    if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return NSA_ERR_NO_DEVICE;
+    return NSA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Tensor map over a bf16 [T, hkv, 128] tensor; box = (64 columns, 1 head, bs keys),
+// 128-byte swizzle (the layout the tensor-core descriptors expect).
+bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)hkv, (cuuint64_t)(T > 0 ? T : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)hkv * kHeadDim * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)bs};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct Carved {
+    DevStatus* st;
+    InvertPlan inv;
+    uint8_t* base;
+    Layout L;
+};
+
+Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const int32_t* bidx) {
+    Carved c{};
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    c.base = b;
+    c.L = L;
+    c.st = reinterpret_cast<DevStatus*>(b + L.status);
+    InvertPlan& p = c.inv;
+    p.cu = cu;
+    p.nseq = D.nseq;
+    p.T = D.T;
+    p.hkv = D.hkv;
+    p.bidx = bidx;
+    p.topk = D.topk;
+    p.bs = D.bs;
+    p.tokens_per_tile = kTileRows / D.G;
+    p.chunk_tiles = kChunkTiles;
+    p.nent = D.nent;
+    p.nbk_cap = D.nbk_cap;
+    p.key_bits = D.key_bits;
+    p.sort_tiles = D.sort_tiles;
+    p.blkoff = reinterpret_cast<int32_t*>(b + L.blkoff);
+    p.keys[0] = reinterpret_cast<uint32_t*>(b + L.keys0);
+    p.keys[1] = reinterpret_cast<uint32_t*>(b + L.keys1);
+    p.vals[0] = reinterpret_cast<uint32_t*>(b + L.vals0);
+    p.vals[1] = reinterpret_cast<uint32_t*>(b + L.vals1);
+    p.hist = reinterpret_cast<uint32_t*>(b + L.hist);
+    p.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
+    p.tile_off = reinterpret_cast<int32_t*>(b + L.tile_off);
+    p.chunk_off = reinterpret_cast<int32_t*>(b + L.chunk_off);
+    p.st = c.st;
+    p.final_buf = 0;
+    return c;
+}
+
+nsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA; }
+
+// Common checks of the index inputs and the workspace; returns NSA_OK and fills D.
+nsa_status_t check_common(const int32_t* cu, int nseq, int T, int hq, int hkv, int d,
+                          const int32_t* bidx, int topk, int bs, void* ws, size_t ws_bytes,
+                          bool bwd, Dims* D) {
+    nsa_status_t s = check_dims(T, nseq, hq, hkv, d, topk, bs, D);
+    if (s != NSA_OK) return s;
+    if (!cu || !ws || (T > 0 && !bidx)) return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu, 4) || !aligned(bidx, 4) || !aligned(ws, 256)) return NSA_ERR_INVALID_ARG;
+    if (ws_bytes < make_layout(*D, bwd).total) return NSA_ERR_WORKSPACE;
+    return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nsa_sel_attn_workspace_size(int total_tokens, int num_seqs, int hq, int hkv, int head_dim,
+                                   int topk, int block_size, int for_bwd) {
+    Dims D;
+    if (check_dims(total_tokens, num_seqs, hq, hkv, head_dim, topk, block_size, &D) != NSA_OK)
+        return 0;
+    return make_layout(D, for_bwd != 0).total;
+}
+
+const char* nsa_sel_status_string(nsa_status_t s) {
+    switch (s) {
+        case NSA_OK: return "ok";
+        case NSA_ERR_INVALID_ARG: return "invalid argument";
+        case NSA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+        case NSA_ERR_WORKSPACE: return "workspace too small";
+        case NSA_ERR_CUDA: return "CUDA error";
+        case NSA_ERR_TIMEOUT: return "device-side wait timed out";
+        case NSA_ERR_BAD_INDEX: return "invalid block_idx or cu_seqlens";
+        case NSA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"
+
+namespace {
+
+// Records ev[i] (when given) on the stream at phase boundary i.
+struct PhaseMarks {
+    void* const* ev;
+    int n;
+    cudaStream_t stream;
+    int* launches;
+    void mark(int i) const {
+        if (ev && i < n && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream);
+    }
+    void add(int k) const {
+        if (launches) *launches += k;
+    }
+};
+
+int invert_launches(const Dims& D) {
+    const int passes = D.key_bits <= 8 ? 1 : (D.key_bits + 7) / 8;
+    return 1 + 3 * passes + 2;
+}
+
+nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                      int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                      const int32_t* block_idx, int topk, int block_size, float scale, void* out,
+                      float* lse, void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
+                      void* const* events, int num_events, int* launches) {
+    Dims D;
+    nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
+                                  block_idx, topk, block_size, workspace, workspace_bytes, false, &D);
+    if (s != NSA_OK) return s;
+    if (total_tokens > 0 && (!q || !k || !v || !out || !lse)) return NSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4))
+        return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const Layout L = make_layout(D, false);
+    Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
+    const PhaseMarks pm{events, num_events, stream, launches};
+    if (launches) *launches = 0;
+    pm.mark(0);
+    if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) {
+        for (int i = 1; i < 4; ++i) pm.mark(i);
+        return NSA_OK;
+    }
+
+    CUtensorMap kmap, vmap;
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
+        return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+    pm.add(invert_launches(D));
+    pm.mark(1);
+
+    FwdPlan fp{};
+    fp.q = q;
+    fp.cu = cu_seqlens;
+    fp.nseq = D.nseq; fp.T = D.T; fp.hq = D.hq; fp.hkv = D.hkv; fp.topk = D.topk; fp.bs = D.bs;
+    fp.G = D.G;
+    fp.scale_log2 = scale * 1.4426950408889634f;
+    fp.blkoff = c.inv.blkoff;
+    fp.offsets = c.inv.offsets;
+    fp.tile_off = c.inv.tile_off;
+    fp.entries = c.inv.vals[c.inv.final_buf];
+    fp.nbk_cap = D.nbk_cap;
+    fp.part_o = c.base + L.part_o;
+    fp.part_lse = reinterpret_cast<float*>(c.base + L.part_lse);
+    fp.st = c.st;
+    fp.num_sms = num_sms;
+    if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, stream))) != NSA_OK) return s;
+    pm.add(1);
+    pm.mark(2);
+
+    MergePlan mp{};
+    mp.cu = cu_seqlens;
+    mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
+    mp.bidx = block_idx;
+    mp.part_o = fp.part_o;
+    mp.part_lse = fp.part_lse;
+    mp.out = out;
+    mp.lse = lse;
+    if ((s = cuda_status(launch_merge(mp, stream))) != NSA_OK) return s;
+    pm.add(1);
+    pm.mark(3);
+    return NSA_OK;
+}
+
+nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* out,
+                      const float* lse, const void* dout, const int32_t* cu_seqlens, int num_seqs,
+                      int total_tokens, int hq, int hkv, int head_dim, const int32_t* block_idx,
+                      int topk, int block_size, float scale, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
+                      void* const* events, int num_events, int* launches) {
+    Dims D;
+    nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
+                                  block_idx, topk, block_size, workspace, workspace_bytes, true, &D);
+    if (s != NSA_OK) return s;
+    if (total_tokens > 0 && (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4))
+        return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const Layout L = make_layout(D, true);
+    Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
+    const PhaseMarks pm{events, num_events, stream, launches};
+    if (launches) *launches = 0;
+    pm.mark(0);
+    if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) {
+        for (int i = 1; i < 6; ++i) pm.mark(i);
+        return NSA_OK;
+    }
+
+    CUtensorMap kmap, vmap;
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
+        return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+    pm.add(invert_launches(D));
+    pm.mark(1);
+
+    BwdPlan bp{};
+    bp.q = q;
+    bp.dout = dout;
+    bp.lse = lse;
+    bp.delta = reinterpret_cast<float*>(c.base + L.delta);
+    bp.cu = cu_seqlens;
+    bp.nseq = D.nseq; bp.T = D.T; bp.hq = D.hq; bp.hkv = D.hkv; bp.topk = D.topk; bp.bs = D.bs;
+    bp.G = D.G;
+    bp.scale = scale;
+    bp.scale_log2 = scale * 1.4426950408889634f;
+    bp.blkoff = c.inv.blkoff;
+    bp.offsets = c.inv.offsets;
+    bp.tile_off = c.inv.tile_off;
+    bp.chunk_off = c.inv.chunk_off;
+    bp.entries = c.inv.vals[c.inv.final_buf];
+    bp.nbk_cap = D.nbk_cap;
+    bp.chunk_tiles = kChunkTiles;
+    bp.part_dq = c.base + L.part_o;
+    bp.part_dkdv = reinterpret_cast<float*>(c.base + L.part_dkdv);
+    bp.st = c.st;
+    bp.num_sms = num_sms;
+    if ((s = cuda_status(launch_bwd_preprocess(out, dout, bp.delta, D.T, D.hq, stream))) != NSA_OK)
+        return s;
+    pm.add(1);
+    pm.mark(2);
+    if ((s = cuda_status(launch_bwd_tiles(bp, &kmap, &vmap, stream))) != NSA_OK) return s;
+    pm.add(1);
+    pm.mark(3);
+    if ((s = cuda_status(launch_bwd_dq_merge(bp, block_idx, dq, stream))) != NSA_OK) return s;
+    pm.add(1);
+    pm.mark(4);
+    if ((s = cuda_status(launch_bwd_dkdv_reduce(bp, dk, dv, stream))) != NSA_OK) return s;
+    pm.add(1);
+    pm.mark(5);
+    return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nsa_status_t nsa_sel_attn_fwd(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens, int num_seqs, int total_tokens, int hq,
+                              int hkv, int head_dim, const int32_t* block_idx, int topk,
+                              int block_size, float scale, void* out, float* lse, void* workspace,
+                              size_t workspace_bytes, nsa_stream_t stream) {
+    return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
+                    topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, nullptr,
+                    0, nullptr);
+}
+
+nsa_status_t nsa_sel_attn_fwd_profiled(const void* q, const void* k, const void* v,
+                                       const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                       int hq, int hkv, int head_dim, const int32_t* block_idx,
+                                       int topk, int block_size, float scale, void* out,
+                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       nsa_stream_t stream, void* const* events, int num_events,
+                                       int* num_launches) {
+    return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
+                    topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
+                    num_events, num_launches);
+}
+
+nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                              const float* lse, const void* dout, const int32_t* cu_seqlens,
+                              int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                              const int32_t* block_idx, int topk, int block_size, float scale,
+                              void* dq, void* dk, void* dv, void* workspace,
+                              size_t workspace_bytes, nsa_stream_t stream) {
+    return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
+                    head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
+                    workspace_bytes, stream, nullptr, 0, nullptr);
+}
+
+nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void* v,
+                                       const void* out, const float* lse, const void* dout,
+                                       const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                       int hq, int hkv, int head_dim, const int32_t* block_idx,
+                                       int topk, int block_size, float scale, void* dq, void* dk,
+                                       void* dv, void* workspace, size_t workspace_bytes,
+                                       nsa_stream_t stream, void* const* events, int num_events,
+                                       int* num_launches) {
+    return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
+                    head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
+                    workspace_bytes, stream, events, num_events, num_launches);
+}
+
+nsa_status_t nsa_sel_invert_index(const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                  int hkv, const int32_t* block_idx, int topk, int block_size,
+                                  int32_t* offsets, int32_t* entries, int32_t* counts,
+                                  void* workspace, size_t workspace_bytes, nsa_stream_t stream_) {
+    Dims D;
+    // hq = hkv (group 1) fixes the tile geometry; it does not change the inversion.
+    nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hkv, hkv, kHeadDim,
+                                  block_idx, topk, block_size, workspace, workspace_bytes, false, &D);
+    if (s != NSA_OK) return s;
+    if (!offsets || !entries || !counts || !aligned(offsets, 4) || !aligned(entries, 4) ||
+        !aligned(counts, 4))
+        return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    const Layout L = make_layout(D, false);
+    Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
+    if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) {
+        if (cudaMemsetAsync(counts, 0, 2 * sizeof(int32_t), stream) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int32_t) * ((size_t)D.nbk_cap + 1), stream) !=
+                cudaSuccess)
+            return NSA_ERR_CUDA;
+        return NSA_OK;
+    }
+    if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+    cudaError_t e = cudaMemcpyAsync(offsets, c.inv.offsets, sizeof(int32_t) * ((size_t)D.nbk_cap + 1),
+                                    cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(entries, c.inv.vals[c.inv.final_buf], sizeof(int32_t) * (size_t)D.nent,
+                            cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(counts, &c.st->nblocks_total, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(counts + 1, &c.st->nentries, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            stream);
+    return cuda_status(e);
+}
+
+nsa_status_t nsa_sel_validate_indices(const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                      int hkv, const int32_t* block_idx, int topk, int block_size,
+                                      long long* n_out_of_range, long long* n_duplicates,
+                                      void* workspace, size_t workspace_bytes,
+                                      nsa_stream_t stream_) {
+    if (!workspace || workspace_bytes < sizeof(DevStatus) || !aligned(workspace, 256))
+        return NSA_ERR_WORKSPACE;
+    if (!cu_seqlens || num_seqs < 1 || total_tokens < 0 || hkv < 1 || topk < 1 ||
+        block_size < 1 || (total_tokens > 0 && !block_idx))
+        return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    nsa_status_t s;
+    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_validate(cu_seqlens, num_seqs, total_tokens, hkv, block_idx, topk,
+                                         block_size, st, stream))) != NSA_OK)
+        return s;
+    DevStatus h;
+    if (cudaMemcpyAsync(&h, st, sizeof(DevStatus), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    if (n_out_of_range) *n_out_of_range = h.bad_range;
+    if (n_duplicates) *n_duplicates = h.bad_dup;
+    return (h.bad_range || h.bad_dup) ? NSA_ERR_BAD_INDEX : NSA_OK;
+}
+
+nsa_status_t nsa_sel_check_status(const void* workspace, nsa_stream_t stream_) {
+    if (!workspace || !aligned(workspace, 256)) return NSA_ERR_INVALID_ARG;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int code = 0;
+    if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return NSA_ERR_CUDA;
+    return static_cast<nsa_status_t>(code);
+}
+
+}  // extern "C"

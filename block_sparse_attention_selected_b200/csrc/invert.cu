@@ -1,0 +1,322 @@
+// invert.cu -- block-index inversion for selected-block attention.
+//
+// The FSA pages describe swapping the outer and inner loops of the NSA selection
+// kernel so that small GQA groups still fill the hardware tiles ("FSA: Efficient
+// Implementation of Native Sparse Attention" blog, second paragraph; the
+// "Relaxed-System-Lab/Flash-Sparse-Attention" project page, key-features table: a
+// main batched query-to-KV kernel).  Swapping the loops needs, for every
+// (KV head g, KV block B), the list of query rows that selected B.  This file builds
+// it as a stable counting sort of the (token, KV head, slot) entries by the bucket
+// key g * NB + B, so every list comes out in ascending token order and the result is
+// deterministic (bit-exact, independent of scheduling).
+//
+// Steps (all on the caller's stream, no host synchronisation):
+//   1. k_seq_blocks      global block offset of every sequence, cu_seqlens check
+//   2. per 8-bit digit:  k_sort_hist -> k_scan_excl -> k_sort_scatter (LSD radix,
+//                        stable: warp-ordered ranks with __match_any_sync)
+//   3. k_bucket_offsets  CSR offsets from the sorted keys
+//   4. k_tile_offsets    per-bucket 128-row tile and backward-chunk prefix sums
+#include "nsa_common.cuh"
+#include "nsa_kernels.h"
+
+namespace nsa {
+namespace {
+
+constexpr int kSortThreads = 256;
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kItems = kSortTile / kSortThreads;   // 16 entries per thread
+constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
+
+struct SortArgs {
+    const int32_t* cu;
+    int nseq, T, hkv, topk, bs;
+    const int32_t* bidx;
+    long long nent;
+    int nbk_cap;
+    const int32_t* blkoff;
+    const DevStatus* st;
+};
+
+// Block-wide inclusive scan of one int64 per thread (blockDim.x <= 1024).
+__device__ __forceinline__ unsigned long long block_incl_scan_u64(unsigned long long x,
+                                                                  unsigned long long* warp_tot) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int o = 1; o < 32; o <<= 1) {
+        unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        unsigned long long t = lane < nw ? warp_tot[lane] : 0ull;
+        for (int o = 1; o < 32; o <<= 1) {
+            unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, t, o);
+            if (lane >= o) t += y;
+        }
+        warp_tot[lane] = t;
+    }
+    __syncthreads();
+    unsigned long long r = x + (w > 0 ? warp_tot[w - 1] : 0ull);
+    __syncthreads();
+    return r;
+}
+
+// 1. blkoff[s] = sum_{s' < s} ceil(L_s' / bs); checks cu_seqlens.
+__global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq, int T, int bs,
+                                                     int32_t* blkoff, DevStatus* st) {
+    __shared__ unsigned long long warp_tot[32];
+    __shared__ unsigned long long round_total;
+    __shared__ int bad;
+    if (threadIdx.x == 0) bad = (cu[0] != 0 || cu[nseq] != T) ? 1 : 0;
+    __syncthreads();
+    unsigned long long carry = 0;
+    for (int base = 0; base < nseq; base += blockDim.x) {
+        int s = base + threadIdx.x;
+        unsigned long long nb = 0;
+        if (s < nseq) {
+            int L = cu[s + 1] - cu[s];
+            if (L < 0) bad = 1;
+            nb = L > 0 ? (unsigned long long)((L + bs - 1) / bs) : 0ull;
+        }
+        unsigned long long incl = block_incl_scan_u64(nb, warp_tot);
+        if (s < nseq) blkoff[s] = (int32_t)(carry + incl - nb);
+        // total of this round = inclusive value of the last thread
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        blkoff[nseq] = (int32_t)carry;
+        st->nblocks_total = (int)carry;
+        if (bad) record_error(st, NSA_ERR_BAD_INDEX, 1);
+    }
+}
+
+// Bucket key of entry e (token-major, then KV head, then slot); kInvalidKey if the
+// entry selects nothing (padding, future or out-of-range block).
+__device__ __forceinline__ uint32_t entry_key(const SortArgs& a, long long e, uint32_t nbtot,
+                                              uint32_t* val) {
+    int j = (int)(e % a.topk);
+    long long r = e / a.topk;
+    int g = (int)(r % a.hkv);
+    int t = (int)(r / a.hkv);
+    *val = (uint32_t)t * 64u + (uint32_t)j;
+    int b = __ldg(a.bidx + e);
+    int s = seq_of_token(a.cu, a.nseq, t);
+    int i = t - __ldg(a.cu + s);
+    int qb = i >= 0 ? i / a.bs : -1;
+    if (!block_valid(b, qb)) return kInvalidKey;
+    uint32_t key = (uint32_t)g * nbtot + (uint32_t)__ldg(a.blkoff + s) + (uint32_t)b;
+    return key < (uint32_t)a.nbk_cap ? key : kInvalidKey;
+}
+
+// 2a. per-tile digit histogram, stored digit-major: hist[d * ntiles + tile].
+template <bool kFirst>
+__global__ void __launch_bounds__(kSortThreads) k_sort_hist(SortArgs a, const uint32_t* keys_in,
+                                                           int shift, uint32_t* hist) {
+    __shared__ uint32_t h[256];
+    h[threadIdx.x] = 0;
+    __syncthreads();
+    const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
+    const long long base = (long long)blockIdx.x * kSortTile;
+    for (int it = 0; it < kItems; ++it) {
+        long long e = base + it * kSortThreads + threadIdx.x;
+        if (e < a.nent) {
+            uint32_t v;
+            uint32_t key = kFirst ? entry_key(a, e, nbtot, &v) : keys_in[e];
+            atomicAdd(&h[(key >> shift) & 255u], 1u);
+        }
+    }
+    __syncthreads();
+    hist[(size_t)threadIdx.x * gridDim.x + blockIdx.x] = h[threadIdx.x];
+}
+
+// 2b. in-place exclusive scan of n uint32 values by one block.
+__global__ void __launch_bounds__(1024) k_scan_excl(uint32_t* a, long long n) {
+    __shared__ unsigned long long warp_tot[32];
+    const long long per = (n + blockDim.x - 1) / blockDim.x;
+    const long long lo = per * threadIdx.x;
+    const long long hi = min(lo + per, n);
+    unsigned long long sum = 0;
+    for (long long i = lo; i < hi; ++i) sum += a[i];
+    unsigned long long incl = block_incl_scan_u64(sum, warp_tot);
+    unsigned long long run = incl - sum;
+    for (long long i = lo; i < hi; ++i) {
+        uint32_t x = a[i];
+        a[i] = (uint32_t)run;
+        run += x;
+    }
+}
+
+// 2c. stable scatter of one tile by the digit at `shift`.
+template <bool kFirst>
+__global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const uint32_t* keys_in,
+                                                              const uint32_t* vals_in, int shift,
+                                                              const uint32_t* hist_scan,
+                                                              uint32_t* keys_out,
+                                                              uint32_t* vals_out) {
+    __shared__ uint32_t whist[kSortWarps][256];
+    __shared__ uint32_t tile_base[256];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    for (int i = tid; i < kSortWarps * 256; i += kSortThreads) (&whist[0][0])[i] = 0;
+    tile_base[tid] = hist_scan[(size_t)tid * gridDim.x + blockIdx.x];
+    __syncthreads();
+    const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
+    const long long base = (long long)blockIdx.x * kSortTile + (long long)w * (kItems * 32);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t key[kItems], val[kItems], rank[kItems];
+    for (int it = 0; it < kItems; ++it) {
+        long long e = base + it * 32 + lane;
+        uint32_t d = 256u;   // sentinel for entries past the end
+        if (e < a.nent) {
+            key[it] = kFirst ? entry_key(a, e, nbtot, &val[it]) : keys_in[e];
+            if (!kFirst) val[it] = vals_in[e];
+            d = (key[it] >> shift) & 255u;
+        }
+        uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
+        uint32_t before = __popc(peers & lt_mask);
+        if (d < 256u) rank[it] = whist[w][d] + before;
+        __syncwarp();
+        if (d < 256u && before == 0) whist[w][d] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    {   // exclusive prefix of each digit over the warps of the tile
+        uint32_t run = 0;
+        for (int ww = 0; ww < kSortWarps; ++ww) {
+            uint32_t c = whist[ww][tid];
+            whist[ww][tid] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (int it = 0; it < kItems; ++it) {
+        long long e = base + it * 32 + lane;
+        if (e < a.nent) {
+            uint32_t d = (key[it] >> shift) & 255u;
+            uint32_t pos = tile_base[d] + whist[w][d] + rank[it];
+            keys_out[pos] = key[it];
+            vals_out[pos] = val[it];
+        }
+    }
+}
+
+// 3. offsets[B] = number of sorted keys below B, for B in [0, hkv * NB].
+__global__ void k_bucket_offsets(const uint32_t* keys, long long nent, const DevStatus* st,
+                                 int hkv, int32_t* offsets) {
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i > nent) return;
+    const long long nbk = (long long)hkv * st->nblocks_total;
+    long long prev = i == 0 ? -1 : min((long long)keys[i - 1], nbk);
+    long long cur = i == nent ? nbk : min((long long)keys[i], nbk);
+    for (long long B = prev + 1; B <= cur; ++B) offsets[B] = (int32_t)i;
+}
+
+// 4. tile and chunk prefix sums per bucket; totals into the status block.
+__global__ void __launch_bounds__(1024) k_tile_offsets(const int32_t* offsets, DevStatus* st,
+                                                       int hkv, int tpt, int chunk_tiles,
+                                                       int32_t* tile_off, int32_t* chunk_off) {
+    __shared__ unsigned long long warp_tot[32];
+    __shared__ unsigned long long round_total;
+    const long long nbk = (long long)hkv * st->nblocks_total;
+    unsigned long long carry = 0;   // (chunks << 32) | tiles
+    for (long long base = 0; base < nbk; base += blockDim.x) {
+        long long B = base + threadIdx.x;
+        unsigned long long x = 0;
+        if (B < nbk) {
+            long long cnt = offsets[B + 1] - offsets[B];
+            unsigned long long nt = (unsigned long long)((cnt + tpt - 1) / tpt);
+            unsigned long long nc = (nt + chunk_tiles - 1) / chunk_tiles;
+            x = (nc << 32) | nt;
+        }
+        unsigned long long incl = block_incl_scan_u64(x, warp_tot);
+        unsigned long long ex = carry + incl - x;
+        if (B < nbk) {
+            tile_off[B] = (int32_t)(ex & 0xFFFFFFFFull);
+            chunk_off[B] = (int32_t)(ex >> 32);
+        }
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        tile_off[nbk] = (int32_t)(carry & 0xFFFFFFFFull);
+        chunk_off[nbk] = (int32_t)(carry >> 32);
+        st->ntiles = (int)(carry & 0xFFFFFFFFull);
+        st->nchunks = (int)(carry >> 32);
+        st->nentries = offsets[nbk];
+    }
+}
+
+// Range / duplicate check of block_idx (one thread per (token, KV head) row).
+__global__ void k_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
+                           int topk, int bs, DevStatus* st) {
+    long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= (long long)T * hkv) return;
+    int t = (int)(r / hkv);
+    int s = seq_of_token(cu, nseq, t);
+    int L = cu[s + 1] - cu[s];
+    int nb = L > 0 ? (L + bs - 1) / bs : 0;
+    const int32_t* row = bidx + r * topk;
+    long long bad = 0, dup = 0;
+    for (int j = 0; j < topk; ++j) {
+        int b = row[j];
+        if (b == -1) continue;
+        if (b < -1 || b >= nb) ++bad;
+        if (b >= 0)
+            for (int j2 = 0; j2 < j; ++j2)
+                if (row[j2] == b) { ++dup; break; }
+    }
+    if (bad) atomicAdd(reinterpret_cast<unsigned long long*>(&st->bad_range),
+                       (unsigned long long)bad);
+    if (dup) atomicAdd(reinterpret_cast<unsigned long long*>(&st->bad_dup),
+                       (unsigned long long)dup);
+}
+
+}  // namespace
+
+cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
+    k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st);
+    SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
+    const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
+    const uint32_t* kin = nullptr;
+    const uint32_t* vin = nullptr;
+    for (int pass = 0; pass < passes; ++pass) {
+        const int shift = 8 * pass;
+        uint32_t* kout = p.keys[pass & 1];
+        uint32_t* vout = p.vals[pass & 1];
+        if (pass == 0)
+            k_sort_hist<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, nullptr, shift, p.hist);
+        else
+            k_sort_hist<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, shift, p.hist);
+        k_scan_excl<<<1, 1024, 0, stream>>>(p.hist, 256ll * p.sort_tiles);
+        if (pass == 0)
+            k_sort_scatter<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(
+                a, nullptr, nullptr, shift, p.hist, kout, vout);
+        else
+            k_sort_scatter<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, vin, shift,
+                                                                            p.hist, kout, vout);
+        kin = kout;
+        vin = vout;
+    }
+    p.final_buf = (passes - 1) & 1;
+    const long long n1 = p.nent + 1;
+    k_bucket_offsets<<<(unsigned)((n1 + 255) / 256), 256, 0, stream>>>(p.keys[p.final_buf], p.nent,
+                                                                      p.st, p.hkv, p.offsets);
+    k_tile_offsets<<<1, 1024, 0, stream>>>(p.offsets, p.st, p.hkv, p.tokens_per_tile,
+                                           p.chunk_tiles, p.tile_off, p.chunk_off);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
+                            int topk, int bs, DevStatus* st, cudaStream_t stream) {
+    long long rows = (long long)T * hkv;
+    if (rows > 0)
+        k_validate<<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(cu, nseq, T, hkv, bidx,
+                                                                        topk, bs, st);
+    return cudaGetLastError();
+}
+
+}  // namespace nsa

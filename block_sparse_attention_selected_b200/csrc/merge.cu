@@ -1,0 +1,180 @@
+// merge.cu -- the memory-bound passes around the tensor-core kernels.
+//
+//  k_merge         forward: per (token, query head) the log-sum-exp merge of the
+//                  per-block partials, O = sum_j e^{lse_j - LSE} o_j and
+//                  LSE = log sum_j e^{lse_j}; one warp per row, no atomics (the
+//                  reduction / online-softmax kernels of the key-features table on
+//                  the "Relaxed-System-Lab/Flash-Sparse-Attention" project page).
+//  k_bwd_delta     backward preprocess D = rowsum(dO * O) (fp32, [hq, T]).
+//  k_dq_merge      backward: dQ = sum over the row's slots of the dQ partials.
+//  k_dkdv_reduce   backward: dK, dV of every key = sum over the backward work
+//                  units of its (KV head, block), in unit order (deterministic).
+#include <math_constants.h>
+
+#include "nsa_common.cuh"
+#include "nsa_kernels.h"
+
+namespace nsa {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ float warp_max(float x) {
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    return x;
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= (long long)p.T * p.hq) return;
+    const int t = (int)(row / p.hq);
+    const int h = (int)(row - (long long)t * p.hq);
+    const int g = h / (p.hq / p.hkv);
+    const int s = seq_of_token(p.cu, p.nseq, t);
+    const int qb = (t - __ldg(p.cu + s)) / p.bs;
+    const int32_t* bi = p.bidx + ((size_t)t * p.hkv + g) * p.topk;
+    const size_t prow0 = (size_t)row * p.topk;
+
+    float l0 = -CUDART_INF_F, l1 = -CUDART_INF_F;
+    if (lane < p.topk && block_valid(__ldg(bi + lane), qb)) l0 = __ldg(p.part_lse + prow0 + lane);
+    if (lane + 32 < p.topk && block_valid(__ldg(bi + lane + 32), qb))
+        l1 = __ldg(p.part_lse + prow0 + lane + 32);
+    const float M = warp_max(fmaxf(l0, l1));
+    uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                           (size_t)row * kHeadDim) + lane;
+    if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
+        *outp = make_uint2(0u, 0u);
+        if (lane == 0) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
+        return;
+    }
+    const float w0 = l0 == -CUDART_INF_F ? 0.f : __expf(l0 - M);
+    const float w1 = l1 == -CUDART_INF_F ? 0.f : __expf(l1 - M);
+    const float Lam = warp_sum(w0 + w1);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint2* po = reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.part_o) +
+                                                     prow0 * kHeadDim) + lane;
+    for (int j = 0; j < p.topk; ++j) {
+        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? w0 : w1, j & 31);
+        if (wj == 0.f) continue;       // warp-uniform
+        const uint2 u = __ldg(po + (size_t)j * (kHeadDim / 4));
+        const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+        acc[0] = fmaf(wj, a.x, acc[0]);
+        acc[1] = fmaf(wj, a.y, acc[1]);
+        acc[2] = fmaf(wj, b.x, acc[2]);
+        acc[3] = fmaf(wj, b.y, acc[3]);
+    }
+    const float inv = 1.f / Lam;
+    *outp = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    if (lane == 0) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* out, const void* dout,
+                                                                  float* delta, int T, int hq) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= (long long)T * hq) return;
+    const uint2 o = __ldg(reinterpret_cast<const uint2*>(out) + row * (kHeadDim / 4) + lane);
+    const uint2 d = __ldg(reinterpret_cast<const uint2*>(dout) + row * (kHeadDim / 4) + lane);
+    const float2 o0 = unpack_bf16x2(o.x), o1 = unpack_bf16x2(o.y);
+    const float2 d0 = unpack_bf16x2(d.x), d1 = unpack_bf16x2(d.y);
+    float x = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
+    x = warp_sum(x);
+    if (lane == 0) {
+        const int t = (int)(row / hq), h = (int)(row - (long long)t * hq);
+        delta[(size_t)h * T + t] = x;
+    }
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan p, const int32_t* bidx,
+                                                                 void* dq) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= (long long)p.T * p.hq) return;
+    const int t = (int)(row / p.hq);
+    const int h = (int)(row - (long long)t * p.hq);
+    const int g = h / p.G;
+    const int s = seq_of_token(p.cu, p.nseq, t);
+    const int qb = (t - __ldg(p.cu + s)) / p.bs;
+    const int32_t* bi = bidx + ((size_t)t * p.hkv + g) * p.topk;
+    const uint2* pd = reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.part_dq) +
+                                                     (size_t)row * p.topk * kHeadDim) + lane;
+    const int b0 = lane < p.topk ? __ldg(bi + lane) : -1;
+    const int b1 = lane + 32 < p.topk ? __ldg(bi + lane + 32) : -1;
+    const unsigned v0 = __ballot_sync(0xFFFFFFFFu, block_valid(b0, qb));
+    const unsigned v1 = __ballot_sync(0xFFFFFFFFu, block_valid(b1, qb));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < p.topk; ++j) {
+        const bool ok = j < 32 ? ((v0 >> j) & 1u) : ((v1 >> (j - 32)) & 1u);
+        if (!ok) continue;
+        const uint2 u = __ldg(pd + (size_t)j * (kHeadDim / 4));
+        const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+        acc[0] += a.x;
+        acc[1] += a.y;
+        acc[2] += b.x;
+        acc[3] += b.y;
+    }
+    uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dq) + (size_t)row * kHeadDim) + lane;
+    *o = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+}
+
+// One warp per (key token, KV head); each lane owns 4 of the 128 columns.
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dkdv_reduce(const BwdPlan p, void* dk, void* dv) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= (long long)p.T * p.hkv) return;
+    const int t = (int)(row / p.hkv);
+    const int g = (int)(row - (long long)t * p.hkv);
+    const int s = seq_of_token(p.cu, p.nseq, t);
+    const int i = t - __ldg(p.cu + s);
+    const int b = i / p.bs;
+    const int r = i - b * p.bs;
+    const int nbtot = __ldg(p.blkoff + p.nseq);
+    const int bucket = g * nbtot + __ldg(p.blkoff + s) + b;
+    const int c0 = __ldg(p.chunk_off + bucket), c1 = __ldg(p.chunk_off + bucket + 1);
+    float4 av = make_float4(0.f, 0.f, 0.f, 0.f), ak = av;
+    for (int c = c0; c < c1; ++c) {
+        const float* base = p.part_dkdv + ((size_t)c * 2 * p.bs + r) * kHeadDim;
+        const float4 x = __ldg(reinterpret_cast<const float4*>(base) + lane);
+        const float4 y = __ldg(reinterpret_cast<const float4*>(base + (size_t)p.bs * kHeadDim) + lane);
+        av.x += x.x; av.y += x.y; av.z += x.z; av.w += x.w;
+        ak.x += y.x; ak.y += y.y; ak.z += y.z; ak.w += y.w;
+    }
+    uint2* ov = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dv) + (size_t)row * kHeadDim) + lane;
+    uint2* ok = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dk) + (size_t)row * kHeadDim) + lane;
+    *ov = make_uint2(pack_bf16x2(av.x, av.y), pack_bf16x2(av.z, av.w));
+    *ok = make_uint2(pack_bf16x2(ak.x, ak.y), pack_bf16x2(ak.z, ak.w));
+}
+
+inline unsigned blocks_for(long long rows) {
+    return (unsigned)((rows + kWarpsPerBlock - 1) / kWarpsPerBlock);
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
+    k_merge<<<blocks_for((long long)p.T * p.hq), kWarpsPerBlock * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
+                                  cudaStream_t stream) {
+    k_bwd_delta<<<blocks_for((long long)T * hq), kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq, cudaStream_t stream) {
+    k_dq_merge<<<blocks_for((long long)p.T * p.hq), kWarpsPerBlock * 32, 0, stream>>>(p, bidx, dq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStream_t stream) {
+    k_dkdv_reduce<<<blocks_for((long long)p.T * p.hkv), kWarpsPerBlock * 32, 0, stream>>>(p, dk, dv);
+    return cudaGetLastError();
+}
+
+}  // namespace nsa

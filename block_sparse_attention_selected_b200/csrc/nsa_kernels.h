@@ -1,0 +1,109 @@
+// nsa_kernels.h -- internal launch interface between the C ABI (api.cu) and the
+// kernels.  Not installed; the public interface is include/nsa_sel.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nsa {
+
+struct DevStatus;
+
+// Everything the index inversion reads and writes.
+struct InvertPlan {
+    const int32_t* cu;       // [nseq + 1]
+    int nseq;
+    int T;
+    int hkv;
+    const int32_t* bidx;     // [T, hkv, topk]
+    int topk;
+    int bs;
+    int tokens_per_tile;     // 128 / G (query heads per KV head)
+    int chunk_tiles;         // tiles per backward work unit
+    long long nent;          // T * hkv * topk
+    int nbk_cap;             // hkv * (T / bs + nseq): bound on buckets
+    int key_bits;            // bits of the bucket key
+    int sort_tiles;          // ceil(nent / kSortTile)
+    // workspace views
+    int32_t* blkoff;         // [nseq + 1]
+    uint32_t* keys[2];       // [nent] ping-pong
+    uint32_t* vals[2];       // [nent] ping-pong
+    uint32_t* hist;          // [256 * sort_tiles]
+    int32_t* offsets;        // [nbk_cap + 1]
+    int32_t* tile_off;       // [nbk_cap + 1]
+    int32_t* chunk_off;      // [nbk_cap + 1]
+    DevStatus* st;
+    // result: the sorted values live in vals[final_buf]
+    int final_buf;
+};
+
+constexpr int kSortTile = 4096;  // entries per sort tile (256 threads x 16)
+
+// Runs the inversion on `stream`; returns the first launch error.
+cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream);
+
+struct FwdPlan {
+    const void* q;
+    const int32_t* cu;
+    int nseq, T, hq, hkv, topk, bs, G;
+    float scale_log2;        // scale * log2(e)
+    const int32_t* blkoff;
+    const int32_t* offsets;  // bucket offsets into entries
+    const int32_t* tile_off; // bucket tile offsets
+    const uint32_t* entries; // token * 64 + slot
+    int nbk_cap;
+    void* part_o;            // bf16 [T * hq * topk, 128]
+    float* part_lse;         // fp32 [T * hq * topk]
+    DevStatus* st;
+    int num_sms;
+};
+
+cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                             cudaStream_t stream);
+
+struct MergePlan {
+    const int32_t* cu;
+    int nseq, T, hq, hkv, topk, bs;
+    const int32_t* bidx;
+    const void* part_o;
+    const float* part_lse;
+    void* out;
+    float* lse;
+};
+
+cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream);
+
+struct BwdPlan {
+    const void* q;
+    const void* dout;
+    const float* lse;        // [hq, T]
+    float* delta;            // [hq, T]  rowsum(dout * out)
+    const int32_t* cu;
+    int nseq, T, hq, hkv, topk, bs, G;
+    float scale, scale_log2;
+    const int32_t* blkoff;
+    const int32_t* offsets;
+    const int32_t* tile_off;
+    const int32_t* chunk_off;
+    const uint32_t* entries;
+    int nbk_cap;
+    int chunk_tiles;
+    void* part_dq;           // bf16 [T * hq * topk, 128]
+    float* part_dkdv;        // fp32 [chunks, 2, bs, 128]
+    DevStatus* st;
+    int num_sms;
+};
+
+cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
+                                  cudaStream_t stream);
+cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                             cudaStream_t stream);
+cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq,
+                                cudaStream_t stream);
+cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStream_t stream);
+
+cudaError_t launch_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
+                            int topk, int bs, DevStatus* st, cudaStream_t stream);
+
+}  // namespace nsa

@@ -1,0 +1,165 @@
+/*
+ * nsa_sel.h -- C ABI of the B200 (sm_100a) selected-block attention library
+ * (Native Sparse Attention, selection branch: each query attends only to the
+ * KV blocks chosen for its sequence and KV head).
+ *
+ * Sources for the operation:
+ *  - "Relaxed-System-Lab/Flash-Sparse-Attention" project page, Quick-start section:
+ *    block_size (64), topk (16), init_blocks (1), local_blocks (2), GQA head counts,
+ *    head_dim 128, and varlen packing through cu_seqlens (int32 cumulative lengths
+ *    with a leading 0).  Same page, Limitations section: Q, K and V share one head
+ *    dimension.  Same page, key-features table: a main query-to-KV kernel plus
+ *    reduction and online-softmax kernels with no atomics; forward-only prefill and
+ *    full backward.
+ *  - "FSA: Efficient Implementation of Native Sparse Attention" blog page, second
+ *    paragraph: the kernel swaps the loop order so that small GQA groups still fill
+ *    the hardware tiles.
+ *
+ * Definition computed (token t of sequence s, local position i, query block
+ * qb = i / block_size, query head h, KV head g = h / (hq / hkv)):
+ *     Sel  = { block_idx[t, g, j] : 0 <= value <= qb }        (-1 pads)
+ *     J    = { keys j of the blocks in Sel : j <= i }        (causal)
+ *     O[t, h]   = softmax_j(scale * q[t,h] . k[j,g]) . v[j,g]
+ *     LSE[h, t] = natural log of sum_j exp(scale * q[t,h] . k[j,g])
+ * An empty J gives O = 0 and LSE = -inf.  Block numbers are local to each sequence.
+ * Indices in one (t, g) row must be distinct (nsa_sel_validate_indices checks).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers, contiguous, in the layouts stated.
+ *    bf16 tensors and the workspace must be 16-byte aligned, int32/fp32 ones
+ *    4-byte aligned.
+ *  - The caller owns every buffer, including the workspace; the library allocates
+ *    nothing and keeps no state between calls.
+ *  - Work is enqueued on `stream` (a cudaStream_t); no call synchronises except
+ *    nsa_sel_validate_indices and nsa_sel_check_status.
+ *  - Argument errors are detected on the host before any launch and leave the
+ *    outputs untouched.  Launch failures return NSA_ERR_CUDA.  Device-side
+ *    problems (a bounded wait that expired, malformed cu_seqlens) are recorded
+ *    in the status block at the start of the workspace and read with
+ *    nsa_sel_check_status.  No C++ exception crosses this interface.
+ *  - Supported domain: bf16, head_dim == 128, block_size in {64, 128},
+ *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv <= 16, total_tokens < 2^25.
+ *    Anything else returns NSA_ERR_UNSUPPORTED.
+ */
+#ifndef NSA_SEL_H
+#define NSA_SEL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NSA_API __attribute__((visibility("default")))
+#else
+#define NSA_API
+#endif
+
+typedef struct CUstream_st *nsa_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+    NSA_OK = 0,
+    NSA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, negative size, bad shape */
+    NSA_ERR_UNSUPPORTED = 2,  /* outside the supported domain above */
+    NSA_ERR_WORKSPACE = 3,    /* workspace smaller than nsa_sel_attn_workspace_size() */
+    NSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    NSA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (kernel returned) */
+    NSA_ERR_BAD_INDEX = 6,    /* block_idx or cu_seqlens content is invalid */
+    NSA_ERR_NO_DEVICE = 7     /* no sm_100 device is current */
+} nsa_status_t;
+
+/* Bytes of workspace that nsa_sel_attn_fwd (for_bwd = 0) or nsa_sel_attn_bwd
+ * (for_bwd = 1) needs for these sizes; 0 when the sizes are unsupported.  The first
+ * 256 bytes are the device status block. */
+NSA_API size_t nsa_sel_attn_workspace_size(int total_tokens, int num_seqs, int hq, int hkv,
+                                   int head_dim, int topk, int block_size, int for_bwd);
+
+/* Forward selected-block attention (definition in the file header).
+ *   q   bf16 [total_tokens, hq, head_dim]        k, v bf16 [total_tokens, hkv, head_dim]
+ *   cu_seqlens int32 [num_seqs + 1], cu_seqlens[0] = 0, non-decreasing,
+ *              cu_seqlens[num_seqs] = total_tokens
+ *   block_idx  int32 [total_tokens, hkv, topk], block numbers local to the sequence
+ *   out  bf16 [total_tokens, hq, head_dim] (written)
+ *   lse  fp32 [hq, total_tokens] (written; natural log)
+ * Steps on `stream`: block-index inversion, the tensor-core tile kernel over
+ * (KV block, gathered query rows), and the log-sum-exp merge of the per-block
+ * partial results. */
+NSA_API nsa_status_t nsa_sel_attn_fwd(const void *q, const void *k, const void *v,
+                              const int32_t *cu_seqlens, int num_seqs, int total_tokens,
+                              int hq, int hkv, int head_dim, const int32_t *block_idx,
+                              int topk, int block_size, float scale, void *out, float *lse,
+                              void *workspace, size_t workspace_bytes, nsa_stream_t stream);
+
+/* Backward of the forward above for the loss gradient dout = dL/dO.
+ *   out, lse   the forward's outputs (same layouts)
+ *   dout       bf16 [total_tokens, hq, head_dim]
+ *   dq         bf16 [total_tokens, hq, head_dim] (written)
+ *   dk, dv     bf16 [total_tokens, hkv, head_dim] (written; keys that no query
+ *              attends get 0)
+ * Uses D = rowsum(dout * out) from the bf16 `out`.  Deterministic: the sums over
+ * query rows run in a fixed order. */
+NSA_API nsa_status_t nsa_sel_attn_bwd(const void *q, const void *k, const void *v, const void *out,
+                              const float *lse, const void *dout, const int32_t *cu_seqlens,
+                              int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                              const int32_t *block_idx, int topk, int block_size, float scale,
+                              void *dq, void *dk, void *dv, void *workspace,
+                              size_t workspace_bytes, nsa_stream_t stream);
+
+/* Instrumented forms of the two calls above, used for measurement.  Identical work;
+ * in addition, when events is non-null, events[i] (cudaEvent_t, created by the caller)
+ * is recorded on `stream` at phase boundary i, for i < num_events:
+ *   forward:  0 start, 1 inversion done, 2 tile kernel done, 3 merge done
+ *   backward: 0 start, 1 inversion done, 2 D = rowsum(dO * O) done, 3 tile kernel
+ *             done, 4 dQ merge done, 5 dK / dV reduction done
+ * and *num_launches (when non-null) receives the number of kernels launched. */
+NSA_API nsa_status_t nsa_sel_attn_fwd_profiled(
+    const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
+    int total_tokens, int hq, int hkv, int head_dim, const int32_t *block_idx, int topk,
+    int block_size, float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+    nsa_stream_t stream, void *const *events, int num_events, int *num_launches);
+NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
+    const void *q, const void *k, const void *v, const void *out, const float *lse,
+    const void *dout, const int32_t *cu_seqlens, int num_seqs, int total_tokens, int hq, int hkv,
+    int head_dim, const int32_t *block_idx, int topk, int block_size, float scale, void *dq,
+    void *dk, void *dv, void *workspace, size_t workspace_bytes, nsa_stream_t stream,
+    void *const *events, int num_events, int *num_launches);
+
+/* The block-index inversion on its own (the loop swap named in the file header):
+ * for KV head g and global block B (blocks of earlier sequences first), the list of
+ * entries token * 64 + slot with block_idx[token, g, slot] = local block of B and
+ * 0 <= value <= qb(token), ascending.
+ *   offsets  int32 [hkv * NB + 1], NB = sum_s ceil(L_s / block_size); exclusive
+ *            prefix sums over (g major, B minor).  Room for
+ *            hkv * (total_tokens / block_size + num_seqs) + 1 values is required.
+ *   entries  int32 [total_tokens * hkv * topk] room; the first offsets[hkv*NB] are set.
+ *   counts   int32 [2] (written): NB and the number of entries.
+ * Uses the forward workspace size. */
+NSA_API nsa_status_t nsa_sel_invert_index(const int32_t *cu_seqlens, int num_seqs, int total_tokens,
+                                  int hkv, const int32_t *block_idx, int topk, int block_size,
+                                  int32_t *offsets, int32_t *entries, int32_t *counts,
+                                  void *workspace, size_t workspace_bytes, nsa_stream_t stream);
+
+/* Host-synchronous check of block_idx: counts values outside {-1} U [0, NB_s) and
+ * repeated non-negative values within one (token, KV head) row.  Returns
+ * NSA_ERR_BAD_INDEX when either count is non-zero, NSA_OK otherwise.  Future blocks
+ * (qb < value < NB_s) are allowed and contribute nothing. */
+NSA_API nsa_status_t nsa_sel_validate_indices(const int32_t *cu_seqlens, int num_seqs,
+                                      int total_tokens, int hkv, const int32_t *block_idx,
+                                      int topk, int block_size, long long *n_out_of_range,
+                                      long long *n_duplicates, void *workspace,
+                                      size_t workspace_bytes, nsa_stream_t stream);
+
+/* Synchronises `stream` and returns the device-side status of the last call that
+ * used this workspace (NSA_OK, NSA_ERR_TIMEOUT or NSA_ERR_BAD_INDEX). */
+NSA_API nsa_status_t nsa_sel_check_status(const void *workspace, nsa_stream_t stream);
+
+/* Static string for a status code. */
+NSA_API const char *nsa_sel_status_string(nsa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_SEL_H */

@@ -28,13 +28,28 @@ import numpy as np
 INDEX_SEED_OFFSET = 1_000_003
 
 
-def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to the nearest bfloat16 (ties to even); return float32."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    bits = x.view(np.uint32).astype(np.uint64)
-    lsb = (bits >> 16) & 1
-    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
-    return rounded.astype(np.uint32).view(np.float32).reshape(x.shape)
+def bf16_round(x: np.ndarray, inplace: bool = False) -> np.ndarray:
+    """Round finite float32 values to the nearest bfloat16 (ties to even); return float32.
+
+    On the uint32 bit patterns: add 0x7FFF plus the lowest kept bit, then clear the
+    16 dropped bits.  Chunked, so that large arrays need no big temporaries.
+    """
+    if inplace and isinstance(x, np.ndarray) and x.dtype == np.float32 and x.flags.c_contiguous:
+        out = x
+    else:
+        out = np.array(x, dtype=np.float32, copy=True, order="C")
+    bits = out.reshape(-1).view(np.uint32)
+    chunk = 1 << 22
+    lsb = np.empty(min(chunk, bits.size), dtype=np.uint32)
+    for a in range(0, bits.size, chunk):
+        seg = bits[a:a + chunk]
+        t = lsb[:seg.size]
+        np.right_shift(seg, 16, out=t)
+        t &= np.uint32(1)
+        seg += np.uint32(0x7FFF)
+        seg += t
+        seg &= np.uint32(0xFFFF0000)
+    return out
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -153,10 +168,11 @@ def make_problem(lengths, hq: int, hkv: int, head_dim: int = 128, block_size: in
     cu = cu_seqlens_from_lengths(lengths)
     T = int(cu[-1])
     rng = np.random.Generator(np.random.PCG64(seed))
-    q = bf16_round(rng.standard_normal((T, hq, head_dim), dtype=np.float32))
-    k = bf16_round(rng.standard_normal((T, hkv, head_dim), dtype=np.float32))
-    v = bf16_round(rng.standard_normal((T, hkv, head_dim), dtype=np.float32))
-    dout = bf16_round(rng.standard_normal((T, hq, head_dim), dtype=np.float32)) if with_dout else None
+    draw = lambda shape: bf16_round(rng.standard_normal(shape, dtype=np.float32), inplace=True)
+    q = draw((T, hq, head_dim))
+    k = draw((T, hkv, head_dim))
+    v = draw((T, hkv, head_dim))
+    dout = draw((T, hq, head_dim)) if with_dout else None
     if block_idx is None:
         block_idx = make_block_idx(cu, hkv, topk, block_size, seed)
     return Problem(name=name, cu_seqlens=cu, hq=hq, hkv=hkv, head_dim=head_dim,

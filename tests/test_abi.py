@@ -1,0 +1,103 @@
+"""The C ABI library builds, loads and exports every symbol of include/nsa_sel.h.
+
+CPU only: no call here reaches a CUDA kernel.  Argument checks run on the host
+before any device work, so their error codes can be checked without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_selected_b200 as nsa
+from block_sparse_attention_selected_b200 import build as nsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nsa_sel.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nsa_build.build()
+    return nsa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_sel_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(nsa.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        s = lib.nsa_sel_status_string(code)
+        assert s and s != b"unknown status"
+    assert lib.nsa_sel_status_string(99) == b"unknown status"
+
+
+def test_workspace_size_domain(lib):
+    ws = nsa.nsa_sel_attn_workspace_size
+    base = ws(65536, 1, 16, 4, 128, 16, 64, False)
+    # partial results dominate: T * hq * topk rows of 128 bf16 + one fp32
+    assert base >= 65536 * 16 * 16 * (256 + 4)
+    assert ws(65536, 1, 16, 4, 128, 16, 64, True) > base
+    assert ws(0, 1, 4, 4, 128, 8, 64, False) > 0
+    f = lib.nsa_sel_attn_workspace_size
+    assert f(1024, 1, 4, 4, 64, 8, 64, 0) == 0          # head_dim 64 not supported
+    assert f(1024, 1, 4, 4, 128, 8, 32, 0) == 0         # block 32 not supported
+    assert f(1024, 1, 4, 4, 128, 65, 64, 0) == 0        # topk > 64
+    assert f(1024, 1, 64, 2, 128, 8, 64, 0) == 0        # group 32 > 16
+    assert f(1024, 1, 6, 4, 128, 8, 64, 0) == 0         # hq % hkv != 0
+    assert f(1 << 25, 1, 4, 4, 128, 8, 64, 0) == 0      # too many tokens
+
+
+def test_host_argument_errors(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)           # never dereferenced: checks fail first
+    # unsupported head_dim
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 64, fake, 8, 64, 0.1,
+                              fake, fake, fake, 1 << 30, None)
+    assert rc == 2
+    # null cu_seqlens
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, None, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
+                              fake, fake, fake, 1 << 30, None)
+    assert rc == 1
+    # workspace too small
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
+                              fake, fake, fake, 256, None)
+    assert rc == 3
+    # misaligned q
+    rc = lib.nsa_sel_attn_fwd(P((1 << 20) + 2), fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64,
+                              0.1, fake, fake, fake, 1 << 30, None)
+    assert rc == 1
+    # bad scale
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, -1.0,
+                              fake, fake, fake, 1 << 30, None)
+    assert rc == 1
+    # backward: hq % hkv
+    rc = lib.nsa_sel_attn_bwd(fake, fake, fake, fake, fake, fake, fake, 1, 64, 6, 4, 128, fake,
+                              8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None)
+    assert rc == 1
+    # inversion: bad block size
+    rc = lib.nsa_sel_invert_index(fake, 1, 64, 4, fake, 8, 96, fake, fake, fake, fake, 1 << 30,
+                                  None)
+    assert rc == 2
+    assert lib.nsa_sel_check_status(None, None) == 1
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The package and its sources never import, link or call the oracle."""
+    pkg = os.path.join(ROOT, "block_sparse_attention_selected_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.lower().replace("oracle_", ""), f

@@ -1,0 +1,277 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small problems are compared element by element over every output; the workloads
+at their full sizes are compared on stratified token / block samples that the
+oracle computes one by one.  Tolerances: max |dO| <= 1e-2 on bf16 O, <= 1e-3 on
+fp32 LSE, relative Frobenius <= 2e-2 on dQ, dK, dV; the inversion is bit-exact.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_selected_b200 as nsa
+import nsa_inputs as ni
+import oracle
+from gpu_util import TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, rel_fro, sample_tokens, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _perturb(p: ni.Problem, seed: int, frac: float = 0.05) -> ni.Problem:
+    """Shuffle every index row (moving the -1 pads) and plant future, out-of-range and
+    negative values in random slots (all must contribute nothing)."""
+    rng = np.random.default_rng(seed)
+    bi = p.block_idx.copy()
+    T, hkv, topk = bi.shape
+    idx = np.argsort(rng.random(bi.shape), axis=2)
+    bi = np.take_along_axis(bi, idx, axis=2)
+    pad = np.argwhere(bi == -1)
+    if len(pad):
+        pick = pad[rng.random(len(pad)) < frac * 4]
+        cu = p.cu_seqlens.astype(np.int64)
+        seq = np.searchsorted(cu, pick[:, 0], side="right") - 1
+        L = cu[seq + 1] - cu[seq]
+        nb = (L + p.block_size - 1) // p.block_size
+        kind = rng.integers(0, 3, size=len(pick))
+        vals = np.where(kind == 0, nb + 3, np.where(kind == 1, -7, nb - 1))   # oob, negative, last
+        bi[pick[:, 0], pick[:, 1], pick[:, 2]] = vals.astype(np.int32)
+        # "last block" is a future block for most tokens; keep rows distinct
+        for (t, g, _), v in zip(pick, vals):
+            row = bi[t, g]
+            if (row == v).sum() > 1:
+                row[np.nonzero(row == v)[0][1:]] = -1
+    p.block_idx = np.ascontiguousarray(bi)
+    return p
+
+
+def _fwd(p):
+    d = to_device(p)
+    out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], p.block_size,
+                                    p.scale)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    return d, out, lse
+
+
+def _check_fwd(p, out, lse, tokens=None):
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+                              tokens=tokens)
+    o = f64(out) if tokens is None else f64(out[torch.from_numpy(tokens).cuda()])
+    l = f64(lse).T if tokens is None else f64(lse[:, torch.from_numpy(tokens).cuda()]).T
+    eo, el = max_abs(o, o_ref), max_abs(l, l_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
+    return eo, el
+
+
+# ------------------------------------------------------------------------- inversion
+
+INV_CASES = [
+    ("tiny", dict(lengths=[2048], hq=4, hkv=4, block_size=64, topk=8, seed=1), False),
+    ("varlen_ragged", dict(lengths=[700, 37, 1, 515], hq=2, hkv=2, block_size=64, topk=16, seed=3), True),
+    ("bs128_k64", dict(lengths=[3000, 129], hq=4, hkv=1, block_size=128, topk=64, seed=5), True),
+    ("empty_seq", dict(lengths=[0, 300, 0, 65], hq=3, hkv=3, block_size=64, topk=5, seed=6), True),
+]
+
+
+@pytest.mark.parametrize("name,spec,perturb", INV_CASES, ids=[c[0] for c in INV_CASES])
+def test_invert_bit_exact_small(name, spec, perturb):
+    p = ni.make_problem(head_dim=8, with_dout=False, **spec)
+    if perturb:
+        p = _perturb(p, 11)
+    cu = torch.from_numpy(p.cu_seqlens).cuda()
+    bi = torch.from_numpy(p.block_idx).cuda()
+    off, ent = nsa.nsa_sel_invert_index(cu, bi, p.block_size)
+    roff, rent = oracle.invert(p.cu_seqlens, p.block_idx, p.block_size)
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.array_equal(ent.cpu().numpy(), rent)
+
+
+@pytest.mark.parametrize("wl", [ni.HEADLINE, "varlen_64k_32k_g1_k16", "train_t32k_hq64_g8_k16",
+                                "sweep_t64k_g1_bs128_k32"])
+def test_invert_bit_exact_full(wl):
+    spec = ni.WORKLOADS[wl]
+    cu = ni.cu_seqlens_from_lengths(spec["lengths"])
+    bidx = ni.make_block_idx(cu, spec["hkv"], spec["topk"], spec["block_size"], spec["seed"])
+    off, ent = nsa.nsa_sel_invert_index(torch.from_numpy(cu).cuda(), torch.from_numpy(bidx).cuda(),
+                                        spec["block_size"])
+    roff, rent = oracle.invert(cu, bidx, spec["block_size"])
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.array_equal(ent.cpu().numpy(), rent)
+
+
+# --------------------------------------------------------------------------- forward
+
+FWD_SMALL = [
+    ("tiny_t2k_g1_k8", None, False),
+    ("g1_bs64_k16", dict(lengths=[700, 37, 1, 515], hq=2, hkv=2, block_size=64, topk=16, seed=7), True),
+    ("g2_bs64_k3", dict(lengths=[1500, 130], hq=4, hkv=2, block_size=64, topk=3, seed=8), True),
+    ("g4_bs64_k16", dict(lengths=[2500, 64, 63], hq=8, hkv=2, block_size=64, topk=16, seed=9), True),
+    ("g8_bs128_k8", dict(lengths=[2000, 1], hq=16, hkv=2, block_size=128, topk=8, seed=10), True),
+    ("g16_bs128_k64", dict(lengths=[1800], hq=16, hkv=1, block_size=128, topk=64, seed=11), True),
+    ("g16_bs64_k1", dict(lengths=[999, 333], hq=32, hkv=2, block_size=64, topk=1, seed=12), False),
+    ("g4_dense_causal", dict(lengths=[640, 300], hq=8, hkv=2, block_size=64, topk=12, seed=13), False),
+]
+
+
+@pytest.mark.parametrize("name,spec,perturb", FWD_SMALL, ids=[c[0] for c in FWD_SMALL])
+def test_fwd_small_full_compare(name, spec, perturb):
+    if spec is None:
+        p = ni.workload(name, with_dout=False)
+    else:
+        p = ni.make_problem(name=name, with_dout=False, **spec)
+    if name == "g4_dense_causal":   # topk covers every block: dense causal attention
+        cu = p.cu_seqlens.astype(np.int64)
+        for s in range(p.nseq):
+            L = int(cu[s + 1] - cu[s])
+            nb = (L + 63) // 64
+            p.block_idx[cu[s]:cu[s + 1]] = -1
+            p.block_idx[cu[s]:cu[s + 1], :, :nb] = np.arange(nb, dtype=np.int32)[::-1]
+    if perturb:
+        p = _perturb(p, 5)
+    _, out, lse = _fwd(p)
+    _check_fwd(p, out, lse)
+
+
+# Every (group, block) pair of the T=65536 sweep at topk 16, plus the topk ends; all
+# 30 points with NSA_FULL_SWEEP=1.
+_SWEEP = [(g, bs, 16) for g in (1, 2, 4, 8, 16) for bs in (64, 128)] + \
+    [(4, 64, 8), (4, 64, 32), (1, 64, 8), (16, 128, 32)]
+if os.environ.get("NSA_FULL_SWEEP") == "1":
+    _SWEEP = list(ni.SWEEP_POINTS)
+FWD_FULL = ["fwd_t32k_hq32_g4_k16", "varlen_64k_32k_g1_k16", "train_t32k_hq64_g8_k16"] + \
+    [f"sweep_t64k_g{g}_bs{bs}_k{k}" for g, bs, k in _SWEEP]
+
+
+@pytest.mark.parametrize("wl", FWD_FULL)
+def test_fwd_full_size_sampled(wl):
+    p = ni.workload(wl, with_dout=False)
+    _, out, lse = _fwd(p)
+    toks = sample_tokens(p.cu_seqlens, p.block_size, n_random=96, seed=1)
+    _check_fwd(p, out, lse, tokens=toks)
+    # properties that hold everywhere: finite outputs, LSE >= the LSE of the
+    # structural blocks alone is not checkable cheaply, but finiteness is
+    assert torch.isfinite(out.float()).all()
+    assert torch.isfinite(lse).all()
+
+
+def test_fwd_deterministic_and_zero_tokens():
+    p = ni.make_problem([1200, 77], hq=8, hkv=2, block_size=64, topk=16, seed=21, with_dout=False)
+    d, o1, l1 = _fwd(p)
+    o2, l2 = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], 64, p.scale)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    # T = 0: a no-op that still succeeds
+    z = torch.empty((0, 8, 128), dtype=torch.bfloat16, device="cuda")
+    zk = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(2, dtype=torch.int32, device="cuda")
+    bi = torch.empty((0, 2, 16), dtype=torch.int32, device="cuda")
+    o, l = nsa.nsa_sel_attn_fwd(z, zk, zk, cu, bi, 64)
+    assert o.shape == (0, 8, 128) and l.shape == (8, 0)
+
+
+def test_fwd_empty_rows_give_zero_and_neg_inf():
+    p = ni.make_problem([500], hq=4, hkv=2, block_size=64, topk=4, seed=22, with_dout=False)
+    p.block_idx[100, 0] = -1
+    p.block_idx[200, 1] = [-1, 9, -4, 8]        # only out-of-range / future values
+    _, out, lse = _fwd(p)
+    assert (out[100, 0:2].float() == 0).all() and torch.isneginf(lse[0:2, 100]).all()
+    assert (out[200, 2:4].float() == 0).all() and torch.isneginf(lse[2:4, 200]).all()
+    _check_fwd(p, out, lse)
+
+
+def test_bad_cu_seqlens_reported():
+    p = ni.make_problem([256, 256], hq=2, hkv=2, block_size=64, topk=4, seed=23, with_dout=False)
+    d = to_device(p)
+    cu = torch.tensor([0, 300, 200], dtype=torch.int32, device="cuda")   # decreasing, wrong end
+    nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], cu, d["bidx"], 64)
+    assert nsa.nsa_sel_check_status() == 6
+
+
+def test_validate_indices_counts():
+    p = ni.make_problem([300, 100], hq=2, hkv=2, block_size=64, topk=6, seed=24, with_dout=False)
+    bi = p.block_idx.copy()
+    bi[10, 0, 5] = 99        # out of range
+    bi[150, 1, 4] = -3       # out of range
+    bi[299, 1, 5] = bi[299, 1, 0]   # duplicate
+    d_cu = torch.from_numpy(p.cu_seqlens).cuda()
+    assert nsa.nsa_sel_validate_indices(d_cu, torch.from_numpy(p.block_idx).cuda(), 64) == (0, 0)
+    assert nsa.nsa_sel_validate_indices(d_cu, torch.from_numpy(bi).cuda(), 64) == (2, 1)
+
+
+# -------------------------------------------------------------------------- backward
+
+def _bwd(p, d, out, lse):
+    dq, dk, dv = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"],
+                                      d["bidx"], p.block_size, p.scale)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    return dq, dk, dv
+
+
+BWD_SMALL = [
+    ("tiny_t2k_g1_k8", None, False),
+    ("g4_bs64_k16", dict(lengths=[1500, 40, 300], hq=8, hkv=2, block_size=64, topk=16, seed=31), True),
+    ("g1_bs128_k8", dict(lengths=[1100, 1], hq=2, hkv=2, block_size=128, topk=8, seed=32), True),
+    ("g16_bs64_k5", dict(lengths=[700], hq=16, hkv=1, block_size=64, topk=5, seed=33), False),
+    ("g8_bs128_k64", dict(lengths=[900, 129], hq=8, hkv=1, block_size=128, topk=64, seed=34), True),
+]
+
+
+@pytest.mark.parametrize("name,spec,perturb", BWD_SMALL, ids=[c[0] for c in BWD_SMALL])
+def test_bwd_small_full_compare(name, spec, perturb):
+    p = ni.workload(name) if spec is None else ni.make_problem(name=name, **spec)
+    if perturb:
+        p = _perturb(p, 6)
+    d, out, lse = _fwd(p)
+    dq, dk, dv = _bwd(p, d, out, lse)
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
+                               p.scale)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    assert max(e) <= TOL_GRAD, (name, e)
+
+
+def _check_bwd_sampled(p, dq, dk, dv, blocks, seed=0, n_random=48):
+    toks = sample_tokens(p.cu_seqlens, p.block_size, n_random=n_random, seed=seed)
+    rdq = oracle.bwd_dq(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+                        toks)
+    e_dq = rel_fro(f64(dq[torch.from_numpy(toks).cuda()]), rdq)
+    gk, rk, gv, rv = [], [], [], []
+    for g, key0, n in blocks:
+        k_ref, v_ref = oracle.bwd_dkdv_keys(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx,
+                                            p.block_size, p.scale, g, key0, n)
+        gk.append(f64(dk[key0:key0 + n, g]))
+        gv.append(f64(dv[key0:key0 + n, g]))
+        rk.append(k_ref)
+        rv.append(v_ref)
+    e_dk = rel_fro(np.concatenate(gk), np.concatenate(rk))
+    e_dv = rel_fro(np.concatenate(gv), np.concatenate(rv))
+    assert max(e_dq, e_dk, e_dv) <= TOL_GRAD, (p.name, e_dq, e_dk, e_dv)
+
+
+def test_bwd_medium_multi_unit():
+    """Block 0 is selected by every token: 512 tiles, 16 backward work units."""
+    p = ni.make_problem([8192], hq=16, hkv=2, block_size=64, topk=16, seed=35, name="bwd_medium")
+    d, out, lse = _fwd(p)
+    dq, dk, dv = _bwd(p, d, out, lse)
+    _check_bwd_sampled(p, dq, dk, dv, blocks=[(0, 0, 64), (1, 64, 64), (1, 4096, 64),
+                                              (0, 8128, 64)])
+
+
+def test_bwd_full_size_training_shape_sampled():
+    p = ni.workload("train_t32k_hq64_g8_k16")
+    d, out, lse = _fwd(p)
+    dq, dk, dv = _bwd(p, d, out, lse)
+    assert torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all()
+    assert torch.isfinite(dv.float()).all()
+    _check_bwd_sampled(p, dq, dk, dv, blocks=[(3, 64 * 300, 64), (7, 32768 - 64, 64),
+                                              (0, 64 * 20, 64)], n_random=24)
+
+
+def test_bwd_deterministic():
+    p = ni.make_problem([3000], hq=8, hkv=2, block_size=64, topk=16, seed=36)
+    d, out, lse = _fwd(p)
+    a = _bwd(p, d, out, lse)
+    b = _bwd(p, d, out, lse)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
