@@ -54,9 +54,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_bwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, I, I, F,
                                              P, P, P, P, Z, P]
             lib.nsa_sel_attn_bwd.restype = I
-            lib.nsa_sel_attn_fwd_profiled.argtypes = lib.nsa_sel_attn_fwd.argtypes + [P, I, P]
+            IP = ctypes.POINTER(ctypes.c_int)
+            lib.nsa_sel_attn_fwd_profiled.argtypes = lib.nsa_sel_attn_fwd.argtypes + [P, I, IP]
             lib.nsa_sel_attn_fwd_profiled.restype = I
-            lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, P]
+            lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, IP]
             lib.nsa_sel_attn_bwd_profiled.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I

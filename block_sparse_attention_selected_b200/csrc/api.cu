@@ -30,7 +30,7 @@ struct Dims {
 };
 
 struct Layout {
-    size_t status, blkoff, keys0, keys1, vals0, vals1, hist, offsets, tile_off, chunk_off;
+    size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
     size_t part_o, part_lse, delta, part_dkdv;
     size_t total;
 };
@@ -72,12 +72,13 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.vals0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.vals1 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.hist = take(sizeof(uint32_t) * 256 * (size_t)std::max(D.sort_tiles, 1));
+    L.digit_tot = take(sizeof(uint32_t) * 256);
     L.offsets = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.tile_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.chunk_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     const size_t rows = (size_t)D.T * D.hq * D.topk;
-    L.part_o = take(rows * kHeadDim * 2);   // bf16 partial O (forward) / dQ (backward)
-    L.part_lse = take(rows * sizeof(float));
+    L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
+    L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
     if (bwd) {
         L.delta = take(sizeof(float) * (size_t)D.hq * D.T);
         L.part_dkdv = take(sizeof(float) * 2 * (size_t)D.bs * kHeadDim * (size_t)D.units_cap);
@@ -163,6 +164,7 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.vals[0] = reinterpret_cast<uint32_t*>(b + L.vals0);
     p.vals[1] = reinterpret_cast<uint32_t*>(b + L.vals1);
     p.hist = reinterpret_cast<uint32_t*>(b + L.hist);
+    p.digit_tot = reinterpret_cast<uint32_t*>(b + L.digit_tot);
     p.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
     p.tile_off = reinterpret_cast<int32_t*>(b + L.tile_off);
     p.chunk_off = reinterpret_cast<int32_t*>(b + L.chunk_off);
@@ -281,7 +283,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.entries = c.inv.vals[c.inv.final_buf];
     fp.nbk_cap = D.nbk_cap;
     fp.part_o = c.base + L.part_o;
-    fp.part_lse = reinterpret_cast<float*>(c.base + L.part_lse);
+    fp.part_meta = reinterpret_cast<float2*>(c.base + L.part_lse);
     fp.st = c.st;
     fp.num_sms = num_sms;
     if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, stream))) != NSA_OK) return s;
@@ -293,7 +295,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
     mp.bidx = block_idx;
     mp.part_o = fp.part_o;
-    mp.part_lse = fp.part_lse;
+    mp.part_meta = fp.part_meta;
     mp.out = out;
     mp.lse = lse;
     if ((s = cuda_status(launch_merge(mp, stream))) != NSA_OK) return s;

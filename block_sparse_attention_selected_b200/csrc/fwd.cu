@@ -11,7 +11,8 @@
 //   S   = Q K_B^T                      tcgen05.mma, fp32 accumulator in TMEM
 //   P   = exp(scale * S - m), causal mask on the diagonal block, l = sum P
 //   O_B = P V_B                        tcgen05.mma (P from shared memory)
-//   partial (O_B / l as bf16, lse_B = m + log l) stored per (token, head, slot)
+//   partial (O_B / l as fp16 with a power-of-two exponent, lse_B = m + log l)
+//   stored per (token, head, slot)
 //
 // The log-sum-exp merge of the partials over a row's slots (no atomics) is in
 // merge.cu.  Persistent CTAs take contiguous tile ranges, so consecutive tiles of
@@ -242,30 +243,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (tid == 0) mma_unwaited = false;
         tc_fence_after();
 
-        // ---- epilogue: normalised partial O (bf16) and its log-sum-exp
+        // ---- epilogue: normalised partial O as fp16 with a power-of-two row exponent
+        //      (e = 0 unless max|O_B / l| > 2^14), plus lse_B = m + log l
         {
-            const float inv_l = 1.f / l;
-            const size_t prow = ((size_t)(my_t < 0 ? 0 : my_t) * p.hq + my_h) * p.topk + my_j;
-            uint4* dst = reinterpret_cast<uint4*>(
-                reinterpret_cast<__nv_bfloat16*>(p.part_o) + prow * kHeadDim);
+            float o[128];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float o[32];
-                tmem_ld32(tO + lane_off + c * 32, o);
-                tmem_wait_ld();
-                if (my_t >= 0) {
+            for (int c = 0; c < 4; ++c) tmem_ld32(tO + lane_off + c * 32, o + c * 32);
+            tmem_wait_ld();
+            if (my_t >= 0) {
+                const float inv_l = 1.f / l;
+                float mx = 0.f;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
-                        w.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
-                        w.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
-                        w.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
-                        dst[c * 4 + q4] = w;
-                    }
+                for (int c = 0; c < 128; ++c) mx = fmaxf(mx, fabsf(o[c]));
+                mx *= inv_l;
+                const int e = mx > 16384.f ? ilogbf(mx) - 14 : 0;
+                const float sc = ldexpf(inv_l, -e);
+                const size_t prow = ((size_t)my_t * p.hq + my_h) * p.topk + my_j;
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.part_o) +
+                                                      prow * kHeadDim);
+#pragma unroll
+                for (int q8 = 0; q8 < 16; ++q8) {
+                    const float* x = o + q8 * 8;
+                    uint4 w;
+                    w.x = pack_f16x2(x[0] * sc, x[1] * sc);
+                    w.y = pack_f16x2(x[2] * sc, x[3] * sc);
+                    w.z = pack_f16x2(x[4] * sc, x[5] * sc);
+                    w.w = pack_f16x2(x[6] * sc, x[7] * sc);
+                    dst[q8] = w;
                 }
+                p.part_meta[prow] = make_float2((m + __log2f(l)) * kLn2, (float)e);
             }
-            if (my_t >= 0) p.part_lse[prow] = (m + __log2f(l)) * kLn2;
         }
         tc_fence_before();
         __syncthreads();

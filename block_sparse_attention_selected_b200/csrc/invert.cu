@@ -12,7 +12,7 @@
 //
 // Steps (all on the caller's stream, no host synchronisation):
 //   1. k_seq_blocks      global block offset of every sequence, cu_seqlens check
-//   2. per 8-bit digit:  k_sort_hist -> k_scan_excl -> k_sort_scatter (LSD radix,
+//   2. per 8-bit digit:  k_sort_hist -> k_scan_digits -> k_sort_scatter (LSD radix,
 //                        stable: warp-ordered ranks with __match_any_sync)
 //   3. k_bucket_offsets  CSR offsets from the sorted keys
 //   4. k_tile_offsets    per-bucket 128-row tile and backward-chunk prefix sums
@@ -132,21 +132,25 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(SortArgs a, const ui
     hist[(size_t)threadIdx.x * gridDim.x + blockIdx.x] = h[threadIdx.x];
 }
 
-// 2b. in-place exclusive scan of n uint32 values by one block.
-__global__ void __launch_bounds__(1024) k_scan_excl(uint32_t* a, long long n) {
+// 2b. per digit (one block each): exclusive scan of hist[d * ntiles + tile] over the
+//     tiles, in place, and the digit's total into digit_tot[d].
+__global__ void __launch_bounds__(1024) k_scan_digits(uint32_t* hist, int ntiles,
+                                                      uint32_t* digit_tot) {
     __shared__ unsigned long long warp_tot[32];
-    const long long per = (n + blockDim.x - 1) / blockDim.x;
-    const long long lo = per * threadIdx.x;
-    const long long hi = min(lo + per, n);
+    uint32_t* a = hist + (size_t)blockIdx.x * ntiles;
+    const int per = (ntiles + blockDim.x - 1) / blockDim.x;
+    const int lo = per * threadIdx.x;
+    const int hi = min(lo + per, ntiles);
     unsigned long long sum = 0;
-    for (long long i = lo; i < hi; ++i) sum += a[i];
-    unsigned long long incl = block_incl_scan_u64(sum, warp_tot);
+    for (int i = lo; i < hi; ++i) sum += a[i];
+    const unsigned long long incl = block_incl_scan_u64(sum, warp_tot);
     unsigned long long run = incl - sum;
-    for (long long i = lo; i < hi; ++i) {
-        uint32_t x = a[i];
+    for (int i = lo; i < hi; ++i) {
+        const uint32_t x = a[i];
         a[i] = (uint32_t)run;
         run += x;
     }
+    if (threadIdx.x == blockDim.x - 1) digit_tot[blockIdx.x] = (uint32_t)incl;
 }
 
 // 2c. stable scatter of one tile by the digit at `shift`.
@@ -154,13 +158,19 @@ template <bool kFirst>
 __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const uint32_t* keys_in,
                                                               const uint32_t* vals_in, int shift,
                                                               const uint32_t* hist_scan,
+                                                              const uint32_t* digit_tot,
                                                               uint32_t* keys_out,
                                                               uint32_t* vals_out) {
     __shared__ uint32_t whist[kSortWarps][256];
     __shared__ uint32_t tile_base[256];
+    __shared__ unsigned long long warp_tot[32];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     for (int i = tid; i < kSortWarps * 256; i += kSortThreads) (&whist[0][0])[i] = 0;
-    tile_base[tid] = hist_scan[(size_t)tid * gridDim.x + blockIdx.x];
+    {   // start of digit tid in the output = totals of smaller digits + earlier tiles
+        const uint32_t tot = digit_tot[tid];
+        const unsigned long long incl = block_incl_scan_u64(tot, warp_tot);
+        tile_base[tid] = (uint32_t)(incl - tot) + hist_scan[(size_t)tid * gridDim.x + blockIdx.x];
+    }
     __syncthreads();
     const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
     const long long base = (long long)blockIdx.x * kSortTile + (long long)w * (kItems * 32);
@@ -291,13 +301,13 @@ cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
             k_sort_hist<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, nullptr, shift, p.hist);
         else
             k_sort_hist<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, shift, p.hist);
-        k_scan_excl<<<1, 1024, 0, stream>>>(p.hist, 256ll * p.sort_tiles);
+        k_scan_digits<<<256, 1024, 0, stream>>>(p.hist, p.sort_tiles, p.digit_tot);
         if (pass == 0)
             k_sort_scatter<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(
-                a, nullptr, nullptr, shift, p.hist, kout, vout);
+                a, nullptr, nullptr, shift, p.hist, p.digit_tot, kout, vout);
         else
-            k_sort_scatter<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, vin, shift,
-                                                                            p.hist, kout, vout);
+            k_sort_scatter<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(
+                a, kin, vin, shift, p.hist, p.digit_tot, kout, vout);
         kin = kout;
         vin = vout;
     }

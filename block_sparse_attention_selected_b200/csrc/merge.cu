@@ -40,10 +40,18 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
     const int32_t* bi = p.bidx + ((size_t)t * p.hkv + g) * p.topk;
     const size_t prow0 = (size_t)row * p.topk;
 
-    float l0 = -CUDART_INF_F, l1 = -CUDART_INF_F;
-    if (lane < p.topk && block_valid(__ldg(bi + lane), qb)) l0 = __ldg(p.part_lse + prow0 + lane);
-    if (lane + 32 < p.topk && block_valid(__ldg(bi + lane + 32), qb))
-        l1 = __ldg(p.part_lse + prow0 + lane + 32);
+    // lane j holds slot j (and j + 32): (lse_j, exponent_j) of the valid slots
+    float l0 = -CUDART_INF_F, l1 = -CUDART_INF_F, e0 = 0.f, e1 = 0.f;
+    if (lane < p.topk && block_valid(__ldg(bi + lane), qb)) {
+        const float2 m = __ldg(p.part_meta + prow0 + lane);
+        l0 = m.x;
+        e0 = m.y;
+    }
+    if (lane + 32 < p.topk && block_valid(__ldg(bi + lane + 32), qb)) {
+        const float2 m = __ldg(p.part_meta + prow0 + lane + 32);
+        l1 = m.x;
+        e1 = m.y;
+    }
     const float M = warp_max(fmaxf(l0, l1));
     uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
                                            (size_t)row * kHeadDim) + lane;
@@ -55,14 +63,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
     const float w0 = l0 == -CUDART_INF_F ? 0.f : __expf(l0 - M);
     const float w1 = l1 == -CUDART_INF_F ? 0.f : __expf(l1 - M);
     const float Lam = warp_sum(w0 + w1);
+    const float s0 = ldexpf(w0, (int)e0), s1 = ldexpf(w1, (int)e1);   // weight x 2^e
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint2* po = reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.part_o) +
+    const uint2* po = reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(p.part_o) +
                                                      prow0 * kHeadDim) + lane;
     for (int j = 0; j < p.topk; ++j) {
-        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? w0 : w1, j & 31);
+        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
         if (wj == 0.f) continue;       // warp-uniform
         const uint2 u = __ldg(po + (size_t)j * (kHeadDim / 4));
-        const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+        const float2 a = unpack_f16x2(u.x), b = unpack_f16x2(u.y);
         acc[0] = fmaf(wj, a.x, acc[0]);
         acc[1] = fmaf(wj, a.y, acc[1]);
         acc[2] = fmaf(wj, b.x, acc[2]);

@@ -30,6 +30,7 @@ struct InvertPlan {
     uint32_t* keys[2];       // [nent] ping-pong
     uint32_t* vals[2];       // [nent] ping-pong
     uint32_t* hist;          // [256 * sort_tiles]
+    uint32_t* digit_tot;     // [256]
     int32_t* offsets;        // [nbk_cap + 1]
     int32_t* tile_off;       // [nbk_cap + 1]
     int32_t* chunk_off;      // [nbk_cap + 1]
@@ -53,8 +54,8 @@ struct FwdPlan {
     const int32_t* tile_off; // bucket tile offsets
     const uint32_t* entries; // token * 64 + slot
     int nbk_cap;
-    void* part_o;            // bf16 [T * hq * topk, 128]
-    float* part_lse;         // fp32 [T * hq * topk]
+    void* part_o;            // fp16 [T * hq * topk, 128]: O_B / l_B * 2^-e
+    float2* part_meta;       // [T * hq * topk]: (lse_B, e)
     DevStatus* st;
     int num_sms;
 };
@@ -67,7 +68,7 @@ struct MergePlan {
     int nseq, T, hq, hkv, topk, bs;
     const int32_t* bidx;
     const void* part_o;
-    const float* part_lse;
+    const float2* part_meta;
     void* out;
     float* lse;
 };

@@ -186,6 +186,8 @@ WORKLOADS = {
     "fwd_t32k_hq32_g4_k16": dict(lengths=[32768], hq=32, hkv=8, block_size=64, topk=16, seed=2),
     "varlen_64k_32k_g1_k16": dict(lengths=[65536, 32768], hq=4, hkv=4, block_size=64, topk=16, seed=3),
     "train_t32k_hq64_g8_k16": dict(lengths=[32768], hq=64, hkv=8, block_size=64, topk=16, seed=5),
+    # half of the headline sequence, same heads: the profiling capture size
+    "prof_t32k_hq16_g4_k16": dict(lengths=[32768], hq=16, hkv=4, block_size=64, topk=16, seed=4),
 }
 
 

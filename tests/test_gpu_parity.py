@@ -2,8 +2,9 @@
 
 Small problems are compared element by element over every output; the workloads
 at their full sizes are compared on stratified token / block samples that the
-oracle computes one by one.  Tolerances: max |dO| <= 1e-2 on bf16 O, <= 1e-3 on
-fp32 LSE, relative Frobenius <= 2e-2 on dQ, dK, dV; the inversion is bit-exact.
+oracle computes one by one.  Tolerances: |O - O_ref| <= 1e-2 beyond half a bf16 ulp
+of O_ref (the rounding of the exact answer to the bf16 output), <= 1e-3 on fp32 LSE,
+relative Frobenius <= 2e-2 on dQ, dK, dV; the inversion is bit-exact.
 """
 import os
 
@@ -14,7 +15,8 @@ import torch
 import block_sparse_attention_selected_b200 as nsa
 import nsa_inputs as ni
 import oracle
-from gpu_util import TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, rel_fro, sample_tokens, to_device
+from gpu_util import (TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, o_excess, rel_fro, sample_tokens,
+                      to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,8 +62,8 @@ def _check_fwd(p, out, lse, tokens=None):
                               tokens=tokens)
     o = f64(out) if tokens is None else f64(out[torch.from_numpy(tokens).cuda()])
     l = f64(lse).T if tokens is None else f64(lse[:, torch.from_numpy(tokens).cuda()]).T
-    eo, el = max_abs(o, o_ref), max_abs(l, l_ref)
-    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
+    eo, el = o_excess(o, o_ref), max_abs(l, l_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el, max_abs(o, o_ref))
     return eo, el
 
 
