@@ -117,8 +117,8 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
         self.proc = None
         self.path = None
 
@@ -207,8 +207,14 @@ def run_ours(args, rank, world, local_rank, dist):
     n_bwd = ctypes.c_int(0)
 
     def ev_array(evs):
-        arr = (ctypes.c_void_p * len(evs))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
-        return arr
+        # torch creates the CUDA event lazily: record once so that the handle exists
+        for e in evs:
+            e.record(stream)
+        torch.cuda.synchronize()
+        handles = [e.cuda_event for e in evs]
+        assert all(handles), "CUDA events were not created"
+        arr = (ctypes.c_void_p * len(evs))(*handles)
+        return ctypes.cast(arr, ctypes.c_void_p), arr
 
     def step(fwd_ev=None, bwd_ev=None, q_=q, k_=k, v_=v, do_=do, cu_=cu, bi_=bi):
         rc = lib.nsa_sel_attn_fwd_profiled(
@@ -247,11 +253,17 @@ def run_ours(args, rank, world, local_rank, dist):
     K = args.steps
     fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    farr = [ev_array(e) for e in fevs]
-    barr = [ev_array(e) for e in bevs]
+    farr_keep = [ev_array(e) for e in fevs]
+    barr_keep = [ev_array(e) for e in bevs]
+    farr = [a for a, _ in farr_keep]
+    barr = [a for a, _ in barr_keep]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local_rank)
+    clocks = ClockSampler(gpu_id)
     barrier()
     torch.cuda.synchronize()
     clocks.start()

@@ -17,6 +17,7 @@ using namespace nsa;
 namespace {
 
 constexpr int kChunkTiles = 32;   // tiles per backward work unit
+constexpr int kWindowRows = 8192; // query rows per forward token window (tokens x group)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -27,11 +28,14 @@ struct Dims {
     int key_bits;
     int sort_tiles;
     long long tiles_cap, units_cap;
+    int wtok, nwin, nb_stride;   // forward token windows
+    long long fwd_tiles_cap;     // bound on the number of forward tiles
 };
 
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
-    size_t part_o, part_lse, delta, part_dkdv;
+    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc;
+    size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket;
     size_t total;
 };
 
@@ -47,6 +51,7 @@ nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int b
     if (nent >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;
     const long long nbk_cap = (long long)hkv * ((long long)T / bs + nseq);
     if (nbk_cap >= (1ll << 30)) return NSA_ERR_UNSUPPORTED;
+    if ((long long)T * hq >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;   // TMA row coordinate
     D->T = T; D->nseq = nseq; D->hq = hq; D->hkv = hkv; D->d = d; D->topk = topk; D->bs = bs;
     D->G = G;
     D->nent = nent;
@@ -58,6 +63,12 @@ nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int b
     const int tpt = kTileRows / G;
     D->tiles_cap = (nent + tpt - 1) / tpt + nbk_cap;
     D->units_cap = (D->tiles_cap + kChunkTiles - 1) / kChunkTiles + nbk_cap;
+    D->wtok = kWindowRows / G;
+    D->nwin = std::max(1, (T + D->wtok - 1) / D->wtok);
+    D->nb_stride = (int)((long long)T / bs + nseq);
+    if ((long long)hkv * D->nwin * (D->nb_stride + 1) >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;
+    D->fwd_tiles_cap = (nent + tpt - 1) / tpt +
+                       std::min<long long>(nent, (long long)hkv * D->nwin * D->nb_stride);
     return NSA_OK;
 }
 
@@ -76,12 +87,20 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.offsets = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.tile_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.chunk_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
+    const size_t wrows = (size_t)D.hkv * D.nwin;
+    L.win_rng = take(sizeof(int2) * wrows * (size_t)D.nb_stride);
+    L.wtile_off = take(sizeof(int32_t) * wrows * ((size_t)D.nb_stride + 1));
+    L.row_tiles = take(sizeof(int32_t) * wrows);
+    L.row_off = take(sizeof(int32_t) * (wrows + 1));
+    L.tile_desc = take(sizeof(int4) * (size_t)std::max<long long>(D.fwd_tiles_cap, 1));
     const size_t rows = (size_t)D.T * D.hq * D.topk;
     L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
     if (bwd) {
         L.delta = take(sizeof(float) * (size_t)D.hq * D.T);
         L.part_dkdv = take(sizeof(float) * 2 * (size_t)D.bs * kHeadDim * (size_t)D.units_cap);
+        L.udesc = take(sizeof(int4) * (size_t)D.units_cap);
+        L.ubucket = take(sizeof(int) * (size_t)D.units_cap);
     }
     L.total = o;
     return L;
@@ -268,7 +287,18 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
-    pm.add(invert_launches(D));
+    WindowPlan wp{};
+    wp.nwin = D.nwin;
+    wp.wtok = D.wtok;
+    wp.nb_stride = D.nb_stride;
+    wp.win_rng = reinterpret_cast<int2*>(c.base + L.win_rng);
+    wp.tile_off = reinterpret_cast<int32_t*>(c.base + L.wtile_off);
+    wp.row_tiles = reinterpret_cast<int32_t*>(c.base + L.row_tiles);
+    wp.row_off = reinterpret_cast<int32_t*>(c.base + L.row_off);
+    wp.tile_desc = reinterpret_cast<int4*>(c.base + L.tile_desc);
+    wp.tiles_cap = D.fwd_tiles_cap;
+    if ((s = cuda_status(launch_window_split(c.inv, wp, stream))) != NSA_OK) return s;
+    pm.add(invert_launches(D) + 4);
     pm.mark(1);
 
     FwdPlan fp{};
@@ -282,6 +312,12 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.tile_off = c.inv.tile_off;
     fp.entries = c.inv.vals[c.inv.final_buf];
     fp.nbk_cap = D.nbk_cap;
+    fp.nwin = wp.nwin;
+    fp.nb_stride = wp.nb_stride;
+    fp.win_rng = wp.win_rng;
+    fp.wtile_off = wp.tile_off;
+    fp.row_off = wp.row_off;
+    fp.tile_desc = wp.tile_desc;
     fp.part_o = c.base + L.part_o;
     fp.part_meta = reinterpret_cast<float2*>(c.base + L.part_lse);
     fp.st = c.st;
@@ -339,7 +375,11 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
-    pm.add(invert_launches(D));
+    int4* udesc = reinterpret_cast<int4*>(c.base + L.udesc);
+    int* ubucket = reinterpret_cast<int*>(c.base + L.ubucket);
+    if ((s = cuda_status(launch_unit_desc(c.inv, D.units_cap, udesc, ubucket, stream))) != NSA_OK)
+        return s;
+    pm.add(invert_launches(D) + 1);
     pm.mark(1);
 
     BwdPlan bp{};
@@ -359,6 +399,8 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.entries = c.inv.vals[c.inv.final_buf];
     bp.nbk_cap = D.nbk_cap;
     bp.chunk_tiles = kChunkTiles;
+    bp.udesc = udesc;
+    bp.ubucket = ubucket;
     bp.part_dq = c.base + L.part_o;
     bp.part_dkdv = reinterpret_cast<float*>(c.base + L.part_dkdv);
     bp.st = c.st;

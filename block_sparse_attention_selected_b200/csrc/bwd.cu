@@ -12,8 +12,19 @@
 //
 // At the end of a unit dV and scale*dK of its block are written as fp32 partials;
 // k_dkdv_reduce sums the units of each block in order and k_dq_merge sums the dQ
-// partials of each row over its slots.  No atomics anywhere: the result is
-// deterministic.
+// partials of each row over its slots.  No atomics: the result is deterministic.
+//
+// One persistent CTA per SM takes units round-robin; it is warp-specialised:
+//
+//   warps 0-1   loaders: row metadata, cp.async gather of the Q and dO rows (NQ
+//               stages; rows past the list are zero, so they add nothing to dV / dK)
+//   warp 2      TMA producer: K_B and V_B of each unit
+//   warp 3      MMA issuer (one thread): S/dP of tile i+1 go ahead of the dV/dK/dQ
+//               products of tile i when there are two TMEM slots
+//   warps 4-7   P / dS, dQ epilogue, unit epilogue of even tiles  } NSLOT = 2: one
+//   warps 8-11  the same for odd tiles                             } TMEM slot each
+//
+// Work descriptors come from k_unit_desc; every wait is bounded (nsa_common.cuh).
 #include <math_constants.h>
 
 #include "nsa_common.cuh"
@@ -22,28 +33,32 @@
 namespace nsa {
 namespace {
 
-constexpr int kBwdThreads = 128;
+constexpr int kThreads = 384;
+constexpr int kLoaderThreads = 64;
+constexpr int kWgThreads = 128;
 
-template <int BS>
+template <int BS, int NQ, int NSLOT>
 struct alignas(1024) BwdSmem {
-    uint8_t q[2][kTileRows * 128];
-    uint8_t dout[2][kTileRows * 128];
-    uint8_t k[2][BS * 128];
+    uint8_t q[NQ][2][kTileRows * 128];        // [stage][64-column half]
+    uint8_t dout[NQ][2][kTileRows * 128];
+    uint8_t k[2][BS * 128];                   // [half]
     uint8_t v[2][BS * 128];
-    uint8_t p[BS / 64][kTileRows * 128];
-    uint8_t ds[BS / 64][kTileRows * 128];
-    uint64_t bar_kv;
-    uint64_t bar_mma;
+    uint8_t p[BS / 64][kTileRows * 128];      // P bf16 [row][key], 64-key chunks
+    uint8_t ds[BS / 64][kTileRows * 128];     // dS bf16 [row][key]
+    int4 meta[NQ][kTileRows];                 // (token or -1, head, slot, causal limit)
+    uint64_t q_full[NQ], q_empty[NQ], meta_full[NQ], meta_empty[NQ];
+    uint64_t kv_full, kv_empty;
+    uint64_t sdp_full[NSLOT], dq_full[NSLOT], tmem_empty[NSLOT];
+    uint64_t pds_full, pds_empty, acc_full, acc_empty, drain;
     uint32_t tmem_base;
     int abort_flag;
+    int loader_stop;
     int nunits;
-    int row_tok[kTileRows];
-    int row_head[kTileRows];
 };
 
-template <int BS>
+template <int BS, int NQ, int NSLOT>
 constexpr size_t bwd_smem_bytes() {
-    return sizeof(BwdSmem<BS>) + 1024;
+    return sizeof(BwdSmem<BS, NQ, NSLOT>) + 1024;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -53,118 +68,155 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <int BS>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int BS, int NQ, int NSLOT>
+__global__ void __launch_bounds__(kThreads, 1)
     k_bwd_tiles(const BwdPlan p, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap) {
     extern __shared__ uint8_t smem_raw[];
-    BwdSmem<BS>& S = *reinterpret_cast<BwdSmem<BS>*>(
+    BwdSmem<BS, NQ, NSLOT>& S = *reinterpret_cast<BwdSmem<BS, NQ, NSLOT>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    const int lane = tid & 31;
     DevStatus* st = p.st;
 
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
+        S.loader_stop = 0;
         S.nunits = *reinterpret_cast<volatile int*>(&st->nchunks);
-        mbar_init(&S.bar_kv, 1);
-        mbar_init(&S.bar_mma, 1);
+        for (int i = 0; i < NQ; ++i) {
+            mbar_init(&S.q_full[i], kLoaderThreads);
+            mbar_init(&S.q_empty[i], 1);
+            mbar_init(&S.meta_full[i], kLoaderThreads);
+            mbar_init(&S.meta_empty[i], kWgThreads);
+        }
+        for (int i = 0; i < NSLOT; ++i) {
+            mbar_init(&S.sdp_full[i], 1);
+            mbar_init(&S.dq_full[i], 1);
+            mbar_init(&S.tmem_empty[i], kWgThreads);
+        }
+        mbar_init(&S.kv_full, 1);
+        mbar_init(&S.kv_empty, 1);
+        mbar_init(&S.pds_full, kWgThreads);
+        mbar_init(&S.pds_empty, 1);
+        mbar_init(&S.acc_full, 1);
+        mbar_init(&S.acc_empty, kWgThreads);
+        mbar_init(&S.drain, 1);
         fence_barrier_init();
-        prefetch_tmap(&kmap);
-        prefetch_tmap(&vmap);
     }
     if (warp == 0) {
+        __syncwarp();
         tmem_alloc(&S.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+
     const uint32_t tmem = S.tmem_base;
-    const uint32_t tS = tmem;          // S, later dQ: columns [0, 128)
-    const uint32_t tdP = tmem + 128;   // dP
-    const uint32_t tdV = tmem + 256;   // dV^T  (lane = head-dim index, column = key)
-    const uint32_t tdK = tmem + 384;   // dK^T
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-
-    const int nbtot = __ldg(p.blkoff + p.nseq);
-    const int nbk = p.hkv * nbtot;
     const int nunits = S.nunits;
-    const long long ub = (long long)nunits * blockIdx.x / gridDim.x;
-    const long long ue = (long long)nunits * (blockIdx.x + 1) / gridDim.x;
+    const int nk = (!S.abort_flag && (int)blockIdx.x < nunits)
+                       ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
+                       : 0;
+    auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+    auto ld_unit = [&](int k) {
+        return k < nk ? __ldg(p.udesc + unit_of(k)) : make_int4(0, 0, 0, 0);
+    };
+    auto ld_bucket = [&](int k) { return k < nk ? __ldg(p.ubucket + unit_of(k)) : -1; };
     const int tpt = kTileRows / p.G;
-    constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);    // S, dP
-    constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);      // dV^T, dK^T
-    constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);    // dQ
-    const float kLog2e = 1.4426950408889634f;
+    volatile int* abort_flag = &S.abort_flag;
+    auto wait = [&](uint64_t* bar, uint32_t parity, int where) -> bool {
+        if (*abort_flag) return false;
+        if (!mbar_wait(bar, parity, st, where)) {
+            *abort_flag = 1;
+            return false;
+        }
+        return true;
+    };
+    // TMEM columns: per slot [S | dP] (2*BS, dQ aliases its first 128), then dV^T, dK^T
+    constexpr int kSlotCols = 2 * BS;
+    constexpr int kColDV = NSLOT * kSlotCols;
+    constexpr int kColDK = kColDV + BS;
+    static_assert(kColDK + BS <= 512, "TMEM budget");
 
-    uint32_t kv_phase = 0, mma_phase = 0;
-    bool kv_unwaited = false, mma_unwaited = false;
-    int cached_bucket = -1;
-
-    for (long long unit = ub; unit < ue && !S.abort_flag; ++unit) {
-        const int bucket = upper_index(p.chunk_off, nbk, (int)unit);
-        const int g = bucket / nbtot;
-        const int gb = bucket - g * nbtot;
-        const int s = upper_index(p.blkoff, p.nseq, gb);
-        const int b = gb - __ldg(p.blkoff + s);
-        const int seq0 = __ldg(p.cu + s);
-        const int key0 = seq0 + b * BS;
-        const int tile_lo = __ldg(p.tile_off + bucket) +
-                            ((int)unit - __ldg(p.chunk_off + bucket)) * p.chunk_tiles;
-        const int tile_hi = min(tile_lo + p.chunk_tiles, __ldg(p.tile_off + bucket + 1));
-        const int ent_lo = __ldg(p.offsets + bucket);
-        const int ent_hi = __ldg(p.offsets + bucket + 1);
-
-        for (int tile = tile_lo; tile < tile_hi; ++tile) {
-            const bool first = tile == tile_lo;
-            const int e0 = ent_lo + (tile - __ldg(p.tile_off + bucket)) * tpt;
-            const int e1 = min(e0 + tpt, ent_hi);
-            const int nrows = (e1 - e0) * p.G;
-
-            int my_t = -1, my_h = 0, my_j = 0, my_lim = -1;
-            float my_lse2 = 0.f, my_delta = 0.f;
-            if (tid < nrows) {
-                const uint32_t ent = __ldg(p.entries + e0 + tid / p.G);
-                my_t = (int)(ent >> 6);
-                my_j = (int)(ent & 63u);
-                my_h = g * p.G + tid % p.G;
-                my_lim = (my_t - seq0) - b * BS;
-                my_lse2 = __ldg(p.lse + (size_t)my_h * p.T + my_t) * kLog2e;
-                my_delta = __ldg(p.delta + (size_t)my_h * p.T + my_t);
-            }
-            S.row_tok[tid] = my_t;
-            S.row_head[tid] = my_h;
-            __syncthreads();
-
-            if (first && bucket != cached_bucket && tid == 0) {
-                mbar_arrive_expect_tx(&S.bar_kv, 4u * BS * 128u);
-                tma_load_3d(S.k[0], &kmap, &S.bar_kv, 0, g, key0);
-                tma_load_3d(S.k[1], &kmap, &S.bar_kv, 64, g, key0);
-                tma_load_3d(S.v[0], &vmap, &S.bar_kv, 0, g, key0);
-                tma_load_3d(S.v[1], &vmap, &S.bar_kv, 64, g, key0);
-                kv_unwaited = true;
-            }
-            cached_bucket = bucket;
-
-            // gather Q and dO rows; rows past the list are zero so that they add
-            // nothing to the dV / dK sums over rows
-            {
-                const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-                const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(p.dout);
-                const uint32_t q0 = smem_u32(S.q[0]), q1 = smem_u32(S.q[1]);
-                const uint32_t d0 = smem_u32(S.dout[0]), d1 = smem_u32(S.dout[1]);
+    if (warp < 2) {
+        // ------------------------------------------------------------------ loaders
+        // 64 threads; each tile's row metadata is shared through shared memory (named
+        // barrier 1).  A tile is published as soon as its own copies have landed: the
+        // stage it waits for next is freed by MMA work that needs this tile first.
+        const int lt = tid;
+        const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+        const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(p.dout);
+        volatile int* stop = &S.loader_stop;
+        int4 u0 = ld_unit(0), u1 = ld_unit(1), u2 = ld_unit(2);
+        auto ld_ent = [&](int e0, int ehi, int r) -> uint32_t {
+            return (e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0u;
+        };
+        uint32_t ent0 = 0u, ent1 = 0u;
+        if (nk > 0) {
+            ent0 = ld_ent(u0.y, u0.z, 2 * lt);
+            ent1 = ld_ent(u0.y, u0.z, 2 * lt + 1);
+        }
+        int i = 0;
+        bool stopped = false;
+        for (int k = 0; k < nk && !stopped; ++k) {
+            const int4 d = u0;
+            u0 = u1; u1 = u2; u2 = ld_unit(k + 3);
+            const int ntl = d.w & 255, g = d.w >> 8;
+            for (int tt = 0; tt < ntl; ++tt, ++i) {
+                const int e0 = d.y + tt * tpt;
+                const int nrows = min(tpt, d.z - e0) * p.G;
+                const int stg = i % NQ;
+                const uint32_t ph_empty = ((i / NQ) & 1) ^ 1;
+                const bool ok = wait(&S.meta_empty[stg], ph_empty, 50) &&
+                                wait(&S.q_empty[stg], ph_empty, 51);
+                if (!ok) *stop = 1;
+                if (ok) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int r = 2 * lt + rr;
+                        const uint32_t ent = rr ? ent1 : ent0;
+                        int4 m = make_int4(-1, 0, 0, -1);
+                        if (r < nrows) {
+                            m.x = (int)(ent >> 6);
+                            m.y = g * p.G + r % p.G;
+                            m.z = (int)(ent & 63u);
+                            m.w = m.x - d.x;
+                        }
+                        S.meta[stg][r] = m;
+                    }
+                }
+                // index entries of the next tile (this unit's or the next unit's first)
+                if (tt + 1 < ntl) {
+                    ent0 = ld_ent(e0 + tpt, d.z, 2 * lt);
+                    ent1 = ld_ent(e0 + tpt, d.z, 2 * lt + 1);
+                } else if (k + 1 < nk) {
+                    ent0 = ld_ent(u0.y, u0.z, 2 * lt);
+                    ent1 = ld_ent(u0.y, u0.z, 2 * lt + 1);
+                }
+                named_bar_sync(1, kLoaderThreads);
+                if (*stop) { stopped = true; break; }   // read after the barrier: uniform
+                mbar_arrive(&S.meta_full[stg]);
+                // gather Q and dO: 4096 16-byte chunks, 64 per thread; zero rows past the list
 #pragma unroll 4
-                for (int it = 0; it < 32; ++it) {
-                    const int idx = tid + it * kBwdThreads;     // 0 .. 4095
-                    const int which = idx >> 11;                // 0: Q, 1: dO
-                    const int row = (idx >> 4) & 127, c = idx & 15;
-                    const int t = S.row_tok[row];
-                    const uint32_t dst = (which ? (c < 8 ? d0 : d1) : (c < 8 ? q0 : q1)) +
-                                         sw128_offset(row, c & 7);
-                    if (t >= 0) {
+                for (int c = 0; c < 64; ++c) {
+                    const int idx = lt + c * kLoaderThreads;
+                    const int which = idx >> 11;
+                    const int row = (idx >> 4) & 127, ch = idx & 15;
+                    const uint32_t dst = smem_u32(which ? S.dout[stg][ch >> 3] : S.q[stg][ch >> 3]) +
+                                         sw128_offset(row, ch & 7);
+                    const int4 m = S.meta[stg][row];
+                    if (m.x >= 0) {
                         const __nv_bfloat16* src = (which ? dO : q) +
-                                                   ((size_t)t * p.hq + S.row_head[row]) * kHeadDim + c * 8;
+                                                   ((size_t)m.x * p.hq + m.y) * kHeadDim + ch * 8;
                         cp_async_16(dst, src);
                     } else {
                         st_shared_v4(dst, 0u, 0u, 0u, 0u);
@@ -173,168 +225,263 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 cp_async_commit();
                 cp_async_wait_all();
                 fence_async_smem();
+                mbar_arrive(&S.q_full[stg]);
             }
-            __syncthreads();
-
-            // S = Q K^T and dP = dO V^T
-            if (tid == 0) {
-                bool ok = true;
-                if (kv_unwaited) {
-                    ok = mbar_wait(&S.bar_kv, kv_phase, st, 20);
-                    if (ok) { kv_phase ^= 1; kv_unwaited = false; }
-                }
-                if (ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (uint32_t)(ks & 3) * 32u;
-                        mma_bf16_ss(tS, smem_desc_sw128(smem_u32(S.q[ks >> 2]) + off, 16, 1024),
-                                    smem_desc_sw128(smem_u32(S.k[ks >> 2]) + off, 16, 1024),
-                                    kIdescS, ks > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (uint32_t)(ks & 3) * 32u;
-                        mma_bf16_ss(tdP, smem_desc_sw128(smem_u32(S.dout[ks >> 2]) + off, 16, 1024),
-                                    smem_desc_sw128(smem_u32(S.v[ks >> 2]) + off, 16, 1024),
-                                    kIdescS, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&S.bar_mma);
-                    mma_unwaited = true;
-                } else {
-                    S.abort_flag = 1;
-                }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------- K/V producer
+        if (lane == 0) {
+            prefetch_tmap(&kmap);
+            prefetch_tmap(&vmap);
+            int prev = -1, loads = 0, last_parity = 0;
+            bool loaded = false;
+            int4 u0 = ld_unit(0), u1 = ld_unit(1);
+            int b0 = ld_bucket(0), b1 = ld_bucket(1);
+            for (int k = 0; k < nk; ++k) {
+                const int4 d = u0;
+                const int b = b0;
+                u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
+                if (b == prev) continue;
+                prev = b;
+                if (!wait(&S.kv_empty, (loads & 1) ^ 1, 52)) break;
+                const int g = d.w >> 8;
+                mbar_arrive_expect_tx(&S.kv_full, 4u * BS * 128u);
+                tma_load_3d(S.k[0], &kmap, &S.kv_full, 0, g, d.x);
+                tma_load_3d(S.k[1], &kmap, &S.kv_full, 64, g, d.x);
+                tma_load_3d(S.v[0], &vmap, &S.kv_full, 0, g, d.x);
+                tma_load_3d(S.v[1], &vmap, &S.kv_full, 64, g, d.x);
+                last_parity = loads & 1;
+                loaded = true;
+                ++loads;
             }
-            __syncthreads();
-            if (S.abort_flag) break;
-            {
-                const bool ok = mbar_wait(&S.bar_mma, mma_phase, st, 21);
-                if (!ok) S.abort_flag = 1;
-                mma_phase ^= 1;
-                if (tid == 0 && ok) mma_unwaited = false;
-            }
-            tc_fence_after();
-
-            // P and dS of this thread's row, 32 columns at a time
-#pragma unroll
-            for (int c32 = 0; c32 < BS / 32; ++c32) {
-                float sv[32], dp[32];
-                tmem_ld32(tS + lane_off + c32 * 32, sv);
-                tmem_ld32(tdP + lane_off + c32 * 32, dp);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int key = c32 * 32 + c;
-                    const float pr = (key <= my_lim) ? exp2f(sv[c] * p.scale_log2 - my_lse2) : 0.f;
-                    sv[c] = pr;
-                    dp[c] = pr * (dp[c] - my_delta);
+            if (*abort_flag && loaded) mbar_wait(&S.kv_full, last_parity, st, 53);
+        }
+    } else if (warp == 3) {
+        // -------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);   // S, dP
+            constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);     // dV^T, dK^T
+            constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
+            int kv_loads = 0, prev_bucket = -1;
+            bool ok = true;
+            auto sdp = [&](int i, bool first, int bucket) -> bool {
+                if (first && bucket != prev_bucket) {
+                    if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
+                    ++kv_loads;
+                    prev_bucket = bucket;
                 }
-                const int chunk = c32 >> 1;
-                const uint32_t pb = smem_u32(S.p[chunk]);
-                const uint32_t db = smem_u32(S.ds[chunk]);
-#pragma unroll
-                for (int pc4 = 0; pc4 < 4; ++pc4) {
-                    const int pc = (c32 & 1) * 4 + pc4;
-                    const float* x = sv + pc4 * 8;
-                    const float* y = dp + pc4 * 8;
-                    st_shared_v4(pb + sw128_offset(tid, pc), pack_bf16x2(x[0], x[1]),
-                                 pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                                 pack_bf16x2(x[6], x[7]));
-                    st_shared_v4(db + sw128_offset(tid, pc), pack_bf16x2(y[0], y[1]),
-                                 pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                                 pack_bf16x2(y[6], y[7]));
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (S.abort_flag) break;
-
-            // dV^T += dO^T P,  dK^T += Q^T dS,  dQ = dS K
-            if (tid == 0) {
+                const int s = i % NSLOT, stg = i % NQ;
+                if (!wait(&S.tmem_empty[s], ((i / NSLOT) & 1) ^ 1, 55)) return false;
+                if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
                 tc_fence_after();
+                const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {     // K = 128 rows, 16 per step
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ss(tS, smem_desc_sw128(smem_u32(S.q[stg][ks >> 2]) + off, 16, 1024),
+                                smem_desc_sw128(smem_u32(S.k[ks >> 2]) + off, 16, 1024), kIdescS,
+                                ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = (uint32_t)(ks & 3) * 32u;
+                    mma_bf16_ss(tdP, smem_desc_sw128(smem_u32(S.dout[stg][ks >> 2]) + off, 16, 1024),
+                                smem_desc_sw128(smem_u32(S.v[ks >> 2]) + off, 16, 1024), kIdescS,
+                                ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&S.sdp_full[s]);
+                return true;
+            };
+            auto rest = [&](int i, bool first, bool last, int k, bool release_kv) -> bool {
+                const int s = i % NSLOT, stg = i % NQ;
+                if (!wait(&S.pds_full, i & 1, 57)) return false;
+                if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
+                tc_fence_after();
+                const uint32_t q0 = smem_u32(S.q[stg][0]), d0 = smem_u32(S.dout[stg][0]);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step
                     const uint32_t off = (uint32_t)ks * 2048u;
                     const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                    mma_bf16_ss(tdV, smem_desc_sw128(smem_u32(S.dout[0]) + off, 16384, 1024),
+                    mma_bf16_ss(tmem + kColDV, smem_desc_sw128(d0 + off, 16384, 1024),
                                 smem_desc_sw128(smem_u32(S.p[0]) + off, 16384, 1024), kIdescT, acc);
-                    mma_bf16_ss(tdK, smem_desc_sw128(smem_u32(S.q[0]) + off, 16384, 1024),
+                    mma_bf16_ss(tmem + kColDK, smem_desc_sw128(q0 + off, 16384, 1024),
                                 smem_desc_sw128(smem_u32(S.ds[0]) + off, 16384, 1024), kIdescT, acc);
                 }
 #pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks) {   // K = BS keys
-                    mma_bf16_ss(tS,
+                for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
+                    mma_bf16_ss(tmem + s * kSlotCols,
                                 smem_desc_sw128(smem_u32(S.ds[ks >> 2]) + (uint32_t)(ks & 3) * 32u, 16, 1024),
                                 smem_desc_sw128(smem_u32(S.k[0]) + (uint32_t)ks * 2048u, BS * 128, 1024),
                                 kIdescQ, ks > 0 ? 1u : 0u);
+                mma_commit(&S.dq_full[s]);
+                mma_commit(&S.pds_empty);
+                mma_commit(&S.q_empty[stg]);
+                if (last) {
+                    mma_commit(&S.acc_full);
+                    if (release_kv) mma_commit(&S.kv_empty);
                 }
-                mma_commit(&S.bar_mma);
-                mma_unwaited = true;
+                return true;
+            };
+            // tile sequence with one tile of look-ahead
+            int4 u0 = ld_unit(0), u1 = ld_unit(1);
+            int b0 = ld_bucket(0), b1 = ld_bucket(1);
+            bool have_prev = false;
+            int pi = 0, pk = 0, pb = -1;
+            bool pfirst = false, plast = false;
+            int i = 0;
+            for (int k = 0; k < nk && ok; ++k) {
+                const int4 d = u0;
+                const int b = b0;
+                u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
+                const int ntl = d.w & 255;
+                for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
+                    const bool first = tt == 0, last = tt == ntl - 1;
+                    // S/dP of this tile may go ahead of the previous tile's products when
+                    // it needs no other K/V block, Q/dO stage or TMEM slot
+                    const bool early = have_prev && NSLOT == 2 && NQ == 2 && !(first && b != pb);
+                    if (early && !(ok = sdp(i, first, b))) break;
+                    if (have_prev && !(ok = rest(pi, pfirst, plast, pk, plast && b != pb))) break;
+                    if (!early && !(ok = sdp(i, first, b))) break;
+                    have_prev = true;
+                    pi = i; pk = k; pb = b; pfirst = first; plast = last;
+                }
             }
-            {
-                const bool ok = mbar_wait(&S.bar_mma, mma_phase, st, 22);
-                if (!ok) S.abort_flag = 1;
-                mma_phase ^= 1;
-                if (tid == 0 && ok) mma_unwaited = false;
-            }
-            tc_fence_after();
-
-            // dQ partial of this row and slot
-            {
-                const size_t prow = ((size_t)(my_t < 0 ? 0 : my_t) * p.hq + my_h) * p.topk + my_j;
-                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.part_dq) +
-                                                      prow * kHeadDim);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float o[32];
-                    tmem_ld32(tS + lane_off + c * 32, o);
-                    tmem_wait_ld();
+            if (ok && have_prev) rest(pi, pfirst, plast, pk, true);
+            mma_commit(&S.drain);
+            mbar_wait(&S.drain, 0, st, 59);
+        }
+    } else {
+        // ------------------------------------------------- P / dS and the epilogues
+        const int wg = (warp - 4) >> 2;
+        const int r = (warp & 3) * 32 + lane;            // row = TMEM lane (= d for dV^T/dK^T)
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const float kLog2e = 1.4426950408889634f;
+        if (wg < NSLOT) {
+            int4 u0 = ld_unit(0), u1 = ld_unit(1);
+            int i = 0;
+            bool ok = true;
+            for (int k = 0; k < nk && ok; ++k) {
+                const int4 d = u0;
+                u0 = u1; u1 = ld_unit(k + 2);
+                const int ntl = d.w & 255;
+                for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
+                    if (i % NSLOT != wg) continue;
+                    const int stg = i % NQ, s = i % NSLOT;
+                    if (!(ok = wait(&S.meta_full[stg], (i / NQ) & 1, 60))) break;
+                    const int4 m = S.meta[stg][r];
+                    mbar_arrive(&S.meta_empty[stg]);
+                    const int my_t = m.x, my_h = m.y, my_j = m.z, my_lim = m.w;
+                    float lse2 = 0.f, delta = 0.f;
                     if (my_t >= 0) {
+                        lse2 = __ldg(p.lse + (size_t)my_h * p.T + my_t) * kLog2e;
+                        delta = __ldg(p.delta + (size_t)my_h * p.T + my_t);
+                    }
+                    if (!(ok = wait(&S.sdp_full[s], (i / NSLOT) & 1, 61))) break;
+                    tc_fence_after();
+                    const uint32_t tS = tmem + s * kSlotCols + lane_off, tdP = tS + BS;
+                    // P and dS of this row, 64 keys per batch of TMEM loads
+                    auto pds_chunk = [&](int c64, uint32_t* pk, uint32_t* dk) {
+                        float sv[64], dp[64];
+                        tmem_ld32(tS + c64 * 64, sv);
+                        tmem_ld32(tS + c64 * 64 + 32, sv + 32);
+                        tmem_ld32(tdP + c64 * 64, dp);
+                        tmem_ld32(tdP + c64 * 64 + 32, dp + 32);
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float* x = o + q4 * 8;
-                            uint4 w;
-                            w.x = pack_bf16x2(x[0] * p.scale, x[1] * p.scale);
-                            w.y = pack_bf16x2(x[2] * p.scale, x[3] * p.scale);
-                            w.z = pack_bf16x2(x[4] * p.scale, x[5] * p.scale);
-                            w.w = pack_bf16x2(x[6] * p.scale, x[7] * p.scale);
-                            dst[c * 4 + q4] = w;
+                        for (int c = 0; c < 64; c += 2) {
+                            const int key = c64 * 64 + c;
+                            const float p0 = key <= my_lim ? exp2f(sv[c] * p.scale_log2 - lse2) : 0.f;
+                            const float p1 = key + 1 <= my_lim ? exp2f(sv[c + 1] * p.scale_log2 - lse2) : 0.f;
+                            pk[c / 2] = pack_bf16x2(p0, p1);
+                            dk[c / 2] = pack_bf16x2(p0 * (dp[c] - delta), p1 * (dp[c + 1] - delta));
+                        }
+                    };
+                    auto store_chunk = [&](int c64, const uint32_t* pk, const uint32_t* dk) {
+#pragma unroll
+                        for (int pc = 0; pc < 8; ++pc) {   // 16-byte pieces of 8 keys
+                            st_shared_v4(smem_u32(S.p[c64]) + sw128_offset(r, pc), pk[pc * 4],
+                                         pk[pc * 4 + 1], pk[pc * 4 + 2], pk[pc * 4 + 3]);
+                            st_shared_v4(smem_u32(S.ds[c64]) + sw128_offset(r, pc), dk[pc * 4],
+                                         dk[pc * 4 + 1], dk[pc * 4 + 2], dk[pc * 4 + 3]);
+                        }
+                    };
+                    if constexpr (NSLOT == 1) {
+                        // single slot: nothing to overlap, stream each 64-key chunk out
+                        if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;
+#pragma unroll 1
+                        for (int c64 = 0; c64 < BS / 64; ++c64) {
+                            uint32_t pk[32], dk[32];
+                            pds_chunk(c64, pk, dk);
+                            store_chunk(c64, pk, dk);
+                        }
+                        tc_fence_before();
+                    } else {
+                        // two slots: compute the row while the previous tile's products
+                        // still read the P / dS tile, then store it
+                        uint32_t pk[BS / 2], dk[BS / 2];
+#pragma unroll
+                        for (int c64 = 0; c64 < BS / 64; ++c64) pds_chunk(c64, pk + c64 * 32, dk + c64 * 32);
+                        tc_fence_before();
+                        if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;
+#pragma unroll
+                        for (int c64 = 0; c64 < BS / 64; ++c64) store_chunk(c64, pk + c64 * 32, dk + c64 * 32);
+                    }
+                    fence_async_smem();
+                    mbar_arrive(&S.pds_full);
+                    // dQ partial of this row and slot
+                    if (!(ok = wait(&S.dq_full[s], (i / NSLOT) & 1, 63))) break;
+                    tc_fence_after();
+                    {
+                        const size_t prow = ((size_t)(my_t < 0 ? 0 : my_t) * p.hq + my_h) * p.topk + my_j;
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            reinterpret_cast<__nv_bfloat16*>(p.part_dq) + prow * kHeadDim);
+                        const uint32_t tq = tmem + s * kSlotCols + lane_off;
+                        float o[128];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) tmem_ld32(tq + c * 32, o + c * 32);
+                        tmem_wait_ld();
+                        if (my_t >= 0) {
+#pragma unroll
+                            for (int q8 = 0; q8 < 16; ++q8) {
+                                const float* x = o + q8 * 8;
+                                uint4 w;
+                                w.x = pack_bf16x2(x[0] * p.scale, x[1] * p.scale);
+                                w.y = pack_bf16x2(x[2] * p.scale, x[3] * p.scale);
+                                w.z = pack_bf16x2(x[4] * p.scale, x[5] * p.scale);
+                                w.w = pack_bf16x2(x[6] * p.scale, x[7] * p.scale);
+                                dst[q8] = w;
+                            }
                         }
                     }
+                    if (tt == ntl - 1) {
+                        // unit epilogue: dV and scale*dK of the block as fp32 [2][BS][128]
+                        if (!(ok = wait(&S.acc_full, k & 1, 64))) break;
+                        tc_fence_after();
+                        float* dvp = p.part_dkdv + (size_t)unit_of(k) * 2 * BS * kHeadDim;
+                        float* dkp = dvp + (size_t)BS * kHeadDim;
+#pragma unroll 1
+                        for (int c32 = 0; c32 < BS / 32; ++c32) {
+                            float xv[32], xk[32];
+                            tmem_ld32(tmem + kColDV + lane_off + c32 * 32, xv);
+                            tmem_ld32(tmem + kColDK + lane_off + c32 * 32, xk);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const int key = c32 * 32 + c;
+                                dvp[(size_t)key * kHeadDim + r] = xv[c];
+                                dkp[(size_t)key * kHeadDim + r] = xk[c] * p.scale;
+                            }
+                        }
+                        tc_fence_before();
+                        mbar_arrive(&S.acc_empty);
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&S.tmem_empty[s]);
                 }
             }
-            tc_fence_before();
-            __syncthreads();
         }
-        if (S.abort_flag) break;
-
-        // unit epilogue: dV and scale*dK of this block as fp32 partials [2][BS][128]
-        {
-            float* dvp = p.part_dkdv + (size_t)unit * 2 * BS * kHeadDim;
-            float* dkp = dvp + (size_t)BS * kHeadDim;
-#pragma unroll
-            for (int c32 = 0; c32 < BS / 32; ++c32) {
-                float xv[32], xk[32];
-                tmem_ld32(tdV + lane_off + c32 * 32, xv);
-                tmem_ld32(tdK + lane_off + c32 * 32, xk);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int key = c32 * 32 + c;
-                    dvp[(size_t)key * kHeadDim + tid] = xv[c];
-                    dkp[(size_t)key * kHeadDim + tid] = xk[c] * p.scale;
-                }
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
     }
 
-    if (tid == 0 && S.abort_flag) {
-        if (kv_unwaited) mbar_wait(&S.bar_kv, kv_phase, st, 23);
-        if (mma_unwaited) mbar_wait(&S.bar_mma, mma_phase, st, 24);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -346,13 +493,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              cudaStream_t stream) {
     if (p.bs == 64) {
-        constexpr size_t smem = bwd_smem_bytes<64>();
-        cudaFuncSetAttribute(k_bwd_tiles<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_bwd_tiles<64><<<p.num_sms, kBwdThreads, smem, stream>>>(p, *kmap, *vmap);
+        constexpr size_t smem = bwd_smem_bytes<64, 2, 2>();
+        cudaFuncSetAttribute(k_bwd_tiles<64, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        k_bwd_tiles<64, 2, 2><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
     } else {
-        constexpr size_t smem = bwd_smem_bytes<128>();
-        cudaFuncSetAttribute(k_bwd_tiles<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_bwd_tiles<128><<<p.num_sms, kBwdThreads, smem, stream>>>(p, *kmap, *vmap);
+        constexpr size_t smem = bwd_smem_bytes<128, 1, 1>();
+        cudaFuncSetAttribute(k_bwd_tiles<128, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        k_bwd_tiles<128, 1, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
     }
     return cudaGetLastError();
 }

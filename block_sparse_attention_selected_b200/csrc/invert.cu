@@ -260,6 +260,134 @@ __global__ void __launch_bounds__(1024) k_tile_offsets(const int32_t* offsets, D
     }
 }
 
+// 5. Window split for the forward's tile order.  Tokens are cut into windows of
+//    `wtok` (packed) tokens; for every (g, window w, global block B) the sub-range of
+//    the (g, B) list whose tokens lie in w (the list is sorted by token, so it is a
+//    contiguous run found by binary search on the entry value token * 64 + slot).
+//    win_rng[(g * nwin + w) * nb_stride + B] = (first entry, count).
+__device__ __forceinline__ int lower_bound_u32(const uint32_t* a, int lo, int hi, uint32_t x) {
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a + mid) < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+__global__ void k_window_split(const uint32_t* entries, const int32_t* offsets, const DevStatus* st,
+                               int hkv, int nwin, int wtok, int nb_stride, int2* win_rng) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nbtot = st->nblocks_total;
+    const long long n = (long long)hkv * nwin * nbtot;
+    if (idx >= n) return;
+    const int B = (int)(idx % nbtot);
+    const long long r = idx / nbtot;          // (g * nwin + w)
+    const int w = (int)(r % nwin);
+    const int g = (int)(r / nwin);
+    const int lo = offsets[g * nbtot + B], hi = offsets[g * nbtot + B + 1];
+    const uint32_t v0 = (uint32_t)w * (uint32_t)wtok * 64u;
+    const uint32_t v1 = (uint32_t)(w + 1) * (uint32_t)wtok * 64u;
+    const int a = lower_bound_u32(entries, lo, hi, v0);
+    const int b = (w + 1 == nwin) ? hi : lower_bound_u32(entries, a, hi, v1);
+    win_rng[r * nb_stride + B] = make_int2(a, b - a);
+}
+
+// 6. Per (g, w) row: exclusive scan over B of ceil(count / tpt) tiles, and the row's
+//    total.  One block per row.
+__global__ void __launch_bounds__(1024) k_window_tiles(const int2* win_rng, const DevStatus* st,
+                                                       int nb_stride, int tpt, int32_t* tile_off,
+                                                       int32_t* row_tiles) {
+    __shared__ unsigned long long warp_tot[32];
+    __shared__ unsigned long long round_total;
+    const int nbtot = st->nblocks_total;
+    const int2* rng = win_rng + (size_t)blockIdx.x * nb_stride;
+    int32_t* out = tile_off + (size_t)blockIdx.x * (nb_stride + 1);
+    unsigned long long carry = 0;
+    for (int base = 0; base < nbtot; base += blockDim.x) {
+        const int B = base + threadIdx.x;
+        unsigned long long x = 0;
+        if (B < nbtot) x = (unsigned long long)((rng[B].y + tpt - 1) / tpt);
+        const unsigned long long incl = block_incl_scan_u64(x, warp_tot);
+        if (B < nbtot) out[B] = (int32_t)(carry + incl - x);
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        out[nbtot] = (int32_t)carry;
+        row_tiles[blockIdx.x] = (int32_t)carry;
+    }
+}
+
+// 7. Exclusive scan of the rows' tile counts; total into the status block.
+__global__ void __launch_bounds__(1024) k_row_offsets(const int32_t* row_tiles, int nrows,
+                                                      int32_t* row_off, DevStatus* st) {
+    __shared__ unsigned long long warp_tot[32];
+    __shared__ unsigned long long round_total;
+    unsigned long long carry = 0;
+    for (int base = 0; base < nrows; base += blockDim.x) {
+        const int r = base + threadIdx.x;
+        const unsigned long long x = r < nrows ? (unsigned long long)row_tiles[r] : 0ull;
+        const unsigned long long incl = block_incl_scan_u64(x, warp_tot);
+        if (r < nrows) row_off[r] = (int32_t)(carry + incl - x);
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        row_off[nrows] = (int32_t)carry;
+        st->ntiles_fwd = (int)carry;
+    }
+}
+
+// 8. One descriptor per forward tile, so that the tile kernel's roles read a tile's
+//    geometry with one load instead of three dependent binary searches:
+//    (first key of the block, first entry, nrows | g << 8, g * NB + B).
+__global__ void k_tile_desc(const DevStatus* st, const int32_t* row_off, const int32_t* tile_off,
+                            const int2* win_rng, const int32_t* blkoff, const int32_t* cu,
+                            int nseq, int hkv, int nwin, int nb_stride, int G, int bs,
+                            int4* desc) {
+    const int tile = blockIdx.x * blockDim.x + threadIdx.x;
+    if (tile >= st->ntiles_fwd) return;
+    const int nbtot = st->nblocks_total;
+    const int row = upper_index(row_off, hkv * nwin, tile);
+    const int tr = tile - row_off[row];
+    const int32_t* toff = tile_off + (size_t)row * (nb_stride + 1);
+    const int B = upper_index(toff, nbtot, tr);
+    const int2 rng = win_rng[(size_t)row * nb_stride + B];
+    const int tpt = kTileRows / G;
+    const int g = row / nwin;
+    const int s = upper_index(blkoff, nseq, B);
+    const int key0 = cu[s] + (B - blkoff[s]) * bs;
+    const int e0 = rng.x + (tr - toff[B]) * tpt;
+    const int nrows = (min(e0 + tpt, rng.x + rng.y) - e0) * G;
+    desc[tile] = make_int4(key0, e0, nrows | (g << 8), g * nbtot + B);
+}
+
+// 9. One descriptor per backward work unit (up to chunk_tiles consecutive tiles of one
+//    (g, B) list): (first key of the block, first entry, end of the list's entries,
+//    ntiles | g << 8) and the bucket id g * NB + B.
+__global__ void k_unit_desc(const DevStatus* st, const int32_t* chunk_off, const int32_t* tile_off,
+                            const int32_t* offsets, const int32_t* blkoff, const int32_t* cu,
+                            int nseq, int hkv, int tpt, int chunk_tiles, int bs, int4* udesc,
+                            int* ubucket) {
+    const int u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= st->nchunks) return;
+    const int nbtot = st->nblocks_total;
+    const int bucket = upper_index(chunk_off, hkv * nbtot, u);
+    const int t0 = tile_off[bucket];
+    const int tlo = t0 + (u - chunk_off[bucket]) * chunk_tiles;
+    const int thi = min(tlo + chunk_tiles, tile_off[bucket + 1]);
+    const int g = bucket / nbtot;
+    const int B = bucket - g * nbtot;
+    const int s = upper_index(blkoff, nseq, B);
+    const int key0 = cu[s] + (B - blkoff[s]) * bs;
+    udesc[u] = make_int4(key0, offsets[bucket] + (tlo - t0) * tpt, offsets[bucket + 1],
+                         (thi - tlo) | (g << 8));
+    ubucket[u] = bucket;
+}
+
 // Range / duplicate check of block_idx (one thread per (token, KV head) row).
 __global__ void k_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
                            int topk, int bs, DevStatus* st) {
@@ -317,6 +445,28 @@ cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
                                                                       p.st, p.hkv, p.offsets);
     k_tile_offsets<<<1, 1024, 0, stream>>>(p.offsets, p.st, p.hkv, p.tokens_per_tile,
                                            p.chunk_tiles, p.tile_off, p.chunk_off);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaStream_t stream) {
+    const int nrows = p.hkv * w.nwin;
+    const long long n = (long long)nrows * w.nb_stride;      // upper bound (device NB <= stride)
+    k_window_split<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+        p.vals[p.final_buf], p.offsets, p.st, p.hkv, w.nwin, w.wtok, w.nb_stride, w.win_rng);
+    k_window_tiles<<<nrows, 1024, 0, stream>>>(w.win_rng, p.st, w.nb_stride, p.tokens_per_tile,
+                                               w.tile_off, w.row_tiles);
+    k_row_offsets<<<1, 1024, 0, stream>>>(w.row_tiles, nrows, w.row_off, p.st);
+    k_tile_desc<<<(unsigned)((w.tiles_cap + 255) / 256), 256, 0, stream>>>(
+        p.st, w.row_off, w.tile_off, w.win_rng, p.blkoff, p.cu, p.nseq, p.hkv, w.nwin, w.nb_stride,
+        kTileRows / p.tokens_per_tile, p.bs, w.tile_desc);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
+                             cudaStream_t stream) {
+    k_unit_desc<<<(unsigned)((units_cap + 255) / 256), 256, 0, stream>>>(
+        p.st, p.chunk_off, p.tile_off, p.offsets, p.blkoff, p.cu, p.nseq, p.hkv,
+        p.tokens_per_tile, p.chunk_tiles, p.bs, udesc, ubucket);
     return cudaGetLastError();
 }
 

@@ -32,7 +32,8 @@ struct DevStatus {
     int nchunks;       // number of backward work units of the last inversion
     int nentries;      // number of valid (token, KV head, slot) entries
     long long bad_range, bad_dup;   // validation counters
-    int pad[52];
+    int ntiles_fwd;    // number of forward tiles in window order
+    int pad[51];
 };
 static_assert(sizeof(DevStatus) == 256, "status block is 256 bytes");
 
@@ -190,6 +191,7 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 
 // 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32*(w%4)..).
+// Several loads may be issued before one tmem_wait_ld().
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     uint32_t* r = reinterpret_cast<uint32_t*>(v);
     asm volatile(

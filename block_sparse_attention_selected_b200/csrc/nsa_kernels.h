@@ -41,8 +41,24 @@ struct InvertPlan {
 
 constexpr int kSortTile = 4096;  // entries per sort tile (256 threads x 16)
 
+// Window split of the (g, B) lists for the forward's tile order (g, window, B).
+struct WindowPlan {
+    int nwin;                // number of token windows
+    int wtok;                // tokens per window
+    int nb_stride;           // row stride of the tables: T / bs + nseq >= NB
+    int2* win_rng;           // [hkv * nwin * nb_stride]: (first entry, count)
+    int32_t* tile_off;       // [hkv * nwin * (nb_stride + 1)]: tile offsets within a row
+    int32_t* row_tiles;      // [hkv * nwin]
+    int32_t* row_off;        // [hkv * nwin + 1]
+    int4* tile_desc;         // [tiles_cap]: (key0, e0, nrows | g << 8, g * NB + B)
+    long long tiles_cap;     // bound on the number of forward tiles
+};
+
 // Runs the inversion on `stream`; returns the first launch error.
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream);
+cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaStream_t stream);
+cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
+                             cudaStream_t stream);
 
 struct FwdPlan {
     const void* q;
@@ -54,6 +70,12 @@ struct FwdPlan {
     const int32_t* tile_off; // bucket tile offsets
     const uint32_t* entries; // token * 64 + slot
     int nbk_cap;
+    // window order of the tiles (see WindowPlan)
+    int nwin, nb_stride;
+    const int2* win_rng;
+    const int32_t* wtile_off;
+    const int32_t* row_off;
+    const int4* tile_desc;
     void* part_o;            // fp16 [T * hq * topk, 128]: O_B / l_B * 2^-e
     float2* part_meta;       // [T * hq * topk]: (lse_B, e)
     DevStatus* st;
@@ -90,6 +112,8 @@ struct BwdPlan {
     const uint32_t* entries;
     int nbk_cap;
     int chunk_tiles;
+    const int4* udesc;       // per unit: (key0, first entry, list end, ntiles | g << 8)
+    const int* ubucket;      // per unit: g * NB + B
     void* part_dq;           // bf16 [T * hq * topk, 128]
     float* part_dkdv;        // fp32 [chunks, 2, bs, 128]
     DevStatus* st;
