@@ -24,8 +24,9 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
                 3: "NSA_ERR_WORKSPACE", 4: "NSA_ERR_CUDA", 5: "NSA_ERR_TIMEOUT",
                 6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
-            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_invert_index", "nsa_sel_validate_indices", "nsa_sel_check_status",
-            "nsa_sel_status_string"]
+            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_invert_index",
+            "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
+            "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
 
 _lib = None
 _lock = threading.Lock()
@@ -61,6 +62,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_bwd_profiled.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
+            lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
+            lib.nsa_sel_invert_index_noalloc.restype = I
+            lib.nsa_sel_invert_index_noalloc_max_bytes.argtypes = []
+            lib.nsa_sel_invert_index_noalloc_max_bytes.restype = Z
             lib.nsa_sel_validate_indices.argtypes = [P, I, I, I, P, I, I, P, P, P, Z, P]
             lib.nsa_sel_validate_indices.restype = I
             lib.nsa_sel_check_status.argtypes = [P, P]
@@ -205,6 +210,30 @@ def nsa_sel_invert_index(cu_seqlens, block_idx, block_size, workspace=None):
     _check("nsa_sel_invert_index", load_library().nsa_sel_invert_index(
         _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
         _ptr(entries), _ptr(counts), _ptr(ws), ws.numel(), _stream(dev)))
+    nb, n = (int(x) for x in counts.tolist())
+    return offsets[:hkv * nb + 1], entries[:n]
+
+
+def nsa_sel_invert_index_noalloc(cu_seqlens, block_idx, block_size):
+    """The block-index inversion without a caller workspace.
+
+    For callers that cannot allocate device memory (a plug-in inside a framework
+    that owns all device memory, or a loop where cudaMalloc is not allowed): the
+    library uses a fixed device array of its own as scratch.  Output buffers are
+    still the caller's.  Calls sharing a device must not overlap on the GPU.
+    Returns (offsets int32 [hkv*NB+1], entries int32 [n]).
+    """
+    dev = block_idx.device
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(block_idx, "block_idx", torch.int32, 3, dev)
+    T, hkv, topk = block_idx.shape
+    nseq = cu_seqlens.numel() - 1
+    offsets = torch.empty(hkv * (T // block_size + nseq) + 1, dtype=torch.int32, device=dev)
+    entries = torch.empty(max(T * hkv * topk, 1), dtype=torch.int32, device=dev)
+    counts = torch.zeros(2, dtype=torch.int32, device=dev)
+    _check("nsa_sel_invert_index_noalloc", load_library().nsa_sel_invert_index_noalloc(
+        _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
+        _ptr(entries), _ptr(counts), _stream(dev)))
     nb, n = (int(x) for x in counts.tolist())
     return offsets[:hkv * nb + 1], entries[:n]
 

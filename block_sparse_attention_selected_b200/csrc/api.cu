@@ -551,3 +551,98 @@ nsa_status_t nsa_sel_check_status(const void* workspace, nsa_stream_t stream_) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Index inversion with library-owned scratch.
+//
+// For callers that cannot allocate device memory themselves -- a plug-in running
+// inside a framework that owns every byte of device memory and gives plug-ins no
+// allocation hook, or a latency-critical loop where cudaMalloc (which may
+// synchronise the device) is not allowed -- this entry point takes its scratch from
+// a fixed array in the library's own device data instead of a caller workspace.
+//
+// The array (kInvertScratchBytes, 64 MiB) exists once per device that loads the
+// library and stays allocated until the process exits.  Its device address is looked
+// up with cudaGetSymbolAddress the first time the entry point runs on a device (with
+// that device current); make that first call before any stream capture.  All calls
+// share the array and it keeps the last call's contents (everything a call reads is
+// first written by the same call, and its status block is cleared on entry), so
+// calls whose work overlaps on the GPU -- on different streams, or from different
+// host threads -- race with one another: serialise them.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kInvertScratchBytes = size_t(64) << 20;
+__device__ __align__(256) unsigned char g_invert_scratch[kInvertScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_address[kMaxScratchDevices] = {};
+
+// Device address of this device's scratch array (resolved once per device).
+nsa_status_t scratch_for_current_device(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_NO_DEVICE;
+    if (dev < 0 || dev >= kMaxScratchDevices) return NSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_address[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_invert_scratch) != cudaSuccess || !ptr) return NSA_ERR_CUDA;
+        g_scratch_address[dev] = ptr;
+    }
+    *out = g_scratch_address[dev];
+    return NSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nsa_sel_invert_index_noalloc_max_bytes(void) { return kInvertScratchBytes; }
+
+nsa_status_t nsa_sel_invert_index_noalloc(const int32_t* cu_seqlens, int num_seqs,
+                                          int total_tokens, int hkv, const int32_t* block_idx,
+                                          int topk, int block_size, int32_t* offsets,
+                                          int32_t* entries, int32_t* counts,
+                                          nsa_stream_t stream_) {
+    Dims D;
+    // hq = hkv (group 1) fixes the tile geometry; it does not change the inversion.
+    nsa_status_t s = check_dims(total_tokens, num_seqs, hkv, hkv, kHeadDim, topk, block_size, &D);
+    if (s != NSA_OK) return s;
+    if (!cu_seqlens || (total_tokens > 0 && !block_idx) || !offsets || !entries || !counts)
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4) || !aligned(block_idx, 4) || !aligned(offsets, 4) ||
+        !aligned(entries, 4) || !aligned(counts, 4))
+        return NSA_ERR_INVALID_ARG;
+    const Layout L = make_layout(D, false);
+    if (L.win_rng > kInvertScratchBytes) return NSA_ERR_WORKSPACE;   // too large for the array
+    int num_sms = 0;
+    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    void* scratch = nullptr;
+    if ((s = scratch_for_current_device(&scratch)) != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    Carved c = carve(D, L, scratch, cu_seqlens, block_idx);
+    if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) {
+        if (cudaMemsetAsync(counts, 0, 2 * sizeof(int32_t), stream) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int32_t) * ((size_t)D.nbk_cap + 1), stream) !=
+                cudaSuccess)
+            return NSA_ERR_CUDA;
+        return NSA_OK;
+    }
+    if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+    cudaError_t e = cudaMemcpyAsync(offsets, c.inv.offsets, sizeof(int32_t) * ((size_t)D.nbk_cap + 1),
+                                    cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(entries, c.inv.vals[c.inv.final_buf], sizeof(int32_t) * (size_t)D.nent,
+                            cudaMemcpyDeviceToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(counts, &c.st->nblocks_total, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(counts + 1, &c.st->nentries, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                            stream);
+    return cuda_status(e);
+}
+
+}  // extern "C"

@@ -141,6 +141,30 @@ NSA_API nsa_status_t nsa_sel_invert_index(const int32_t *cu_seqlens, int num_seq
                                   int32_t *offsets, int32_t *entries, int32_t *counts,
                                   void *workspace, size_t workspace_bytes, nsa_stream_t stream);
 
+/* The block-index inversion above, for callers that cannot allocate device memory
+ * (for example a plug-in whose host framework owns all device memory and offers no
+ * allocation hook, or a loop where cudaMalloc's possible device synchronisation is
+ * not allowed).  The pages have no counterpart for this entry point.
+ *   Arguments and outputs are those of nsa_sel_invert_index, without the workspace:
+ *   the scratch is a fixed array in the library's device data, of
+ *   nsa_sel_invert_index_noalloc_max_bytes() bytes (64 MiB) per device, held until
+ *   the process exits.  Problems whose inversion scratch would not fit return
+ *   NSA_ERR_WORKSPACE before any device work (about 17 bytes per (token, KV head,
+ *   slot) entry: T * hkv * topk up to roughly 3.5 million).
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents; each call
+ *   clears what it reads before writing it, but calls whose work overlaps on the GPU
+ *   (other streams, other host threads) race: serialise them. */
+NSA_API nsa_status_t nsa_sel_invert_index_noalloc(const int32_t *cu_seqlens, int num_seqs,
+                                                  int total_tokens, int hkv,
+                                                  const int32_t *block_idx, int topk,
+                                                  int block_size, int32_t *offsets,
+                                                  int32_t *entries, int32_t *counts,
+                                                  nsa_stream_t stream);
+/* Size in bytes of the scratch array used by nsa_sel_invert_index_noalloc. */
+NSA_API size_t nsa_sel_invert_index_noalloc_max_bytes(void);
+
 /* Host-synchronous check of block_idx: counts values outside {-1} U [0, NB_s) and
  * repeated non-negative values within one (token, KV head) row.  Returns
  * NSA_ERR_BAD_INDEX when either count is non-zero, NSA_OK otherwise.  Future blocks
