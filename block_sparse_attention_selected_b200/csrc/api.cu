@@ -17,7 +17,7 @@ using namespace nsa;
 namespace {
 
 constexpr int kChunkTiles = 32;   // tiles per backward work unit
-constexpr int kWindowRows = 8192; // query rows per forward token window (tokens x group)
+constexpr int kWindowRows = 32768; // query rows per forward token window (tokens x group)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -34,7 +34,7 @@ struct Dims {
 
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
-    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc;
+    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket;
     size_t total;
 };
@@ -93,6 +93,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.row_tiles = take(sizeof(int32_t) * wrows);
     L.row_off = take(sizeof(int32_t) * (wrows + 1));
     L.tile_desc = take(sizeof(int4) * (size_t)std::max<long long>(D.fwd_tiles_cap, 1));
+    L.posmap = take(sizeof(int32_t) * (size_t)std::max<long long>(D.nent, 1));
     const size_t rows = (size_t)D.T * D.hq * D.topk;
     L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
@@ -298,7 +299,9 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     wp.tile_desc = reinterpret_cast<int4*>(c.base + L.tile_desc);
     wp.tiles_cap = D.fwd_tiles_cap;
     if ((s = cuda_status(launch_window_split(c.inv, wp, stream))) != NSA_OK) return s;
-    pm.add(invert_launches(D) + 4);
+    int32_t* posmap = reinterpret_cast<int32_t*>(c.base + L.posmap);
+    if ((s = cuda_status(launch_posmap(c.inv, D.nent, posmap, stream))) != NSA_OK) return s;
+    pm.add(invert_launches(D) + 5);
     pm.mark(1);
 
     FwdPlan fp{};
@@ -329,11 +332,14 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     MergePlan mp{};
     mp.cu = cu_seqlens;
     mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
+    mp.G = D.G;
     mp.bidx = block_idx;
+    mp.posmap = posmap;
     mp.part_o = fp.part_o;
     mp.part_meta = fp.part_meta;
     mp.out = out;
     mp.lse = lse;
+    mp.st = c.st;
     if ((s = cuda_status(launch_merge(mp, stream))) != NSA_OK) return s;
     pm.add(1);
     pm.mark(3);

@@ -72,10 +72,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 template <int BS, int NQ, int NSLOT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_tiles(const BwdPlan p, const __grid_constant__ CUtensorMap kmap,

@@ -388,6 +388,20 @@ __global__ void k_unit_desc(const DevStatus* st, const int32_t* chunk_off, const
     ubucket[u] = bucket;
 }
 
+// 10. Position map: for every sorted position pos of a valid entry (token t, KV head
+//     g, slot j), posmap[(t * hkv + g) * topk + j] = pos.  The forward's partial
+//     results are stored in sorted order; the merge finds them through this map.
+__global__ void k_posmap(const uint32_t* keys, const uint32_t* vals, const DevStatus* st, int hkv,
+                         int topk, int32_t* posmap) {
+    const int pos = blockIdx.x * blockDim.x + threadIdx.x;
+    // malformed cu_seqlens (recorded by k_seq_blocks) leave the keys inconsistent
+    if (st->code != 0 || pos >= st->nentries) return;
+    const uint32_t g = keys[pos] / (uint32_t)st->nblocks_total;
+    const uint32_t v = vals[pos];
+    if (g >= (uint32_t)hkv || (int)(v & 63u) >= topk) return;
+    posmap[((size_t)(v >> 6) * hkv + g) * topk + (v & 63u)] = pos;
+}
+
 // Range / duplicate check of block_idx (one thread per (token, KV head) row).
 __global__ void k_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
                            int topk, int bs, DevStatus* st) {
@@ -459,6 +473,14 @@ cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaSt
     k_tile_desc<<<(unsigned)((w.tiles_cap + 255) / 256), 256, 0, stream>>>(
         p.st, w.row_off, w.tile_off, w.win_rng, p.blkoff, p.cu, p.nseq, p.hkv, w.nwin, w.nb_stride,
         kTileRows / p.tokens_per_tile, p.bs, w.tile_desc);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_posmap(const InvertPlan& p, long long nent, int32_t* posmap,
+                          cudaStream_t stream) {
+    if (nent > 0)
+        k_posmap<<<(unsigned)((nent + 255) / 256), 256, 0, stream>>>(
+            p.keys[p.final_buf], p.vals[p.final_buf], p.st, p.hkv, p.topk, posmap);
     return cudaGetLastError();
 }
 

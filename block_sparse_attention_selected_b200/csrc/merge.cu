@@ -28,29 +28,46 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: it finds the
+// slot's partial through the position map (row = sorted position * G + head offset)
+// and reads its (lse_j, exponent_j).  The 128 columns are split 4 per lane; partial
+// rows are fetched eight slots at a time so that eight 256-byte reads are in flight.
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p) {
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hq) return;
+    // after a recorded device error (malformed cu_seqlens, an expired wait) the
+    // position map and partials are incomplete: leave the outputs untouched
+    if (*reinterpret_cast<const volatile int*>(&p.st->code) != 0) return;
     const int t = (int)(row / p.hq);
     const int h = (int)(row - (long long)t * p.hq);
-    const int g = h / (p.hq / p.hkv);
+    const int g = h / p.G;
+    const int hoff = h - g * p.G;
+    const unsigned nrows_part = (unsigned)p.st->nentries * (unsigned)p.G;
     const int s = seq_of_token(p.cu, p.nseq, t);
     const int qb = (t - __ldg(p.cu + s)) / p.bs;
-    const int32_t* bi = p.bidx + ((size_t)t * p.hkv + g) * p.topk;
-    const size_t prow0 = (size_t)row * p.topk;
+    const size_t base = ((size_t)t * p.hkv + g) * p.topk;
+    const int32_t* bi = p.bidx + base;
+    const int32_t* pm = p.posmap + base;
 
-    // lane j holds slot j (and j + 32): (lse_j, exponent_j) of the valid slots
+    // lane j holds slot j (and j + 32): partial row and (lse_j, exponent_j)
     float l0 = -CUDART_INF_F, l1 = -CUDART_INF_F, e0 = 0.f, e1 = 0.f;
+    unsigned r0 = 0u, r1 = 0u;
     if (lane < p.topk && block_valid(__ldg(bi + lane), qb)) {
-        const float2 m = __ldg(p.part_meta + prow0 + lane);
-        l0 = m.x;
-        e0 = m.y;
+        r0 = (unsigned)__ldg(pm + lane) * (unsigned)p.G + (unsigned)hoff;
+        if (r0 < nrows_part) {
+            const float2 m = __ldg(p.part_meta + r0);
+            l0 = m.x;
+            e0 = m.y;
+        }
     }
     if (lane + 32 < p.topk && block_valid(__ldg(bi + lane + 32), qb)) {
-        const float2 m = __ldg(p.part_meta + prow0 + lane + 32);
-        l1 = m.x;
-        e1 = m.y;
+        r1 = (unsigned)__ldg(pm + lane + 32) * (unsigned)p.G + (unsigned)hoff;
+        if (r1 < nrows_part) {
+            const float2 m = __ldg(p.part_meta + r1);
+            l1 = m.x;
+            e1 = m.y;
+        }
     }
     const float M = warp_max(fmaxf(l0, l1));
     uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
@@ -65,17 +82,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
     const float Lam = warp_sum(w0 + w1);
     const float s0 = ldexpf(w0, (int)e0), s1 = ldexpf(w1, (int)e1);   // weight x 2^e
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint2* po = reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(p.part_o) +
-                                                     prow0 * kHeadDim) + lane;
-    for (int j = 0; j < p.topk; ++j) {
-        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
-        if (wj == 0.f) continue;       // warp-uniform
-        const uint2 u = __ldg(po + (size_t)j * (kHeadDim / 4));
-        const float2 a = unpack_f16x2(u.x), b = unpack_f16x2(u.y);
-        acc[0] = fmaf(wj, a.x, acc[0]);
-        acc[1] = fmaf(wj, a.y, acc[1]);
-        acc[2] = fmaf(wj, b.x, acc[2]);
-        acc[3] = fmaf(wj, b.y, acc[3]);
+    const uint2* po = reinterpret_cast<const uint2*>(p.part_o) + lane;
+    for (int j0 = 0; j0 < p.topk; j0 += 8) {
+        uint2 u[8];
+        float wv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int j = j0 + k;               // warp-uniform
+            const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
+            const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
+            wv[k] = j < p.topk ? wj : 0.f;
+            u[k] = wv[k] != 0.f ? __ldg(po + (size_t)rj * (kHeadDim / 4)) : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 a = unpack_f16x2(u[k].x), b = unpack_f16x2(u[k].y);
+            acc[0] = fmaf(wv[k], a.x, acc[0]);
+            acc[1] = fmaf(wv[k], a.y, acc[1]);
+            acc[2] = fmaf(wv[k], b.x, acc[2]);
+            acc[3] = fmaf(wv[k], b.y, acc[3]);
+        }
     }
     const float inv = 1.f / Lam;
     *outp = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));

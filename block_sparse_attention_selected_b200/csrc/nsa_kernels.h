@@ -57,6 +57,10 @@ struct WindowPlan {
 // Runs the inversion on `stream`; returns the first launch error.
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream);
 cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaStream_t stream);
+// posmap[(t * hkv + g) * topk + j] = position of entry (t, g, j) in the sorted list
+// (written for valid entries only).
+cudaError_t launch_posmap(const InvertPlan& p, long long nent, int32_t* posmap,
+                          cudaStream_t stream);
 cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
                              cudaStream_t stream);
 
@@ -76,8 +80,9 @@ struct FwdPlan {
     const int32_t* wtile_off;
     const int32_t* row_off;
     const int4* tile_desc;
-    void* part_o;            // fp16 [T * hq * topk, 128]: O_B / l_B * 2^-e
-    float2* part_meta;       // [T * hq * topk]: (lse_B, e)
+    void* part_o;            // fp16 [entries * G, 128]: O_B / l_B * 2^-e, row e * G + head
+                             // offset for the sorted entry e (tile-contiguous)
+    float2* part_meta;       // [entries * G]: (lse_B, e)
     DevStatus* st;
     int num_sms;
 };
@@ -87,12 +92,14 @@ cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CU
 
 struct MergePlan {
     const int32_t* cu;
-    int nseq, T, hq, hkv, topk, bs;
+    int nseq, T, hq, hkv, topk, bs, G;
     const int32_t* bidx;
+    const int32_t* posmap;   // sorted position of each valid (t, g, j) entry
     const void* part_o;
     const float2* part_meta;
     void* out;
     float* lse;
+    const DevStatus* st;
 };
 
 cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream);
