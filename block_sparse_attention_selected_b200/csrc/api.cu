@@ -34,7 +34,7 @@ struct Dims {
 
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
-    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap;
+    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket;
     size_t total;
 };
@@ -94,6 +94,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.row_off = take(sizeof(int32_t) * (wrows + 1));
     L.tile_desc = take(sizeof(int4) * (size_t)std::max<long long>(D.fwd_tiles_cap, 1));
     L.posmap = take(sizeof(int32_t) * (size_t)std::max<long long>(D.nent, 1));
+    L.vexp = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     const size_t rows = (size_t)D.T * D.hq * D.topk;
     L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
@@ -325,8 +326,11 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.part_meta = reinterpret_cast<float2*>(c.base + L.part_lse);
     fp.st = c.st;
     fp.num_sms = num_sms;
+    int32_t* vexp = reinterpret_cast<int32_t*>(c.base + L.vexp);
+    fp.vexp = vexp;
+    if ((s = cuda_status(launch_vblock_exp(fp, v, D.nb_stride, vexp, stream))) != NSA_OK) return s;
     if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, stream))) != NSA_OK) return s;
-    pm.add(1);
+    pm.add(2);
     pm.mark(2);
 
     MergePlan mp{};

@@ -7,10 +7,12 @@
 // Attention" blog, second paragraph).  Per tile:
 //
 //   S   = Q K_B^T                  tcgen05.mma (Q, K from shared memory) -> TMEM
-//   P   = exp2(c S - c m), causal mask on the diagonal block, l = sum P, written
-//         as bf16 back into the S columns of TMEM
+//   P   = exp2(c S - c m), causal mask on the diagonal block, l = sum P; P is
+//         written as bf16 back into the S columns of TMEM
 //   O_B = P V_B                    tcgen05.mma with A = P read from TMEM
-//   partial: O_B / l as fp16 with a power-of-two row exponent, lse_B = m + log l.
+//   partial: O_B * 2^-e / l as fp16, lse_B = m + log l.  e is the block's V
+//         exponent (k_vblock_exp): 0 unless max |V_B| > 2^14, so O_B / l, a convex
+//         combination of V_B's rows, always fits fp16 after the 2^-e.
 //
 // A tile covers the consecutive entries [e0, e0 + ntok) of the sorted index list
 // (invert.cu), so its partial rows (entry * G + head offset) are one contiguous
@@ -22,14 +24,17 @@
 // kChunk consecutive tiles round-robin (consecutive tiles of one (g, window, B) list
 // share K_B / V_B).  Each CTA is warp-specialised and pipelined:
 //
-//   warps 0-1   Q loaders: coalesced cp.async gather (two 256-byte rows per warp
-//               instruction) into the 128B-swizzled Q tile, kNQ stages
-//   warp 2      TMA producer: K_B and V_B (128B swizzle) into NKV stages
-//   warp 3      MMA issuer (one thread): S(i+1) is issued before PV(i)
-//   warps 4-7   softmax + epilogue of even tiles   } TMEM slots 0 / 1: S (P) and
-//   warps 8-11  softmax + epilogue of odd tiles    } O accumulators each
+//   warps 0-1    Q loaders: coalesced cp.async gather (two 256-byte rows per warp
+//                instruction) into the 128B-swizzled Q tile, kNQ stages
+//   warp 2       TMA producer: K_B and V_B (128B swizzle) into NKV stages
+//   warp 3       MMA issuer (one thread): S(i+1) is issued before PV(i)
+//   warps 4-7    softmax of even tiles  } TMEM slot 0 / 1: S (P) and O accumulators
+//   warps 8-11   softmax of odd tiles   }
+//   warps 12-15  epilogue of every tile: O from TMEM, scale, fp16, store
 //
-// Producer/consumer hand-offs are mbarriers; every wait is bounded (nsa_common.cuh).
+// The softmax hands each row's scale 2^-e / l to the epilogue in shared memory
+// (double-buffered per slot, with its own barrier).  Producer/consumer hand-offs are
+// mbarriers; every wait is bounded (nsa_common.cuh).
 #include <math_constants.h>
 
 #include "nsa_common.cuh"
@@ -38,9 +43,9 @@
 namespace nsa {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kLoaderThreads = 64;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kWgThreads = 128;
 constexpr int kNQ = 2;         // Q stages
 constexpr int kChunk = 2;      // consecutive tiles per scheduling chunk
 
@@ -48,10 +53,12 @@ template <int BS, int NKV>
 struct alignas(1024) FwdSmem {
     uint8_t q[kNQ][2][kTileRows * 128];       // Q tile per stage: [64-column half][row]
     uint8_t kv[NKV][2][2][BS * 128];          // [stage][K, V][64-column half][key]
-    uint8_t stage[8][32 * 128];               // epilogue staging, 4 KB per softmax warp
+    uint8_t stage[4][32 * 128];               // epilogue staging, 4 KB per epilogue warp
+    float sc[2][2][kTileRows];                // row scale 2^-e / l: [slot][tile parity][row]
     uint64_t q_full[kNQ], q_empty[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
     uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+    uint64_t l_full[2][2];                    // sc[slot][parity] written
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -107,9 +114,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
-            mbar_init(&S.p_full[i], kSoftmaxThreads);
+            mbar_init(&S.p_full[i], kWgThreads);
             mbar_init(&S.o_full[i], 1);
-            mbar_init(&S.o_free[i], kSoftmaxThreads);
+            mbar_init(&S.o_free[i], kWgThreads);
+            mbar_init(&S.l_full[i][0], kWgThreads);
+            mbar_init(&S.l_full[i][1], kWgThreads);
         }
         for (int i = 0; i < NKV; ++i) {
             mbar_init(&S.kv_full[i], 1);
@@ -150,6 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
     };
+    // a warp leaves its loop together: every wait of a warp-collective role is voted
+    auto wait_w = [&](uint64_t* bar, uint32_t parity, int where) -> bool {
+        return __all_sync(0xffffffffu, wait(bar, parity, where));
+    };
 
     if (warp < 2) {
         // ---------------------------------------------------------------- Q loaders
@@ -159,8 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 16-byte chunk l % 16 of row 64w + 2k + l / 16 (a 512-byte coalesced read).
         // The copies of tile i are published one tile later (wait for the older
         // cp.async group, fence for the tensor core's async proxy, arrive on q_full),
-        // so two tiles' gathers are in flight.  A warp leaves the loop together: every
-        // wait is followed by a warp vote.
+        // so two tiles' gathers are in flight.
         const int w = warp;
         const uint8_t* qb = static_cast<const uint8_t*>(p.q);
         const int rA = 64 * w + lane, rB = rA + 32;
@@ -175,28 +187,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         int4 d0 = ld_desc(0), d1 = ld_desc(1);
         uint32_t ea = ld_ent(d0, rA), eb = ld_ent(d0, rB);
         int published = 0, issued = 0;
+        const int c = lane & 15;
+        const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
         for (int i = 0; i < n; ++i) {
             const int4 d = d0;
-            const unsigned long long addrA = row_addr(d, rA, ea), addrB = row_addr(d, rB, eb);
+            const unsigned long long addrA = row_addr(d, rA, ea);
+            const unsigned long long addrB = row_addr(d, rB, eb);
             d0 = d1;
             d1 = ld_desc(i + 2);
             ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
             eb = ld_ent(d0, rB);
             const int nrows = d.z & 255;
             const int stg = i % kNQ;
-            const bool ok = wait(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            const uint32_t q0 = smem_u32(S.q[stg][0]);
-            const int c = lane & 15;
-#pragma unroll
+            if (!wait_w(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
+            const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
+#pragma unroll 4
             for (int k = 0; k < 32; ++k) {
                 const int rw = 2 * k + (lane >> 4);          // row within the warp's 64
                 const unsigned long long a =
-                    __shfl_sync(0xffffffffu, k < 16 ? addrA : addrB, rw & 31);
+                    __shfl_sync(0xffffffffu, k < 16 ? addrA : addrB, rw & 31) + c * 16;
                 const int row = 64 * w + rw;
                 if (row < nrows)
-                    cp_async_16(q0 + (c >> 3) * (kTileRows * 128) + sw128_offset(row, c & 7),
-                                reinterpret_cast<const void*>(a + c * 16));
+                    cp_async_16(q0 + sw128_offset(row, c & 7), reinterpret_cast<const void*>(a));
             }
             cp_async_commit();
             issued = i + 1;
@@ -312,80 +324,128 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&S.drain);
             mbar_wait(&S.drain, 0, st, 41);
         }
-    } else {
-        // ---------------------------------------------------- softmax + epilogue
+    } else if (warp < 12) {
+        // ------------------------------------------------------------------ softmax
+        // Thread = tile row = TMEM lane.  Non-diagonal tiles (every row sees the whole
+        // block) skip the causal mask; the test is warp-uniform.
         const int wg = (warp - 4) >> 2;                  // 0: even tiles, 1: odd tiles
         const int quad = warp & 3;                       // TMEM lanes 32*quad ..
-        const int r = quad * 32 + lane;                  // tile row = TMEM lane
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + wg * kSlot + lane_off;
-        const uint32_t tO = tS + BS;
-        const uint32_t stg_base = smem_u32(S.stage[warp - 4]);
+        const int r = quad * 32 + lane;
+        const uint32_t tS = tmem + wg * kSlot + ((uint32_t)(quad * 32) << 16);
         const float c = p.scale_log2;
         const float kLn2 = 0.69314718055994531f;
-        uint8_t* const part_o = static_cast<uint8_t*>(p.part_o);
+        auto ld_row = [&](const int4& d, int i) -> uint32_t {
+            return (i < n && r < (d.z & 255)) ? __ldg(p.entries + d.y + r / p.G) : 0u;
+        };
+        auto ld_vexp = [&](const int4& d, int i) -> int { return i < n ? __ldg(p.vexp + d.w) : 0; };
+        // max over 64 scores; masked: only keys base + k <= lim
+        auto row_max64 = [&](const float* v, bool nomask, int lim, int base) -> float {
+            float a = -CUDART_INF_F, b = -CUDART_INF_F;
+            if (nomask) {
+#pragma unroll
+                for (int k = 0; k < 64; k += 4) {
+                    a = fmax3(a, v[k], v[k + 1]);
+                    b = fmax3(b, v[k + 2], v[k + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 64; k += 2) {
+                    a = fmaxf(a, base + k <= lim ? v[k] : -CUDART_INF_F);
+                    b = fmaxf(b, base + k + 1 <= lim ? v[k + 1] : -CUDART_INF_F);
+                }
+            }
+            return fmaxf(a, b);
+        };
+        // P = 2^(c s - c m) of 64 scores as packed bf16 pairs; l accumulates sum P
+        auto p_chunk = [&](const float* v, float mc, bool nomask, int lim, int base,
+                           uint32_t* pk, float2& l2) {
+            const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
+#pragma unroll
+            for (int k2 = 0; k2 < 32; ++k2) {
+                float2 x = fma2(make_float2(v[2 * k2], v[2 * k2 + 1]), c2, nmc2);
+                x.x = ex2_approx(x.x);
+                x.y = ex2_approx(x.y);
+                if (!nomask) {
+                    if (base + 2 * k2 > lim) x.x = 0.f;
+                    if (base + 2 * k2 + 1 > lim) x.y = 0.f;
+                }
+                l2 = add2(l2, x);
+                pk[k2] = pack_bf16x2(x.x, x.y);
+            }
+        };
         int4 dn = ld_desc(wg);
-        uint32_t en = (wg < n && r < (dn.z & 255)) ? __ldg(p.entries + dn.y + r / p.G) : 0u;
+        uint32_t en = ld_row(dn, wg);
+        int vn = ld_vexp(dn, wg);
         for (int i = wg; i < n; i += 2) {
             const int4 d = dn;
             const uint32_t ent = en;
+            const int ve = vn;
             dn = ld_desc(i + 2);
-            en = (i + 2 < n && r < (dn.z & 255)) ? __ldg(p.entries + dn.y + r / p.G) : 0u;
+            en = ld_row(dn, i + 2);
+            vn = ld_vexp(dn, i + 2);
             const uint32_t ph = (i >> 1) & 1;
-            const int nrows = d.z & 255;
-            const bool valid = r < nrows;
+            const bool valid = r < (d.z & 255);
             // keys 0 .. lim of the block are visible to this row (causal on the diagonal)
             const int lim = valid ? (int)(ent >> 6) - d.x : -1;
-            if (!__all_sync(0xffffffffu, wait(&S.s_full[wg], ph, 38))) break;
+            const bool nomask = __all_sync(0xffffffffu, !valid || lim >= BS - 1);
+            if (!wait_w(&S.s_full[wg], ph, 38)) break;
             tc_fence_after();
-            float sv[BS];
-#pragma unroll
-            for (int c32 = 0; c32 < BS / 32; ++c32) tmem_ld32(tS + c32 * 32, sv + c32 * 32);
+            float sv[64];
+            tmem_ld32(tS, sv);
+            tmem_ld32(tS + 32, sv + 32);
             tmem_wait_ld();
-            float mx = -CUDART_INF_F;
-#pragma unroll
-            for (int k = 0; k < BS; ++k) mx = fmaxf(mx, k <= lim ? sv[k] : -CUDART_INF_F);
-            if (lim < 0) mx = 0.f;
+            float mx = row_max64(sv, nomask, lim, 0);
+            if constexpr (BS == 128) {
+                tmem_ld32(tS + 64, sv);
+                tmem_ld32(tS + 96, sv + 32);
+                tmem_wait_ld();
+                mx = fmaxf(mx, row_max64(sv, nomask, lim, 64));
+            }
+            if (!valid) mx = 0.f;                      // every valid row has lim >= 0
             const float mc = mx * c;
-            // P = 2^(c s - c m) as bf16 over the S columns, l = sum of P (fp32)
-            float l = 0.f;
+            float2 l2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c64 = 0; c64 < BS / 64; ++c64) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int k2 = 0; k2 < 32; ++k2) {
-                    const int k = c64 * 64 + 2 * k2;
-                    const float x0 = k <= lim ? ex2_approx(fmaf(sv[k], c, -mc)) : 0.f;
-                    const float x1 = k + 1 <= lim ? ex2_approx(fmaf(sv[k + 1], c, -mc)) : 0.f;
-                    l += x0 + x1;
-                    pk[k2] = pack_bf16x2(x0, x1);
+                if constexpr (BS == 128) {             // scores of this 64-key chunk again
+                    tmem_ld32(tS + c64 * 64, sv);
+                    tmem_ld32(tS + c64 * 64 + 32, sv + 32);
+                    tmem_wait_ld();
                 }
+                uint32_t pk[32];
+                p_chunk(sv, mc, nomask, lim, c64 * 64, pk, l2);
                 tmem_st32(tS + c64 * 32, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&S.p_full[wg]);
-            if (!__all_sync(0xffffffffu, wait(&S.o_full[wg], ph, 39))) break;
+            const float l = l2.x + l2.y;
+            S.sc[wg][ph][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
+            mbar_arrive(&S.l_full[wg][ph]);
+            if (valid)
+                p.part_meta[(size_t)d.y * p.G + r] = make_float2((mc + __log2f(l)) * kLn2, (float)ve);
+        }
+    } else {
+        // ----------------------------------------------------------------- epilogue
+        // O * (2^-e / l) as fp16 per 64-column half: stage 16-byte pieces XOR-swizzled
+        // by row, then write 4 rows x 128 contiguous bytes per warp instruction.
+        const int quad = warp & 3;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t stg_base = smem_u32(S.stage[warp - 12]);
+        uint8_t* const part_o = static_cast<uint8_t*>(p.part_o);
+        int4 dn = ld_desc(0);
+        for (int i = 0; i < n; ++i) {
+            const int4 d = dn;
+            dn = ld_desc(i + 1);
+            const int slot = i & 1;
+            const uint32_t ph = (i >> 1) & 1;
+            if (!wait_w(&S.o_full[slot], ph, 39)) break;
+            if (!wait_w(&S.l_full[slot][ph], (i >> 2) & 1, 43)) break;
             tc_fence_after();
-            // epilogue pass 1: the row's max |O| picks the exponent e (0 unless
-            // max |O_B / l| > 2^14), so that O_B / l * 2^-e fits fp16
-            float om = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float x[64];
-                tmem_ld32(tO + h * 64, x);
-                tmem_ld32(tO + h * 64 + 32, x + 32);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 64; ++k) om = fmaxf(om, fabsf(x[k]));
-            }
-            const float inv_l = valid ? 1.f / l : 0.f;
-            const float omax = om * inv_l;
-            const int e = omax > 16384.f ? ilogbf(omax) - 14 : 0;
-            const float sc = ldexpf(inv_l, -e);
-            const size_t row0 = (size_t)d.y * p.G + (size_t)quad * 32;   // warp's first partial row
-            // pass 2, per 64-column half: scale, fp16, stage (16-byte pieces XOR-swizzled
-            // by row), then write 4 rows x 128 contiguous bytes per warp instruction
+            const float sc = S.sc[slot][ph][quad * 32 + lane];
+            const float2 sc2 = make_float2(sc, sc);
+            const int nrows = d.z & 255;
+            const size_t row0 = (size_t)d.y * p.G + (size_t)quad * 32;   // warp's first row
+            const uint32_t tO = tmem + slot * kSlot + BS + lane_off;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float x[64];
@@ -394,17 +454,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 if (h == 1) {                 // the slot's O has been read: release it
                     tc_fence_before();
-                    mbar_arrive(&S.o_free[wg]);
+                    mbar_arrive(&S.o_free[slot]);
                 }
 #pragma unroll
                 for (int pc = 0; pc < 8; ++pc) {
                     const float* y = x + pc * 8;
-                    uint4 v;
-                    v.x = pack_f16x2(y[0] * sc, y[1] * sc);
-                    v.y = pack_f16x2(y[2] * sc, y[3] * sc);
-                    v.z = pack_f16x2(y[4] * sc, y[5] * sc);
-                    v.w = pack_f16x2(y[6] * sc, y[7] * sc);
-                    st_shared_v4(stg_base + lane * 128 + ((pc ^ (lane & 7)) << 4), v);
+                    uint32_t u[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 z = mul2(make_float2(y[2 * q2], y[2 * q2 + 1]), sc2);
+                        u[q2] = pack_f16x2(z.x, z.y);
+                    }
+                    st_shared_v4(stg_base + lane * 128 + ((pc ^ (lane & 7)) << 4),
+                                 make_uint4(u[0], u[1], u[2], u[3]));
                 }
                 __syncwarp();
 #pragma unroll
@@ -417,8 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-            if (valid)
-                p.part_meta[row0 + lane] = make_float2((mc + __log2f(l)) * kLn2, (float)e);
         }
     }
 
@@ -430,7 +490,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// Per (KV head g, global block B): e = 0 unless max |V_B| > 2^14, then the exponent
+// that brings it under 2^15 (fp16 partials of O / l stay finite).  One block of 128
+// threads per (B, g), thread = column.
+__global__ void __launch_bounds__(128) k_vblock_exp(const __nv_bfloat16* v, const int32_t* cu,
+                                                    int nseq, int hkv, int bs,
+                                                    const int32_t* blkoff, const DevStatus* st,
+                                                    int32_t* vexp) {
+    __shared__ float wmax[4];
+    const int B = blockIdx.x, g = blockIdx.y;
+    const int nbtot = st->nblocks_total;
+    if (st->code != 0 || B >= nbtot) return;
+    const int s = upper_index(blkoff, nseq, B);
+    const int key0 = __ldg(cu + s) + (B - __ldg(blkoff + s)) * bs;
+    const int kend = min(key0 + bs, __ldg(cu + s + 1));
+    float m = 0.f;
+    for (int key = key0; key < kend; ++key)
+        m = fmaxf(m, fabsf(__bfloat162float(v[((size_t)key * hkv + g) * kHeadDim + threadIdx.x])));
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        m = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+        vexp[g * nbtot + B] = m > 16384.f ? min(ilogbf(m) - 14, 120) : 0;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, int32_t* vexp,
+                              cudaStream_t stream) {
+    if (p.T > 0 && nb_stride > 0)
+        k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), 128, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(v), p.cu, p.nseq, p.hkv, p.bs, p.blkoff, p.st, vexp);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              cudaStream_t stream) {

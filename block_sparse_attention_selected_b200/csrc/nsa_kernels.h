@@ -83,10 +83,14 @@ struct FwdPlan {
     void* part_o;            // fp16 [entries * G, 128]: O_B / l_B * 2^-e, row e * G + head
                              // offset for the sorted entry e (tile-contiguous)
     float2* part_meta;       // [entries * G]: (lse_B, e)
+    const int32_t* vexp;     // [hkv * NB]: exponent e of each (g, B) block's V
     DevStatus* st;
     int num_sms;
 };
 
+// vexp[g * NB + B] = 0, or the exponent that brings max |V_B| under 2^15
+cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, int32_t* vexp,
+                              cudaStream_t stream);
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              cudaStream_t stream);
 
