@@ -17,7 +17,7 @@ using namespace nsa;
 namespace {
 
 constexpr int kChunkTiles = 32;   // tiles per backward work unit
-constexpr int kWindowRows = 32768; // query rows per forward token window (tokens x group)
+constexpr int kWindowRows = 131072; // query rows per forward token window (tokens x group)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -95,7 +95,9 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.tile_desc = take(sizeof(int4) * (size_t)std::max<long long>(D.fwd_tiles_cap, 1));
     L.posmap = take(sizeof(int32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.vexp = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
-    const size_t rows = (size_t)D.T * D.hq * D.topk;
+    // forward: one 128-row slot per tile; backward: one row per (token, head, slot)
+    const size_t rows = std::max((size_t)D.T * D.hq * D.topk,
+                                 (size_t)std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows);
     L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
     if (bwd) {
@@ -149,6 +151,21 @@ bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs) {
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, 8 rows),
+// 128-byte swizzle: the epilogue's TMA stores of 8-row groups.
+bool make_part_map(CUtensorMap* map, void* base, long long rows) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    cuuint32_t box[2] = {64, 8};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -301,7 +318,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     wp.tiles_cap = D.fwd_tiles_cap;
     if ((s = cuda_status(launch_window_split(c.inv, wp, stream))) != NSA_OK) return s;
     int32_t* posmap = reinterpret_cast<int32_t*>(c.base + L.posmap);
-    if ((s = cuda_status(launch_posmap(c.inv, D.nent, posmap, stream))) != NSA_OK) return s;
+    if ((s = cuda_status(launch_posmap(c.inv, wp, posmap, stream))) != NSA_OK) return s;
     pm.add(invert_launches(D) + 5);
     pm.mark(1);
 
@@ -329,7 +346,10 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     int32_t* vexp = reinterpret_cast<int32_t*>(c.base + L.vexp);
     fp.vexp = vexp;
     if ((s = cuda_status(launch_vblock_exp(fp, v, D.nb_stride, vexp, stream))) != NSA_OK) return s;
-    if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, stream))) != NSA_OK) return s;
+    CUtensorMap omap;
+    if (!make_part_map(&omap, fp.part_o, (long long)std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows))
+        return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, &omap, stream))) != NSA_OK) return s;
     pm.add(2);
     pm.mark(2);
 

@@ -47,18 +47,23 @@ constexpr int kThreads = 512;
 constexpr int kLoaderThreads = 64;
 constexpr int kWgThreads = 128;
 constexpr int kNQ = 2;         // Q stages
-constexpr int kChunk = 2;      // consecutive tiles per scheduling chunk
+constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
+// Row-scale buffers: softmax(i + kNSc) may run once PV(i + kNSc - 2) is issued, which
+// waits for the epilogue of tile i + kNSc - 2 - NO; kNSc >= NO + 2 keeps it behind the
+// epilogue's read of sc[i % kNSc].
+constexpr int kNSc = 8;
 
 template <int BS, int NKV>
 struct alignas(1024) FwdSmem {
     uint8_t q[kNQ][2][kTileRows * 128];       // Q tile per stage: [64-column half][row]
     uint8_t kv[NKV][2][2][BS * 128];          // [stage][K, V][64-column half][key]
-    uint8_t stage[4][32 * 128];               // epilogue staging, 4 KB per epilogue warp
-    float sc[2][2][kTileRows];                // row scale 2^-e / l: [slot][tile parity][row]
+    uint8_t stage[4][2][32 * 128];            // epilogue staging: [warp][64-column half]
+    float sc[kNSc][kTileRows];                // row scale 2^-e / l of tile i in sc[i % kNSc]
     uint64_t q_full[kNQ], q_empty[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
-    uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-    uint64_t l_full[2][2];                    // sc[slot][parity] written
+    uint64_t s_full[2], p_full[2];
+    uint64_t o_full[3], o_free[3];            // O accumulator buffers (BS == 64: 3, else 2)
+    uint64_t l_full[kNSc];                    // sc[i % kNSc] written
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -92,7 +97,7 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 template <int BS, int NKV>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tiles(const FwdPlan p, const __grid_constant__ CUtensorMap kmap,
-                const __grid_constant__ CUtensorMap vmap) {
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap) {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<BS, NKV>& S = *reinterpret_cast<FwdSmem<BS, NKV>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -100,10 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     DevStatus* st = p.st;
-    // TMEM columns of slot s: S (and P, bf16, in its first BS/2 columns) at
-    // s * kSlot, the O accumulator at s * kSlot + BS.
-    constexpr int kSlot = BS + kHeadDim;
-    static_assert(2 * kSlot <= 512, "TMEM budget");
+    // TMEM columns: S of slot s (and P, bf16, in its first BS/2 columns) at s * BS;
+    // O accumulator buffer b at 2 * BS + b * 128.
+    constexpr int NO = BS == 64 ? 3 : 2;
+    constexpr int kColO = 2 * BS;
+    static_assert(kColO + NO * kHeadDim <= 512, "TMEM budget");
 
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
@@ -115,11 +121,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.p_full[i], kWgThreads);
+        }
+        for (int i = 0; i < NO; ++i) {
             mbar_init(&S.o_full[i], 1);
             mbar_init(&S.o_free[i], kWgThreads);
-            mbar_init(&S.l_full[i][0], kWgThreads);
-            mbar_init(&S.l_full[i][1], kWgThreads);
         }
+        for (int i = 0; i < kNSc; ++i) mbar_init(&S.l_full[i], kWgThreads);
         for (int i = 0; i < NKV; ++i) {
             mbar_init(&S.kv_full[i], 1);
             mbar_init(&S.kv_empty[i], 1);
@@ -276,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kvs_of[slot] = cur;
                 if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
                 tc_fence_after();
-                const uint32_t tS = tmem + slot * kSlot;
+                const uint32_t tS = tmem + slot * BS;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (uint32_t)(ks & 3) * 32u;
@@ -289,14 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&S.q_empty[stg]);
                 return true;
             };
-            // O(i) = P(i) V into slot i & 1 once the softmax wrote P(i) and the epilogue
-            // of tile i - 2 has read the slot's previous O.
+            // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
+            // epilogue of tile i - NO has read the buffer's previous O.
             auto issue_pv = [&](int i, bool release_kv) -> bool {
-                const int slot = i & 1;
+                const int slot = i & 1, ob = i % NO;
                 if (!wait(&S.p_full[slot], (i >> 1) & 1, 36)) return false;
-                if (!wait(&S.o_free[slot], ((i >> 1) & 1) ^ 1, 34)) return false;
+                if (!wait(&S.o_free[ob], ((i / NO) & 1) ^ 1, 34)) return false;
                 tc_fence_after();
-                const uint32_t tS = tmem + slot * kSlot, tO = tS + BS;
+                const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
                 const int kvs = kvs_of[slot];
 #pragma unroll
                 for (int ks = 0; ks < BS / 16; ++ks) {
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         smem_u32(S.kv[kvs][1][0]) + (uint32_t)ks * 2048u, BS * 128, 1024);
                     mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b, kIdescO, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(&S.o_full[slot]);
+                mma_commit(&S.o_full[ob]);
                 if (release_kv) mma_commit(&S.kv_empty[kvs]);
                 return true;
             };
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wg = (warp - 4) >> 2;                  // 0: even tiles, 1: odd tiles
         const int quad = warp & 3;                       // TMEM lanes 32*quad ..
         const int r = quad * 32 + lane;
-        const uint32_t tS = tmem + wg * kSlot + ((uint32_t)(quad * 32) << 16);
+        const uint32_t tS = tmem + wg * BS + ((uint32_t)(quad * 32) << 16);
         const float c = p.scale_log2;
         const float kLn2 = 0.69314718055994531f;
         auto ld_row = [&](const int4& d, int i) -> uint32_t {
@@ -373,14 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pk[k2] = pack_bf16x2(x.x, x.y);
             }
         };
-        int4 dn = ld_desc(wg);
+        // descriptors two tiles ahead, entries and exponents one tile ahead, so that no
+        // dependent global load sits on the path from S(i) to P(i)
+        int4 dn = ld_desc(wg), dnn = ld_desc(wg + 2);
         uint32_t en = ld_row(dn, wg);
         int vn = ld_vexp(dn, wg);
         for (int i = wg; i < n; i += 2) {
             const int4 d = dn;
             const uint32_t ent = en;
             const int ve = vn;
-            dn = ld_desc(i + 2);
+            dn = dnn;
+            dnn = ld_desc(i + 4);
             en = ld_row(dn, i + 2);
             vn = ld_vexp(dn, i + 2);
             const uint32_t ph = (i >> 1) & 1;
@@ -419,43 +429,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&S.p_full[wg]);
             const float l = l2.x + l2.y;
-            S.sc[wg][ph][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
-            mbar_arrive(&S.l_full[wg][ph]);
+            S.sc[i % kNSc][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
+            mbar_arrive(&S.l_full[i % kNSc]);
             if (valid)
-                p.part_meta[(size_t)d.y * p.G + r] = make_float2((mc + __log2f(l)) * kLn2, (float)ve);
+                p.part_meta[(size_t)tile_of(i) * kTileRows + r] =
+                    make_float2((mc + __log2f(l)) * kLn2, (float)ve);
         }
     } else {
         // ----------------------------------------------------------------- epilogue
-        // O * (2^-e / l) as fp16 per 64-column half: stage 16-byte pieces XOR-swizzled
-        // by row, then write 4 rows x 128 contiguous bytes per warp instruction.
+        // O * (2^-e / l) as fp16, per 64-column half: each thread writes its row into
+        // the warp's staging buffer in the 128-byte-swizzled layout, then one lane
+        // stores the warp's valid rows, rounded up to 8, by TMA into the tile's own
+        // 128-row partial slot (rows past the list only land in the slot's padding).
         const int quad = warp & 3;
+        const int ew = warp - 12;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t stg_base = smem_u32(S.stage[warp - 12]);
-        uint8_t* const part_o = static_cast<uint8_t*>(p.part_o);
         int4 dn = ld_desc(0);
         for (int i = 0; i < n; ++i) {
             const int4 d = dn;
             dn = ld_desc(i + 1);
-            const int slot = i & 1;
-            const uint32_t ph = (i >> 1) & 1;
-            if (!wait_w(&S.o_full[slot], ph, 39)) break;
-            if (!wait_w(&S.l_full[slot][ph], (i >> 2) & 1, 43)) break;
+            const int ob = i % NO;
+            if (!wait_w(&S.o_full[ob], (i / NO) & 1, 39)) break;
+            if (!wait_w(&S.l_full[i % kNSc], (i / kNSc) & 1, 43)) break;
             tc_fence_after();
-            const float sc = S.sc[slot][ph][quad * 32 + lane];
+            const float sc = S.sc[i % kNSc][quad * 32 + lane];
             const float2 sc2 = make_float2(sc, sc);
-            const int nrows = d.z & 255;
-            const size_t row0 = (size_t)d.y * p.G + (size_t)quad * 32;   // warp's first row
-            const uint32_t tO = tmem + slot * kSlot + BS + lane_off;
+            const int valid = min(32, max(0, (d.z & 255) - quad * 32));
+            const int nbox = (valid + 7) >> 3;
+            const int prow0 = tile_of(i) * kTileRows + quad * 32;   // warp's first row
+            const uint32_t tO = tmem + kColO + ob * kHeadDim + lane_off;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float x[64];
                 tmem_ld32(tO + h * 64, x);
                 tmem_ld32(tO + h * 64 + 32, x + 32);
                 tmem_wait_ld();
-                if (h == 1) {                 // the slot's O has been read: release it
+                if (h == 1) {                 // the buffer's O has been read: release it
                     tc_fence_before();
-                    mbar_arrive(&S.o_free[slot]);
+                    mbar_arrive(&S.o_free[ob]);
                 }
+                // the TMA store that last read this staging half (tile i - 1) is done
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+                const uint32_t sb = smem_u32(S.stage[ew][h]);
 #pragma unroll
                 for (int pc = 0; pc < 8; ++pc) {
                     const float* y = x + pc * 8;
@@ -465,21 +481,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float2 z = mul2(make_float2(y[2 * q2], y[2 * q2 + 1]), sc2);
                         u[q2] = pack_f16x2(z.x, z.y);
                     }
-                    st_shared_v4(stg_base + lane * 128 + ((pc ^ (lane & 7)) << 4),
+                    st_shared_v4(sb + lane * 128 + ((pc ^ (lane & 7)) << 4),
                                  make_uint4(u[0], u[1], u[2], u[3]));
                 }
+                fence_async_smem();
                 __syncwarp();
-#pragma unroll
-                for (int it = 0; it < 8; ++it) {
-                    const int rr = it * 4 + (lane >> 3), pc = lane & 7;
-                    const uint4 v = ld_shared_v4(stg_base + rr * 128 + ((pc ^ (rr & 7)) << 4));
-                    if (quad * 32 + rr < nrows)
-                        *reinterpret_cast<uint4*>(part_o + (row0 + rr) * (kHeadDim * 2) + h * 128 +
-                                                  pc * 16) = v;
+                if (lane == 0 && nbox > 0) {
+                    for (int b = 0; b < nbox; ++b)
+                        tma_store_2d(&omap, S.stage[ew][h] + b * 1024, h * 64, prow0 + b * 8);
+                    bulk_commit();
                 }
-                __syncwarp();
             }
         }
+        if (lane == 0) bulk_wait<0>();   // every store performed before the CTA exits
     }
 
     // ---- teardown: every role has left its loop (all waits are bounded) and the MMA
@@ -527,17 +541,17 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
 }
 
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
-                             cudaStream_t stream) {
+                             const CUtensorMap* omap, cudaStream_t stream) {
     if (p.bs == 64) {
         constexpr size_t smem = fwd_smem_bytes<64, 3>();
         cudaFuncSetAttribute(k_fwd_tiles<64, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        k_fwd_tiles<64, 3><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+        k_fwd_tiles<64, 3><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, *omap);
     } else {
         constexpr size_t smem = fwd_smem_bytes<128, 1>();
         cudaFuncSetAttribute(k_fwd_tiles<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        k_fwd_tiles<128, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+        k_fwd_tiles<128, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, *omap);
     }
     return cudaGetLastError();
 }

@@ -388,18 +388,19 @@ __global__ void k_unit_desc(const DevStatus* st, const int32_t* chunk_off, const
     ubucket[u] = bucket;
 }
 
-// 10. Position map: for every sorted position pos of a valid entry (token t, KV head
-//     g, slot j), posmap[(t * hkv + g) * topk + j] = pos.  The forward's partial
-//     results are stored in sorted order; the merge finds them through this map.
-__global__ void k_posmap(const uint32_t* keys, const uint32_t* vals, const DevStatus* st, int hkv,
-                         int topk, int32_t* posmap) {
-    const int pos = blockIdx.x * blockDim.x + threadIdx.x;
-    // malformed cu_seqlens (recorded by k_seq_blocks) leave the keys inconsistent
-    if (st->code != 0 || pos >= st->nentries) return;
-    const uint32_t g = keys[pos] / (uint32_t)st->nblocks_total;
-    const uint32_t v = vals[pos];
-    if (g >= (uint32_t)hkv || (int)(v & 63u) >= topk) return;
-    posmap[((size_t)(v >> 6) * hkv + g) * topk + (v & 63u)] = pos;
+// 10. Position map from the forward tiles: the k-th token of tile tau, entry
+//     (t, g, j), gets posmap[(t * hkv + g) * topk + j] = tau * tpt + k; its partial
+//     rows are posmap * G + head offset, inside the tile's own 128-row slot.
+__global__ void k_posmap_tiles(const int4* desc, const uint32_t* entries, const DevStatus* st,
+                               int hkv, int topk, int tpt, int32_t* posmap) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int tile = (int)(idx / tpt), k = (int)(idx % tpt);
+    if (st->code != 0 || tile >= st->ntiles_fwd) return;
+    const int4 d = desc[tile];
+    const int G = kTileRows / tpt;
+    if (k >= (d.z & 255) / G) return;
+    const uint32_t v = entries[d.y + k];
+    posmap[((size_t)(v >> 6) * hkv + (d.z >> 8)) * topk + (v & 63u)] = tile * tpt + k;
 }
 
 // Range / duplicate check of block_idx (one thread per (token, KV head) row).
@@ -476,11 +477,12 @@ cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaSt
     return cudaGetLastError();
 }
 
-cudaError_t launch_posmap(const InvertPlan& p, long long nent, int32_t* posmap,
+cudaError_t launch_posmap(const InvertPlan& p, const WindowPlan& w, int32_t* posmap,
                           cudaStream_t stream) {
-    if (nent > 0)
-        k_posmap<<<(unsigned)((nent + 255) / 256), 256, 0, stream>>>(
-            p.keys[p.final_buf], p.vals[p.final_buf], p.st, p.hkv, p.topk, posmap);
+    const long long n = w.tiles_cap * p.tokens_per_tile;
+    if (n > 0)
+        k_posmap_tiles<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+            w.tile_desc, p.vals[p.final_buf], p.st, p.hkv, p.topk, p.tokens_per_tile, posmap);
     return cudaGetLastError();
 }
 

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
     const int h = (int)(row - (long long)t * p.hq);
     const int g = h / p.G;
     const int hoff = h - g * p.G;
-    const unsigned nrows_part = (unsigned)p.st->nentries * (unsigned)p.G;
+    const unsigned nrows_part = (unsigned)p.st->ntiles_fwd * (unsigned)kTileRows;
     const int s = seq_of_token(p.cu, p.nseq, t);
     const int qb = (t - __ldg(p.cu + s)) / p.bs;
     const size_t base = ((size_t)t * p.hkv + g) * p.topk;

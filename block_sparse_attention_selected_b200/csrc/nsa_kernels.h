@@ -57,9 +57,9 @@ struct WindowPlan {
 // Runs the inversion on `stream`; returns the first launch error.
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream);
 cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaStream_t stream);
-// posmap[(t * hkv + g) * topk + j] = position of entry (t, g, j) in the sorted list
-// (written for valid entries only).
-cudaError_t launch_posmap(const InvertPlan& p, long long nent, int32_t* posmap,
+// posmap[(t * hkv + g) * topk + j] = tile * (128 / G) + (position of the entry's token
+// in its forward tile) for every valid entry; the partial rows are posmap * G + head.
+cudaError_t launch_posmap(const InvertPlan& p, const WindowPlan& w, int32_t* posmap,
                           cudaStream_t stream);
 cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
                              cudaStream_t stream);
@@ -80,9 +80,8 @@ struct FwdPlan {
     const int32_t* wtile_off;
     const int32_t* row_off;
     const int4* tile_desc;
-    void* part_o;            // fp16 [entries * G, 128]: O_B / l_B * 2^-e, row e * G + head
-                             // offset for the sorted entry e (tile-contiguous)
-    float2* part_meta;       // [entries * G]: (lse_B, e)
+    void* part_o;            // fp16 [tiles * 128, 128]: O_B / l_B * 2^-e, row tile * 128 + r
+    float2* part_meta;       // [tiles * 128]: (lse_B, e)
     const int32_t* vexp;     // [hkv * NB]: exponent e of each (g, B) block's V
     DevStatus* st;
     int num_sms;
@@ -91,8 +90,9 @@ struct FwdPlan {
 // vexp[g * NB + B] = 0, or the exponent that brings max |V_B| under 2^15
 cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, int32_t* vexp,
                               cudaStream_t stream);
+// omap: tensor map over part_o (fp16 [tiles_cap * 128, 128], box 64 x 8, 128B swizzle)
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
-                             cudaStream_t stream);
+                             const CUtensorMap* omap, cudaStream_t stream);
 
 struct MergePlan {
     const int32_t* cu;
