@@ -154,14 +154,14 @@ bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs) {
     return r == CUDA_SUCCESS;
 }
 
-// Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, 8 rows),
-// 128-byte swizzle: the epilogue's TMA stores of 8-row groups.
-bool make_part_map(CUtensorMap* map, void* base, long long rows) {
+// Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, box_rows),
+// 128-byte swizzle: the epilogue's TMA stores of 8-row groups and of whole warps.
+bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    cuuint32_t box[2] = {64, 8};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -346,10 +346,11 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     int32_t* vexp = reinterpret_cast<int32_t*>(c.base + L.vexp);
     fp.vexp = vexp;
     if ((s = cuda_status(launch_vblock_exp(fp, v, D.nb_stride, vexp, stream))) != NSA_OK) return s;
-    CUtensorMap omap;
-    if (!make_part_map(&omap, fp.part_o, (long long)std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows))
+    CUtensorMap omap[2];
+    const long long prow = std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows;
+    if (!make_part_map(&omap[0], fp.part_o, prow, 8) || !make_part_map(&omap[1], fp.part_o, prow, 32))
         return NSA_ERR_CUDA;
-    if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, &omap, stream))) != NSA_OK) return s;
+    if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, omap, stream))) != NSA_OK) return s;
     pm.add(2);
     pm.mark(2);
 

@@ -43,8 +43,15 @@
 namespace nsa {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kLoaderThreads = 64;
+// Warp roles: Q loaders 0 .. kLoaderWarps-1 (2 or 4), softmax warpgroups 4-7 and 8-11,
+// epilogue warpgroup 12-15 (warp % 4 = TMEM lane quadrant), then the TMA producer and
+// the MMA issuer (warps 2, 3 with two loaders; 16, 17 with four).
+constexpr int kLoaderWarps = 2;
+constexpr int kTmaWarp = kLoaderWarps == 2 ? 2 : 16;
+constexpr int kMmaWarp = kTmaWarp + 1;
+constexpr int kThreads = (kLoaderWarps == 2 ? 16 : 18) * 32;
+constexpr int kLoaderThreads = kLoaderWarps * 32;
+constexpr int kRowsPerLoader = kTileRows / kLoaderWarps;   // 64 or 32
 constexpr int kWgThreads = 128;
 constexpr int kNQ = 2;         // Q stages
 constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
@@ -97,7 +104,8 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 template <int BS, int NKV>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tiles(const FwdPlan p, const __grid_constant__ CUtensorMap kmap,
-                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap) {
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap8,
+                const __grid_constant__ CUtensorMap omap32) {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem<BS, NKV>& S = *reinterpret_cast<FwdSmem<BS, NKV>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -171,18 +179,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         return __all_sync(0xffffffffu, wait(bar, parity, where));
     };
 
-    if (warp < 2) {
+    if (warp < kLoaderWarps) {
         // ---------------------------------------------------------------- Q loaders
-        // Warp w fills tile rows [64w, 64w + 64).  Lane l computes the source address of
-        // rows 64w + l and 64w + 32 + l (token from the index entry, head from the row);
-        // in copy step k the warp moves rows 64w + 2k and 64w + 2k + 1, lane l taking the
-        // 16-byte chunk l % 16 of row 64w + 2k + l / 16 (a 512-byte coalesced read).
+        // Warp w fills the R = kRowsPerLoader tile rows [Rw, Rw + R).  Lane l computes the
+        // source address of row Rw + l (and Rw + 32 + l when R = 64) from the index entry
+        // (token) and the row (head); in copy step k the warp moves rows Rw + 2k and
+        // Rw + 2k + 1, lane l taking the 16-byte chunk l % 16 of row Rw + 2k + l / 16 (a
+        // 512-byte coalesced read).
         // The copies of tile i are published one tile later (wait for the older
         // cp.async group, fence for the tensor core's async proxy, arrive on q_full),
         // so two tiles' gathers are in flight.
         const int w = warp;
         const uint8_t* qb = static_cast<const uint8_t*>(p.q);
-        const int rA = 64 * w + lane, rB = rA + 32;
+        const int rA = kRowsPerLoader * w + lane, rB = rA + 32;
         auto ld_ent = [&](const int4& d, int r) -> uint32_t {
             return r < (d.z & 255) ? __ldg(p.entries + d.y + r / p.G) : 0u;
         };
@@ -192,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (kHeadDim * 2));
         };
         int4 d0 = ld_desc(0), d1 = ld_desc(1);
-        uint32_t ea = ld_ent(d0, rA), eb = ld_ent(d0, rB);
+        uint32_t ea = ld_ent(d0, rA), eb = kRowsPerLoader == 64 ? ld_ent(d0, rB) : 0u;
         int published = 0, issued = 0;
         const int c = lane & 15;
         const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
@@ -203,17 +212,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             d0 = d1;
             d1 = ld_desc(i + 2);
             ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
-            eb = ld_ent(d0, rB);
+            eb = kRowsPerLoader == 64 ? ld_ent(d0, rB) : 0u;
             const int nrows = d.z & 255;
             const int stg = i % kNQ;
             if (!wait_w(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
             const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
 #pragma unroll 4
-            for (int k = 0; k < 32; ++k) {
+            for (int k = 0; k < kRowsPerLoader / 2; ++k) {
                 const int rw = 2 * k + (lane >> 4);          // row within the warp's 64
                 const unsigned long long a =
                     __shfl_sync(0xffffffffu, k < 16 ? addrA : addrB, rw & 31) + c * 16;
-                const int row = 64 * w + rw;
+                const int row = kRowsPerLoader * w + rw;
                 if (row < nrows)
                     cp_async_16(q0 + sw128_offset(row, c & 7), reinterpret_cast<const void*>(a));
             }
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();
             mbar_arrive(&S.q_full[(n - 1) % kNQ]);
         }
-    } else if (warp == 2) {
+    } else if (warp == kTmaWarp) {
         // ------------------------------------------------------------- K/V producer
         if (lane == 0) {
             prefetch_tmap(&kmap);
@@ -262,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int s = 0; s < NKV; ++s)
                     if (loaded[s]) mbar_wait(&S.kv_full[s], last_parity[s], st, 40);
         }
-    } else if (warp == 3) {
+    } else if (warp == kMmaWarp) {
         // -------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&S.drain);
             mbar_wait(&S.drain, 0, st, 41);
         }
-    } else if (warp < 12) {
+    } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------------ softmax
         // Thread = tile row = TMEM lane.  Non-diagonal tiles (every row sees the whole
         // block) skip the causal mask; the test is warp-uniform.
@@ -363,9 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return fmaxf(a, b);
         };
-        // P = 2^(c s - c m) of 64 scores as packed bf16 pairs; l accumulates sum P
-        auto p_chunk = [&](const float* v, float mc, bool nomask, int lim, int base,
-                           uint32_t* pk, float2& l2) {
+        // v[k] <- 2^(c v[k] - c m) over 64 scores (0 past the causal limit); l += sum
+        auto exp_chunk = [&](float* v, float mc, bool nomask, int lim, int base, float2& l2) {
             const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
 #pragma unroll
             for (int k2 = 0; k2 < 32; ++k2) {
@@ -377,6 +385,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (base + 2 * k2 + 1 > lim) x.y = 0.f;
                 }
                 l2 = add2(l2, x);
+                v[2 * k2] = x.x;
+                v[2 * k2 + 1] = x.y;
+            }
+        };
+        // 64 values times s as packed bf16 pairs
+        auto pack_chunk = [&](const float* v, float s, uint32_t* pk) {
+            const float2 s2 = make_float2(s, s);
+#pragma unroll
+            for (int k2 = 0; k2 < 32; ++k2) {
+                const float2 x = mul2(make_float2(v[2 * k2], v[2 * k2 + 1]), s2);
                 pk[k2] = pack_bf16x2(x.x, x.y);
             }
         };
@@ -414,23 +432,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!valid) mx = 0.f;                      // every valid row has lim >= 0
             const float mc = mx * c;
             float2 l2 = make_float2(0.f, 0.f);
+            float l;
+            uint32_t pk[32];
+            if constexpr (BS == 64) {
+                // P pre-scaled by 2^-e / l: the epilogue only converts O
+                exp_chunk(sv, mc, nomask, lim, 0, l2);
+                l = l2.x + l2.y;
+                pack_chunk(sv, valid ? ldexpf(1.f / l, -ve) : 0.f, pk);
+                tmem_st32(tS, pk);
+            } else {
 #pragma unroll
-            for (int c64 = 0; c64 < BS / 64; ++c64) {
-                if constexpr (BS == 128) {             // scores of this 64-key chunk again
+                for (int c64 = 0; c64 < 2; ++c64) {    // scores of this 64-key chunk again
                     tmem_ld32(tS + c64 * 64, sv);
                     tmem_ld32(tS + c64 * 64 + 32, sv + 32);
                     tmem_wait_ld();
+                    exp_chunk(sv, mc, nomask, lim, c64 * 64, l2);
+                    pack_chunk(sv, 1.f, pk);
+                    tmem_st32(tS + c64 * 32, pk);
                 }
-                uint32_t pk[32];
-                p_chunk(sv, mc, nomask, lim, c64 * 64, pk, l2);
-                tmem_st32(tS + c64 * 32, pk);
+                l = l2.x + l2.y;
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&S.p_full[wg]);
-            const float l = l2.x + l2.y;
-            S.sc[i % kNSc][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
-            mbar_arrive(&S.l_full[i % kNSc]);
+            if constexpr (BS != 64) {                  // the epilogue applies 2^-e / l
+                S.sc[i % kNSc][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
+                mbar_arrive(&S.l_full[i % kNSc]);
+            }
             if (valid)
                 p.part_meta[(size_t)tile_of(i) * kTileRows + r] =
                     make_float2((mc + __log2f(l)) * kLn2, (float)ve);
@@ -450,9 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             dn = ld_desc(i + 1);
             const int ob = i % NO;
             if (!wait_w(&S.o_full[ob], (i / NO) & 1, 39)) break;
-            if (!wait_w(&S.l_full[i % kNSc], (i / kNSc) & 1, 43)) break;
+            float sc = 1.f;
+            if constexpr (BS != 64) {
+                if (!wait_w(&S.l_full[i % kNSc], (i / kNSc) & 1, 43)) break;
+                sc = S.sc[i % kNSc][quad * 32 + lane];
+            }
             tc_fence_after();
-            const float sc = S.sc[i % kNSc][quad * 32 + lane];
             const float2 sc2 = make_float2(sc, sc);
             const int valid = min(32, max(0, (d.z & 255) - quad * 32));
             const int nbox = (valid + 7) >> 3;
@@ -478,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t u[4];
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
-                        const float2 z = mul2(make_float2(y[2 * q2], y[2 * q2 + 1]), sc2);
+                        float2 z = make_float2(y[2 * q2], y[2 * q2 + 1]);
+                        if constexpr (BS != 64) z = mul2(z, sc2);
                         u[q2] = pack_f16x2(z.x, z.y);
                     }
                     st_shared_v4(sb + lane * 128 + ((pc ^ (lane & 7)) << 4),
@@ -487,8 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0 && nbox > 0) {
-                    for (int b = 0; b < nbox; ++b)
-                        tma_store_2d(&omap, S.stage[ew][h] + b * 1024, h * 64, prow0 + b * 8);
+                    if (nbox == 4) {
+                        tma_store_2d(&omap32, S.stage[ew][h], h * 64, prow0);
+                    } else {
+                        for (int b = 0; b < nbox; ++b)
+                            tma_store_2d(&omap8, S.stage[ew][h] + b * 1024, h * 64, prow0 + b * 8);
+                    }
                     bulk_commit();
                 }
             }
@@ -546,12 +582,12 @@ cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CU
         constexpr size_t smem = fwd_smem_bytes<64, 3>();
         cudaFuncSetAttribute(k_fwd_tiles<64, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        k_fwd_tiles<64, 3><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, *omap);
+        k_fwd_tiles<64, 3><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
     } else {
         constexpr size_t smem = fwd_smem_bytes<128, 1>();
         cudaFuncSetAttribute(k_fwd_tiles<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        k_fwd_tiles<128, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, *omap);
+        k_fwd_tiles<128, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
     }
     return cudaGetLastError();
 }
