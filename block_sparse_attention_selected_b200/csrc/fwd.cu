@@ -53,7 +53,7 @@ constexpr int kThreads = (kLoaderWarps == 2 ? 16 : 18) * 32;
 constexpr int kLoaderThreads = kLoaderWarps * 32;
 constexpr int kRowsPerLoader = kTileRows / kLoaderWarps;   // 64 or 32
 constexpr int kWgThreads = 128;
-constexpr int kNQ = 2;         // Q stages
+constexpr int kNQ = 2;         // Q stages (= S slots: S(i) completing frees stage i % 2)
 constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
 // Row-scale buffers: softmax(i + kNSc) may run once PV(i + kNSc - 2) is issued, which
 // waits for the epilogue of tile i + kNSc - 2 - NO; kNSc >= NO + 2 keeps it behind the
@@ -66,7 +66,7 @@ struct alignas(1024) FwdSmem {
     uint8_t kv[NKV][2][2][BS * 128];          // [stage][K, V][64-column half][key]
     uint8_t stage[4][2][32 * 128];            // epilogue staging: [warp][64-column half]
     float sc[kNSc][kTileRows];                // row scale 2^-e / l of tile i in sc[i % kNSc]
-    uint64_t q_full[kNQ], q_empty[kNQ];
+    uint64_t q_full[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
     uint64_t s_full[2], p_full[2];
     uint64_t o_full[3], o_free[3];            // O accumulator buffers (BS == 64: 3, else 2)
@@ -122,10 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
         S.ntiles = *reinterpret_cast<volatile int*>(&st->ntiles_fwd);
-        for (int i = 0; i < kNQ; ++i) {
-            mbar_init(&S.q_full[i], kLoaderThreads);
-            mbar_init(&S.q_empty[i], 1);
-        }
+        for (int i = 0; i < kNQ; ++i) mbar_init(&S.q_full[i], kLoaderThreads);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.p_full[i], kWgThreads);
@@ -215,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             eb = kRowsPerLoader == 64 ? ld_ent(d0, rB) : 0u;
             const int nrows = d.z & 255;
             const int stg = i % kNQ;
-            if (!wait_w(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
+            // stage i % 2 is free once S(i - 2), which read it, has completed
+            if (!wait_w(&S.s_full[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
             const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
 #pragma unroll 4
             for (int k = 0; k < kRowsPerLoader / 2; ++k) {
@@ -281,6 +279,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
             // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
             // run in issue order.
+            // Shared-memory descriptors are computed once; an MMA step only adds the
+            // byte offset / 16 to the start-address field (addresses stay < 2^18 bytes,
+            // so the 14-bit field never carries).  This keeps the issuing thread's
+            // instruction count per MMA small: it shares its SMSP with busy warps.
+            constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+            constexpr uint64_t kKvStage = sizeof(S.kv[0]) >> 4, kKvHalf = sizeof(S.kv[0][0][0]) >> 4;
+            const uint64_t q_desc0 = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
+            const uint64_t k_desc0 = smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
+            const uint64_t v_desc0 = smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
+            // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
+            // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
+            // run in issue order.  s_full also tells the loaders that the Q stage (i % 2)
+            // is free again.
             auto issue_s = [&](int i, int bucket) -> bool {
                 if (bucket != prev_bucket) {
                     cur = kv_uses % NKV;
@@ -293,16 +304,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
                 tc_fence_after();
                 const uint32_t tS = tmem + slot * BS;
+                const uint64_t a0 = q_desc0 + (uint64_t)stg * kQStage;
+                const uint64_t b0 = k_desc0 + (uint64_t)cur * kKvStage;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (uint32_t)(ks & 3) * 32u;
-                    const uint64_t a = smem_desc_sw128(smem_u32(S.q[stg][ks >> 2]) + off, 16, 1024);
-                    const uint64_t b =
-                        smem_desc_sw128(smem_u32(S.kv[cur][0][ks >> 2]) + off, 16, 1024);
-                    mma_bf16_ss(tS, a, b, kIdescS, ks > 0 ? 1u : 0u);
+                    const uint64_t off = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                    const uint64_t offk = (uint64_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
+                    mma_bf16_ss(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(&S.s_full[slot]);
-                mma_commit(&S.q_empty[stg]);
                 return true;
             };
             // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
@@ -314,12 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
                 const int kvs = kvs_of[slot];
+                const uint64_t b0 = v_desc0 + (uint64_t)kvs * kKvStage;
 #pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks) {
-                    const uint64_t b = smem_desc_sw128(
-                        smem_u32(S.kv[kvs][1][0]) + (uint32_t)ks * 2048u, BS * 128, 1024);
-                    mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b, kIdescO, ks > 0 ? 1u : 0u);
-                }
+                for (int ks = 0; ks < BS / 16; ++ks)    // 16 keys = 2048 bytes per step
+                    mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b0 + (uint64_t)ks * 128u, kIdescO,
+                                ks > 0 ? 1u : 0u);
                 mma_commit(&S.o_full[ob]);
                 if (release_kv) mma_commit(&S.kv_empty[kvs]);
                 return true;
@@ -354,36 +363,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             return (i < n && r < (d.z & 255)) ? __ldg(p.entries + d.y + r / p.G) : 0u;
         };
         auto ld_vexp = [&](const int4& d, int i) -> int { return i < n ? __ldg(p.vexp + d.w) : 0; };
-        // max over 64 scores; masked: only keys base + k <= lim
-        auto row_max64 = [&](const float* v, bool nomask, int lim, int base) -> float {
+        // scores of keys past the causal limit -> -inf (diagonal tiles only)
+        auto mask64 = [&](float* v, int lim, int base) {
+#pragma unroll
+            for (int k = 0; k < 64; ++k)
+                if (base + k > lim) v[k] = -CUDART_INF_F;
+        };
+        auto row_max64 = [&](const float* v) -> float {
             float a = -CUDART_INF_F, b = -CUDART_INF_F;
-            if (nomask) {
 #pragma unroll
-                for (int k = 0; k < 64; k += 4) {
-                    a = fmax3(a, v[k], v[k + 1]);
-                    b = fmax3(b, v[k + 2], v[k + 3]);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 64; k += 2) {
-                    a = fmaxf(a, base + k <= lim ? v[k] : -CUDART_INF_F);
-                    b = fmaxf(b, base + k + 1 <= lim ? v[k + 1] : -CUDART_INF_F);
-                }
+            for (int k = 0; k < 64; k += 4) {
+                a = fmax3(a, v[k], v[k + 1]);
+                b = fmax3(b, v[k + 2], v[k + 3]);
             }
             return fmaxf(a, b);
         };
-        // v[k] <- 2^(c v[k] - c m) over 64 scores (0 past the causal limit); l += sum
-        auto exp_chunk = [&](float* v, float mc, bool nomask, int lim, int base, float2& l2) {
+        // v[k] <- 2^(c v[k] - c m) over 64 scores (a masked -inf gives 0); l += sum
+        auto exp_chunk = [&](float* v, float mc, float2& l2) {
             const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
 #pragma unroll
             for (int k2 = 0; k2 < 32; ++k2) {
                 float2 x = fma2(make_float2(v[2 * k2], v[2 * k2 + 1]), c2, nmc2);
                 x.x = ex2_approx(x.x);
                 x.y = ex2_approx(x.y);
-                if (!nomask) {
-                    if (base + 2 * k2 > lim) x.x = 0.f;
-                    if (base + 2 * k2 + 1 > lim) x.y = 0.f;
-                }
                 l2 = add2(l2, x);
                 v[2 * k2] = x.x;
                 v[2 * k2 + 1] = x.y;
@@ -422,12 +424,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tS, sv);
             tmem_ld32(tS + 32, sv + 32);
             tmem_wait_ld();
-            float mx = row_max64(sv, nomask, lim, 0);
+            if (!nomask) mask64(sv, lim, 0);
+            float mx = row_max64(sv);
             if constexpr (BS == 128) {
                 tmem_ld32(tS + 64, sv);
                 tmem_ld32(tS + 96, sv + 32);
                 tmem_wait_ld();
-                mx = fmaxf(mx, row_max64(sv, nomask, lim, 64));
+                if (!nomask) mask64(sv, lim, 64);
+                mx = fmaxf(mx, row_max64(sv));
             }
             if (!valid) mx = 0.f;                      // every valid row has lim >= 0
             const float mc = mx * c;
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[32];
             if constexpr (BS == 64) {
                 // P pre-scaled by 2^-e / l: the epilogue only converts O
-                exp_chunk(sv, mc, nomask, lim, 0, l2);
+                exp_chunk(sv, mc, l2);
                 l = l2.x + l2.y;
                 pack_chunk(sv, valid ? ldexpf(1.f / l, -ve) : 0.f, pk);
                 tmem_st32(tS, pk);
@@ -446,7 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(tS + c64 * 64, sv);
                     tmem_ld32(tS + c64 * 64 + 32, sv + 32);
                     tmem_wait_ld();
-                    exp_chunk(sv, mc, nomask, lim, c64 * 64, l2);
+                    if (!nomask) mask64(sv, lim, c64 * 64);
+                    exp_chunk(sv, mc, l2);
                     pack_chunk(sv, 1.f, pk);
                     tmem_st32(tS + c64 * 32, pk);
                 }

@@ -106,15 +106,17 @@ constexpr long long kWaitBudgetCycles = 2000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DevStatus* st,
                                           int where) {
     if (mbar_try_wait(bar, parity)) return true;
-    long long start = clock64();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+    const long long start = clock64();
+    // a compact loop: this function is inlined at every wait of the warp-specialised
+    // kernels, whose code must stay small enough for the instruction caches
+#pragma unroll 1
+    while (!mbar_try_wait(bar, parity)) {
         if (clock64() - start > kWaitBudgetCycles) {
             record_error(st, NSA_ERR_TIMEOUT, where, blockIdx.x);
             return false;
         }
     }
+    return true;
 }
 
 // ---------------------------------------------------------------------------- TMA
