@@ -46,13 +46,14 @@ struct alignas(1024) BwdSmem {
     uint8_t p[BS / 64][kTileRows * 128];      // P bf16 [row][key], 64-key chunks
     uint8_t ds[BS / 64][kTileRows * 128];     // dS bf16 [row][key]
     int4 meta[NQ][kTileRows];                 // (token or -1, head, slot, causal limit)
+    float rlse[NQ][kTileRows];                // row LSE * log2(e)
+    float rdelta[NQ][kTileRows];              // row D = rowsum(dO * O)
     uint64_t q_full[NQ], q_empty[NQ], meta_full[NQ], meta_empty[NQ];
     uint64_t kv_full, kv_empty;
     uint64_t sdp_full[NSLOT], dq_full[NSLOT], tmem_empty[NSLOT];
     uint64_t pds_full, pds_empty, acc_full, acc_empty, drain;
     uint32_t tmem_base;
     int abort_flag;
-    int loader_stop;
     int nunits;
 };
 
@@ -66,10 +67,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 template <int BS, int NQ, int NSLOT>
@@ -86,7 +83,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
-        S.loader_stop = 0;
         S.nunits = *reinterpret_cast<volatile int*>(&st->nchunks);
         for (int i = 0; i < NQ; ++i) {
             mbar_init(&S.q_full[i], kLoaderThreads);
@@ -145,23 +141,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 2) {
         // ------------------------------------------------------------------ loaders
-        // 64 threads; each tile's row metadata is shared through shared memory (named
-        // barrier 1).  A tile is published as soon as its own copies have landed: the
-        // stage it waits for next is freed by MMA work that needs this tile first.
-        const int lt = tid;
-        const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-        const __nv_bfloat16* dO = reinterpret_cast<const __nv_bfloat16*>(p.dout);
-        volatile int* stop = &S.loader_stop;
+        // 64 threads.  Lane l of warp w owns tile rows r = 64w + l and 64w + 32 + l: it
+        // writes their metadata, LSE (times log2 e) and D into shared memory for the
+        // P / dS warps, and computes their Q / dO source addresses.  In copy step k the
+        // warp moves rows 64w + 2k and 64w + 2k + 1 (lane l: 16-byte chunk l % 16 of row
+        // 64w + 2k + l / 16, a 512-byte coalesced read); rows past the list are zeroed,
+        // so that they add nothing to dV and dK.  Tile i - 1's copies are published
+        // (wait, fence, arrive on q_full) after tile i's metadata is out and before the
+        // loader waits for tile i's stage: that stage is released by the dV / dK / dQ
+        // products of tile i - 2, which the MMA issuer may queue behind S / dP of tile
+        // i - 1, so publishing later than this could wait in a cycle.
+        const int w = warp;
+        const uint8_t* qb = static_cast<const uint8_t*>(p.q);
+        const uint8_t* db = static_cast<const uint8_t*>(p.dout);
+        const float kLog2e = 1.4426950408889634f;
         int4 u0 = ld_unit(0), u1 = ld_unit(1), u2 = ld_unit(2);
         auto ld_ent = [&](int e0, int ehi, int r) -> uint32_t {
-            return (e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0u;
+            return (e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0xFFFFFFFFu;
         };
-        uint32_t ent0 = 0u, ent1 = 0u;
+        const int rA = 64 * w + lane, rB = rA + 32;
+        uint32_t entA = 0xFFFFFFFFu, entB = 0xFFFFFFFFu;
         if (nk > 0) {
-            ent0 = ld_ent(u0.y, u0.z, 2 * lt);
-            ent1 = ld_ent(u0.y, u0.z, 2 * lt + 1);
+            entA = ld_ent(u0.y, u0.z, rA);
+            entB = ld_ent(u0.y, u0.z, rB);
         }
-        int i = 0;
+        const int c = lane & 15;
+        const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
+        int i = 0, issued = 0, published = 0;
         bool stopped = false;
         for (int k = 0; k < nk && !stopped; ++k) {
             const int4 d = u0;
@@ -169,60 +175,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ntl = d.w & 255, g = d.w >> 8;
             for (int tt = 0; tt < ntl; ++tt, ++i) {
                 const int e0 = d.y + tt * tpt;
-                const int nrows = min(tpt, d.z - e0) * p.G;
                 const int stg = i % NQ;
                 const uint32_t ph_empty = ((i / NQ) & 1) ^ 1;
-                const bool ok = wait(&S.meta_empty[stg], ph_empty, 50) &&
-                                wait(&S.q_empty[stg], ph_empty, 51);
-                if (!ok) *stop = 1;
-                if (ok) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int r = 2 * lt + rr;
-                        const uint32_t ent = rr ? ent1 : ent0;
-                        int4 m = make_int4(-1, 0, 0, -1);
-                        if (r < nrows) {
-                            m.x = (int)(ent >> 6);
-                            m.y = g * p.G + r % p.G;
-                            m.z = (int)(ent & 63u);
-                            m.w = m.x - d.x;
-                        }
-                        S.meta[stg][r] = m;
-                    }
-                }
+                const uint32_t ea = entA, eb = entB;
                 // index entries of the next tile (this unit's or the next unit's first)
                 if (tt + 1 < ntl) {
-                    ent0 = ld_ent(e0 + tpt, d.z, 2 * lt);
-                    ent1 = ld_ent(e0 + tpt, d.z, 2 * lt + 1);
+                    entA = ld_ent(e0 + tpt, d.z, rA);
+                    entB = ld_ent(e0 + tpt, d.z, rB);
                 } else if (k + 1 < nk) {
-                    ent0 = ld_ent(u0.y, u0.z, 2 * lt);
-                    ent1 = ld_ent(u0.y, u0.z, 2 * lt + 1);
+                    entA = ld_ent(u0.y, u0.z, rA);
+                    entB = ld_ent(u0.y, u0.z, rB);
                 }
-                named_bar_sync(1, kLoaderThreads);
-                if (*stop) { stopped = true; break; }   // read after the barrier: uniform
+                // this lane's two rows: metadata, LSE, D, source offsets (-1: past the list)
+                long long offA = -1, offB = -1;
+                float lA = 0.f, lB = 0.f, dA = 0.f, dB = 0.f;
+                int4 mA = make_int4(-1, 0, 0, -1), mB = mA;
+                if (ea != 0xFFFFFFFFu) {
+                    mA = make_int4((int)(ea >> 6), g * p.G + rA % p.G, (int)(ea & 63u), (int)(ea >> 6) - d.x);
+                    offA = ((long long)mA.x * p.hq + mA.y) * (kHeadDim * 2);
+                    lA = __ldg(p.lse + (size_t)mA.y * p.T + mA.x) * kLog2e;
+                    dA = __ldg(p.delta + (size_t)mA.y * p.T + mA.x);
+                }
+                if (eb != 0xFFFFFFFFu) {
+                    mB = make_int4((int)(eb >> 6), g * p.G + rB % p.G, (int)(eb & 63u), (int)(eb >> 6) - d.x);
+                    offB = ((long long)mB.x * p.hq + mB.y) * (kHeadDim * 2);
+                    lB = __ldg(p.lse + (size_t)mB.y * p.T + mB.x) * kLog2e;
+                    dB = __ldg(p.delta + (size_t)mB.y * p.T + mB.x);
+                }
+                if (!__all_sync(0xffffffffu, wait(&S.meta_empty[stg], ph_empty, 50))) {
+                    stopped = true;
+                    break;
+                }
+                S.meta[stg][rA] = mA;
+                S.meta[stg][rB] = mB;
+                S.rlse[stg][rA] = lA;
+                S.rlse[stg][rB] = lB;
+                S.rdelta[stg][rA] = dA;
+                S.rdelta[stg][rB] = dB;
                 mbar_arrive(&S.meta_full[stg]);
-                // gather Q and dO: 4096 16-byte chunks, 64 per thread; zero rows past the list
+                if (i > 0) {                       // publish tile i - 1
+                    cp_async_wait_all();
+                    fence_async_smem();
+                    mbar_arrive(&S.q_full[(i - 1) % NQ]);
+                    published = i;
+                }
+                if (!__all_sync(0xffffffffu, wait(&S.q_empty[stg], ph_empty, 51))) {
+                    stopped = true;
+                    break;
+                }
+                // gather Q and dO
+                const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c, d0 = smem_u32(S.dout[stg][0]) + dst_c;
 #pragma unroll 4
-                for (int c = 0; c < 64; ++c) {
-                    const int idx = lt + c * kLoaderThreads;
-                    const int which = idx >> 11;
-                    const int row = (idx >> 4) & 127, ch = idx & 15;
-                    const uint32_t dst = smem_u32(which ? S.dout[stg][ch >> 3] : S.q[stg][ch >> 3]) +
-                                         sw128_offset(row, ch & 7);
-                    const int4 m = S.meta[stg][row];
-                    if (m.x >= 0) {
-                        const __nv_bfloat16* src = (which ? dO : q) +
-                                                   ((size_t)m.x * p.hq + m.y) * kHeadDim + ch * 8;
-                        cp_async_16(dst, src);
+                for (int kk = 0; kk < 32; ++kk) {
+                    const int rw = 2 * kk + (lane >> 4);          // row within the warp's 64
+                    const long long off = __shfl_sync(0xffffffffu, kk < 16 ? offA : offB, rw & 31);
+                    const uint32_t so = sw128_offset(64 * w + rw, c & 7);
+                    if (off >= 0) {
+                        cp_async_16(q0 + so, qb + off + c * 16);
+                        cp_async_16(d0 + so, db + off + c * 16);
                     } else {
-                        st_shared_v4(dst, 0u, 0u, 0u, 0u);
+                        st_shared_v4(q0 + so, 0u, 0u, 0u, 0u);
+                        st_shared_v4(d0 + so, 0u, 0u, 0u, 0u);
                     }
                 }
                 cp_async_commit();
-                cp_async_wait_all();
-                fence_async_smem();
-                mbar_arrive(&S.q_full[stg]);
+                issued = i + 1;
             }
+        }
+        cp_async_wait_all();   // nothing may still be in flight when the CTA exits
+        if (!stopped && issued > 0 && published == issued - 1) {
+            fence_async_smem();
+            mbar_arrive(&S.q_full[(issued - 1) % NQ]);
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------- K/V producer
@@ -260,6 +283,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
             int kv_loads = 0, prev_bucket = -1;
             bool ok = true;
+            // Shared-memory descriptors are computed once; an MMA step adds its byte
+            // offset / 16 to the start-address field (addresses < 2^18 bytes: no carry
+            // out of the 14-bit field).  K-major operands: LBO 16, SBO 1024 (the 64-column
+            // half of a tile is a separate base); MN-major ones: LBO = the stride between
+            // 64-element halves (or 64-key chunks), SBO 1024.
+            constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+            constexpr uint64_t kKHalf = sizeof(S.k[0]) >> 4, kPChunk = sizeof(S.p[0]) >> 4;
+            const uint64_t dq_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);       // Q, K-major
+            const uint64_t dq_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16, 1024);   // dO, K-major
+            const uint64_t dq_k = smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);          // K, K-major
+            const uint64_t dq_v = smem_desc_sw128(smem_u32(S.v[0]), 16, 1024);          // V, K-major
+            const uint64_t dt_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16384, 1024);    // Q^T
+            const uint64_t dt_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16384, 1024); // dO^T
+            const uint64_t dt_p = smem_desc_sw128(smem_u32(S.p[0]), 16384, 1024);       // P (keys x rows)
+            const uint64_t dt_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16384, 1024);     // dS (keys x rows)
+            const uint64_t dk_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16, 1024);        // dS, K-major
+            const uint64_t dk_kmn = smem_desc_sw128(smem_u32(S.k[0]), BS * 128, 1024);  // K, MN-major
             auto sdp = [&](int i, bool first, int bucket) -> bool {
                 if (first && bucket != prev_bucket) {
                     if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
@@ -271,19 +311,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
                 tc_fence_after();
                 const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
+                const uint64_t aq = dq_q + (uint64_t)stg * kQStage, ad = dq_do + (uint64_t)stg * kQStage;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ss(tS, smem_desc_sw128(smem_u32(S.q[stg][ks >> 2]) + off, 16, 1024),
-                                smem_desc_sw128(smem_u32(S.k[ks >> 2]) + off, 16, 1024), kIdescS,
-                                ks > 0 ? 1u : 0u);
+                    const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                    const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                    mma_bf16_ss(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (uint32_t)(ks & 3) * 32u;
-                    mma_bf16_ss(tdP, smem_desc_sw128(smem_u32(S.dout[stg][ks >> 2]) + off, 16, 1024),
-                                smem_desc_sw128(smem_u32(S.v[ks >> 2]) + off, 16, 1024), kIdescS,
-                                ks > 0 ? 1u : 0u);
+                    const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                    const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                    mma_bf16_ss(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(&S.sdp_full[s]);
                 return true;
@@ -293,22 +332,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait(&S.pds_full, i & 1, 57)) return false;
                 if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
                 tc_fence_after();
-                const uint32_t q0 = smem_u32(S.q[stg][0]), d0 = smem_u32(S.dout[stg][0]);
+                const uint64_t aq = dt_q + (uint64_t)stg * kQStage, ad = dt_do + (uint64_t)stg * kQStage;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step
-                    const uint32_t off = (uint32_t)ks * 2048u;
+                for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
+                    const uint64_t off = (uint64_t)ks * 128u;
                     const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                    mma_bf16_ss(tmem + kColDV, smem_desc_sw128(d0 + off, 16384, 1024),
-                                smem_desc_sw128(smem_u32(S.p[0]) + off, 16384, 1024), kIdescT, acc);
-                    mma_bf16_ss(tmem + kColDK, smem_desc_sw128(q0 + off, 16384, 1024),
-                                smem_desc_sw128(smem_u32(S.ds[0]) + off, 16384, 1024), kIdescT, acc);
+                    mma_bf16_ss(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
+                    mma_bf16_ss(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
                 }
 #pragma unroll
                 for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
                     mma_bf16_ss(tmem + s * kSlotCols,
-                                smem_desc_sw128(smem_u32(S.ds[ks >> 2]) + (uint32_t)(ks & 3) * 32u, 16, 1024),
-                                smem_desc_sw128(smem_u32(S.k[0]) + (uint32_t)ks * 2048u, BS * 128, 1024),
-                                kIdescQ, ks > 0 ? 1u : 0u);
+                                dk_ds + (uint64_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
+                                dk_kmn + (uint64_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
                 mma_commit(&S.dq_full[s]);
                 mma_commit(&S.pds_empty);
                 mma_commit(&S.q_empty[stg]);
@@ -351,7 +387,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wg = (warp - 4) >> 2;
         const int r = (warp & 3) * 32 + lane;            // row = TMEM lane (= d for dV^T/dK^T)
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const float kLog2e = 1.4426950408889634f;
         if (wg < NSLOT) {
             int4 u0 = ld_unit(0), u1 = ld_unit(1);
             int i = 0;
@@ -365,13 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int stg = i % NQ, s = i % NSLOT;
                     if (!(ok = wait(&S.meta_full[stg], (i / NQ) & 1, 60))) break;
                     const int4 m = S.meta[stg][r];
+                    const float lse2 = S.rlse[stg][r], delta = S.rdelta[stg][r];
                     mbar_arrive(&S.meta_empty[stg]);
                     const int my_t = m.x, my_h = m.y, my_j = m.z, my_lim = m.w;
-                    float lse2 = 0.f, delta = 0.f;
-                    if (my_t >= 0) {
-                        lse2 = __ldg(p.lse + (size_t)my_h * p.T + my_t) * kLog2e;
-                        delta = __ldg(p.delta + (size_t)my_h * p.T + my_t);
-                    }
                     if (!(ok = wait(&S.sdp_full[s], (i / NSLOT) & 1, 61))) break;
                     tc_fence_after();
                     const uint32_t tS = tmem + s * kSlotCols + lane_off, tdP = tS + BS;
@@ -383,13 +414,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_ld32(tdP + c64 * 64, dp);
                         tmem_ld32(tdP + c64 * 64 + 32, dp + 32);
                         tmem_wait_ld();
+                        const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+                        const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
 #pragma unroll
                         for (int c = 0; c < 64; c += 2) {
                             const int key = c64 * 64 + c;
-                            const float p0 = key <= my_lim ? exp2f(sv[c] * p.scale_log2 - lse2) : 0.f;
-                            const float p1 = key + 1 <= my_lim ? exp2f(sv[c + 1] * p.scale_log2 - lse2) : 0.f;
-                            pk[c / 2] = pack_bf16x2(p0, p1);
-                            dk[c / 2] = pack_bf16x2(p0 * (dp[c] - delta), p1 * (dp[c + 1] - delta));
+                            float2 x = fma2(make_float2(sv[c], sv[c + 1]), c2, nl2);
+                            x.x = key <= my_lim ? ex2_approx(x.x) : 0.f;
+                            x.y = key + 1 <= my_lim ? ex2_approx(x.y) : 0.f;
+                            const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
+                            pk[c / 2] = pack_bf16x2(x.x, x.y);
+                            dk[c / 2] = pack_bf16x2(ds.x, ds.y);
                         }
                     };
                     auto store_chunk = [&](int c64, const uint32_t* pk, const uint32_t* dk) {
