@@ -43,15 +43,31 @@
 namespace nsa {
 namespace {
 
-// Warp roles: Q loaders 0 .. kLoaderWarps-1 (2 or 4), softmax warpgroups 4-7 and 8-11,
-// epilogue warpgroup 12-15 (warp % 4 = TMEM lane quadrant), then the TMA producer and
-// the MMA issuer (warps 2, 3 with two loaders; 16, 17 with four).
-constexpr int kLoaderWarps = 2;
-constexpr int kTmaWarp = kLoaderWarps == 2 ? 2 : 16;
-constexpr int kMmaWarp = kTmaWarp + 1;
-constexpr int kThreads = (kLoaderWarps == 2 ? 16 : 18) * 32;
+// Warp roles (five warpgroups; warp % 4 = TMEM lane quadrant):
+//   warpgroup 0 (warps 0-3)    Q loaders 0-3
+//   warpgroups 1, 2 (4-11)     softmax of even / odd tiles
+//   warpgroup 3 (12-15)        epilogue
+//   warpgroup 4 (16-19)        TMA producer (16), MMA issuer (17), Q loaders 4-5 (18, 19)
+// The gather's throughput grows with the number of warps issuing cp.async, so six
+// warps load Q.  Registers are rebalanced with setmaxnreg: the launch gives every
+// thread 96; warpgroups 0 and 4 drop to 56, the softmax warpgroups rise to 136
+// (2 x 128 x 56 + 128 x 96 + 2 x 128 x 136 = 640 x 96).
+constexpr int kThreads = 640;
+constexpr int kLoaderWarps = 6;
 constexpr int kLoaderThreads = kLoaderWarps * 32;
-constexpr int kRowsPerLoader = kTileRows / kLoaderWarps;   // 64 or 32
+constexpr int kRowsPerLoader = (kTileRows + kLoaderWarps - 1) / kLoaderWarps;   // 22
+static_assert(kRowsPerLoader <= 32, "one row per loader lane");
+constexpr int kTmaWarp = 16, kMmaWarp = 17;
+constexpr int kRegsLow = 56, kRegsSoftmax = 136;
+
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 constexpr int kWgThreads = 128;
 constexpr int kNQ = 2;         // Q stages (= S slots: S(i) completing frees stage i % 2)
 constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
@@ -176,180 +192,184 @@ __global__ void __launch_bounds__(kThreads, 1)
         return __all_sync(0xffffffffu, wait(bar, parity, where));
     };
 
-    if (warp < kLoaderWarps) {
-        // ---------------------------------------------------------------- Q loaders
-        // Warp w fills the R = kRowsPerLoader tile rows [Rw, Rw + R).  Lane l computes the
-        // source address of row Rw + l (and Rw + 32 + l when R = 64) from the index entry
-        // (token) and the row (head); in copy step k the warp moves rows Rw + 2k and
-        // Rw + 2k + 1, lane l taking the 16-byte chunk l % 16 of row Rw + 2k + l / 16 (a
-        // 512-byte coalesced read).
-        // The copies of tile i are published one tile later (wait for the older
-        // cp.async group, fence for the tensor core's async proxy, arrive on q_full),
-        // so two tiles' gathers are in flight.
-        const int w = warp;
-        const uint8_t* qb = static_cast<const uint8_t*>(p.q);
-        const int rA = kRowsPerLoader * w + lane, rB = rA + 32;
-        auto ld_ent = [&](const int4& d, int r) -> uint32_t {
-            return r < (d.z & 255) ? __ldg(p.entries + d.y + r / p.G) : 0u;
-        };
-        auto row_addr = [&](const int4& d, int r, uint32_t ent) -> unsigned long long {
-            const int g = d.z >> 8;
-            return reinterpret_cast<unsigned long long>(
-                qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (kHeadDim * 2));
-        };
-        int4 d0 = ld_desc(0), d1 = ld_desc(1);
-        uint32_t ea = ld_ent(d0, rA), eb = kRowsPerLoader == 64 ? ld_ent(d0, rB) : 0u;
-        int published = 0, issued = 0;
-        const int c = lane & 15;
-        const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
-        for (int i = 0; i < n; ++i) {
-            const int4 d = d0;
-            const unsigned long long addrA = row_addr(d, rA, ea);
-            const unsigned long long addrB = row_addr(d, rB, eb);
-            d0 = d1;
-            d1 = ld_desc(i + 2);
-            ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
-            eb = kRowsPerLoader == 64 ? ld_ent(d0, rB) : 0u;
-            const int nrows = d.z & 255;
-            const int stg = i % kNQ;
-            // stage i % 2 is free once S(i - 2), which read it, has completed
-            if (!wait_w(&S.s_full[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
-            const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
-#pragma unroll 4
-            for (int k = 0; k < kRowsPerLoader / 2; ++k) {
-                const int rw = 2 * k + (lane >> 4);          // row within the warp's 64
-                const unsigned long long a =
-                    __shfl_sync(0xffffffffu, k < 16 ? addrA : addrB, rw & 31) + c * 16;
-                const int row = kRowsPerLoader * w + rw;
-                if (row < nrows)
-                    cp_async_16(q0 + sw128_offset(row, c & 7), reinterpret_cast<const void*>(a));
-            }
-            cp_async_commit();
-            issued = i + 1;
-            if (i > 0) {
-                cp_async_wait_one_pending();
-                fence_async_smem();
-                mbar_arrive(&S.q_full[(i - 1) % kNQ]);
-                published = i;
-            }
-        }
-        cp_async_wait_all();   // nothing may still be in flight when the CTA exits
-        if (issued == n && published == n - 1 && n > 0) {
-            fence_async_smem();
-            mbar_arrive(&S.q_full[(n - 1) % kNQ]);
-        }
-    } else if (warp == kTmaWarp) {
-        // ------------------------------------------------------------- K/V producer
-        if (lane == 0) {
-            prefetch_tmap(&kmap);
-            prefetch_tmap(&vmap);
-            int prev = -1, uses = 0;
-            int last_parity[NKV];
-            bool loaded[NKV];
-            for (int s = 0; s < NKV; ++s) { last_parity[s] = 0; loaded[s] = false; }
-            int4 d0 = ld_desc(0), d1 = ld_desc(1), d2 = ld_desc(2);
+    const int wgrp = warp >> 2;
+    const int li = wgrp == 0 ? warp : (warp >= 18 ? warp - 14 : -1);   // loader index
+
+    if (wgrp == 0 || wgrp == 4) {
+        reg_dealloc<kRegsLow>();
+        if (li >= 0) {
+            // ---------------------------------------------------------------- Q loaders
+            // Loader w fills the tile rows [R w, min(R w + R, 128)), R = kRowsPerLoader.
+            // Lane l computes the source address of row R w + l from the index entry (token)
+            // and the row (head); in copy step k the loader moves rows R w + 2k and
+            // R w + 2k + 1, lane l taking the 16-byte chunk l % 16 of row R w + 2k + l / 16
+            // (a 512-byte coalesced read).  The copies of tile i are published one tile
+            // later (wait for the older cp.async group, fence for the tensor core's async
+            // proxy, arrive on q_full), so two tiles' gathers are in flight.
+            const int w = li;
+            const int nr_w = min(kRowsPerLoader, kTileRows - kRowsPerLoader * w);   // rows of this loader
+            const uint8_t* qb = static_cast<const uint8_t*>(p.q);
+            const int rA = kRowsPerLoader * w + lane;
+            auto ld_ent = [&](const int4& d, int r) -> uint32_t {
+                return (lane < nr_w && r < (d.z & 255)) ? __ldg(p.entries + d.y + r / p.G) : 0u;
+            };
+            auto row_addr = [&](const int4& d, int r, uint32_t ent) -> unsigned long long {
+                const int g = d.z >> 8;
+                return reinterpret_cast<unsigned long long>(
+                    qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (kHeadDim * 2));
+            };
+            int4 d0 = ld_desc(0), d1 = ld_desc(1);
+            uint32_t ea = ld_ent(d0, rA);
+            int published = 0, issued = 0;
+            const int c = lane & 15;
+            const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
             for (int i = 0; i < n; ++i) {
                 const int4 d = d0;
-                d0 = d1; d1 = d2; d2 = ld_desc(i + 3);
-                if (d.w == prev) continue;
-                prev = d.w;
-                const int stg = uses % NKV;
-                if (!wait(&S.kv_empty[stg], ((uses / NKV) & 1) ^ 1, 32)) break;
-                const int g = d.z >> 8;
-                mbar_arrive_expect_tx(&S.kv_full[stg], 4u * BS * 128u);
-                tma_load_3d(S.kv[stg][0][0], &kmap, &S.kv_full[stg], 0, g, d.x);
-                tma_load_3d(S.kv[stg][0][1], &kmap, &S.kv_full[stg], 64, g, d.x);
-                tma_load_3d(S.kv[stg][1][0], &vmap, &S.kv_full[stg], 0, g, d.x);
-                tma_load_3d(S.kv[stg][1][1], &vmap, &S.kv_full[stg], 64, g, d.x);
-                last_parity[stg] = (uses / NKV) & 1;
-                loaded[stg] = true;
-                ++uses;
-            }
-            if (*abort_flag)   // let copies still in flight land before the CTA exits
-                for (int s = 0; s < NKV; ++s)
-                    if (loaded[s]) mbar_wait(&S.kv_full[s], last_parity[s], st, 40);
-        }
-    } else if (warp == kMmaWarp) {
-        // -------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);
-            constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
-            int kv_uses = 0, prev_bucket = -1, cur = 0;
-            int kvs_of[2] = {0, 0};
-            // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
-            // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
-            // run in issue order.
-            // Shared-memory descriptors are computed once; an MMA step only adds the
-            // byte offset / 16 to the start-address field (addresses stay < 2^18 bytes,
-            // so the 14-bit field never carries).  This keeps the issuing thread's
-            // instruction count per MMA small: it shares its SMSP with busy warps.
-            constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
-            constexpr uint64_t kKvStage = sizeof(S.kv[0]) >> 4, kKvHalf = sizeof(S.kv[0][0][0]) >> 4;
-            const uint64_t q_desc0 = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
-            const uint64_t k_desc0 = smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
-            const uint64_t v_desc0 = smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
-            // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
-            // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
-            // run in issue order.  s_full also tells the loaders that the Q stage (i % 2)
-            // is free again.
-            auto issue_s = [&](int i, int bucket) -> bool {
-                if (bucket != prev_bucket) {
-                    cur = kv_uses % NKV;
-                    if (!wait(&S.kv_full[cur], (kv_uses / NKV) & 1, 33)) return false;
-                    ++kv_uses;
-                    prev_bucket = bucket;
+                const unsigned long long addrA = row_addr(d, rA, ea);
+                d0 = d1;
+                d1 = ld_desc(i + 2);
+                ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
+                const int nrows = d.z & 255;
+                const int stg = i % kNQ;
+                // stage i % 2 is free once S(i - 2), which read it, has completed
+                if (!wait_w(&S.s_full[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
+                const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
+    #pragma unroll 4
+                for (int k = 0; k < (kRowsPerLoader + 1) / 2; ++k) {
+                    const int rw = 2 * k + (lane >> 4);          // row within the loader's rows
+                    const unsigned long long a = __shfl_sync(0xffffffffu, addrA, rw & 31) + c * 16;
+                    const int row = kRowsPerLoader * w + rw;
+                    if (rw < nr_w && row < nrows)
+                        cp_async_16(q0 + sw128_offset(row, c & 7), reinterpret_cast<const void*>(a));
                 }
-                const int slot = i & 1, stg = i % kNQ;
-                kvs_of[slot] = cur;
-                if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
-                tc_fence_after();
-                const uint32_t tS = tmem + slot * BS;
-                const uint64_t a0 = q_desc0 + (uint64_t)stg * kQStage;
-                const uint64_t b0 = k_desc0 + (uint64_t)cur * kKvStage;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t off = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                    const uint64_t offk = (uint64_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
-                    mma_bf16_ss(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u);
+                cp_async_commit();
+                issued = i + 1;
+                if (i > 0) {
+                    cp_async_wait_one_pending();
+                    fence_async_smem();
+                    mbar_arrive(&S.q_full[(i - 1) % kNQ]);
+                    published = i;
                 }
-                mma_commit(&S.s_full[slot]);
-                return true;
-            };
-            // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
-            // epilogue of tile i - NO has read the buffer's previous O.
-            auto issue_pv = [&](int i, bool release_kv) -> bool {
-                const int slot = i & 1, ob = i % NO;
-                if (!wait(&S.p_full[slot], (i >> 1) & 1, 36)) return false;
-                if (!wait(&S.o_free[ob], ((i / NO) & 1) ^ 1, 34)) return false;
-                tc_fence_after();
-                const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
-                const int kvs = kvs_of[slot];
-                const uint64_t b0 = v_desc0 + (uint64_t)kvs * kKvStage;
-#pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks)    // 16 keys = 2048 bytes per step
-                    mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b0 + (uint64_t)ks * 128u, kIdescO,
-                                ks > 0 ? 1u : 0u);
-                mma_commit(&S.o_full[ob]);
-                if (release_kv) mma_commit(&S.kv_empty[kvs]);
-                return true;
-            };
-            int4 dc = ld_desc(0), dn = ld_desc(1), dnn = ld_desc(2);
-            bool ok = n > 0 && issue_s(0, dc.w);
-            for (int i = 0; i < n && ok; ++i) {
-                const bool more = i + 1 < n;
-                const bool same = more && dn.w == dc.w;
-                // S(i+1) goes ahead of PV(i) unless it needs the only K/V stage
-                const bool ahead = more && (NKV > 1 || same);
-                if (ahead && !(ok = issue_s(i + 1, dn.w))) break;
-                if (!(ok = issue_pv(i, !same))) break;
-                if (more && !ahead && !(ok = issue_s(i + 1, dn.w))) break;
-                dc = dn; dn = dnn; dnn = ld_desc(i + 3);
             }
-            // every MMA issued above has finished once this commit arrives
-            mma_commit(&S.drain);
-            mbar_wait(&S.drain, 0, st, 41);
+            cp_async_wait_all();   // nothing may still be in flight when the CTA exits
+            if (issued == n && published == n - 1 && n > 0) {
+                fence_async_smem();
+                mbar_arrive(&S.q_full[(n - 1) % kNQ]);
+            }
+        } else if (warp == kTmaWarp) {
+            // ------------------------------------------------------------- K/V producer
+            if (lane == 0) {
+                prefetch_tmap(&kmap);
+                prefetch_tmap(&vmap);
+                int prev = -1, uses = 0;
+                int last_parity[NKV];
+                bool loaded[NKV];
+                for (int s = 0; s < NKV; ++s) { last_parity[s] = 0; loaded[s] = false; }
+                int4 d0 = ld_desc(0), d1 = ld_desc(1), d2 = ld_desc(2);
+                for (int i = 0; i < n; ++i) {
+                    const int4 d = d0;
+                    d0 = d1; d1 = d2; d2 = ld_desc(i + 3);
+                    if (d.w == prev) continue;
+                    prev = d.w;
+                    const int stg = uses % NKV;
+                    if (!wait(&S.kv_empty[stg], ((uses / NKV) & 1) ^ 1, 32)) break;
+                    const int g = d.z >> 8;
+                    mbar_arrive_expect_tx(&S.kv_full[stg], 4u * BS * 128u);
+                    tma_load_3d(S.kv[stg][0][0], &kmap, &S.kv_full[stg], 0, g, d.x);
+                    tma_load_3d(S.kv[stg][0][1], &kmap, &S.kv_full[stg], 64, g, d.x);
+                    tma_load_3d(S.kv[stg][1][0], &vmap, &S.kv_full[stg], 0, g, d.x);
+                    tma_load_3d(S.kv[stg][1][1], &vmap, &S.kv_full[stg], 64, g, d.x);
+                    last_parity[stg] = (uses / NKV) & 1;
+                    loaded[stg] = true;
+                    ++uses;
+                }
+                if (*abort_flag)   // let copies still in flight land before the CTA exits
+                    for (int s = 0; s < NKV; ++s)
+                        if (loaded[s]) mbar_wait(&S.kv_full[s], last_parity[s], st, 40);
+            }
+        } else if (warp == kMmaWarp) {
+            // -------------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);
+                constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
+                int kv_uses = 0, prev_bucket = -1, cur = 0;
+                int kvs_of[2] = {0, 0};
+                // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
+                // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
+                // run in issue order.
+                // Shared-memory descriptors are computed once; an MMA step only adds the
+                // byte offset / 16 to the start-address field (addresses stay < 2^18 bytes,
+                // so the 14-bit field never carries).  This keeps the issuing thread's
+                // instruction count per MMA small: it shares its SMSP with busy warps.
+                constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+                constexpr uint64_t kKvStage = sizeof(S.kv[0]) >> 4, kKvHalf = sizeof(S.kv[0][0][0]) >> 4;
+                const uint64_t q_desc0 = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
+                const uint64_t k_desc0 = smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
+                const uint64_t v_desc0 = smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
+                // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
+                // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
+                // run in issue order.  s_full also tells the loaders that the Q stage (i % 2)
+                // is free again.
+                auto issue_s = [&](int i, int bucket) -> bool {
+                    if (bucket != prev_bucket) {
+                        cur = kv_uses % NKV;
+                        if (!wait(&S.kv_full[cur], (kv_uses / NKV) & 1, 33)) return false;
+                        ++kv_uses;
+                        prev_bucket = bucket;
+                    }
+                    const int slot = i & 1, stg = i % kNQ;
+                    kvs_of[slot] = cur;
+                    if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
+                    tc_fence_after();
+                    const uint32_t tS = tmem + slot * BS;
+                    const uint64_t a0 = q_desc0 + (uint64_t)stg * kQStage;
+                    const uint64_t b0 = k_desc0 + (uint64_t)cur * kKvStage;
+    #pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t off = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint64_t offk = (uint64_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
+                        mma_bf16_ss(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&S.s_full[slot]);
+                    return true;
+                };
+                // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
+                // epilogue of tile i - NO has read the buffer's previous O.
+                auto issue_pv = [&](int i, bool release_kv) -> bool {
+                    const int slot = i & 1, ob = i % NO;
+                    if (!wait(&S.p_full[slot], (i >> 1) & 1, 36)) return false;
+                    if (!wait(&S.o_free[ob], ((i / NO) & 1) ^ 1, 34)) return false;
+                    tc_fence_after();
+                    const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
+                    const int kvs = kvs_of[slot];
+                    const uint64_t b0 = v_desc0 + (uint64_t)kvs * kKvStage;
+    #pragma unroll
+                    for (int ks = 0; ks < BS / 16; ++ks)    // 16 keys = 2048 bytes per step
+                        mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b0 + (uint64_t)ks * 128u, kIdescO,
+                                    ks > 0 ? 1u : 0u);
+                    mma_commit(&S.o_full[ob]);
+                    if (release_kv) mma_commit(&S.kv_empty[kvs]);
+                    return true;
+                };
+                int4 dc = ld_desc(0), dn = ld_desc(1), dnn = ld_desc(2);
+                bool ok = n > 0 && issue_s(0, dc.w);
+                for (int i = 0; i < n && ok; ++i) {
+                    const bool more = i + 1 < n;
+                    const bool same = more && dn.w == dc.w;
+                    // S(i+1) goes ahead of PV(i) unless it needs the only K/V stage
+                    const bool ahead = more && (NKV > 1 || same);
+                    if (ahead && !(ok = issue_s(i + 1, dn.w))) break;
+                    if (!(ok = issue_pv(i, !same))) break;
+                    if (more && !ahead && !(ok = issue_s(i + 1, dn.w))) break;
+                    dc = dn; dn = dnn; dnn = ld_desc(i + 3);
+                }
+                // every MMA issued above has finished once this commit arrives
+                mma_commit(&S.drain);
+                mbar_wait(&S.drain, 0, st, 41);
+            }
         }
-    } else if (warp >= 4 && warp < 12) {
+    } else if (wgrp == 1 || wgrp == 2) {
+        reg_alloc<kRegsSoftmax>();
         // ------------------------------------------------------------------ softmax
         // Thread = tile row = TMEM lane.  Non-diagonal tiles (every row sees the whole
         // block) skip the causal mask; the test is warp-uniform.
