@@ -33,9 +33,31 @@
 namespace nsa {
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kLoaderThreads = 64;
+// Warp roles (four warpgroups; warp % 4 = TMEM lane quadrant):
+//   warpgroup 0 (warps 0-3)      Q / dO loaders 0-3
+//   warpgroups 1, 2 (4-11)       P / dS and epilogues of even / odd tiles
+//   warpgroup 3 (12-15)          TMA producer (12), MMA issuer (13), loaders 4-5 (14, 15)
+// A cp.async gather's throughput grows with the number of issuing warps, and a tile
+// needs 64 KB of gathered Q and dO rows, so six warps load.  setmaxnreg rebalances
+// the launch's 128 registers per thread: warpgroups 0 and 3 take 64, the P / dS
+// warpgroups 192 (2 x 128 x 64 + 2 x 128 x 192 = 512 x 128).
+constexpr int kThreads = 512;
+constexpr int kLoaderWarps = 6;
+constexpr int kLoaderThreads = kLoaderWarps * 32;
+constexpr int kRowsPerLoader = (kTileRows + kLoaderWarps - 1) / kLoaderWarps;   // 22
+static_assert(kRowsPerLoader <= 32, "one row per loader lane");
+constexpr int kTmaWarp = 12, kMmaWarp = 13;
+constexpr int kRegsLow = 64, kRegsWg = 192;
 constexpr int kWgThreads = 128;
+
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 template <int BS, int NQ, int NSLOT>
 struct alignas(1024) BwdSmem {
@@ -139,250 +161,244 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kColDK = kColDV + BS;
     static_assert(kColDK + BS <= 512, "TMEM budget");
 
-    if (warp < 2) {
-        // ------------------------------------------------------------------ loaders
-        // 64 threads.  Lane l of warp w owns tile rows r = 64w + l and 64w + 32 + l: it
-        // writes their metadata, LSE (times log2 e) and D into shared memory for the
-        // P / dS warps, and computes their Q / dO source addresses.  In copy step k the
-        // warp moves rows 64w + 2k and 64w + 2k + 1 (lane l: 16-byte chunk l % 16 of row
-        // 64w + 2k + l / 16, a 512-byte coalesced read); rows past the list are zeroed,
-        // so that they add nothing to dV and dK.  Tile i - 1's copies are published
-        // (wait, fence, arrive on q_full) after tile i's metadata is out and before the
-        // loader waits for tile i's stage: that stage is released by the dV / dK / dQ
-        // products of tile i - 2, which the MMA issuer may queue behind S / dP of tile
-        // i - 1, so publishing later than this could wait in a cycle.
-        const int w = warp;
-        const uint8_t* qb = static_cast<const uint8_t*>(p.q);
-        const uint8_t* db = static_cast<const uint8_t*>(p.dout);
-        const float kLog2e = 1.4426950408889634f;
-        int4 u0 = ld_unit(0), u1 = ld_unit(1), u2 = ld_unit(2);
-        auto ld_ent = [&](int e0, int ehi, int r) -> uint32_t {
-            return (e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0xFFFFFFFFu;
-        };
-        const int rA = 64 * w + lane, rB = rA + 32;
-        uint32_t entA = 0xFFFFFFFFu, entB = 0xFFFFFFFFu;
-        if (nk > 0) {
-            entA = ld_ent(u0.y, u0.z, rA);
-            entB = ld_ent(u0.y, u0.z, rB);
-        }
-        const int c = lane & 15;
-        const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
-        int i = 0, issued = 0, published = 0;
-        bool stopped = false;
-        for (int k = 0; k < nk && !stopped; ++k) {
-            const int4 d = u0;
-            u0 = u1; u1 = u2; u2 = ld_unit(k + 3);
-            const int ntl = d.w & 255, g = d.w >> 8;
-            for (int tt = 0; tt < ntl; ++tt, ++i) {
-                const int e0 = d.y + tt * tpt;
-                const int stg = i % NQ;
-                const uint32_t ph_empty = ((i / NQ) & 1) ^ 1;
-                const uint32_t ea = entA, eb = entB;
-                // index entries of the next tile (this unit's or the next unit's first)
-                if (tt + 1 < ntl) {
-                    entA = ld_ent(e0 + tpt, d.z, rA);
-                    entB = ld_ent(e0 + tpt, d.z, rB);
-                } else if (k + 1 < nk) {
-                    entA = ld_ent(u0.y, u0.z, rA);
-                    entB = ld_ent(u0.y, u0.z, rB);
+    const int wgrp = warp >> 2;
+    const int li = wgrp == 0 ? warp : warp >= 14 ? warp - 10 : -1;
+
+    if (wgrp == 0 || wgrp == 3) {
+        reg_dealloc<kRegsLow>();
+        if (li >= 0) {
+            // ------------------------------------------------------------------ loaders
+            // Loader w fills tile rows [R w, min(R w + R, 128)), R = kRowsPerLoader; lane l
+            // owns row R w + l: it writes the row's metadata, LSE (times log2 e) and D into
+            // shared memory for the P / dS warps and computes its Q / dO source address.  In
+            // copy step k the loader moves rows R w + 2k and R w + 2k + 1 (lane l: 16-byte
+            // chunk l % 16 of row R w + 2k + l / 16, a 512-byte coalesced read); rows past
+            // the list are zeroed, so that they add nothing to dV and dK.  Tile i - 1's copies are published
+            // (wait, fence, arrive on q_full) after tile i's metadata is out and before the
+            // loader waits for tile i's stage: that stage is released by the dV / dK / dQ
+            // products of tile i - 2, which the MMA issuer may queue behind S / dP of tile
+            // i - 1, so publishing later than this could wait in a cycle.
+            const int w = li;
+            const int nr_w = min(kRowsPerLoader, kTileRows - kRowsPerLoader * w);   // rows of this loader
+            const uint8_t* qb = static_cast<const uint8_t*>(p.q);
+            const uint8_t* db = static_cast<const uint8_t*>(p.dout);
+            const float kLog2e = 1.4426950408889634f;
+            int4 u0 = ld_unit(0), u1 = ld_unit(1), u2 = ld_unit(2);
+            auto ld_ent = [&](int e0, int ehi, int r) -> uint32_t {
+                return (lane < nr_w && e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0xFFFFFFFFu;
+            };
+            const int rA = kRowsPerLoader * w + lane;
+            uint32_t entA = 0xFFFFFFFFu;
+            if (nk > 0) entA = ld_ent(u0.y, u0.z, rA);
+            const int c = lane & 15;
+            const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
+            int i = 0, issued = 0, published = 0;
+            bool stopped = false;
+            for (int k = 0; k < nk && !stopped; ++k) {
+                const int4 d = u0;
+                u0 = u1; u1 = u2; u2 = ld_unit(k + 3);
+                const int ntl = d.w & 255, g = d.w >> 8;
+                for (int tt = 0; tt < ntl; ++tt, ++i) {
+                    const int e0 = d.y + tt * tpt;
+                    const int stg = i % NQ;
+                    const uint32_t ph_empty = ((i / NQ) & 1) ^ 1;
+                    const uint32_t ea = entA;
+                    // index entries of the next tile (this unit's or the next unit's first)
+                    if (tt + 1 < ntl) entA = ld_ent(e0 + tpt, d.z, rA);
+                    else if (k + 1 < nk) entA = ld_ent(u0.y, u0.z, rA);
+                    // this lane's row: metadata, LSE, D, source offset (-1: past the list)
+                    long long offA = -1;
+                    float lA = 0.f, dA = 0.f;
+                    int4 mA = make_int4(-1, 0, 0, -1);
+                    if (ea != 0xFFFFFFFFu) {
+                        mA = make_int4((int)(ea >> 6), g * p.G + rA % p.G, (int)(ea & 63u), (int)(ea >> 6) - d.x);
+                        offA = ((long long)mA.x * p.hq + mA.y) * (kHeadDim * 2);
+                        lA = __ldg(p.lse + (size_t)mA.y * p.T + mA.x) * kLog2e;
+                        dA = __ldg(p.delta + (size_t)mA.y * p.T + mA.x);
+                    }
+                    if (!__all_sync(0xffffffffu, wait(&S.meta_empty[stg], ph_empty, 50))) {
+                        stopped = true;
+                        break;
+                    }
+                    if (lane < nr_w) {
+                        S.meta[stg][rA] = mA;
+                        S.rlse[stg][rA] = lA;
+                        S.rdelta[stg][rA] = dA;
+                    }
+                    mbar_arrive(&S.meta_full[stg]);
+                    if (i > 0) {                       // publish tile i - 1
+                        cp_async_wait_all();
+                        fence_async_smem();
+                        mbar_arrive(&S.q_full[(i - 1) % NQ]);
+                        published = i;
+                    }
+                    if (!__all_sync(0xffffffffu, wait(&S.q_empty[stg], ph_empty, 51))) {
+                        stopped = true;
+                        break;
+                    }
+                    // gather Q and dO
+                    const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c, d0 = smem_u32(S.dout[stg][0]) + dst_c;
+    #pragma unroll 1
+                    for (int kk = 0; kk < (kRowsPerLoader + 1) / 2; ++kk) {
+                        const int rw = 2 * kk + (lane >> 4);          // row within the loader's rows
+                        const long long off = __shfl_sync(0xffffffffu, offA, rw & 31);
+                        if (rw >= nr_w) continue;
+                        const uint32_t so = sw128_offset(kRowsPerLoader * w + rw, c & 7);
+                        if (off >= 0) {
+                            cp_async_16(q0 + so, qb + off + c * 16);
+                            cp_async_16(d0 + so, db + off + c * 16);
+                        } else {
+                            st_shared_v4(q0 + so, 0u, 0u, 0u, 0u);
+                            st_shared_v4(d0 + so, 0u, 0u, 0u, 0u);
+                        }
+                    }
+                    cp_async_commit();
+                    issued = i + 1;
                 }
-                // this lane's two rows: metadata, LSE, D, source offsets (-1: past the list)
-                long long offA = -1, offB = -1;
-                float lA = 0.f, lB = 0.f, dA = 0.f, dB = 0.f;
-                int4 mA = make_int4(-1, 0, 0, -1), mB = mA;
-                if (ea != 0xFFFFFFFFu) {
-                    mA = make_int4((int)(ea >> 6), g * p.G + rA % p.G, (int)(ea & 63u), (int)(ea >> 6) - d.x);
-                    offA = ((long long)mA.x * p.hq + mA.y) * (kHeadDim * 2);
-                    lA = __ldg(p.lse + (size_t)mA.y * p.T + mA.x) * kLog2e;
-                    dA = __ldg(p.delta + (size_t)mA.y * p.T + mA.x);
+            }
+            cp_async_wait_all();   // nothing may still be in flight when the CTA exits
+            if (!stopped && issued > 0 && published == issued - 1) {
+                fence_async_smem();
+                mbar_arrive(&S.q_full[(issued - 1) % NQ]);
+            }
+        } else if (warp == kTmaWarp) {
+            // ------------------------------------------------------------- K/V producer
+            if (lane == 0) {
+                prefetch_tmap(&kmap);
+                prefetch_tmap(&vmap);
+                int prev = -1, loads = 0, last_parity = 0;
+                bool loaded = false;
+                int4 u0 = ld_unit(0), u1 = ld_unit(1);
+                int b0 = ld_bucket(0), b1 = ld_bucket(1);
+                for (int k = 0; k < nk; ++k) {
+                    const int4 d = u0;
+                    const int b = b0;
+                    u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
+                    if (b == prev) continue;
+                    prev = b;
+                    if (!wait(&S.kv_empty, (loads & 1) ^ 1, 52)) break;
+                    const int g = d.w >> 8;
+                    mbar_arrive_expect_tx(&S.kv_full, 4u * BS * 128u);
+                    tma_load_3d(S.k[0], &kmap, &S.kv_full, 0, g, d.x);
+                    tma_load_3d(S.k[1], &kmap, &S.kv_full, 64, g, d.x);
+                    tma_load_3d(S.v[0], &vmap, &S.kv_full, 0, g, d.x);
+                    tma_load_3d(S.v[1], &vmap, &S.kv_full, 64, g, d.x);
+                    last_parity = loads & 1;
+                    loaded = true;
+                    ++loads;
                 }
-                if (eb != 0xFFFFFFFFu) {
-                    mB = make_int4((int)(eb >> 6), g * p.G + rB % p.G, (int)(eb & 63u), (int)(eb >> 6) - d.x);
-                    offB = ((long long)mB.x * p.hq + mB.y) * (kHeadDim * 2);
-                    lB = __ldg(p.lse + (size_t)mB.y * p.T + mB.x) * kLog2e;
-                    dB = __ldg(p.delta + (size_t)mB.y * p.T + mB.x);
-                }
-                if (!__all_sync(0xffffffffu, wait(&S.meta_empty[stg], ph_empty, 50))) {
-                    stopped = true;
-                    break;
-                }
-                S.meta[stg][rA] = mA;
-                S.meta[stg][rB] = mB;
-                S.rlse[stg][rA] = lA;
-                S.rlse[stg][rB] = lB;
-                S.rdelta[stg][rA] = dA;
-                S.rdelta[stg][rB] = dB;
-                mbar_arrive(&S.meta_full[stg]);
-                if (i > 0) {                       // publish tile i - 1
-                    cp_async_wait_all();
-                    fence_async_smem();
-                    mbar_arrive(&S.q_full[(i - 1) % NQ]);
-                    published = i;
-                }
-                if (!__all_sync(0xffffffffu, wait(&S.q_empty[stg], ph_empty, 51))) {
-                    stopped = true;
-                    break;
-                }
-                // gather Q and dO
-                const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c, d0 = smem_u32(S.dout[stg][0]) + dst_c;
-#pragma unroll 4
-                for (int kk = 0; kk < 32; ++kk) {
-                    const int rw = 2 * kk + (lane >> 4);          // row within the warp's 64
-                    const long long off = __shfl_sync(0xffffffffu, kk < 16 ? offA : offB, rw & 31);
-                    const uint32_t so = sw128_offset(64 * w + rw, c & 7);
-                    if (off >= 0) {
-                        cp_async_16(q0 + so, qb + off + c * 16);
-                        cp_async_16(d0 + so, db + off + c * 16);
-                    } else {
-                        st_shared_v4(q0 + so, 0u, 0u, 0u, 0u);
-                        st_shared_v4(d0 + so, 0u, 0u, 0u, 0u);
+                if (*abort_flag && loaded) mbar_wait(&S.kv_full, last_parity, st, 53);
+            }
+        } else if (warp == kMmaWarp) {
+            // -------------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);   // S, dP
+                constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);     // dV^T, dK^T
+                constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
+                int kv_loads = 0, prev_bucket = -1;
+                bool ok = true;
+                // Shared-memory descriptors are computed once; an MMA step adds its byte
+                // offset / 16 to the start-address field (addresses < 2^18 bytes: no carry
+                // out of the 14-bit field).  K-major operands: LBO 16, SBO 1024 (the 64-column
+                // half of a tile is a separate base); MN-major ones: LBO = the stride between
+                // 64-element halves (or 64-key chunks), SBO 1024.
+                constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+                constexpr uint64_t kKHalf = sizeof(S.k[0]) >> 4, kPChunk = sizeof(S.p[0]) >> 4;
+                const uint64_t dq_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);       // Q, K-major
+                const uint64_t dq_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16, 1024);   // dO, K-major
+                const uint64_t dq_k = smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);          // K, K-major
+                const uint64_t dq_v = smem_desc_sw128(smem_u32(S.v[0]), 16, 1024);          // V, K-major
+                const uint64_t dt_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16384, 1024);    // Q^T
+                const uint64_t dt_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16384, 1024); // dO^T
+                const uint64_t dt_p = smem_desc_sw128(smem_u32(S.p[0]), 16384, 1024);       // P (keys x rows)
+                const uint64_t dt_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16384, 1024);     // dS (keys x rows)
+                const uint64_t dk_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16, 1024);        // dS, K-major
+                const uint64_t dk_kmn = smem_desc_sw128(smem_u32(S.k[0]), BS * 128, 1024);  // K, MN-major
+                auto sdp = [&](int i, bool first, int bucket) -> bool {
+                    if (first && bucket != prev_bucket) {
+                        if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
+                        ++kv_loads;
+                        prev_bucket = bucket;
+                    }
+                    const int s = i % NSLOT, stg = i % NQ;
+                    if (!wait(&S.tmem_empty[s], ((i / NSLOT) & 1) ^ 1, 55)) return false;
+                    if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
+                    tc_fence_after();
+                    const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
+                    const uint64_t aq = dq_q + (uint64_t)stg * kQStage, ad = dq_do + (uint64_t)stg * kQStage;
+    #pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                        mma_bf16_ss(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
+                    }
+    #pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                        mma_bf16_ss(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&S.sdp_full[s]);
+                    return true;
+                };
+                auto rest = [&](int i, bool first, bool last, int k, bool release_kv) -> bool {
+                    const int s = i % NSLOT, stg = i % NQ;
+                    if (!wait(&S.pds_full, i & 1, 57)) return false;
+                    if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
+                    tc_fence_after();
+                    const uint64_t aq = dt_q + (uint64_t)stg * kQStage, ad = dt_do + (uint64_t)stg * kQStage;
+    #pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
+                        const uint64_t off = (uint64_t)ks * 128u;
+                        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
+                        mma_bf16_ss(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
+                        mma_bf16_ss(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
+                    }
+    #pragma unroll
+                    for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
+                        mma_bf16_ss(tmem + s * kSlotCols,
+                                    dk_ds + (uint64_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
+                                    dk_kmn + (uint64_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
+                    mma_commit(&S.dq_full[s]);
+                    mma_commit(&S.pds_empty);
+                    mma_commit(&S.q_empty[stg]);
+                    if (last) {
+                        mma_commit(&S.acc_full);
+                        if (release_kv) mma_commit(&S.kv_empty);
+                    }
+                    return true;
+                };
+                // tile sequence with one tile of look-ahead
+                int4 u0 = ld_unit(0), u1 = ld_unit(1);
+                int b0 = ld_bucket(0), b1 = ld_bucket(1);
+                bool have_prev = false;
+                int pi = 0, pk = 0, pb = -1;
+                bool pfirst = false, plast = false;
+                int i = 0;
+                for (int k = 0; k < nk && ok; ++k) {
+                    const int4 d = u0;
+                    const int b = b0;
+                    u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
+                    const int ntl = d.w & 255;
+                    for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
+                        const bool first = tt == 0, last = tt == ntl - 1;
+                        // S/dP of this tile may go ahead of the previous tile's products when
+                        // it needs no other K/V block, Q/dO stage or TMEM slot
+                        const bool early = have_prev && NSLOT == 2 && NQ == 2 && !(first && b != pb);
+                        if (early && !(ok = sdp(i, first, b))) break;
+                        if (have_prev && !(ok = rest(pi, pfirst, plast, pk, plast && b != pb))) break;
+                        if (!early && !(ok = sdp(i, first, b))) break;
+                        have_prev = true;
+                        pi = i; pk = k; pb = b; pfirst = first; plast = last;
                     }
                 }
-                cp_async_commit();
-                issued = i + 1;
+                if (ok && have_prev) rest(pi, pfirst, plast, pk, true);
+                mma_commit(&S.drain);
+                mbar_wait(&S.drain, 0, st, 59);
             }
-        }
-        cp_async_wait_all();   // nothing may still be in flight when the CTA exits
-        if (!stopped && issued > 0 && published == issued - 1) {
-            fence_async_smem();
-            mbar_arrive(&S.q_full[(issued - 1) % NQ]);
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------- K/V producer
-        if (lane == 0) {
-            prefetch_tmap(&kmap);
-            prefetch_tmap(&vmap);
-            int prev = -1, loads = 0, last_parity = 0;
-            bool loaded = false;
-            int4 u0 = ld_unit(0), u1 = ld_unit(1);
-            int b0 = ld_bucket(0), b1 = ld_bucket(1);
-            for (int k = 0; k < nk; ++k) {
-                const int4 d = u0;
-                const int b = b0;
-                u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
-                if (b == prev) continue;
-                prev = b;
-                if (!wait(&S.kv_empty, (loads & 1) ^ 1, 52)) break;
-                const int g = d.w >> 8;
-                mbar_arrive_expect_tx(&S.kv_full, 4u * BS * 128u);
-                tma_load_3d(S.k[0], &kmap, &S.kv_full, 0, g, d.x);
-                tma_load_3d(S.k[1], &kmap, &S.kv_full, 64, g, d.x);
-                tma_load_3d(S.v[0], &vmap, &S.kv_full, 0, g, d.x);
-                tma_load_3d(S.v[1], &vmap, &S.kv_full, 64, g, d.x);
-                last_parity = loads & 1;
-                loaded = true;
-                ++loads;
-            }
-            if (*abort_flag && loaded) mbar_wait(&S.kv_full, last_parity, st, 53);
-        }
-    } else if (warp == 3) {
-        // -------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);   // S, dP
-            constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);     // dV^T, dK^T
-            constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
-            int kv_loads = 0, prev_bucket = -1;
-            bool ok = true;
-            // Shared-memory descriptors are computed once; an MMA step adds its byte
-            // offset / 16 to the start-address field (addresses < 2^18 bytes: no carry
-            // out of the 14-bit field).  K-major operands: LBO 16, SBO 1024 (the 64-column
-            // half of a tile is a separate base); MN-major ones: LBO = the stride between
-            // 64-element halves (or 64-key chunks), SBO 1024.
-            constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
-            constexpr uint64_t kKHalf = sizeof(S.k[0]) >> 4, kPChunk = sizeof(S.p[0]) >> 4;
-            const uint64_t dq_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);       // Q, K-major
-            const uint64_t dq_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16, 1024);   // dO, K-major
-            const uint64_t dq_k = smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);          // K, K-major
-            const uint64_t dq_v = smem_desc_sw128(smem_u32(S.v[0]), 16, 1024);          // V, K-major
-            const uint64_t dt_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16384, 1024);    // Q^T
-            const uint64_t dt_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16384, 1024); // dO^T
-            const uint64_t dt_p = smem_desc_sw128(smem_u32(S.p[0]), 16384, 1024);       // P (keys x rows)
-            const uint64_t dt_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16384, 1024);     // dS (keys x rows)
-            const uint64_t dk_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16, 1024);        // dS, K-major
-            const uint64_t dk_kmn = smem_desc_sw128(smem_u32(S.k[0]), BS * 128, 1024);  // K, MN-major
-            auto sdp = [&](int i, bool first, int bucket) -> bool {
-                if (first && bucket != prev_bucket) {
-                    if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
-                    ++kv_loads;
-                    prev_bucket = bucket;
-                }
-                const int s = i % NSLOT, stg = i % NQ;
-                if (!wait(&S.tmem_empty[s], ((i / NSLOT) & 1) ^ 1, 55)) return false;
-                if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
-                tc_fence_after();
-                const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
-                const uint64_t aq = dq_q + (uint64_t)stg * kQStage, ad = dq_do + (uint64_t)stg * kQStage;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                    const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                    mma_bf16_ss(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                    const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                    mma_bf16_ss(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(&S.sdp_full[s]);
-                return true;
-            };
-            auto rest = [&](int i, bool first, bool last, int k, bool release_kv) -> bool {
-                const int s = i % NSLOT, stg = i % NQ;
-                if (!wait(&S.pds_full, i & 1, 57)) return false;
-                if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
-                tc_fence_after();
-                const uint64_t aq = dt_q + (uint64_t)stg * kQStage, ad = dt_do + (uint64_t)stg * kQStage;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
-                    const uint64_t off = (uint64_t)ks * 128u;
-                    const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                    mma_bf16_ss(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
-                    mma_bf16_ss(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
-                }
-#pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
-                    mma_bf16_ss(tmem + s * kSlotCols,
-                                dk_ds + (uint64_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
-                                dk_kmn + (uint64_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
-                mma_commit(&S.dq_full[s]);
-                mma_commit(&S.pds_empty);
-                mma_commit(&S.q_empty[stg]);
-                if (last) {
-                    mma_commit(&S.acc_full);
-                    if (release_kv) mma_commit(&S.kv_empty);
-                }
-                return true;
-            };
-            // tile sequence with one tile of look-ahead
-            int4 u0 = ld_unit(0), u1 = ld_unit(1);
-            int b0 = ld_bucket(0), b1 = ld_bucket(1);
-            bool have_prev = false;
-            int pi = 0, pk = 0, pb = -1;
-            bool pfirst = false, plast = false;
-            int i = 0;
-            for (int k = 0; k < nk && ok; ++k) {
-                const int4 d = u0;
-                const int b = b0;
-                u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
-                const int ntl = d.w & 255;
-                for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
-                    const bool first = tt == 0, last = tt == ntl - 1;
-                    // S/dP of this tile may go ahead of the previous tile's products when
-                    // it needs no other K/V block, Q/dO stage or TMEM slot
-                    const bool early = have_prev && NSLOT == 2 && NQ == 2 && !(first && b != pb);
-                    if (early && !(ok = sdp(i, first, b))) break;
-                    if (have_prev && !(ok = rest(pi, pfirst, plast, pk, plast && b != pb))) break;
-                    if (!early && !(ok = sdp(i, first, b))) break;
-                    have_prev = true;
-                    pi = i; pk = k; pb = b; pfirst = first; plast = last;
-                }
-            }
-            if (ok && have_prev) rest(pi, pfirst, plast, pk, true);
-            mma_commit(&S.drain);
-            mbar_wait(&S.drain, 0, st, 59);
         }
     } else {
+        reg_alloc<kRegsWg>();
         // ------------------------------------------------- P / dS and the epilogues
         const int wg = (warp - 4) >> 2;
         const int r = (warp & 3) * 32 + lane;            // row = TMEM lane (= d for dV^T/dK^T)
@@ -409,11 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // P and dS of this row, 64 keys per batch of TMEM loads
                     auto pds_chunk = [&](int c64, uint32_t* pk, uint32_t* dk) {
                         float sv[64], dp[64];
-                        tmem_ld32(tS + c64 * 64, sv);
-                        tmem_ld32(tS + c64 * 64 + 32, sv + 32);
-                        tmem_ld32(tdP + c64 * 64, dp);
-                        tmem_ld32(tdP + c64 * 64 + 32, dp + 32);
-                        tmem_wait_ld();
+                        tmem_ld64_sync(tS + c64 * 64, sv);
+                        tmem_ld64_sync(tdP + c64 * 64, dp);
                         const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
                         const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
 #pragma unroll
@@ -469,8 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t tq = tmem + s * kSlotCols + lane_off;
                         float o[128];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) tmem_ld32(tq + c * 32, o + c * 32);
-                        tmem_wait_ld();
+                        for (int c = 0; c < 2; ++c) tmem_ld64_sync(tq + c * 64, o + c * 64);
                         if (my_t >= 0) {
 #pragma unroll
                             for (int q8 = 0; q8 < 16; ++q8) {
@@ -493,9 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                         for (int c32 = 0; c32 < BS / 32; ++c32) {
                             float xv[32], xk[32];
-                            tmem_ld32(tmem + kColDV + lane_off + c32 * 32, xv);
-                            tmem_ld32(tmem + kColDK + lane_off + c32 * 32, xk);
-                            tmem_wait_ld();
+                            tmem_ld32_sync(tmem + kColDV + lane_off + c32 * 32, xv);
+                            tmem_ld32_sync(tmem + kColDK + lane_off + c32 * 32, xk);
 #pragma unroll
                             for (int c = 0; c < 32; ++c) {
                                 const int key = c32 * 32 + c;

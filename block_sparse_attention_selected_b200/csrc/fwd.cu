@@ -441,15 +441,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_w(&S.s_full[wg], ph, 38)) break;
             tc_fence_after();
             float sv[64];
-            tmem_ld32(tS, sv);
-            tmem_ld32(tS + 32, sv + 32);
-            tmem_wait_ld();
+            tmem_ld64_sync(tS, sv);
             if (!nomask) mask64(sv, lim, 0);
             float mx = row_max64(sv);
             if constexpr (BS == 128) {
-                tmem_ld32(tS + 64, sv);
-                tmem_ld32(tS + 96, sv + 32);
-                tmem_wait_ld();
+                tmem_ld64_sync(tS + 64, sv);
                 if (!nomask) mask64(sv, lim, 64);
                 mx = fmaxf(mx, row_max64(sv));
             }
@@ -463,21 +459,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 exp_chunk(sv, mc, l2);
                 l = l2.x + l2.y;
                 pack_chunk(sv, valid ? ldexpf(1.f / l, -ve) : 0.f, pk);
-                tmem_st32(tS, pk);
+                tmem_st32_sync(tS, pk);
             } else {
 #pragma unroll
                 for (int c64 = 0; c64 < 2; ++c64) {    // scores of this 64-key chunk again
-                    tmem_ld32(tS + c64 * 64, sv);
-                    tmem_ld32(tS + c64 * 64 + 32, sv + 32);
-                    tmem_wait_ld();
+                    tmem_ld64_sync(tS + c64 * 64, sv);
                     if (!nomask) mask64(sv, lim, c64 * 64);
                     exp_chunk(sv, mc, l2);
                     pack_chunk(sv, 1.f, pk);
-                    tmem_st32(tS + c64 * 32, pk);
+                    tmem_st32_sync(tS + c64 * 32, pk);
                 }
                 l = l2.x + l2.y;
             }
-            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&S.p_full[wg]);
             if constexpr (BS != 64) {                  // the epilogue applies 2^-e / l
@@ -517,9 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float x[64];
-                tmem_ld32(tO + h * 64, x);
-                tmem_ld32(tO + h * 64 + 32, x + 32);
-                tmem_wait_ld();
+                tmem_ld64_sync(tO + h * 64, x);
                 if (h == 1) {                 // the buffer's O has been read: release it
                     tc_fence_before();
                     mbar_arrive(&S.o_free[ob]);
