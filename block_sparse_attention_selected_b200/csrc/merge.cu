@@ -28,11 +28,14 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: it finds the
-// slot's partial through the position map (row = sorted position * G + head offset)
-// and reads its (lse_j, exponent_j).  The 128 columns are split 4 per lane; partial
-// rows are fetched eight slots at a time so that eight 256-byte reads are in flight.
+// One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: its block
+// index (validity) and its position in the forward tiles (partial row = position * G +
+// head offset) are loaded first; then, in one round of requests, every valid slot's
+// 256-byte partial row (4 columns per lane) and each lane's (lse_j, exponent_j), so
+// that the row costs two dependent memory latencies.
+template <int kS>   // slots held by the warp: 16, 32 or 64 (>= topk)
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p) {
+    constexpr bool kTopk32 = kS <= 32;
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hq) return;
@@ -47,29 +50,30 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
     const int s = seq_of_token(p.cu, p.nseq, t);
     const int qb = (t - __ldg(p.cu + s)) / p.bs;
     const size_t base = ((size_t)t * p.hkv + g) * p.topk;
-    const int32_t* bi = p.bidx + base;
-    const int32_t* pm = p.posmap + base;
-
-    // lane j holds slot j (and j + 32): partial row and (lse_j, exponent_j)
-    float l0 = -CUDART_INF_F, l1 = -CUDART_INF_F, e0 = 0.f, e1 = 0.f;
-    unsigned r0 = 0u, r1 = 0u;
-    if (lane < p.topk && block_valid(__ldg(bi + lane), qb)) {
-        r0 = (unsigned)__ldg(pm + lane) * (unsigned)p.G + (unsigned)hoff;
-        if (r0 < nrows_part) {
-            const float2 m = __ldg(p.part_meta + r0);
-            l0 = m.x;
-            e0 = m.y;
-        }
+    // level 1: validity and partial row of slots lane, lane + 32
+    unsigned r0 = 0xFFFFFFFFu, r1 = 0xFFFFFFFFu;   // partial row, or none
+    if (lane < p.topk && block_valid(__ldg(p.bidx + base + lane), qb)) {
+        const unsigned r = (unsigned)__ldg(p.posmap + base + lane) * (unsigned)p.G + (unsigned)hoff;
+        if (r < nrows_part) r0 = r;
     }
-    if (lane + 32 < p.topk && block_valid(__ldg(bi + lane + 32), qb)) {
-        r1 = (unsigned)__ldg(pm + lane + 32) * (unsigned)p.G + (unsigned)hoff;
-        if (r1 < nrows_part) {
-            const float2 m = __ldg(p.part_meta + r1);
-            l1 = m.x;
-            e1 = m.y;
-        }
+    if (!kTopk32 && lane + 32 < p.topk && block_valid(__ldg(p.bidx + base + lane + 32), qb)) {
+        const unsigned r = (unsigned)__ldg(p.posmap + base + lane + 32) * (unsigned)p.G + (unsigned)hoff;
+        if (r < nrows_part) r1 = r;
     }
-    const float M = warp_max(fmaxf(l0, l1));
+    // level 2: the (lse, exponent) of this lane's slots and every valid partial row
+    float2 m0 = make_float2(-CUDART_INF_F, 0.f), m1 = m0;
+    if (r0 != 0xFFFFFFFFu) m0 = __ldg(p.part_meta + r0);
+    if (r1 != 0xFFFFFFFFu) m1 = __ldg(p.part_meta + r1);
+    const uint2* po = reinterpret_cast<const uint2*>(p.part_o) + lane;
+    const int nslot = min(p.topk, kS);
+    uint2 u[kS];
+#pragma unroll
+    for (int j = 0; j < kS; ++j) {
+        const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
+        u[j] = (j < nslot && rj != 0xFFFFFFFFu) ? __ldg(po + (size_t)rj * (kHeadDim / 4))
+                                                : make_uint2(0u, 0u);
+    }
+    const float M = warp_max(fmaxf(m0.x, m1.x));
     uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
                                            (size_t)row * kHeadDim) + lane;
     if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
@@ -77,31 +81,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_merge(const MergePlan p
         if (lane == 0) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
         return;
     }
-    const float w0 = l0 == -CUDART_INF_F ? 0.f : __expf(l0 - M);
-    const float w1 = l1 == -CUDART_INF_F ? 0.f : __expf(l1 - M);
+    const float w0 = m0.x == -CUDART_INF_F ? 0.f : __expf(m0.x - M);
+    const float w1 = m1.x == -CUDART_INF_F ? 0.f : __expf(m1.x - M);
     const float Lam = warp_sum(w0 + w1);
-    const float s0 = ldexpf(w0, (int)e0), s1 = ldexpf(w1, (int)e1);   // weight x 2^e
+    const float s0 = ldexpf(w0, (int)m0.y), s1 = ldexpf(w1, (int)m1.y);   // weight x 2^e
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint2* po = reinterpret_cast<const uint2*>(p.part_o) + lane;
-    for (int j0 = 0; j0 < p.topk; j0 += 8) {
-        uint2 u[8];
-        float wv[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int j = j0 + k;               // warp-uniform
-            const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
-            const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
-            wv[k] = j < p.topk ? wj : 0.f;
-            u[k] = wv[k] != 0.f ? __ldg(po + (size_t)rj * (kHeadDim / 4)) : make_uint2(0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float2 a = unpack_f16x2(u[k].x), b = unpack_f16x2(u[k].y);
-            acc[0] = fmaf(wv[k], a.x, acc[0]);
-            acc[1] = fmaf(wv[k], a.y, acc[1]);
-            acc[2] = fmaf(wv[k], b.x, acc[2]);
-            acc[3] = fmaf(wv[k], b.y, acc[3]);
-        }
+    for (int j = 0; j < kS; ++j) {
+        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
+        const float2 a = unpack_f16x2(u[j].x), b = unpack_f16x2(u[j].y);
+        acc[0] = fmaf(wj, a.x, acc[0]);
+        acc[1] = fmaf(wj, a.y, acc[1]);
+        acc[2] = fmaf(wj, b.x, acc[2]);
+        acc[3] = fmaf(wj, b.y, acc[3]);
     }
     const float inv = 1.f / Lam;
     *outp = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
@@ -192,7 +184,13 @@ inline unsigned blocks_for(long long rows) {
 }  // namespace
 
 cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
-    k_merge<<<blocks_for((long long)p.T * p.hq), kWarpsPerBlock * 32, 0, stream>>>(p);
+    const unsigned nb = blocks_for((long long)p.T * p.hq);
+    if (p.topk <= 16)
+        k_merge<16><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
+    else if (p.topk <= 32)
+        k_merge<32><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
+    else
+        k_merge<64><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
