@@ -70,6 +70,7 @@ struct alignas(1024) BwdSmem {
     int4 meta[NQ][kTileRows];                 // (token or -1, head, slot, causal limit)
     float rlse[NQ][kTileRows];                // row LSE * log2(e)
     float rdelta[NQ][kTileRows];              // row D = rowsum(dO * O)
+    uint8_t dqs[8][32 * 64];                  // dQ staging: 32 rows x 32 columns per warp
     uint64_t q_full[NQ], q_empty[NQ], meta_full[NQ], meta_empty[NQ];
     uint64_t kv_full, kv_empty;
     uint64_t sdp_full[NSLOT], dq_full[NSLOT], tmem_empty[NSLOT];
@@ -476,24 +477,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = wait(&S.dq_full[s], (i / NSLOT) & 1, 63))) break;
                     tc_fence_after();
                     {
-                        const size_t prow = ((size_t)(my_t < 0 ? 0 : my_t) * p.hq + my_h) * p.topk + my_j;
-                        uint4* dst = reinterpret_cast<uint4*>(
-                            reinterpret_cast<__nv_bfloat16*>(p.part_dq) + prow * kHeadDim);
+                        // per 32-column quarter: scale, bf16, stage the warp's 32 rows (16-byte
+                        // pieces XOR-swizzled so that both phases are conflict-free), then
+                        // write 8 rows x 64 contiguous bytes per warp instruction.  The
+                        // TMEM slot is released as soon as the last quarter is read.
+                        const long long prow =
+                            my_t < 0 ? -1ll : ((long long)my_t * p.hq + my_h) * p.topk + my_j;
+                        uint8_t* const dqb = static_cast<uint8_t*>(p.part_dq);
                         const uint32_t tq = tmem + s * kSlotCols + lane_off;
-                        float o[128];
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) tmem_ld64_sync(tq + c * 64, o + c * 64);
-                        if (my_t >= 0) {
-#pragma unroll
-                            for (int q8 = 0; q8 < 16; ++q8) {
-                                const float* x = o + q8 * 8;
-                                uint4 w;
-                                w.x = pack_bf16x2(x[0] * p.scale, x[1] * p.scale);
-                                w.y = pack_bf16x2(x[2] * p.scale, x[3] * p.scale);
-                                w.z = pack_bf16x2(x[4] * p.scale, x[5] * p.scale);
-                                w.w = pack_bf16x2(x[6] * p.scale, x[7] * p.scale);
-                                dst[q8] = w;
+                        const uint32_t sb = smem_u32(S.dqs[warp - 4]);
+                        const float2 sc2 = make_float2(p.scale, p.scale);
+#pragma unroll 1
+                        for (int qtr = 0; qtr < 4; ++qtr) {
+                            float o[32];
+                            tmem_ld32_sync(tq + qtr * 32, o);
+                            if (qtr == 3) {
+                                tc_fence_before();
+                                mbar_arrive(&S.tmem_empty[s]);
                             }
+#pragma unroll
+                            for (int pc = 0; pc < 4; ++pc) {
+                                uint32_t u[4];
+#pragma unroll
+                                for (int q2 = 0; q2 < 4; ++q2) {
+                                    const float2 z = mul2(make_float2(o[pc * 8 + 2 * q2], o[pc * 8 + 2 * q2 + 1]), sc2);
+                                    u[q2] = pack_bf16x2(z.x, z.y);
+                                }
+                                st_shared_v4(sb + lane * 64 + ((pc ^ ((lane >> 1) & 3)) << 4), u[0], u[1],
+                                             u[2], u[3]);
+                            }
+                            __syncwarp();
+#pragma unroll
+                            for (int it = 0; it < 4; ++it) {
+                                const int rr = it * 8 + (lane >> 2), pc = lane & 3;
+                                const long long gr = __shfl_sync(0xffffffffu, prow, rr);
+                                uint4 v;
+                                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                             : "r"(sb + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4))
+                                             : "memory");
+                                if (gr >= 0)
+                                    *reinterpret_cast<uint4*>(dqb + gr * (kHeadDim * 2) + qtr * 64 + pc * 16) = v;
+                            }
+                            __syncwarp();
                         }
                     }
                     if (tt == ntl - 1) {
@@ -517,8 +543,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                         mbar_arrive(&S.acc_empty);
                     }
-                    tc_fence_before();
-                    mbar_arrive(&S.tmem_empty[s]);
                 }
             }
         }
