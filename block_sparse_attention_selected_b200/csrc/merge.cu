@@ -34,7 +34,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 // 256-byte partial row (4 columns per lane) and each lane's (lse_j, exponent_j), so
 // that the row costs two dependent memory latencies.
 template <int kS>   // slots held by the warp: 16, 32 or 64 (>= topk)
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, 5) k_merge(const MergePlan p) {
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge(const MergePlan p) {
     constexpr bool kTopk32 = kS <= 32;
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
