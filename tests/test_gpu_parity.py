@@ -146,6 +146,24 @@ FWD_FULL = ["fwd_t32k_hq32_g4_k16", "varlen_64k_32k_g1_k16", "train_t32k_hq64_g8
     [f"sweep_t64k_g{g}_bs{bs}_k{k}" for g, bs, k in _SWEEP]
 
 
+@pytest.mark.parametrize("bs", [64, 128])
+def test_fwd_large_v_uses_block_exponent(bs):
+    """V scaled by 2^15 (exact in bf16): |V| reaches ~1.6e5, above fp16's range, so the
+    forward must carry the per-block exponent e > 0 through its fp16 partials."""
+    p = ni.make_problem([1500, 300], hq=8, hkv=2, block_size=bs, topk=8, seed=41,
+                        name=f"large_v_bs{bs}")
+    p.v = (p.v * 32768.0).astype(p.v.dtype)
+    assert np.abs(p.v).max() > 65504.0
+    _, out, lse = _fwd(p)
+    assert torch.isfinite(out.float()).all()
+    # O scales exactly with V (a power of two), LSE does not change: compare O / 2^15
+    # with the standard tolerance (bf16 rounding is invariant under that scaling)
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale)
+    eo = o_excess(f64(out) / 32768.0, o_ref / 32768.0)
+    el = max_abs(f64(lse).T, l_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
+
+
 @pytest.mark.parametrize("wl", FWD_FULL)
 def test_fwd_full_size_sampled(wl):
     p = ni.workload(wl, with_dout=False)
