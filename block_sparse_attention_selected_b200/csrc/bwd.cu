@@ -19,8 +19,8 @@
 //   warps 0-1   loaders: row metadata, cp.async gather of the Q and dO rows (NQ
 //               stages; rows past the list are zero, so they add nothing to dV / dK)
 //   warp 2      TMA producer: K_B and V_B of each unit
-//   warp 3      MMA issuer (one thread): S/dP of tile i+1 go ahead of the dV/dK/dQ
-//               products of tile i when there are two TMEM slots
+//   warp 3      MMA issuer (one thread): S/dP may run one tile ahead of the dV/dK/dQ
+//               products; it issues whichever of the two is ready first
 //   warps 4-7   P / dS, dQ epilogue, unit epilogue of even tiles  } NSLOT = 2: one
 //   warps 8-11  the same for odd tiles                             } TMEM slot each
 //
@@ -303,41 +303,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // out of the 14-bit field).  K-major operands: LBO 16, SBO 1024 (the 64-column
                 // half of a tile is a separate base); MN-major ones: LBO = the stride between
                 // 64-element halves (or 64-key chunks), SBO 1024.
-                constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
-                constexpr uint64_t kKHalf = sizeof(S.k[0]) >> 4, kPChunk = sizeof(S.p[0]) >> 4;
-                const uint64_t dq_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);       // Q, K-major
-                const uint64_t dq_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16, 1024);   // dO, K-major
-                const uint64_t dq_k = smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);          // K, K-major
-                const uint64_t dq_v = smem_desc_sw128(smem_u32(S.v[0]), 16, 1024);          // V, K-major
-                const uint64_t dt_q = smem_desc_sw128(smem_u32(S.q[0][0]), 16384, 1024);    // Q^T
-                const uint64_t dt_do = smem_desc_sw128(smem_u32(S.dout[0][0]), 16384, 1024); // dO^T
-                const uint64_t dt_p = smem_desc_sw128(smem_u32(S.p[0]), 16384, 1024);       // P (keys x rows)
-                const uint64_t dt_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16384, 1024);     // dS (keys x rows)
-                const uint64_t dk_ds = smem_desc_sw128(smem_u32(S.ds[0]), 16, 1024);        // dS, K-major
-                const uint64_t dk_kmn = smem_desc_sw128(smem_u32(S.k[0]), BS * 128, 1024);  // K, MN-major
-                auto sdp = [&](int i, bool first, int bucket) -> bool {
-                    if (first && bucket != prev_bucket) {
+                constexpr uint32_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+                constexpr uint32_t kKHalf = sizeof(S.k[0]) >> 4, kPChunk = sizeof(S.p[0]) >> 4;
+                const uint32_t dq_q = (uint32_t)smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);       // Q, K-major
+                const uint32_t dq_do = (uint32_t)smem_desc_sw128(smem_u32(S.dout[0][0]), 16, 1024);   // dO, K-major
+                const uint32_t dq_k = (uint32_t)smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);          // K, K-major
+                const uint32_t dq_v = (uint32_t)smem_desc_sw128(smem_u32(S.v[0]), 16, 1024);          // V, K-major
+                const uint32_t dt_q = (uint32_t)smem_desc_sw128(smem_u32(S.q[0][0]), 16384, 1024);    // Q^T
+                const uint32_t dt_do = (uint32_t)smem_desc_sw128(smem_u32(S.dout[0][0]), 16384, 1024); // dO^T
+                const uint32_t dt_p = (uint32_t)smem_desc_sw128(smem_u32(S.p[0]), 16384, 1024);       // P (keys x rows)
+                const uint32_t dt_ds = (uint32_t)smem_desc_sw128(smem_u32(S.ds[0]), 16384, 1024);     // dS (keys x rows)
+                const uint32_t dk_ds = (uint32_t)smem_desc_sw128(smem_u32(S.ds[0]), 16, 1024);        // dS, K-major
+                const uint32_t dk_kmn = (uint32_t)smem_desc_sw128(smem_u32(S.k[0]), BS * 128, 1024);  // K, MN-major
+                auto sdp = [&](int i, bool newkv) -> bool {
+                    if (newkv) {
                         if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
                         ++kv_loads;
-                        prev_bucket = bucket;
                     }
                     const int s = i % NSLOT, stg = i % NQ;
                     if (!wait(&S.tmem_empty[s], ((i / NSLOT) & 1) ^ 1, 55)) return false;
                     if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
                     tc_fence_after();
                     const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
-                    const uint64_t aq = dq_q + (uint64_t)stg * kQStage, ad = dq_do + (uint64_t)stg * kQStage;
+                    const uint32_t aq = dq_q + (uint32_t)stg * kQStage, ad = dq_do + (uint32_t)stg * kQStage;
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                        const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
+                        const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                        mma_bf16_ss_lo(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
                     }
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t oa = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                        const uint64_t ob = (uint64_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
+                        const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
+                        mma_bf16_ss_lo(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
                     }
                     mma_commit(&S.sdp_full[s]);
                     return true;
@@ -347,19 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!wait(&S.pds_full, i & 1, 57)) return false;
                     if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
                     tc_fence_after();
-                    const uint64_t aq = dt_q + (uint64_t)stg * kQStage, ad = dt_do + (uint64_t)stg * kQStage;
+                    const uint32_t aq = dt_q + (uint32_t)stg * kQStage, ad = dt_do + (uint32_t)stg * kQStage;
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
-                        const uint64_t off = (uint64_t)ks * 128u;
+                        const uint32_t off = (uint32_t)ks * 128u;
                         const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                        mma_bf16_ss(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
-                        mma_bf16_ss(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
+                        mma_bf16_ss_lo(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
+                        mma_bf16_ss_lo(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
                     }
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
-                        mma_bf16_ss(tmem + s * kSlotCols,
-                                    dk_ds + (uint64_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
-                                    dk_kmn + (uint64_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
+                        mma_bf16_ss_lo(tmem + s * kSlotCols,
+                                    dk_ds + (uint32_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
+                                    dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
                     mma_commit(&S.dq_full[s]);
                     mma_commit(&S.pds_empty);
                     mma_commit(&S.q_empty[stg]);
@@ -369,31 +368,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     return true;
                 };
-                // tile sequence with one tile of look-ahead
-                int4 u0 = ld_unit(0), u1 = ld_unit(1);
-                int b0 = ld_bucket(0), b1 = ld_bucket(1);
-                bool have_prev = false;
-                int pi = 0, pk = 0, pb = -1;
-                bool pfirst = false, plast = false;
-                int i = 0;
-                for (int k = 0; k < nk && ok; ++k) {
-                    const int4 d = u0;
-                    const int b = b0;
-                    u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
-                    const int ntl = d.w & 255;
-                    for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
-                        const bool first = tt == 0, last = tt == ntl - 1;
-                        // S/dP of this tile may go ahead of the previous tile's products when
-                        // it needs no other K/V block, Q/dO stage or TMEM slot
-                        const bool early = have_prev && NSLOT == 2 && NQ == 2 && !(first && b != pb);
-                        if (early && !(ok = sdp(i, first, b))) break;
-                        if (have_prev && !(ok = rest(pi, pfirst, plast, pk, plast && b != pb))) break;
-                        if (!early && !(ok = sdp(i, first, b))) break;
-                        have_prev = true;
-                        pi = i; pk = k; pb = b; pfirst = first; plast = last;
+                // Tiles in order, S/dP running at most one tile ahead of the products (two
+                // TMEM slots, two Q/dO stages).  The issuer serves whichever is ready first:
+                // the products of the oldest tile whose S/dP is done (preferred: they release
+                // its Q/dO stage for the gather two tiles on) or S/dP of the next tile.  A
+                // fixed order would make each stage's release wait for the next tile's gather.
+                // S/dP of a tile that needs a new K/V block waits until every product of the
+                // previous block is issued (a single K/V buffer).
+                int fk = 0, ftt = 0, fi = 0;                 // next S/dP: unit, tile in unit, index
+                int4 fu = ld_unit(0), fu1 = ld_unit(1);
+                int fb = ld_bucket(0), fb1 = ld_bucket(1);
+                int ri = 0;                                  // next products: tile index
+                // pending tiles' flags, even / odd tile index: unit << 3 | release K/V << 2 |
+                // last of unit << 1 | first of unit (registers, no local-memory array)
+                int pend0 = 0, pend1 = 0;
+                long long idle_since = clock64();
+                while (ok && (fk < nk || ri < fi)) {
+                    bool go_r = false, go_s = false, newkv = false;
+                    const int pend = (ri & 1) ? pend1 : pend0;
+                    if (ri < fi)
+                        go_r = mbar_test(&S.pds_full, ri & 1) &&
+                               (!(pend & 1) || mbar_test(&S.acc_empty, ((pend >> 3) & 1) ^ 1));
+                    if (!go_r && fk < nk && fi - ri <= 1) {
+                        newkv = ftt == 0 && fb != prev_bucket;
+                        go_s = (!newkv || ri == fi) &&
+                               mbar_test(&S.q_full[fi % NQ], (fi / NQ) & 1) &&
+                               mbar_test(&S.tmem_empty[fi % NSLOT], ((fi / NSLOT) & 1) ^ 1) &&
+                               (!newkv || mbar_test(&S.kv_full, kv_loads & 1));
+                    }
+                    if (go_r) {
+                        ok = rest(ri, pend & 1, (pend >> 1) & 1, pend >> 3, (pend >> 2) & 1);
+                        ++ri;
+                        idle_since = clock64();
+                    } else if (go_s) {
+                        const int ntl = fu.w & 255;
+                        const bool lst = ftt == ntl - 1;
+                        const int info = (fk << 3) | ((lst && (fk + 1 >= nk || fb1 != fb)) << 2) |
+                                         (lst << 1) | (ftt == 0);
+                        if (fi & 1) pend1 = info; else pend0 = info;
+                        ok = sdp(fi, newkv);
+                        if (newkv) prev_bucket = fb;
+                        ++fi;
+                        if (++ftt == ntl) {
+                            ftt = 0;
+                            ++fk;
+                            fu = fu1; fb = fb1;
+                            fu1 = ld_unit(fk + 1); fb1 = ld_bucket(fk + 1);
+                        }
+                        idle_since = clock64();
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (clock64() - idle_since > kWaitBudgetCycles) {
+                        record_error(st, NSA_ERR_TIMEOUT, 56, blockIdx.x);
+                        *abort_flag = 1;
+                        ok = false;
                     }
                 }
-                if (ok && have_prev) rest(pi, pfirst, plast, pk, true);
                 mma_commit(&S.drain);
                 mbar_wait(&S.drain, 0, st, 59);
             }
