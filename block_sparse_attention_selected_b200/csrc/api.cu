@@ -35,7 +35,7 @@ struct Dims {
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
     size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
-    size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket;
+    size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket, uorder;
     size_t total;
 };
 
@@ -105,6 +105,7 @@ Layout make_layout(const Dims& D, bool bwd) {
         L.part_dkdv = take(sizeof(float) * 2 * (size_t)D.bs * kHeadDim * (size_t)D.units_cap);
         L.udesc = take(sizeof(int4) * (size_t)D.units_cap);
         L.ubucket = take(sizeof(int) * (size_t)D.units_cap);
+        L.uorder = take(sizeof(int) * (size_t)D.units_cap);
     }
     L.total = o;
     return L;
@@ -410,7 +411,9 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     int* ubucket = reinterpret_cast<int*>(c.base + L.ubucket);
     if ((s = cuda_status(launch_unit_desc(c.inv, D.units_cap, udesc, ubucket, stream))) != NSA_OK)
         return s;
-    pm.add(invert_launches(D) + 1);
+    int* uorder = reinterpret_cast<int*>(c.base + L.uorder);
+    if ((s = cuda_status(launch_unit_order(c.st, udesc, uorder, stream))) != NSA_OK) return s;
+    pm.add(invert_launches(D) + 2);
     pm.mark(1);
 
     BwdPlan bp{};
@@ -432,6 +435,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.chunk_tiles = kChunkTiles;
     bp.udesc = udesc;
     bp.ubucket = ubucket;
+    bp.uorder = uorder;
     bp.part_dq = c.base + L.part_o;
     bp.part_dkdv = reinterpret_cast<float*>(c.base + L.part_dkdv);
     bp.st = c.st;

@@ -14,15 +14,16 @@
 // k_dkdv_reduce sums the units of each block in order and k_dq_merge sums the dQ
 // partials of each row over its slots.  No atomics: the result is deterministic.
 //
-// One persistent CTA per SM takes units round-robin; it is warp-specialised:
+// One persistent CTA per SM takes units (largest first, dealt in snake order); it is
+// warp-specialised:
 //
-//   warps 0-1   loaders: row metadata, cp.async gather of the Q and dO rows (NQ
-//               stages; rows past the list are zero, so they add nothing to dV / dK)
-//   warp 2      TMA producer: K_B and V_B of each unit
-//   warp 3      MMA issuer (one thread): S/dP may run one tile ahead of the dV/dK/dQ
-//               products; it issues whichever of the two is ready first
-//   warps 4-7   P / dS, dQ epilogue, unit epilogue of even tiles  } NSLOT = 2: one
-//   warps 8-11  the same for odd tiles                             } TMEM slot each
+//   warps 0-3, 14, 15  loaders: row metadata, cp.async gather of the Q and dO rows (NQ
+//                      stages; rows past the list are zero, so they add nothing to dV / dK)
+//   warp 12            TMA producer: K_B and V_B of each unit
+//   warp 13            MMA issuer (one thread): S/dP may run one tile ahead of the
+//                      dV/dK/dQ products; it issues whichever of the two is ready first
+//   warps 4-11         P / dS, dQ epilogue and unit epilogue of every tile, the two
+//                      warpgroups on one half of the columns each
 //
 // Work descriptors come from k_unit_desc; every wait is bounded (nsa_common.cuh).
 #include <math_constants.h>
@@ -35,7 +36,7 @@ namespace {
 
 // Warp roles (four warpgroups; warp % 4 = TMEM lane quadrant):
 //   warpgroup 0 (warps 0-3)      Q / dO loaders 0-3
-//   warpgroups 1, 2 (4-11)       P / dS and epilogues of even / odd tiles
+//   warpgroups 1, 2 (4-11)       P / dS and the epilogues, half of the columns each
 //   warpgroup 3 (12-15)          TMA producer (12), MMA issuer (13), loaders 4-5 (14, 15)
 // A cp.async gather's throughput grows with the number of issuing warps, and a tile
 // needs 64 KB of gathered Q and dO rows, so six warps load.  setmaxnreg rebalances
@@ -59,8 +60,17 @@ __device__ __forceinline__ void reg_alloc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// TMEM slots of [S | dP] (dQ aliases a slot's first 128 columns): a third slot when
+// it fits next to the dV^T / dK^T accumulators, so that S / dP of tile i + 1 need not
+// wait for the dQ epilogue of tile i - 1, which runs after P / dS of tile i.
+template <int BS, int NSLOT>
+constexpr int bwd_tmem_slots() {
+    return (NSLOT == 2 && 3 * 2 * BS + 2 * BS <= 512) ? 3 : NSLOT;
+}
+
 template <int BS, int NQ, int NSLOT>
 struct alignas(1024) BwdSmem {
+    static constexpr int NTS = bwd_tmem_slots<BS, NSLOT>();
     uint8_t q[NQ][2][kTileRows * 128];        // [stage][64-column half]
     uint8_t dout[NQ][2][kTileRows * 128];
     uint8_t k[2][BS * 128];                   // [half]
@@ -73,7 +83,7 @@ struct alignas(1024) BwdSmem {
     uint8_t dqs[8][32 * 64];                  // dQ staging: 32 rows x 32 columns per warp
     uint64_t q_full[NQ], q_empty[NQ], meta_full[NQ], meta_empty[NQ];
     uint64_t kv_full, kv_empty;
-    uint64_t sdp_full[NSLOT], dq_full[NSLOT], tmem_empty[NSLOT];
+    uint64_t sdp_full[NTS], dq_full[NTS], tmem_empty[NTS];
     uint64_t pds_full, pds_empty, acc_full, acc_empty, drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -103,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     DevStatus* st = p.st;
+    constexpr int NTS = BwdSmem<BS, NQ, NSLOT>::NTS;
 
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
@@ -111,19 +122,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S.q_full[i], kLoaderThreads);
             mbar_init(&S.q_empty[i], 1);
             mbar_init(&S.meta_full[i], kLoaderThreads);
-            mbar_init(&S.meta_empty[i], kWgThreads);
+            mbar_init(&S.meta_empty[i], 2 * kWgThreads);
         }
-        for (int i = 0; i < NSLOT; ++i) {
+        for (int i = 0; i < NTS; ++i) {
             mbar_init(&S.sdp_full[i], 1);
             mbar_init(&S.dq_full[i], 1);
-            mbar_init(&S.tmem_empty[i], kWgThreads);
+            mbar_init(&S.tmem_empty[i], 2 * kWgThreads);
         }
         mbar_init(&S.kv_full, 1);
         mbar_init(&S.kv_empty, 1);
-        mbar_init(&S.pds_full, kWgThreads);
+        mbar_init(&S.pds_full, 2 * kWgThreads);
         mbar_init(&S.pds_empty, 1);
         mbar_init(&S.acc_full, 1);
-        mbar_init(&S.acc_empty, kWgThreads);
+        mbar_init(&S.acc_empty, 2 * kWgThreads);
         mbar_init(&S.drain, 1);
         fence_barrier_init();
     }
@@ -138,10 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t tmem = S.tmem_base;
     const int nunits = S.nunits;
-    const int nk = (!S.abort_flag && (int)blockIdx.x < nunits)
-                       ? (nunits - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
-                       : 0;
-    auto unit_of = [&](int k) { return (int)blockIdx.x + k * (int)gridDim.x; };
+    // units dealt in snake order over the list sorted by tile count (k_unit_order)
+    const int ncta = (int)gridDim.x, cta = (int)blockIdx.x;
+    auto rank_of = [&](int k) { return k * ncta + ((k & 1) ? ncta - 1 - cta : cta); };
+    const int nfull = nunits / ncta;
+    const int nk = S.abort_flag ? 0 : nfull + (rank_of(nfull) < nunits ? 1 : 0);
+    auto unit_of = [&](int k) { return __ldg(p.uorder + rank_of(k)); };
     auto ld_unit = [&](int k) {
         return k < nk ? __ldg(p.udesc + unit_of(k)) : make_int4(0, 0, 0, 0);
     };
@@ -158,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // TMEM columns: per slot [S | dP] (2*BS, dQ aliases its first 128), then dV^T, dK^T
     constexpr int kSlotCols = 2 * BS;
-    constexpr int kColDV = NSLOT * kSlotCols;
+    constexpr int kColDV = NTS * kSlotCols;
     constexpr int kColDK = kColDV + BS;
     static_assert(kColDK + BS <= 512, "TMEM budget");
 
@@ -175,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // copy step k the loader moves rows R w + 2k and R w + 2k + 1 (lane l: 16-byte
             // chunk l % 16 of row R w + 2k + l / 16, a 512-byte coalesced read); rows past
             // the list are zeroed, so that they add nothing to dV and dK.  Tile i - 1's copies are published
-            // (wait, fence, arrive on q_full) after tile i's metadata is out and before the
-            // loader waits for tile i's stage: that stage is released by the dV / dK / dQ
-            // products of tile i - 2, which the MMA issuer may queue behind S / dP of tile
-            // i - 1, so publishing later than this could wait in a cycle.
+            // (wait, fence, arrive on q_full) once tile i's row data is requested, before the
+            // loader waits for tile i's metadata slot and stage: that stage is released by the
+            // products of tile i - 2, which may wait for S / dP of tile i - 1, so publishing
+            // after that wait could close a cycle.
             const int w = li;
             const int nr_w = min(kRowsPerLoader, kTileRows - kRowsPerLoader * w);   // rows of this loader
             const uint8_t* qb = static_cast<const uint8_t*>(p.q);
@@ -217,6 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         lA = __ldg(p.lse + (size_t)mA.y * p.T + mA.x) * kLog2e;
                         dA = __ldg(p.delta + (size_t)mA.y * p.T + mA.x);
                     }
+                    if (i > 0) {                       // publish tile i - 1 (the loads above land meanwhile)
+                        cp_async_wait_all();
+                        fence_async_smem();
+                        mbar_arrive(&S.q_full[(i - 1) % NQ]);
+                        published = i;
+                    }
                     if (!__all_sync(0xffffffffu, wait(&S.meta_empty[stg], ph_empty, 50))) {
                         stopped = true;
                         break;
@@ -227,12 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         S.rdelta[stg][rA] = dA;
                     }
                     mbar_arrive(&S.meta_full[stg]);
-                    if (i > 0) {                       // publish tile i - 1
-                        cp_async_wait_all();
-                        fence_async_smem();
-                        mbar_arrive(&S.q_full[(i - 1) % NQ]);
-                        published = i;
-                    }
                     if (!__all_sync(0xffffffffu, wait(&S.q_empty[stg], ph_empty, 51))) {
                         stopped = true;
                         break;
@@ -320,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!wait(&S.kv_full, kv_loads & 1, 54)) return false;
                         ++kv_loads;
                     }
-                    const int s = i % NSLOT, stg = i % NQ;
-                    if (!wait(&S.tmem_empty[s], ((i / NSLOT) & 1) ^ 1, 55)) return false;
+                    const int s = i % NTS, stg = i % NQ;
+                    if (!wait(&S.tmem_empty[s], ((i / NTS) & 1) ^ 1, 55)) return false;
                     if (!wait(&S.q_full[stg], (i / NQ) & 1, 56)) return false;
                     tc_fence_after();
                     const uint32_t tS = tmem + s * kSlotCols, tdP = tS + BS;
@@ -342,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return true;
                 };
                 auto rest = [&](int i, bool first, bool last, int k, bool release_kv) -> bool {
-                    const int s = i % NSLOT, stg = i % NQ;
+                    const int s = i % NTS, stg = i % NQ;
                     if (!wait(&S.pds_full, i & 1, 57)) return false;
                     if (first && !wait(&S.acc_empty, (k & 1) ^ 1, 58)) return false;
                     tc_fence_after();
@@ -354,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ss_lo(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
                         mma_bf16_ss_lo(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
                     }
+                    mma_commit(&S.q_empty[stg]);   // the stage is free once dV / dK have read it
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
                         mma_bf16_ss_lo(tmem + s * kSlotCols,
@@ -361,7 +375,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
                     mma_commit(&S.dq_full[s]);
                     mma_commit(&S.pds_empty);
-                    mma_commit(&S.q_empty[stg]);
                     if (last) {
                         mma_commit(&S.acc_full);
                         if (release_kv) mma_commit(&S.kv_empty);
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         newkv = ftt == 0 && fb != prev_bucket;
                         go_s = (!newkv || ri == fi) &&
                                mbar_test(&S.q_full[fi % NQ], (fi / NQ) & 1) &&
-                               mbar_test(&S.tmem_empty[fi % NSLOT], ((fi / NSLOT) & 1) ^ 1) &&
+                               mbar_test(&S.tmem_empty[fi % NTS], ((fi / NTS) & 1) ^ 1) &&
                                (!newkv || mbar_test(&S.kv_full, kv_loads & 1));
                     }
                     if (go_r) {
@@ -431,151 +444,157 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         reg_alloc<kRegsWg>();
         // ------------------------------------------------- P / dS and the epilogues
+        // Both warpgroups work on every tile, warpgroup wg on half of its columns: keys
+        // [wg BS/2, (wg + 1) BS/2) of P / dS and of the unit's dV / dK, columns
+        // [64 wg, 64 wg + 64) of dQ.  Row r = TMEM lane (= d for dV^T / dK^T).  With two
+        // TMEM slots the dQ epilogue of tile i - 1 runs after P / dS of tile i is stored,
+        // so that the products of tile i can follow those of tile i - 1 at once.
+        constexpr int kKeysWg = BS / 2;
+        constexpr bool kDefer = NSLOT == 2;
         const int wg = (warp - 4) >> 2;
-        const int r = (warp & 3) * 32 + lane;            // row = TMEM lane (= d for dV^T/dK^T)
+        const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        if (wg < NSLOT) {
-            int4 u0 = ld_unit(0), u1 = ld_unit(1);
-            int i = 0;
-            bool ok = true;
-            for (int k = 0; k < nk && ok; ++k) {
-                const int4 d = u0;
-                u0 = u1; u1 = ld_unit(k + 2);
-                const int ntl = d.w & 255;
-                for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
-                    if (i % NSLOT != wg) continue;
-                    const int stg = i % NQ, s = i % NSLOT;
-                    if (!(ok = wait(&S.meta_full[stg], (i / NQ) & 1, 60))) break;
-                    const int4 m = S.meta[stg][r];
-                    const float lse2 = S.rlse[stg][r], delta = S.rdelta[stg][r];
-                    mbar_arrive(&S.meta_empty[stg]);
-                    const int my_t = m.x, my_h = m.y, my_j = m.z, my_lim = m.w;
-                    if (!(ok = wait(&S.sdp_full[s], (i / NSLOT) & 1, 61))) break;
-                    tc_fence_after();
-                    const uint32_t tS = tmem + s * kSlotCols + lane_off, tdP = tS + BS;
-                    // P and dS of this row, 64 keys per batch of TMEM loads
-                    auto pds_chunk = [&](int c64, uint32_t* pk, uint32_t* dk) {
-                        float sv[64], dp[64];
-                        tmem_ld64_sync(tS + c64 * 64, sv);
-                        tmem_ld64_sync(tdP + c64 * 64, dp);
-                        const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
-                        const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
-#pragma unroll
-                        for (int c = 0; c < 64; c += 2) {
-                            const int key = c64 * 64 + c;
-                            float2 x = fma2(make_float2(sv[c], sv[c + 1]), c2, nl2);
-                            x.x = key <= my_lim ? ex2_approx(x.x) : 0.f;
-                            x.y = key + 1 <= my_lim ? ex2_approx(x.y) : 0.f;
-                            const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
-                            pk[c / 2] = pack_bf16x2(x.x, x.y);
-                            dk[c / 2] = pack_bf16x2(ds.x, ds.y);
-                        }
-                    };
-                    auto store_chunk = [&](int c64, const uint32_t* pk, const uint32_t* dk) {
-#pragma unroll
-                        for (int pc = 0; pc < 8; ++pc) {   // 16-byte pieces of 8 keys
-                            st_shared_v4(smem_u32(S.p[c64]) + sw128_offset(r, pc), pk[pc * 4],
-                                         pk[pc * 4 + 1], pk[pc * 4 + 2], pk[pc * 4 + 3]);
-                            st_shared_v4(smem_u32(S.ds[c64]) + sw128_offset(r, pc), dk[pc * 4],
-                                         dk[pc * 4 + 1], dk[pc * 4 + 2], dk[pc * 4 + 3]);
-                        }
-                    };
-                    if constexpr (NSLOT == 1) {
-                        // single slot: nothing to overlap, stream each 64-key chunk out
-                        if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;
+        uint8_t* const dqb = static_cast<uint8_t*>(p.part_dq);
+        const uint32_t sb = smem_u32(S.dqs[warp - 4]);
+        const float2 sc2 = make_float2(p.scale, p.scale);
+        // dQ partial of tile j (row r, this warpgroup's 64 columns); then, after the
+        // unit's last tile, dV and scale*dK of its block as fp32 [2][BS][128]
+        auto epilogue = [&](int j, long long prow, bool unit_last, int k) -> bool {
+            const int s = j % NTS;
+            if (!wait(&S.dq_full[s], (j / NTS) & 1, 63)) return false;
+            tc_fence_after();
+            const uint32_t tq = tmem + s * kSlotCols + lane_off;
+            // per 32-column quarter: scale, bf16, stage the warp's 32 rows (16-byte pieces
+            // XOR-swizzled so that both phases are conflict-free), then write 8 rows x 64
+            // contiguous bytes per warp instruction.  The TMEM slot is released as soon as
+            // the warpgroup's last quarter is read.
 #pragma unroll 1
-                        for (int c64 = 0; c64 < BS / 64; ++c64) {
-                            uint32_t pk[32], dk[32];
-                            pds_chunk(c64, pk, dk);
-                            store_chunk(c64, pk, dk);
-                        }
-                        tc_fence_before();
+            for (int h = 0; h < 2; ++h) {
+                const int qtr = 2 * wg + h;
+                float o[32];
+                tmem_ld32_sync(tq + qtr * 32, o);
+                if (h == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&S.tmem_empty[s]);
+                }
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc) {
+                    uint32_t u[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float2 z = mul2(make_float2(o[pc * 8 + 2 * q2], o[pc * 8 + 2 * q2 + 1]), sc2);
+                        u[q2] = pack_bf16x2(z.x, z.y);
+                    }
+                    st_shared_v4(sb + lane * 64 + ((pc ^ ((lane >> 1) & 3)) << 4), u[0], u[1], u[2], u[3]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int rr = it * 8 + (lane >> 2), pc = lane & 3;
+                    const long long gr = __shfl_sync(0xffffffffu, prow, rr);
+                    uint4 v;
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(sb + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4))
+                                 : "memory");
+                    if (gr >= 0)
+                        *reinterpret_cast<uint4*>(dqb + gr * (kHeadDim * 2) + qtr * 64 + pc * 16) = v;
+                }
+                __syncwarp();
+            }
+            if (unit_last) {
+                if (!wait(&S.acc_full, k & 1, 64)) return false;
+                tc_fence_after();
+                float* dvp = p.part_dkdv + (size_t)unit_of(k) * 2 * BS * kHeadDim;
+                float* dkp = dvp + (size_t)BS * kHeadDim;
+#pragma unroll 1
+                for (int c32 = wg * (kKeysWg / 32); c32 < (wg + 1) * (kKeysWg / 32); ++c32) {
+                    float xv[32], xk[32];
+                    tmem_ld32_sync(tmem + kColDV + lane_off + c32 * 32, xv);
+                    tmem_ld32_sync(tmem + kColDK + lane_off + c32 * 32, xk);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int key = c32 * 32 + c;
+                        dvp[(size_t)key * kHeadDim + r] = xv[c];
+                        dkp[(size_t)key * kHeadDim + r] = xk[c] * p.scale;
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&S.acc_empty);
+            }
+            return true;
+        };
+        int4 u0 = ld_unit(0), u1 = ld_unit(1);
+        int i = 0;
+        bool ok = true;
+        long long prev_prow = -1;
+        bool prev_last = false;
+        int prev_k = 0;
+        for (int k = 0; k < nk && ok; ++k) {
+            const int4 d = u0;
+            u0 = u1; u1 = ld_unit(k + 2);
+            const int ntl = d.w & 255;
+            for (int tt = 0; tt < ntl && ok; ++tt, ++i) {
+                const int stg = i % NQ, s = i % NTS;
+                if (!(ok = wait(&S.meta_full[stg], (i / NQ) & 1, 60))) break;
+                const int4 m = S.meta[stg][r];
+                const float lse2 = S.rlse[stg][r], delta = S.rdelta[stg][r];
+                mbar_arrive(&S.meta_empty[stg]);
+                const int my_lim = m.w;
+                const long long prow = m.x < 0 ? -1ll : ((long long)m.x * p.hq + m.y) * p.topk + m.z;
+                if (!(ok = wait(&S.sdp_full[s], (i / NTS) & 1, 61))) break;
+                tc_fence_after();
+                // P and dS of this row over the warpgroup's keys, into registers while the
+                // products of the previous tile may still read the P / dS tile
+                const uint32_t tS = tmem + s * kSlotCols + lane_off + wg * kKeysWg, tdP = tS + BS;
+                uint32_t pk[kKeysWg / 2], dk[kKeysWg / 2];
+                {
+                    float sv[kKeysWg], dp[kKeysWg];
+                    if constexpr (kKeysWg == 32) {
+                        tmem_ld32_sync(tS, sv);
+                        tmem_ld32_sync(tdP, dp);
                     } else {
-                        // two slots: compute the row while the previous tile's products
-                        // still read the P / dS tile, then store it
-                        uint32_t pk[BS / 2], dk[BS / 2];
-#pragma unroll
-                        for (int c64 = 0; c64 < BS / 64; ++c64) pds_chunk(c64, pk + c64 * 32, dk + c64 * 32);
-                        tc_fence_before();
-                        if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;
-#pragma unroll
-                        for (int c64 = 0; c64 < BS / 64; ++c64) store_chunk(c64, pk + c64 * 32, dk + c64 * 32);
+                        tmem_ld64_sync(tS, sv);
+                        tmem_ld64_sync(tdP, dp);
                     }
-                    fence_async_smem();
-                    mbar_arrive(&S.pds_full);
-                    // dQ partial of this row and slot
-                    if (!(ok = wait(&S.dq_full[s], (i / NSLOT) & 1, 63))) break;
-                    tc_fence_after();
-                    {
-                        // per 32-column quarter: scale, bf16, stage the warp's 32 rows (16-byte
-                        // pieces XOR-swizzled so that both phases are conflict-free), then
-                        // write 8 rows x 64 contiguous bytes per warp instruction.  The
-                        // TMEM slot is released as soon as the last quarter is read.
-                        const long long prow =
-                            my_t < 0 ? -1ll : ((long long)my_t * p.hq + my_h) * p.topk + my_j;
-                        uint8_t* const dqb = static_cast<uint8_t*>(p.part_dq);
-                        const uint32_t tq = tmem + s * kSlotCols + lane_off;
-                        const uint32_t sb = smem_u32(S.dqs[warp - 4]);
-                        const float2 sc2 = make_float2(p.scale, p.scale);
-#pragma unroll 1
-                        for (int qtr = 0; qtr < 4; ++qtr) {
-                            float o[32];
-                            tmem_ld32_sync(tq + qtr * 32, o);
-                            if (qtr == 3) {
-                                tc_fence_before();
-                                mbar_arrive(&S.tmem_empty[s]);
-                            }
+                    const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+                    const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
 #pragma unroll
-                            for (int pc = 0; pc < 4; ++pc) {
-                                uint32_t u[4];
-#pragma unroll
-                                for (int q2 = 0; q2 < 4; ++q2) {
-                                    const float2 z = mul2(make_float2(o[pc * 8 + 2 * q2], o[pc * 8 + 2 * q2 + 1]), sc2);
-                                    u[q2] = pack_bf16x2(z.x, z.y);
-                                }
-                                st_shared_v4(sb + lane * 64 + ((pc ^ ((lane >> 1) & 3)) << 4), u[0], u[1],
-                                             u[2], u[3]);
-                            }
-                            __syncwarp();
-#pragma unroll
-                            for (int it = 0; it < 4; ++it) {
-                                const int rr = it * 8 + (lane >> 2), pc = lane & 3;
-                                const long long gr = __shfl_sync(0xffffffffu, prow, rr);
-                                uint4 v;
-                                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                                             : "r"(sb + rr * 64 + ((pc ^ ((rr >> 1) & 3)) << 4))
-                                             : "memory");
-                                if (gr >= 0)
-                                    *reinterpret_cast<uint4*>(dqb + gr * (kHeadDim * 2) + qtr * 64 + pc * 16) = v;
-                            }
-                            __syncwarp();
-                        }
+                    for (int c = 0; c < kKeysWg; c += 2) {
+                        const int key = wg * kKeysWg + c;
+                        float2 x = fma2(make_float2(sv[c], sv[c + 1]), c2, nl2);
+                        x.x = key <= my_lim ? ex2_approx(x.x) : 0.f;
+                        x.y = key + 1 <= my_lim ? ex2_approx(x.y) : 0.f;
+                        const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
+                        pk[c / 2] = pack_bf16x2(x.x, x.y);
+                        dk[c / 2] = pack_bf16x2(ds.x, ds.y);
                     }
-                    if (tt == ntl - 1) {
-                        // unit epilogue: dV and scale*dK of the block as fp32 [2][BS][128]
-                        if (!(ok = wait(&S.acc_full, k & 1, 64))) break;
-                        tc_fence_after();
-                        float* dvp = p.part_dkdv + (size_t)unit_of(k) * 2 * BS * kHeadDim;
-                        float* dkp = dvp + (size_t)BS * kHeadDim;
-#pragma unroll 1
-                        for (int c32 = 0; c32 < BS / 32; ++c32) {
-                            float xv[32], xk[32];
-                            tmem_ld32_sync(tmem + kColDV + lane_off + c32 * 32, xv);
-                            tmem_ld32_sync(tmem + kColDK + lane_off + c32 * 32, xk);
+                }
+                tc_fence_before();
+                if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int key = c32 * 32 + c;
-                                dvp[(size_t)key * kHeadDim + r] = xv[c];
-                                dkp[(size_t)key * kHeadDim + r] = xk[c] * p.scale;
-                            }
-                        }
-                        tc_fence_before();
-                        mbar_arrive(&S.acc_empty);
-                    }
+                for (int pc = 0; pc < kKeysWg / 8; ++pc) {   // 16-byte pieces of 8 keys
+                    const int gp = wg * (kKeysWg / 8) + pc;
+                    const int c64 = gp >> 3, pp = gp & 7;
+                    st_shared_v4(smem_u32(S.p[c64]) + sw128_offset(r, pp), pk[pc * 4], pk[pc * 4 + 1],
+                                 pk[pc * 4 + 2], pk[pc * 4 + 3]);
+                    st_shared_v4(smem_u32(S.ds[c64]) + sw128_offset(r, pp), dk[pc * 4], dk[pc * 4 + 1],
+                                 dk[pc * 4 + 2], dk[pc * 4 + 3]);
+                }
+                fence_async_smem();
+                mbar_arrive(&S.pds_full);
+                const bool last = tt == ntl - 1;
+                if constexpr (kDefer) {
+                    if (i > 0 && !(ok = epilogue(i - 1, prev_prow, prev_last, prev_k))) break;
+                    prev_prow = prow;
+                    prev_last = last;
+                    prev_k = k;
+                } else {
+                    if (!(ok = epilogue(i, prow, last, k))) break;
                 }
             }
         }
+        if (kDefer && ok && i > 0) epilogue(i - 1, prev_prow, prev_last, prev_k);
     }
 
     tc_fence_before();

@@ -388,6 +388,31 @@ __global__ void k_unit_desc(const DevStatus* st, const int32_t* chunk_off, const
     ubucket[u] = bucket;
 }
 
+// Units sorted by tile count, largest first (a counting sort in one block; units of
+// equal count in any order).  The backward tile kernel deals them out in snake order
+// (round k: CTA c takes rank k P + c for even k and k P + P - 1 - c for odd k), which
+// evens out the tiles per CTA; which CTA runs a unit does not change its arithmetic.
+__global__ void __launch_bounds__(1024) k_unit_order(const DevStatus* st, const int4* udesc,
+                                                     int* uorder) {
+    __shared__ int hist[256];
+    if (st->code != 0) return;
+    const int n = st->nchunks;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int u = threadIdx.x; u < n; u += blockDim.x) atomicAdd(&hist[udesc[u].w & 255], 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {   // exclusive prefix from the largest count down
+        int acc = 0;
+        for (int c = 255; c >= 0; --c) {
+            const int h = hist[c];
+            hist[c] = acc;
+            acc += h;
+        }
+    }
+    __syncthreads();
+    for (int u = threadIdx.x; u < n; u += blockDim.x) uorder[atomicAdd(&hist[udesc[u].w & 255], 1)] = u;
+}
+
 // 10. Position map from the forward tiles: the k-th token of tile tau, entry
 //     (t, g, j), gets posmap[(t * hkv + g) * topk + j] = tau * tpt + k; its partial
 //     rows are posmap * G + head offset, inside the tile's own 128-row slot.
@@ -491,6 +516,12 @@ cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* ude
     k_unit_desc<<<(unsigned)((units_cap + 255) / 256), 256, 0, stream>>>(
         p.st, p.chunk_off, p.tile_off, p.offsets, p.blkoff, p.cu, p.nseq, p.hkv,
         p.tokens_per_tile, p.chunk_tiles, p.bs, udesc, ubucket);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unit_order(const DevStatus* st, const int4* udesc, int* uorder,
+                              cudaStream_t stream) {
+    k_unit_order<<<1, 1024, 0, stream>>>(st, udesc, uorder);
     return cudaGetLastError();
 }
 

@@ -63,6 +63,9 @@ cudaError_t launch_posmap(const InvertPlan& p, const WindowPlan& w, int32_t* pos
                           cudaStream_t stream);
 cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
                              cudaStream_t stream);
+// Units ordered by tile count, largest first, for the snake deal of the backward kernel.
+cudaError_t launch_unit_order(const DevStatus* st, const int4* udesc, int* uorder,
+                              cudaStream_t stream);
 
 struct FwdPlan {
     const void* q;
@@ -126,6 +129,7 @@ struct BwdPlan {
     int chunk_tiles;
     const int4* udesc;       // per unit: (key0, first entry, list end, ntiles | g << 8)
     const int* ubucket;      // per unit: g * NB + B
+    const int* uorder;       // units by tile count, largest first (k_unit_order)
     void* part_dq;           // bf16 [T * hq * topk, 128]
     float* part_dkdv;        // fp32 [chunks, 2, bs, 128]
     DevStatus* st;
