@@ -305,7 +305,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else if (warp == kMmaWarp) {
             // -------------------------------------------------------------- MMA issuer
-            if (lane == 0) {
+            // The whole warp runs the issue loop (warp-uniform state and decisions); one
+            // elected lane executes the tcgen05 instructions.
+            {
+                const uint32_t elected = elect_one();
                 constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);   // S, dP
                 constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);     // dV^T, dK^T
                 constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
@@ -343,15 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss_lo(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u);
+                        mma_bf16_ss_lo_e(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss_lo(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u);
+                        mma_bf16_ss_lo_e(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
-                    mma_commit(&S.sdp_full[s]);
+                    mma_commit_e(&S.sdp_full[s], elected);
                     return true;
                 };
                 auto rest = [&](int i, bool first, bool last, int k, bool release_kv) -> bool {
@@ -364,20 +367,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
                         const uint32_t off = (uint32_t)ks * 128u;
                         const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                        mma_bf16_ss_lo(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc);
-                        mma_bf16_ss_lo(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc);
+                        mma_bf16_ss_lo_e(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc, elected);
+                        mma_bf16_ss_lo_e(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc, elected);
                     }
-                    mma_commit(&S.q_empty[stg]);   // the stage is free once dV / dK have read it
+                    mma_commit_e(&S.q_empty[stg], elected);   // the stage is free once dV / dK have read it
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
-                        mma_bf16_ss_lo(tmem + s * kSlotCols,
+                        mma_bf16_ss_lo_e(tmem + s * kSlotCols,
                                     dk_ds + (uint32_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
-                                    dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u);
-                    mma_commit(&S.dq_full[s]);
-                    mma_commit(&S.pds_empty);
+                                    dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u, elected);
+                    mma_commit_e(&S.dq_full[s], elected);
+                    mma_commit_e(&S.pds_empty, elected);
                     if (last) {
-                        mma_commit(&S.acc_full);
-                        if (release_kv) mma_commit(&S.kv_empty);
+                        mma_commit_e(&S.acc_full, elected);
+                        if (release_kv) mma_commit_e(&S.kv_empty, elected);
                     }
                     return true;
                 };
@@ -409,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                mbar_test(&S.tmem_empty[fi % NTS], ((fi / NTS) & 1) ^ 1) &&
                                (!newkv || mbar_test(&S.kv_full, kv_loads & 1));
                     }
+                    go_r = __shfl_sync(0xffffffffu, go_r, 0);
+                    go_s = __shfl_sync(0xffffffffu, go_s, 0);
                     if (go_r) {
                         ok = rest(ri, pend & 1, (pend >> 1) & 1, pend >> 3, (pend >> 2) & 1);
                         ++ri;
@@ -429,15 +434,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             fu1 = ld_unit(fk + 1); fb1 = ld_bucket(fk + 1);
                         }
                         idle_since = clock64();
-                    } else if (*abort_flag) {
+                    } else if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
                         ok = false;
-                    } else if (clock64() - idle_since > kWaitBudgetCycles) {
-                        record_error(st, NSA_ERR_TIMEOUT, 56, blockIdx.x);
+                    } else if (__shfl_sync(0xffffffffu, clock64() - idle_since > kWaitBudgetCycles, 0)) {
+                        if (lane == 0) record_error(st, NSA_ERR_TIMEOUT, 56, blockIdx.x);
                         *abort_flag = 1;
                         ok = false;
                     }
                 }
-                mma_commit(&S.drain);
+                mma_commit_e(&S.drain, elected);
                 mbar_wait(&S.drain, 0, st, 59);
             }
         }

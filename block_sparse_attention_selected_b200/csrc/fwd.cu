@@ -27,7 +27,8 @@
 //   warps 0-1    Q loaders: coalesced cp.async gather (two 256-byte rows per warp
 //                instruction) into the 128B-swizzled Q tile, kNQ stages
 //   warp 2       TMA producer: K_B and V_B (128B swizzle) into NKV stages
-//   warp 3       MMA issuer (one thread): S(i+1) is issued before PV(i)
+//   warp 17      MMA issuer (one elected lane of a warp-uniform loop): S(i+1) is
+//                issued before PV(i)
 //   warps 4-7    softmax of even tiles  } TMEM slot 0 / 1: S (P) and O accumulators
 //   warps 8-11   softmax of odd tiles   }
 //   warps 12-15  epilogue of every tile: O from TMEM, scale, fp16, store
@@ -289,7 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else if (warp == kMmaWarp) {
             // -------------------------------------------------------------- MMA issuer
-            if (lane == 0) {
+            // The whole warp runs the issue loop (warp-uniform state); one elected lane
+            // executes the tcgen05 instructions.
+            {
+                const uint32_t elected = elect_one();
                 constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);
                 constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
                 int kv_uses = 0, prev_bucket = -1, cur = 0;
@@ -301,11 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // byte offset / 16 to the start-address field (addresses stay < 2^18 bytes,
                 // so the 14-bit field never carries).  This keeps the issuing thread's
                 // instruction count per MMA small: it shares its SMSP with busy warps.
-                constexpr uint64_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
-                constexpr uint64_t kKvStage = sizeof(S.kv[0]) >> 4, kKvHalf = sizeof(S.kv[0][0][0]) >> 4;
-                const uint64_t q_desc0 = smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
-                const uint64_t k_desc0 = smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
-                const uint64_t v_desc0 = smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
+                constexpr uint32_t kQStage = sizeof(S.q[0]) >> 4, kQHalf = sizeof(S.q[0][0]) >> 4;
+                constexpr uint32_t kKvStage = sizeof(S.kv[0]) >> 4, kKvHalf = sizeof(S.kv[0][0][0]) >> 4;
+                const uint32_t q_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
+                const uint32_t k_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
+                const uint32_t v_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
                 // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
                 // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
                 // run in issue order.  s_full also tells the loaders that the Q stage (i % 2)
@@ -322,15 +326,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
                     tc_fence_after();
                     const uint32_t tS = tmem + slot * BS;
-                    const uint64_t a0 = q_desc0 + (uint64_t)stg * kQStage;
-                    const uint64_t b0 = k_desc0 + (uint64_t)cur * kKvStage;
+                    const uint32_t a0 = q_desc0 + (uint32_t)stg * kQStage;
+                    const uint32_t b0 = k_desc0 + (uint32_t)cur * kKvStage;
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t off = (uint64_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
-                        const uint64_t offk = (uint64_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
-                        mma_bf16_ss(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u);
+                        const uint32_t off = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
+                        const uint32_t offk = (uint32_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
+                        mma_bf16_ss_lo_e(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
-                    mma_commit(&S.s_full[slot]);
+                    mma_commit_e(&S.s_full[slot], elected);
                     return true;
                 };
                 // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
@@ -342,13 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
                     const int kvs = kvs_of[slot];
-                    const uint64_t b0 = v_desc0 + (uint64_t)kvs * kKvStage;
+                    const uint32_t b0 = v_desc0 + (uint32_t)kvs * kKvStage;
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)    // 16 keys = 2048 bytes per step
-                        mma_bf16_ts(tO, tS + (uint32_t)ks * 8u, b0 + (uint64_t)ks * 128u, kIdescO,
-                                    ks > 0 ? 1u : 0u);
-                    mma_commit(&S.o_full[ob]);
-                    if (release_kv) mma_commit(&S.kv_empty[kvs]);
+                        mma_bf16_ts_lo_e(tO, tS + (uint32_t)ks * 8u, b0 + (uint32_t)ks * 128u, kIdescO,
+                                         ks > 0 ? 1u : 0u, elected);
+                    mma_commit_e(&S.o_full[ob], elected);
+                    if (release_kv) mma_commit_e(&S.kv_empty[kvs], elected);
                     return true;
                 };
                 int4 dc = ld_desc(0), dn = ld_desc(1), dnn = ld_desc(2);
@@ -364,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dc = dn; dn = dnn; dnn = ld_desc(i + 3);
                 }
                 // every MMA issued above has finished once this commit arrives
-                mma_commit(&S.drain);
+                mma_commit_e(&S.drain, elected);
                 mbar_wait(&S.drain, 0, st, 41);
             }
         }

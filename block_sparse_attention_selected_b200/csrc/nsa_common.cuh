@@ -234,6 +234,58 @@ __device__ __forceinline__ void mma_bf16_ss_lo(uint32_t d_tmem, uint32_t a_lo, u
         : "memory");
 }
 
+// Warp-uniform MMA issue.  The issuing warp runs its whole loop with every lane (so
+// that descriptors and loop state stay warp-uniform) and one elected lane executes the
+// tcgen05 instructions.  A single issuing lane inside a divergent branch was measured
+// to lose most of its issue slots to busy warps on the same SM sub-partition (about
+// 150 instead of 50 cycles per M=128, N=64 MMA).
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e;
+}
+__device__ __forceinline__ void mma_bf16_ss_lo_e(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                                 uint32_t idesc, uint32_t accumulate,
+                                                 uint32_t elected) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 e, %5, 0;\n\t"
+        "mov.b64 da, {%1, %6};\n\t"
+        "mov.b64 db, {%2, %6};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(elected),
+        "r"(kSw128Sbo1024DescHi)
+        : "memory");
+}
+// TS form (A from TMEM), B from the low word of an SBO-1024 SW128 descriptor.
+__device__ __forceinline__ void mma_bf16_ts_lo_e(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                                 uint32_t idesc, uint32_t accumulate,
+                                                 uint32_t elected) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 e, %5, 0;\n\t"
+        "mov.b64 db, {%2, %6};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(elected),
+        "r"(kSw128Sbo1024DescHi)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_e(uint64_t* bar, uint32_t elected) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "setp.ne.b32 e, %1, 0;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_u32(bar)),
+        "r"(elected)
+        : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M rows x K, two bf16 per 32-bit
 // column, row = TMEM lane) is read from tensor memory (kind::f16).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
