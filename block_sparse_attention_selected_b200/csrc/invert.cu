@@ -97,10 +97,19 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
 // entry selects nothing (padding, future or out-of-range block).
 __device__ __forceinline__ uint32_t entry_key(const SortArgs& a, long long e, uint32_t nbtot,
                                               uint32_t* val) {
-    int j = (int)(e % a.topk);
-    long long r = e / a.topk;
-    int g = (int)(r % a.hkv);
-    int t = (int)(r / a.hkv);
+    int j, g, t;
+    if (a.nent <= 0x7FFFFFFFll) {   // 32-bit division (the 64-bit one is far longer)
+        const uint32_t e32 = (uint32_t)e, tk = (uint32_t)a.topk, hk = (uint32_t)a.hkv;
+        const uint32_t r = e32 / tk;
+        j = (int)(e32 - r * tk);
+        t = (int)(r / hk);
+        g = (int)(r - (uint32_t)t * hk);
+    } else {
+        j = (int)(e % a.topk);
+        const long long r = e / a.topk;
+        g = (int)(r % a.hkv);
+        t = (int)(r / a.hkv);
+    }
     *val = (uint32_t)t * 64u + (uint32_t)j;
     int b = __ldg(a.bidx + e);
     int s = seq_of_token(a.cu, a.nseq, t);
@@ -419,7 +428,15 @@ __global__ void __launch_bounds__(1024) k_unit_order(const DevStatus* st, const 
 __global__ void k_posmap_tiles(const int4* desc, const uint32_t* entries, const DevStatus* st,
                                int hkv, int topk, int tpt, int32_t* posmap) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const int tile = (int)(idx / tpt), k = (int)(idx % tpt);
+    int tile, k;
+    if (idx <= 0x7FFFFFFFll) {   // 32-bit division where the index allows it
+        const uint32_t i32 = (uint32_t)idx;
+        tile = (int)(i32 / (uint32_t)tpt);
+        k = (int)(i32 - (uint32_t)tile * (uint32_t)tpt);
+    } else {
+        tile = (int)(idx / tpt);
+        k = (int)(idx % tpt);
+    }
     if (st->code != 0 || tile >= st->ntiles_fwd) return;
     const int4 d = desc[tile];
     const int G = kTileRows / tpt;

@@ -100,20 +100,42 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     if (lane == 0) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
 }
 
+// Eight rows per warp, half a warp per row and 16-byte loads: four rows' loads of O and
+// dO are in flight per lane before the first reduction.
+constexpr int kDeltaRowsPerWarp = 8;
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* out, const void* dout,
                                                                   float* delta, int T, int hq) {
-    const int lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-    if (row >= (long long)T * hq) return;
-    const uint2 o = __ldg(reinterpret_cast<const uint2*>(out) + row * (kHeadDim / 4) + lane);
-    const uint2 d = __ldg(reinterpret_cast<const uint2*>(dout) + row * (kHeadDim / 4) + lane);
-    const float2 o0 = unpack_bf16x2(o.x), o1 = unpack_bf16x2(o.y);
-    const float2 d0 = unpack_bf16x2(d.x), d1 = unpack_bf16x2(d.y);
-    float x = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
-    x = warp_sum(x);
-    if (lane == 0) {
-        const int t = (int)(row / hq), h = (int)(row - (long long)t * hq);
-        delta[(size_t)h * T + t] = x;
+    const int lane = threadIdx.x & 31, half = lane >> 4, c = lane & 15;
+    const long long nrows = (long long)T * hq;
+    const long long row0 =
+        ((long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * kDeltaRowsPerWarp;
+    uint4 o[kDeltaRowsPerWarp / 2], d[kDeltaRowsPerWarp / 2];
+#pragma unroll
+    for (int it = 0; it < kDeltaRowsPerWarp / 2; ++it) {
+        const long long row = row0 + 2 * it + half;
+        o[it] = d[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (row < nrows) {
+            o[it] = __ldg(reinterpret_cast<const uint4*>(out) + row * (kHeadDim / 8) + c);
+            d[it] = __ldg(reinterpret_cast<const uint4*>(dout) + row * (kHeadDim / 8) + c);
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < kDeltaRowsPerWarp / 2; ++it) {
+        const uint32_t ow[4] = {o[it].x, o[it].y, o[it].z, o[it].w};
+        const uint32_t dw[4] = {d[it].x, d[it].y, d[it].z, d[it].w};
+        float x = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 a = unpack_bf16x2(ow[q]), b = unpack_bf16x2(dw[q]);
+            x = fmaf(a.x, b.x, x);
+            x = fmaf(a.y, b.y, x);
+        }
+        for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, off);
+        const long long row = row0 + 2 * it + half;
+        if (c == 0 && row < nrows) {
+            const int t = (int)(row / hq), h = (int)(row - (long long)t * hq);
+            delta[(size_t)h * T + t] = x;
+        }
     }
 }
 
@@ -196,7 +218,11 @@ cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
                                   cudaStream_t stream) {
-    k_bwd_delta<<<blocks_for((long long)T * hq), kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
+    const long long rows = (long long)T * hq;
+    const long long per_block = (long long)kWarpsPerBlock * kDeltaRowsPerWarp;
+    if (rows > 0)
+        k_bwd_delta<<<(unsigned)((rows + per_block - 1) / per_block), kWarpsPerBlock * 32, 0,
+                      stream>>>(out, dout, delta, T, hq);
     return cudaGetLastError();
 }
 
