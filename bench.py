@@ -83,12 +83,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+# source file of each kernel whose DRAM traffic the committed ncu summary records
+KERNEL_SOURCES = {"k_fwd_tiles": "fwd.cu", "k_bwd_tiles": "bwd.cu", "k_merge": "merge.cu",
+                  "k_dq_merge": "merge.cu"}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the kernel's source file and the shared headers."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_attention_selected_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in (KERNEL_SOURCES[kernel], "nsa_common.cuh", "nsa_kernels.h"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -99,10 +104,8 @@ def profiled_traffic(kernel: str, launch_units: float):
         d = json.load(open(path))
     except Exception:
         return None
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     k = d.get("kernels", {}).get(kernel)
-    if not k:
+    if not k or kernel not in KERNEL_SOURCES or k.get("source_hash") != kernel_source_hash(kernel):
         return None
     # stored per unit of work (useful FLOP) so that a smaller capture scales
     return float(k["dram_bytes_per_useful_flop"]) * launch_units

@@ -400,17 +400,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int pend0 = 0, pend1 = 0;
                 long long idle_since = clock64();
                 while (ok && (fk < nk || ri < fi)) {
-                    bool go_r = false, go_s = false, newkv = false;
+                    bool go_r = false, go_s = false;
                     const int pend = (ri & 1) ? pend1 : pend0;
-                    if (ri < fi)
-                        go_r = mbar_test(&S.pds_full, ri & 1) &&
-                               (!(pend & 1) || mbar_test(&S.acc_empty, ((pend >> 3) & 1) ^ 1));
-                    if (!go_r && fk < nk && fi - ri <= 1) {
-                        newkv = ftt == 0 && fb != prev_bucket;
-                        go_s = (!newkv || ri == fi) &&
-                               mbar_test(&S.q_full[fi % NQ], (fi / NQ) & 1) &&
-                               mbar_test(&S.tmem_empty[fi % NTS], ((fi / NTS) & 1) ^ 1) &&
-                               (!newkv || mbar_test(&S.kv_full, kv_loads & 1));
+                    const bool newkv = ftt == 0 && fb != prev_bucket;
+                    if (lane == 0) {   // one lane polls (32 lanes on one barrier serialise)
+                        if (ri < fi)
+                            go_r = mbar_test(&S.pds_full, ri & 1) &&
+                                   (!(pend & 1) || mbar_test(&S.acc_empty, ((pend >> 3) & 1) ^ 1));
+                        if (!go_r && fk < nk && fi - ri <= 1)
+                            go_s = (!newkv || ri == fi) &&
+                                   mbar_test(&S.q_full[fi % NQ], (fi / NQ) & 1) &&
+                                   mbar_test(&S.tmem_empty[fi % NTS], ((fi / NTS) & 1) ^ 1) &&
+                                   (!newkv || mbar_test(&S.kv_full, kv_loads & 1));
                     }
                     go_r = __shfl_sync(0xffffffffu, go_r, 0);
                     go_s = __shfl_sync(0xffffffffu, go_s, 0);

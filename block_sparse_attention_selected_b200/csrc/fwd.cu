@@ -324,6 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int slot = i & 1, stg = i % kNQ;
                     kvs_of[slot] = cur;
                     if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
+                    // S(i) overwrites the TMEM slot from which PV(i - 2), the last MMA issued
+                    // before it, reads P(i - 2) as its A operand: S(i) waits until PV(i - 2)
+                    // has completed, so that no write of it can overtake those reads.
+                    if (i >= 2 && !wait(&S.o_full[(i - 2) % NO], ((i - 2) / NO) & 1, 42)) return false;
                     tc_fence_after();
                     const uint32_t tS = tmem + slot * BS;
                     const uint32_t a0 = q_desc0 + (uint32_t)stg * kQStage;
