@@ -24,14 +24,14 @@
 // kChunk consecutive tiles round-robin (consecutive tiles of one (g, window, B) list
 // share K_B / V_B).  Each CTA is warp-specialised and pipelined:
 //
-//   warps 0-1    Q loaders: coalesced cp.async gather (two 256-byte rows per warp
-//                instruction) into the 128B-swizzled Q tile, kNQ stages
-//   warp 2       TMA producer: K_B and V_B (128B swizzle) into NKV stages
-//   warp 17      MMA issuer (one elected lane of a warp-uniform loop): S(i+1) is
-//                issued before PV(i)
-//   warps 4-7    softmax of even tiles  } TMEM slot 0 / 1: S (P) and O accumulators
-//   warps 8-11   softmax of odd tiles   }
-//   warps 12-15  epilogue of every tile: O from TMEM, scale, fp16, store
+//   warps 0-3, 18, 19  Q loaders: coalesced cp.async gather (two 256-byte rows per warp
+//                      instruction) into the 128B-swizzled Q tile, kNQ stages
+//   warp 16            TMA producer: K_B and V_B (128B swizzle) into NKV stages
+//   warp 17            MMA issuer (one elected lane of a warp-uniform loop): S(i+1) is
+//                      issued before PV(i)
+//   warps 4-7          softmax of even tiles  } TMEM slot 0 / 1: S (P)
+//   warps 8-11         softmax of odd tiles   }
+//   warps 12-15        epilogue of every tile: O from TMEM, scale, fp16, store
 //
 // The softmax hands each row's scale 2^-e / l to the epilogue in shared memory
 // (double-buffered per slot, with its own barrier).  Producer/consumer hand-offs are
@@ -70,7 +70,7 @@ __device__ __forceinline__ void reg_alloc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 constexpr int kWgThreads = 128;
-constexpr int kNQ = 2;         // Q stages (= S slots: S(i) completing frees stage i % 2)
+constexpr int kNQ = 3;         // Q stages; S(i) completing frees stage i % kNQ (q_empty)
 constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
 // Row-scale buffers: softmax(i + kNSc) may run once PV(i + kNSc - 2) is issued, which
 // waits for the epilogue of tile i + kNSc - 2 - NO; kNSc >= NO + 2 keeps it behind the
@@ -83,7 +83,7 @@ struct alignas(1024) FwdSmem {
     uint8_t kv[NKV][2][2][BS * 128];          // [stage][K, V][64-column half][key]
     uint8_t stage[4][2][32 * 128];            // epilogue staging: [warp][64-column half]
     float sc[kNSc][kTileRows];                // row scale 2^-e / l of tile i in sc[i % kNSc]
-    uint64_t q_full[kNQ];
+    uint64_t q_full[kNQ], q_empty[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
     uint64_t s_full[2], p_full[2];
     uint64_t o_full[3], o_free[3];            // O accumulator buffers (BS == 64: 3, else 2)
@@ -139,7 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
         S.ntiles = *reinterpret_cast<volatile int*>(&st->ntiles_fwd);
-        for (int i = 0; i < kNQ; ++i) mbar_init(&S.q_full[i], kLoaderThreads);
+        for (int i = 0; i < kNQ; ++i) {
+            mbar_init(&S.q_full[i], kLoaderThreads);
+            mbar_init(&S.q_empty[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.s_full[i], 1);
             mbar_init(&S.p_full[i], kWgThreads);
@@ -232,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
                 const int nrows = d.z & 255;
                 const int stg = i % kNQ;
-                // stage i % 2 is free once S(i - 2), which read it, has completed
-                if (!wait_w(&S.s_full[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
+                // stage i % kNQ is free once S(i - kNQ), which read it, has completed
+                if (!wait_w(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
                 const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
     #pragma unroll 4
                 for (int k = 0; k < (kRowsPerLoader + 1) / 2; ++k) {
@@ -310,9 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t q_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.q[0][0]), 16, 1024);
                 const uint32_t k_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.kv[0][0][0]), 16, 1024);
                 const uint32_t v_desc0 = (uint32_t)smem_desc_sw128(smem_u32(S.kv[0][1][0]), BS * 128, 1024);
-                // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
-                // last read by PV(i - 2), which was issued earlier: tcgen05.mma of one thread
-                // run in issue order.  s_full also tells the loaders that the Q stage (i % 2)
+                // S(i) = Q K^T into slot i & 1, whose previous P (tile i - 2) PV(i - 2) reads
+                // (see the wait below).  q_empty tells the loaders that the Q stage i % kNQ
                 // is free again.
                 auto issue_s = [&](int i, int bucket) -> bool {
                     if (bucket != prev_bucket) {
@@ -339,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ss_lo_e(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
                     mma_commit_e(&S.s_full[slot], elected);
+                    mma_commit_e(&S.q_empty[stg], elected);
                     return true;
                 };
                 // O(i) = P(i) V into buffer i % NO once the softmax wrote P(i) and the
@@ -603,10 +606,10 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream) {
     if (p.bs == 64) {
-        constexpr size_t smem = fwd_smem_bytes<64, 3>();
-        cudaFuncSetAttribute(k_fwd_tiles<64, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        constexpr size_t smem = fwd_smem_bytes<64, 2>();
+        cudaFuncSetAttribute(k_fwd_tiles<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        k_fwd_tiles<64, 3><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
+        k_fwd_tiles<64, 2><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
     } else {
         constexpr size_t smem = fwd_smem_bytes<128, 1>();
         cudaFuncSetAttribute(k_fwd_tiles<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
