@@ -226,11 +226,12 @@ def run_ours(args, rank, world, local_rank, dist):
             fwd_ev, 4 if fwd_ev is not None else 0, ctypes.byref(n_fwd))
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
-        rc = lib.nsa_sel_attn_bwd_profiled(
+        # the backward reuses the index inversion the forward left in the shared workspace
+        rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(out), sp(lse), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq), sp(dk), sp(dv), sp(ws), ws_bytes,
-            ctypes.c_void_p(stream.cuda_stream), bwd_ev, 6 if bwd_ev is not None else 0,
-            ctypes.byref(n_bwd))
+            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX, bwd_ev,
+            6 if bwd_ev is not None else 0, ctypes.byref(n_bwd))
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
 

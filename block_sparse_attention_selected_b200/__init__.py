@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
                 3: "NSA_ERR_WORKSPACE", 4: "NSA_ERR_CUDA", 5: "NSA_ERR_TIMEOUT",
                 6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
-            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_invert_index",
+            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_bwd_ex",
+            "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
 
@@ -60,6 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_fwd_profiled.restype = I
             lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, IP]
             lib.nsa_sel_attn_bwd_profiled.restype = I
+            lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, P, I, IP]
+            lib.nsa_sel_attn_bwd_ex.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
             lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
@@ -172,9 +175,16 @@ def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out
     return out, lse
 
 
+NSA_BWD_REUSE_INDEX = 1
+
+
 def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size, scale=None,
-                     dq=None, dk=None, dv=None, workspace=None):
-    """Backward; returns (dq, dk, dv) bf16."""
+                     dq=None, dk=None, dv=None, workspace=None, reuse_index=False):
+    """Backward; returns (dq, dk, dv) bf16.
+
+    reuse_index: `workspace` (sized for the backward) was given to the forward call for
+    the same cu_seqlens / block_idx tensors and is reused untouched since; the backward
+    then skips the index inversion (nsa_sel_attn_bwd_ex with NSA_BWD_REUSE_INDEX)."""
     dev = q.device
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _need(t, n, torch.bfloat16, 3, dev)
@@ -187,11 +197,14 @@ def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size,
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, True)
+    if reuse_index and workspace is None:
+        raise ValueError("reuse_index needs the workspace the forward used")
     ws = workspace if workspace is not None else get_workspace(nbytes, dev)
-    _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd(
+    _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
         hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(ws), ws.numel(), _stream(dev)))
+        _ptr(ws), ws.numel(), _stream(dev), NSA_BWD_REUSE_INDEX if reuse_index else 0,
+        None, 0, None))
     return dq, dk, dv
 
 

@@ -208,6 +208,17 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.tile_off = reinterpret_cast<int32_t*>(b + L.tile_off);
     p.chunk_off = reinterpret_cast<int32_t*>(b + L.chunk_off);
     p.st = c.st;
+    // identity of the inversion's inputs: the index arrays and every size it depends on
+    unsigned long long h = 1469598103934665603ull;
+    for (unsigned long long x : {(unsigned long long)(uintptr_t)cu, (unsigned long long)(uintptr_t)bidx,
+                                 (unsigned long long)D.T, (unsigned long long)D.nseq,
+                                 (unsigned long long)D.hkv, (unsigned long long)D.topk,
+                                 (unsigned long long)D.bs, (unsigned long long)D.G,
+                                 (unsigned long long)kChunkTiles}) {
+        h ^= x;
+        h *= 1099511628211ull;
+    }
+    p.tag = h;
     p.final_buf = 0;
     return c;
 }
@@ -377,7 +388,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
                       int total_tokens, int hq, int hkv, int head_dim, const int32_t* block_idx,
                       int topk, int block_size, float scale, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
-                      void* const* events, int num_events, int* launches) {
+                      void* const* events, int num_events, int* launches, bool reuse_index) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, true, &D);
@@ -397,7 +408,9 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     const PhaseMarks pm{events, num_events, stream, launches};
     if (launches) *launches = 0;
     pm.mark(0);
-    if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    // a reused inversion keeps the status block the forward left (its counts, any error)
+    if (!reuse_index && cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess)
+        return NSA_ERR_CUDA;
     if (total_tokens == 0) {
         for (int i = 1; i < 6; ++i) pm.mark(i);
         return NSA_OK;
@@ -406,14 +419,20 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     CUtensorMap kmap, vmap;
     if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
         return NSA_ERR_CUDA;
-    if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+    if (reuse_index) {
+        c.inv.final_buf = invert_final_buf(c.inv);
+    } else {
+        if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
+        pm.add(invert_launches(D));
+    }
     int4* udesc = reinterpret_cast<int4*>(c.base + L.udesc);
     int* ubucket = reinterpret_cast<int*>(c.base + L.ubucket);
-    if ((s = cuda_status(launch_unit_desc(c.inv, D.units_cap, udesc, ubucket, stream))) != NSA_OK)
+    if ((s = cuda_status(launch_unit_desc(c.inv, D.units_cap, udesc, ubucket, reuse_index,
+                                          stream))) != NSA_OK)
         return s;
     int* uorder = reinterpret_cast<int*>(c.base + L.uorder);
     if ((s = cuda_status(launch_unit_order(c.st, udesc, uorder, stream))) != NSA_OK) return s;
-    pm.add(invert_launches(D) + 2);
+    pm.add(2);
     pm.mark(1);
 
     BwdPlan bp{};
@@ -490,7 +509,7 @@ nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const
                               size_t workspace_bytes, nsa_stream_t stream) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, nullptr, 0, nullptr);
+                    workspace_bytes, stream, nullptr, 0, nullptr, false);
 }
 
 nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void* v,
@@ -503,7 +522,21 @@ nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void*
                                        int* num_launches) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, events, num_events, num_launches);
+                    workspace_bytes, stream, events, num_events, num_launches, false);
+}
+
+nsa_status_t nsa_sel_attn_bwd_ex(const void* q, const void* k, const void* v, const void* out,
+                                 const float* lse, const void* dout, const int32_t* cu_seqlens,
+                                 int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                                 const int32_t* block_idx, int topk, int block_size, float scale,
+                                 void* dq, void* dk, void* dv, void* workspace,
+                                 size_t workspace_bytes, nsa_stream_t stream, unsigned flags,
+                                 void* const* events, int num_events, int* num_launches) {
+    if (flags & ~(unsigned)NSA_BWD_REUSE_INDEX) return NSA_ERR_INVALID_ARG;
+    return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
+                    head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
+                    workspace_bytes, stream, events, num_events, num_launches,
+                    (flags & NSA_BWD_REUSE_INDEX) != 0);
 }
 
 nsa_status_t nsa_sel_invert_index(const int32_t* cu_seqlens, int num_seqs, int total_tokens,

@@ -63,7 +63,8 @@ __device__ __forceinline__ unsigned long long block_incl_scan_u64(unsigned long 
 
 // 1. blkoff[s] = sum_{s' < s} ceil(L_s' / bs); checks cu_seqlens.
 __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq, int T, int bs,
-                                                     int32_t* blkoff, DevStatus* st) {
+                                                     int32_t* blkoff, DevStatus* st,
+                                                     unsigned long long tag) {
     __shared__ unsigned long long warp_tot[32];
     __shared__ unsigned long long round_total;
     __shared__ int bad;
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
     if (threadIdx.x == 0) {
         blkoff[nseq] = (int32_t)carry;
         st->nblocks_total = (int)carry;
+        st->index_tag = tag;
         if (bad) record_error(st, NSA_ERR_BAD_INDEX, 1);
     }
 }
@@ -377,11 +379,15 @@ __global__ void k_tile_desc(const DevStatus* st, const int32_t* row_off, const i
 // 9. One descriptor per backward work unit (up to chunk_tiles consecutive tiles of one
 //    (g, B) list): (first key of the block, first entry, end of the list's entries,
 //    ntiles | g << 8) and the bucket id g * NB + B.
-__global__ void k_unit_desc(const DevStatus* st, const int32_t* chunk_off, const int32_t* tile_off,
+__global__ void k_unit_desc(DevStatus* st, const int32_t* chunk_off, const int32_t* tile_off,
                             const int32_t* offsets, const int32_t* blkoff, const int32_t* cu,
                             int nseq, int hkv, int tpt, int chunk_tiles, int bs, int4* udesc,
-                            int* ubucket) {
+                            int* ubucket, int check_tag, unsigned long long tag) {
     const int u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (check_tag && st->index_tag != tag) {   // the workspace holds another inversion
+        if (u == 0) record_error(st, NSA_ERR_INVALID_ARG, 80);
+        return;
+    }
     if (u >= st->nchunks) return;
     const int nbtot = st->nblocks_total;
     const int bucket = upper_index(chunk_off, hkv * nbtot, u);
@@ -472,8 +478,13 @@ __global__ void k_validate(const int32_t* cu, int nseq, int T, int hkv, const in
 
 }  // namespace
 
+int invert_final_buf(const InvertPlan& p) {
+    const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
+    return (passes - 1) & 1;
+}
+
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
-    k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st);
+    k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st, p.tag);
     SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
     const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
     const uint32_t* kin = nullptr;
@@ -496,7 +507,7 @@ cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
         kin = kout;
         vin = vout;
     }
-    p.final_buf = (passes - 1) & 1;
+    p.final_buf = invert_final_buf(p);
     const long long n1 = p.nent + 1;
     k_bucket_offsets<<<(unsigned)((n1 + 255) / 256), 256, 0, stream>>>(p.keys[p.final_buf], p.nent,
                                                                       p.st, p.hkv, p.offsets);
@@ -529,10 +540,10 @@ cudaError_t launch_posmap(const InvertPlan& p, const WindowPlan& w, int32_t* pos
 }
 
 cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
-                             cudaStream_t stream) {
+                             bool check_tag, cudaStream_t stream) {
     k_unit_desc<<<(unsigned)((units_cap + 255) / 256), 256, 0, stream>>>(
         p.st, p.chunk_off, p.tile_off, p.offsets, p.blkoff, p.cu, p.nseq, p.hkv,
-        p.tokens_per_tile, p.chunk_tiles, p.bs, udesc, ubucket);
+        p.tokens_per_tile, p.chunk_tiles, p.bs, udesc, ubucket, check_tag ? 1 : 0, p.tag);
     return cudaGetLastError();
 }
 

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan 
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hq) return;
+    if (*reinterpret_cast<const volatile int*>(&p.st->code) != 0) return;
     const int t = (int)(row / p.hq);
     const int h = (int)(row - (long long)t * p.hq);
     const int g = h / p.G;
@@ -176,6 +177,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dkdv_reduce(const BwdPl
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hkv) return;
+    // after a recorded device error the unit lists may not belong to this call
+    if (*reinterpret_cast<const volatile int*>(&p.st->code) != 0) return;
     const int t = (int)(row / p.hkv);
     const int g = (int)(row - (long long)t * p.hkv);
     const int s = seq_of_token(p.cu, p.nseq, t);

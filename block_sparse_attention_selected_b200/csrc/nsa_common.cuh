@@ -33,7 +33,9 @@ struct DevStatus {
     int nentries;      // number of valid (token, KV head, slot) entries
     long long bad_range, bad_dup;   // validation counters
     int ntiles_fwd;    // number of forward tiles in window order
-    int pad[51];
+    int pad0;
+    unsigned long long index_tag;   // identifies the inputs of the inversion held here
+    int pad[48];
 };
 static_assert(sizeof(DevStatus) == 256, "status block is 256 bytes");
 

@@ -35,9 +35,13 @@ struct InvertPlan {
     int32_t* tile_off;       // [nbk_cap + 1]
     int32_t* chunk_off;      // [nbk_cap + 1]
     DevStatus* st;
+    unsigned long long tag;  // written to st->index_tag by the inversion
     // result: the sorted values live in vals[final_buf]
     int final_buf;
 };
+
+// vals buffer that holds the sorted entries after launch_invert
+int invert_final_buf(const InvertPlan& p);
 
 constexpr int kSortTile = 4096;  // entries per sort tile (256 threads x 16)
 
@@ -61,8 +65,10 @@ cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaSt
 // in its forward tile) for every valid entry; the partial rows are posmap * G + head.
 cudaError_t launch_posmap(const InvertPlan& p, const WindowPlan& w, int32_t* posmap,
                           cudaStream_t stream);
+// check_tag: the inversion is reused from an earlier call; a workspace whose
+// st->index_tag differs from p.tag records NSA_ERR_INVALID_ARG (where 80).
 cudaError_t launch_unit_desc(const InvertPlan& p, long long units_cap, int4* udesc, int* ubucket,
-                             cudaStream_t stream);
+                             bool check_tag, cudaStream_t stream);
 // Units ordered by tile count, largest first, for the snake deal of the backward kernel.
 cudaError_t launch_unit_order(const DevStatus* st, const int4* udesc, int* uorder,
                               cudaStream_t stream);

@@ -126,6 +126,27 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
     void *dk, void *dv, void *workspace, size_t workspace_bytes, nsa_stream_t stream,
     void *const *events, int num_events, int *num_launches);
 
+/* The backward with options (flags, OR-ed):
+ *   NSA_BWD_REUSE_INDEX  the workspace holds the block-index inversion that
+ *       nsa_sel_attn_fwd (or _profiled) computed in it for the same cu_seqlens and
+ *       block_idx pointers and sizes, with workspace_bytes at least the backward size,
+ *       and no other call used the workspace since; the backward then skips the
+ *       inversion (a training step uses one index for both passes).  The status block
+ *       is kept as the forward left it.  If the workspace was last inverted for other
+ *       inputs (pointers or sizes), the call records NSA_ERR_INVALID_ARG in the device
+ *       status (nsa_sel_check_status) and the outputs are undefined; the index contents
+ *       themselves are not compared.
+ * Other flag bits return NSA_ERR_INVALID_ARG.  events / num_events / num_launches as in
+ * nsa_sel_attn_bwd_profiled (null / 0 for none).  Otherwise identical to
+ * nsa_sel_attn_bwd. */
+#define NSA_BWD_REUSE_INDEX 1u
+NSA_API nsa_status_t nsa_sel_attn_bwd_ex(
+    const void *q, const void *k, const void *v, const void *out, const float *lse,
+    const void *dout, const int32_t *cu_seqlens, int num_seqs, int total_tokens, int hq, int hkv,
+    int head_dim, const int32_t *block_idx, int topk, int block_size, float scale, void *dq,
+    void *dk, void *dv, void *workspace, size_t workspace_bytes, nsa_stream_t stream,
+    unsigned flags, void *const *events, int num_events, int *num_launches);
+
 /* The block-index inversion on its own (the loop swap named in the file header):
  * for KV head g and global block B (blocks of earlier sequences first), the list of
  * entries token * 64 + slot with block_idx[token, g, slot] = local block of B and

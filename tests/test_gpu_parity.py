@@ -310,3 +310,28 @@ def test_repeat_calls_bitwise_identical():
     for _ in range(30):
         for x, y in zip(_bwd(p, d, out0, lse0), g0):
             assert torch.equal(x, y)
+
+
+def test_bwd_reusing_forward_inversion():
+    p = ni.make_problem([2500, 700], hq=8, hkv=2, block_size=64, topk=16, seed=42)
+    d = to_device(p)
+    T, hq, hkv, topk = p.q.shape[0], p.q.shape[1], p.k.shape[1], p.block_idx.shape[2]
+    nb = nsa.nsa_sel_attn_workspace_size(T, 2, hq, hkv, 128, topk, 64, True)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], 64, p.scale,
+                                    workspace=ws)
+    ref = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"], d["bidx"],
+                               64, p.scale)
+    got = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"], d["bidx"],
+                               64, p.scale, workspace=ws, reuse_index=True)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status(ws) == 0
+    for x, y in zip(got, ref):
+        assert torch.equal(x, y)
+    # an inversion of other index tensors is refused (device status), not used
+    bidx2 = d["bidx"].clone()
+    nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], bidx2, 64, p.scale, workspace=ws)
+    nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"], d["bidx"], 64,
+                         p.scale, workspace=ws, reuse_index=True)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status(ws) == 1   # NSA_ERR_INVALID_ARG
