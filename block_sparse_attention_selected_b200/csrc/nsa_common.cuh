@@ -20,7 +20,7 @@ namespace nsa {
 constexpr int kHeadDim = 128;        // head dimension supported by the kernels
 constexpr int kTileRows = 128;       // MMA M: (token, head) rows per tile
 constexpr int kMaxTopk = 64;         // entry = token * 64 + slot
-constexpr int kMaxGroup = 16;        // query heads per KV head
+constexpr int kMaxGroup = 128;       // query heads per KV head (a divisor of the 128-row tile)
 
 // Device status word layout (int32 slots at the start of the workspace).
 struct DevStatus {

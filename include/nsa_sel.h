@@ -38,7 +38,8 @@
  *    in the status block at the start of the workspace and read with
  *    nsa_sel_check_status.  No C++ exception crosses this interface.
  *  - Supported domain: bf16, head_dim == 128, block_size in {64, 128},
- *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv <= 16, total_tokens < 2^25.
+ *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv a divisor of 128 (a 128-row tile
+ *    holds whole query-head groups), total_tokens < 2^25.
  *    Anything else returns NSA_ERR_UNSUPPORTED.
  */
 #ifndef NSA_SEL_H

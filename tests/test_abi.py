@@ -54,7 +54,9 @@ def test_workspace_size_domain(lib):
     assert f(1024, 1, 4, 4, 64, 8, 64, 0) == 0          # head_dim 64 not supported
     assert f(1024, 1, 4, 4, 128, 8, 32, 0) == 0         # block 32 not supported
     assert f(1024, 1, 4, 4, 128, 65, 64, 0) == 0        # topk > 64
-    assert f(1024, 1, 64, 2, 128, 8, 64, 0) == 0        # group 32 > 16
+    assert f(1024, 1, 64, 2, 128, 8, 64, 0) > 0         # group 32 fills a tile with 4 tokens
+    assert f(1024, 1, 256, 1, 128, 8, 64, 0) == 0       # group 256 > 128 rows of a tile
+    assert f(1024, 1, 6, 2, 128, 8, 64, 0) == 0         # group 3 does not divide 128
     assert f(1024, 1, 6, 4, 128, 8, 64, 0) == 0         # hq % hkv != 0
     assert f(1 << 25, 1, 4, 4, 128, 8, 64, 0) == 0      # too many tokens
 

@@ -114,6 +114,8 @@ FWD_SMALL = [
     ("g16_bs128_k64", dict(lengths=[1800], hq=16, hkv=1, block_size=128, topk=64, seed=11), True),
     ("g16_bs64_k1", dict(lengths=[999, 333], hq=32, hkv=2, block_size=64, topk=1, seed=12), False),
     ("g4_dense_causal", dict(lengths=[640, 300], hq=8, hkv=2, block_size=64, topk=12, seed=13), False),
+    ("g32_bs64_k8", dict(lengths=[600, 77], hq=64, hkv=2, block_size=64, topk=8, seed=14), True),
+    ("g128_bs128_k4", dict(lengths=[300], hq=128, hkv=1, block_size=128, topk=4, seed=15), False),
 ]
 
 
@@ -235,6 +237,8 @@ BWD_SMALL = [
     ("g1_bs128_k8", dict(lengths=[1100, 1], hq=2, hkv=2, block_size=128, topk=8, seed=32), True),
     ("g16_bs64_k5", dict(lengths=[700], hq=16, hkv=1, block_size=64, topk=5, seed=33), False),
     ("g8_bs128_k64", dict(lengths=[900, 129], hq=8, hkv=1, block_size=128, topk=64, seed=34), True),
+    ("g32_bs64_k6", dict(lengths=[500, 70], hq=32, hkv=1, block_size=64, topk=6, seed=35), True),
+    ("g128_bs64_k3", dict(lengths=[260], hq=128, hkv=1, block_size=64, topk=3, seed=37), False),
 ]
 
 
