@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
                 3: "NSA_ERR_WORKSPACE", 4: "NSA_ERR_CUDA", 5: "NSA_ERR_TIMEOUT",
                 6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
-            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_bwd_ex",
+            "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_fwd_ex",
+            "nsa_sel_attn_bwd_ex",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
@@ -61,6 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_fwd_profiled.restype = I
             lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, IP]
             lib.nsa_sel_attn_bwd_profiled.restype = I
+            lib.nsa_sel_attn_fwd_ex.argtypes = lib.nsa_sel_attn_fwd.argtypes + [ctypes.c_uint, P, I, IP]
+            lib.nsa_sel_attn_fwd_ex.restype = I
             lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, P, I, IP]
             lib.nsa_sel_attn_bwd_ex.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
@@ -148,13 +151,30 @@ def _shapes(q, k, cu_seqlens, block_idx):
     return T, hq, hkv, d, topk, cu_seqlens.numel() - 1
 
 
+NSA_BWD_REUSE_INDEX = 1
+NSA_F16 = 2
+
+
+def _elem_type(q):
+    """bf16 or fp16 attention tensors (the flag of the _ex calls)."""
+    if q.dtype == torch.bfloat16:
+        return torch.bfloat16, 0
+    if q.dtype == torch.float16:
+        return torch.float16, NSA_F16
+    raise TypeError(f"q: expected bfloat16 or float16, got {q.dtype}")
+
+
 def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out=None, lse=None,
-                     workspace=None):
-    """Forward selected attention; returns (out bf16 [T,hq,d], lse fp32 [hq,T])."""
+                     workspace=None, with_lse=True):
+    """Forward selected attention; returns (out [T,hq,d], lse fp32 [hq,T]).
+
+    q, k, v (and out) are all bf16 or all fp16.  with_lse=False: a forward with no
+    backward to follow; the LSE is not stored and None is returned in its place."""
     dev = q.device
-    _need(q, "q", torch.bfloat16, 3, dev)
-    _need(k, "k", torch.bfloat16, 3, dev)
-    _need(v, "v", torch.bfloat16, 3, dev)
+    et, flag = _elem_type(q)
+    _need(q, "q", et, 3, dev)
+    _need(k, "k", et, 3, dev)
+    _need(v, "v", et, 3, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
     _need(block_idx, "block_idx", torch.int32, 3, dev)
     T, hq, hkv, d, topk, nseq = _shapes(q, k, cu_seqlens, block_idx)
@@ -163,31 +183,31 @@ def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out
     scale = float(d ** -0.5 if scale is None else scale)
     if out is None:
         out = torch.empty_like(q)
-    if lse is None:
+    if lse is None and with_lse:
         lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
-    _need(out, "out", torch.bfloat16, 3, dev)
-    _need(lse, "lse", torch.float32, 2, dev)
+    _need(out, "out", et, 3, dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2, dev)
     nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, False)
     ws = workspace if workspace is not None else get_workspace(nbytes, dev)
-    _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd(
+    _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, _ptr(block_idx), topk,
-        block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
+        block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev), flag,
+        None, 0, None))
     return out, lse
-
-
-NSA_BWD_REUSE_INDEX = 1
 
 
 def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size, scale=None,
                      dq=None, dk=None, dv=None, workspace=None, reuse_index=False):
-    """Backward; returns (dq, dk, dv) bf16.
+    """Backward; returns (dq, dk, dv) in the type of q (bf16 or fp16).
 
     reuse_index: `workspace` (sized for the backward) was given to the forward call for
     the same cu_seqlens / block_idx tensors and is reused untouched since; the backward
     then skips the index inversion (nsa_sel_attn_bwd_ex with NSA_BWD_REUSE_INDEX)."""
     dev = q.device
+    et, flag = _elem_type(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
-        _need(t, n, torch.bfloat16, 3, dev)
+        _need(t, n, et, 3, dev)
     _need(lse, "lse", torch.float32, 2, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
     _need(block_idx, "block_idx", torch.int32, 3, dev)
@@ -196,6 +216,8 @@ def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, et, 3, dev)
     nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, True)
     if reuse_index and workspace is None:
         raise ValueError("reuse_index needs the workspace the forward used")
@@ -203,7 +225,7 @@ def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size,
     _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
         hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(ws), ws.numel(), _stream(dev), NSA_BWD_REUSE_INDEX if reuse_index else 0,
+        _ptr(ws), ws.numel(), _stream(dev), (NSA_BWD_REUSE_INDEX if reuse_index else 0) | flag,
         None, 0, None))
     return dq, dk, dv
 

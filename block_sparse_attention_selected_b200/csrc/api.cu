@@ -142,14 +142,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // Tensor map over a bf16 [T, hkv, 128] tensor; box = (64 columns, 1 head, bs keys),
 // 128-byte swizzle (the layout the tensor-core descriptors expect).
-bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs) {
+bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs, bool f16) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)hkv, (cuuint64_t)(T > 0 ? T : 1)};
     cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)hkv * kHeadDim * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)bs};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     3, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -290,12 +291,12 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
                       int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
                       const int32_t* block_idx, int topk, int block_size, float scale, void* out,
                       float* lse, void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
-                      void* const* events, int num_events, int* launches) {
+                      void* const* events, int num_events, int* launches, bool f16) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, false, &D);
     if (s != NSA_OK) return s;
-    if (total_tokens > 0 && (!q || !k || !v || !out || !lse)) return NSA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !out)) return NSA_ERR_INVALID_ARG;   // lse may be null
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         !aligned(lse, 4))
         return NSA_ERR_INVALID_ARG;
@@ -315,7 +316,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     }
 
     CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
     WindowPlan wp{};
@@ -339,6 +340,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.cu = cu_seqlens;
     fp.nseq = D.nseq; fp.T = D.T; fp.hq = D.hq; fp.hkv = D.hkv; fp.topk = D.topk; fp.bs = D.bs;
     fp.G = D.G;
+    fp.f16 = f16 ? 1 : 0;
     fp.scale_log2 = scale * 1.4426950408889634f;
     fp.blkoff = c.inv.blkoff;
     fp.offsets = c.inv.offsets;
@@ -370,6 +372,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     mp.cu = cu_seqlens;
     mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
     mp.G = D.G;
+    mp.f16 = f16 ? 1 : 0;
     mp.bidx = block_idx;
     mp.posmap = posmap;
     mp.part_o = fp.part_o;
@@ -388,7 +391,8 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
                       int total_tokens, int hq, int hkv, int head_dim, const int32_t* block_idx,
                       int topk, int block_size, float scale, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
-                      void* const* events, int num_events, int* launches, bool reuse_index) {
+                      void* const* events, int num_events, int* launches, bool reuse_index,
+                      bool f16) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, true, &D);
@@ -417,7 +421,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     }
 
     CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs))
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16))
         return NSA_ERR_CUDA;
     if (reuse_index) {
         c.inv.final_buf = invert_final_buf(c.inv);
@@ -443,6 +447,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.cu = cu_seqlens;
     bp.nseq = D.nseq; bp.T = D.T; bp.hq = D.hq; bp.hkv = D.hkv; bp.topk = D.topk; bp.bs = D.bs;
     bp.G = D.G;
+    bp.f16 = f16 ? 1 : 0;
     bp.scale = scale;
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.blkoff = c.inv.blkoff;
@@ -459,7 +464,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.part_dkdv = reinterpret_cast<float*>(c.base + L.part_dkdv);
     bp.st = c.st;
     bp.num_sms = num_sms;
-    if ((s = cuda_status(launch_bwd_preprocess(out, dout, bp.delta, D.T, D.hq, stream))) != NSA_OK)
+    if ((s = cuda_status(launch_bwd_preprocess(out, dout, bp.delta, D.T, D.hq, bp.f16, stream))) != NSA_OK)
         return s;
     pm.add(1);
     pm.mark(2);
@@ -486,7 +491,7 @@ nsa_status_t nsa_sel_attn_fwd(const void* q, const void* k, const void* v,
                               size_t workspace_bytes, nsa_stream_t stream) {
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, nullptr,
-                    0, nullptr);
+                    0, nullptr, false);
 }
 
 nsa_status_t nsa_sel_attn_fwd_profiled(const void* q, const void* k, const void* v,
@@ -498,7 +503,20 @@ nsa_status_t nsa_sel_attn_fwd_profiled(const void* q, const void* k, const void*
                                        int* num_launches) {
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
-                    num_events, num_launches);
+                    num_events, num_launches, false);
+}
+
+nsa_status_t nsa_sel_attn_fwd_ex(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens, int num_seqs, int total_tokens, int hq,
+                                 int hkv, int head_dim, const int32_t* block_idx, int topk,
+                                 int block_size, float scale, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, nsa_stream_t stream,
+                                 unsigned flags, void* const* events, int num_events,
+                                 int* num_launches) {
+    if (flags & ~(unsigned)NSA_F16) return NSA_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
+                    topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
+                    num_events, num_launches, (flags & NSA_F16) != 0);
 }
 
 nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const void* out,
@@ -509,7 +527,7 @@ nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const
                               size_t workspace_bytes, nsa_stream_t stream) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, nullptr, 0, nullptr, false);
+                    workspace_bytes, stream, nullptr, 0, nullptr, false, false);
 }
 
 nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void* v,
@@ -522,7 +540,7 @@ nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void*
                                        int* num_launches) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, events, num_events, num_launches, false);
+                    workspace_bytes, stream, events, num_events, num_launches, false, false);
 }
 
 nsa_status_t nsa_sel_attn_bwd_ex(const void* q, const void* k, const void* v, const void* out,
@@ -532,11 +550,11 @@ nsa_status_t nsa_sel_attn_bwd_ex(const void* q, const void* k, const void* v, co
                                  void* dq, void* dk, void* dv, void* workspace,
                                  size_t workspace_bytes, nsa_stream_t stream, unsigned flags,
                                  void* const* events, int num_events, int* num_launches) {
-    if (flags & ~(unsigned)NSA_BWD_REUSE_INDEX) return NSA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(NSA_BWD_REUSE_INDEX | NSA_F16)) return NSA_ERR_INVALID_ARG;
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
                     workspace_bytes, stream, events, num_events, num_launches,
-                    (flags & NSA_BWD_REUSE_INDEX) != 0);
+                    (flags & NSA_BWD_REUSE_INDEX) != 0, (flags & NSA_F16) != 0);
 }
 
 nsa_status_t nsa_sel_invert_index(const int32_t* cu_seqlens, int num_seqs, int total_tokens,

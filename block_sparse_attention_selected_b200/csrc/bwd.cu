@@ -102,7 +102,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <int BS, int NQ, int NSLOT>
+template <int BS, int NQ, int NSLOT, int F16>
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_tiles(const BwdPlan p, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap) {
@@ -309,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // elected lane executes the tcgen05 instructions.
             {
                 const uint32_t elected = elect_one();
-                constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);   // S, dP
-                constexpr uint32_t kIdescT = idesc_bf16_f32(128, BS, true, true);     // dV^T, dK^T
-                constexpr uint32_t kIdescQ = idesc_bf16_f32(128, 128, false, true);   // dQ
+                constexpr uint32_t kIdescS = idesc_f16kind_f32(F16, 128, BS, false, false);  // S, dP
+                constexpr uint32_t kIdescT = idesc_f16kind_f32(F16, 128, BS, true, true);    // dV^T, dK^T
+                constexpr uint32_t kIdescQ = idesc_f16kind_f32(F16, 128, 128, false, true);  // dQ
                 int kv_loads = 0, prev_bucket = -1;
                 bool ok = true;
                 // Shared-memory descriptors are computed once; an MMA step adds its byte
@@ -572,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         x.x = key <= my_lim ? ex2_approx(x.x) : 0.f;
                         x.y = key + 1 <= my_lim ? ex2_approx(x.y) : 0.f;
                         const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
-                        pk[c / 2] = pack_bf16x2(x.x, x.y);
-                        dk[c / 2] = pack_bf16x2(ds.x, ds.y);
+                        pk[c / 2] = pack2<F16>(x.x, x.y);    // P, dS in the operands' type
+                        dk[c / 2] = pack2<F16>(ds.x, ds.y);
                     }
                 }
                 tc_fence_before();
@@ -611,18 +611,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+template <int BS, int NQ, int NSLOT, int F16>
+static void launch_bwd_variant(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                               cudaStream_t stream) {
+    constexpr size_t smem = bwd_smem_bytes<BS, NQ, NSLOT>();
+    cudaFuncSetAttribute(k_bwd_tiles<BS, NQ, NSLOT, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    k_bwd_tiles<BS, NQ, NSLOT, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+}
+
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              cudaStream_t stream) {
     if (p.bs == 64) {
-        constexpr size_t smem = bwd_smem_bytes<64, 2, 2>();
-        cudaFuncSetAttribute(k_bwd_tiles<64, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        k_bwd_tiles<64, 2, 2><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+        if (p.f16) launch_bwd_variant<64, 2, 2, 1>(p, kmap, vmap, stream);
+        else launch_bwd_variant<64, 2, 2, 0>(p, kmap, vmap, stream);
     } else {
-        constexpr size_t smem = bwd_smem_bytes<128, 1, 1>();
-        cudaFuncSetAttribute(k_bwd_tiles<128, 1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        k_bwd_tiles<128, 1, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+        if (p.f16) launch_bwd_variant<128, 1, 1, 1>(p, kmap, vmap, stream);
+        else launch_bwd_variant<128, 1, 1, 0>(p, kmap, vmap, stream);
     }
     return cudaGetLastError();
 }

@@ -118,7 +118,7 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
-template <int BS, int NKV>
+template <int BS, int NKV, int F16>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tiles(const FwdPlan p, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap8,
@@ -297,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // executes the tcgen05 instructions.
             {
                 const uint32_t elected = elect_one();
-                constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false, false);
-                constexpr uint32_t kIdescO = idesc_bf16_f32(128, 128, false, true);
+                constexpr uint32_t kIdescS = idesc_f16kind_f32(F16, 128, BS, false, false);
+                constexpr uint32_t kIdescO = idesc_f16kind_f32(F16, 128, 128, false, true);
                 int kv_uses = 0, prev_bucket = -1, cur = 0;
                 int kvs_of[2] = {0, 0};
                 // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k2 = 0; k2 < 32; ++k2) {
                 const float2 x = mul2(make_float2(v[2 * k2], v[2 * k2 + 1]), s2);
-                pk[k2] = pack_bf16x2(x.x, x.y);
+                pk[k2] = pack2<F16>(x.x, x.y);   // P in the type of V (one MMA, one type)
             }
         };
         // descriptors two tiles ahead, entries and exponents one tile ahead, so that no
@@ -597,24 +597,33 @@ __global__ void __launch_bounds__(128) k_vblock_exp(const __nv_bfloat16* v, cons
 
 cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, int32_t* vexp,
                               cudaStream_t stream) {
-    if (p.T > 0 && nb_stride > 0)
+    if (p.T > 0 && nb_stride > 0) {
+        if (p.f16)   // |V| <= 65504 already fits the fp16 partials: every exponent is 0
+            return cudaMemsetAsync(vexp, 0, sizeof(int32_t) * (size_t)p.hkv * nb_stride, stream);
         k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), 128, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(v), p.cu, p.nseq, p.hkv, p.bs, p.blkoff, p.st, vexp);
+    }
     return cudaGetLastError();
+}
+
+template <int BS, int NKV, int F16>
+static void launch_fwd_variant(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                               const CUtensorMap* omap, cudaStream_t stream) {
+    constexpr size_t smem = fwd_smem_bytes<BS, NKV>();
+    cudaFuncSetAttribute(k_fwd_tiles<BS, NKV, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    k_fwd_tiles<BS, NKV, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0],
+                                                                      omap[1]);
 }
 
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream) {
     if (p.bs == 64) {
-        constexpr size_t smem = fwd_smem_bytes<64, 2>();
-        cudaFuncSetAttribute(k_fwd_tiles<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        k_fwd_tiles<64, 2><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
+        if (p.f16) launch_fwd_variant<64, 2, 1>(p, kmap, vmap, omap, stream);
+        else launch_fwd_variant<64, 2, 0>(p, kmap, vmap, omap, stream);
     } else {
-        constexpr size_t smem = fwd_smem_bytes<128, 1>();
-        cudaFuncSetAttribute(k_fwd_tiles<128, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-        k_fwd_tiles<128, 1><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0], omap[1]);
+        if (p.f16) launch_fwd_variant<128, 1, 1>(p, kmap, vmap, omap, stream);
+        else launch_fwd_variant<128, 1, 0>(p, kmap, vmap, omap, stream);
     }
     return cudaGetLastError();
 }

@@ -33,7 +33,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 // head offset) are loaded first; then, in one round of requests, every valid slot's
 // 256-byte partial row (4 columns per lane) and each lane's (lse_j, exponent_j), so
 // that the row costs two dependent memory latencies.
-template <int kS>   // slots held by the warp: 16, 32 or 64 (>= topk)
+template <int kS, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk); fp16 output
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge(const MergePlan p) {
     constexpr bool kTopk32 = kS <= 32;
     const int lane = threadIdx.x & 31;
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
                                            (size_t)row * kHeadDim) + lane;
     if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
         *outp = make_uint2(0u, 0u);
-        if (lane == 0) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
+        if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
         return;
     }
     const float w0 = m0.x == -CUDART_INF_F ? 0.f : __expf(m0.x - M);
@@ -96,13 +96,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
         acc[3] = fmaf(wj, b.y, acc[3]);
     }
     const float inv = 1.f / Lam;
-    *outp = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    if (lane == 0) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
+    *outp = make_uint2(pack2<F16>(acc[0] * inv, acc[1] * inv), pack2<F16>(acc[2] * inv, acc[3] * inv));
+    if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
 }
 
 // Eight rows per warp, half a warp per row and 16-byte loads: four rows' loads of O and
 // dO are in flight per lane before the first reduction.
 constexpr int kDeltaRowsPerWarp = 8;
+template <int F16>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* out, const void* dout,
                                                                   float* delta, int T, int hq) {
     const int lane = threadIdx.x & 31, half = lane >> 4, c = lane & 15;
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* o
         float x = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float2 a = unpack_bf16x2(ow[q]), b = unpack_bf16x2(dw[q]);
+            const float2 a = unpack2<F16>(ow[q]), b = unpack2<F16>(dw[q]);
             x = fmaf(a.x, b.x, x);
             x = fmaf(a.y, b.y, x);
         }
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* o
     }
 }
 
+template <int F16>   // dQ partials are bf16 either way; F16: fp16 output
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan p, const int32_t* bidx,
                                                                  void* dq) {
     const int lane = threadIdx.x & 31;
@@ -169,10 +171,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan 
         acc[3] += b.y;
     }
     uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dq) + (size_t)row * kHeadDim) + lane;
-    *o = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    *o = make_uint2(pack2<F16>(acc[0], acc[1]), pack2<F16>(acc[2], acc[3]));
 }
 
 // One warp per (key token, KV head); each lane owns 4 of the 128 columns.
+template <int F16>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dkdv_reduce(const BwdPlan p, void* dk, void* dv) {
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -198,8 +201,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dkdv_reduce(const BwdPl
     }
     uint2* ov = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dv) + (size_t)row * kHeadDim) + lane;
     uint2* ok = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dk) + (size_t)row * kHeadDim) + lane;
-    *ov = make_uint2(pack_bf16x2(av.x, av.y), pack_bf16x2(av.z, av.w));
-    *ok = make_uint2(pack_bf16x2(ak.x, ak.y), pack_bf16x2(ak.z, ak.w));
+    *ov = make_uint2(pack2<F16>(av.x, av.y), pack2<F16>(av.z, av.w));
+    *ok = make_uint2(pack2<F16>(ak.x, ak.y), pack2<F16>(ak.z, ak.w));
 }
 
 inline unsigned blocks_for(long long rows) {
@@ -210,32 +213,43 @@ inline unsigned blocks_for(long long rows) {
 
 cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
     const unsigned nb = blocks_for((long long)p.T * p.hq);
-    if (p.topk <= 16)
-        k_merge<16><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
-    else if (p.topk <= 32)
-        k_merge<32><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
-    else
-        k_merge<64><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p);
+    const unsigned nt = kWarpsPerBlock * 32;
+    if (p.topk <= 16) {
+        if (p.f16) k_merge<16, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<16, 0><<<nb, nt, 0, stream>>>(p);
+    } else if (p.topk <= 32) {
+        if (p.f16) k_merge<32, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<32, 0><<<nb, nt, 0, stream>>>(p);
+    } else {
+        if (p.f16) k_merge<64, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<64, 0><<<nb, nt, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
-                                  cudaStream_t stream) {
+                                  int f16, cudaStream_t stream) {
     const long long rows = (long long)T * hq;
     const long long per_block = (long long)kWarpsPerBlock * kDeltaRowsPerWarp;
-    if (rows > 0)
-        k_bwd_delta<<<(unsigned)((rows + per_block - 1) / per_block), kWarpsPerBlock * 32, 0,
-                      stream>>>(out, dout, delta, T, hq);
+    const unsigned nb = (unsigned)((rows + per_block - 1) / per_block);
+    if (rows > 0) {
+        if (f16) k_bwd_delta<1><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
+        else k_bwd_delta<0><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq, cudaStream_t stream) {
-    k_dq_merge<<<blocks_for((long long)p.T * p.hq), kWarpsPerBlock * 32, 0, stream>>>(p, bidx, dq);
+    const unsigned nb = blocks_for((long long)p.T * p.hq);
+    if (p.f16) k_dq_merge<1><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p, bidx, dq);
+    else k_dq_merge<0><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p, bidx, dq);
     return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStream_t stream) {
-    k_dkdv_reduce<<<blocks_for((long long)p.T * p.hkv), kWarpsPerBlock * 32, 0, stream>>>(p, dk, dv);
+    const unsigned nb = blocks_for((long long)p.T * p.hkv);
+    if (p.f16) k_dkdv_reduce<1><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p, dk, dv);
+    else k_dkdv_reduce<0><<<nb, kWarpsPerBlock * 32, 0, stream>>>(p, dk, dv);
     return cudaGetLastError();
 }
 

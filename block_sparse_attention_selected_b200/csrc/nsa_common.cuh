@@ -404,14 +404,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 D and A, B both bf16 (f16 = false) or
+// both fp16 (f16 = true): the two operands of one MMA always have the same type.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(bool f16, int M, int N, bool a_mn_major,
+                                                         bool b_mn_major) {
     return (1u << 4)                      // D format: f32
-           | (1u << 7)                    // A format: bf16
-           | (1u << 10)                   // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)       // A format: f16 0, bf16 1
+           | ((f16 ? 0u : 1u) << 10)      // B format: the same
            | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
+                                                      bool b_mn_major) {
+    return idesc_f16kind_f32(false, M, N, a_mn_major, b_mn_major);
 }
 
 // Byte offset of the 16-byte chunk `c16` (0..7) of row `r` inside a K-major tile whose
@@ -438,6 +443,16 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
     __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
     return __bfloat1622float2(v);
+}
+
+// The 16-bit element type of the attention tensors: bf16 (F16 = 0) or fp16 (F16 = 1).
+template <int F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+template <int F16>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+    return F16 ? unpack_f16x2(u) : unpack_bf16x2(u);
 }
 
 // Entry validity shared by every kernel: a selected block b of a token at query block

@@ -77,6 +77,7 @@ struct FwdPlan {
     const void* q;
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
     float scale_log2;        // scale * log2(e)
     const int32_t* blkoff;
     const int32_t* offsets;  // bucket offsets into entries
@@ -107,6 +108,7 @@ cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CU
 struct MergePlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
     const int32_t* bidx;
     const int32_t* posmap;   // sorted position of each valid (t, g, j) entry
     const void* part_o;
@@ -121,6 +123,7 @@ cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream);
 struct BwdPlan {
     const void* q;
     const void* dout;
+    int f16;                 // 1: the attention tensors are fp16; 0: bf16
     const float* lse;        // [hq, T]
     float* delta;            // [hq, T]  rowsum(dout * out)
     const int32_t* cu;
@@ -143,7 +146,7 @@ struct BwdPlan {
 };
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
-                                  cudaStream_t stream);
+                                  int f16, cudaStream_t stream);
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              cudaStream_t stream);
 cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq,

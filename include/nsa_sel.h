@@ -83,7 +83,8 @@ NSA_API size_t nsa_sel_attn_workspace_size(int total_tokens, int num_seqs, int h
  *              cu_seqlens[num_seqs] = total_tokens
  *   block_idx  int32 [total_tokens, hkv, topk], block numbers local to the sequence
  *   out  bf16 [total_tokens, hq, head_dim] (written)
- *   lse  fp32 [hq, total_tokens] (written; natural log)
+ *   lse  fp32 [hq, total_tokens] (written; natural log), or null for a forward
+ *        that will have no backward (nothing is stored then)
  * Steps on `stream`: block-index inversion, the tensor-core tile kernel over
  * (KV block, gathered query rows), and the log-sum-exp merge of the per-block
  * partial results. */
@@ -127,6 +128,19 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
     void *dk, void *dv, void *workspace, size_t workspace_bytes, nsa_stream_t stream,
     void *const *events, int num_events, int *num_launches);
 
+/* Option flags of the _ex calls below (OR-ed). */
+#define NSA_BWD_REUSE_INDEX 1u
+#define NSA_F16 2u
+/* The forward with options: flags = NSA_F16 makes q, k, v and out fp16 instead of bf16
+ * (same layouts; the partials stay fp16 and all arithmetic fp32, as for bf16).  Other
+ * flag bits return NSA_ERR_INVALID_ARG.  events / num_events / num_launches as in
+ * nsa_sel_attn_fwd_profiled (null / 0 for none). */
+NSA_API nsa_status_t nsa_sel_attn_fwd_ex(
+    const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
+    int total_tokens, int hq, int hkv, int head_dim, const int32_t *block_idx, int topk,
+    int block_size, float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+    nsa_stream_t stream, unsigned flags, void *const *events, int num_events, int *num_launches);
+
 /* The backward with options (flags, OR-ed):
  *   NSA_BWD_REUSE_INDEX  the workspace holds the block-index inversion that
  *       nsa_sel_attn_fwd (or _profiled) computed in it for the same cu_seqlens and
@@ -137,10 +151,11 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
  *       inputs (pointers or sizes), the call records NSA_ERR_INVALID_ARG in the device
  *       status (nsa_sel_check_status) and the outputs are undefined; the index contents
  *       themselves are not compared.
+ *   NSA_F16  q, k, v, out, dout, dq, dk, dv are fp16 instead of bf16 (the forward was
+ *       called with NSA_F16 too).
  * Other flag bits return NSA_ERR_INVALID_ARG.  events / num_events / num_launches as in
  * nsa_sel_attn_bwd_profiled (null / 0 for none).  Otherwise identical to
  * nsa_sel_attn_bwd. */
-#define NSA_BWD_REUSE_INDEX 1u
 NSA_API nsa_status_t nsa_sel_attn_bwd_ex(
     const void *q, const void *k, const void *v, const void *out, const float *lse,
     const void *dout, const int32_t *cu_seqlens, int num_seqs, int total_tokens, int hq, int hkv,

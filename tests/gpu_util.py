@@ -12,8 +12,8 @@ TOL_LSE = 1e-3      # max |LSE_gpu - LSE_ref|
 TOL_GRAD = 2e-2     # ||g_gpu - g_ref||_F / ||g_ref||_F for dQ, dK, dV
 
 
-def to_device(p: ni.Problem, dev="cuda"):
-    f = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16).contiguous()
+def to_device(p: ni.Problem, dev="cuda", dtype=torch.bfloat16):
+    f = lambda a: torch.from_numpy(a).to(dev).to(dtype).contiguous()
     d = dict(q=f(p.q), k=f(p.k), v=f(p.v),
              cu=torch.from_numpy(p.cu_seqlens).to(dev),
              bidx=torch.from_numpy(np.ascontiguousarray(p.block_idx)).to(dev))

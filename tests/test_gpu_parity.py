@@ -339,3 +339,44 @@ def test_bwd_reusing_forward_inversion():
                          p.scale, workspace=ws, reuse_index=True)
     torch.cuda.synchronize()
     assert nsa.nsa_sel_check_status(ws) == 1   # NSA_ERR_INVALID_ARG
+
+
+def test_fwd_without_lse():
+    # a forward with no backward: null LSE, the same output
+    p = ni.make_problem([900, 300], hq=8, hkv=2, block_size=64, topk=8, seed=43, with_dout=False)
+    d, out, _ = _fwd(p)
+    o2, l2 = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], 64, p.scale,
+                                  with_lse=False)
+    torch.cuda.synchronize()
+    assert l2 is None and torch.equal(o2, out)
+    assert nsa.nsa_sel_check_status() == 0
+
+
+FP16_CASES = [
+    ("f16_g4_bs64_k16", dict(lengths=[1500, 300], hq=8, hkv=2, block_size=64, topk=16, seed=51), True),
+    ("f16_g2_bs128_k8", dict(lengths=[900, 65], hq=4, hkv=2, block_size=128, topk=8, seed=52), False),
+]
+
+
+@pytest.mark.parametrize("name,spec,perturb", FP16_CASES, ids=[c[0] for c in FP16_CASES])
+def test_fp16_fwd_bwd_full_compare(name, spec, perturb):
+    # fp16 attention tensors: the generator's values rounded to fp16, and the oracle
+    # given exactly those values
+    p = ni.make_problem(name=name, **spec)
+    if perturb:
+        p = _perturb(p, 7)
+    for a in ("q", "k", "v", "dout"):
+        setattr(p, a, getattr(p, a).astype(np.float16).astype(np.float32))
+    d = to_device(p, dtype=torch.float16)
+    out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], p.block_size,
+                                    p.scale)
+    dq, dk, dv = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"],
+                                      d["bidx"], p.block_size, p.scale)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    assert out.dtype == dq.dtype == dk.dtype == dv.dtype == torch.float16
+    _check_fwd(p, out, lse)
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
+                               p.scale)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    assert max(e) <= TOL_GRAD, (name, e)
