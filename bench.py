@@ -191,7 +191,9 @@ def run_ours(args, rank, world, local_rank, dist):
     step_flops = fwd_flops + bwd_flops
     T, hq, hkv, d, topk, bs, nseq = p.T, p.hq, p.hkv, 128, p.topk, p.block_size, p.nseq
 
-    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16).pin_memory()
+    tdt = torch.float16 if args.dtype == "fp16" else torch.bfloat16
+    f16_flag = nsa.NSA_F16 if args.dtype == "fp16" else 0
+    bf = lambda a: torch.from_numpy(a).to(tdt).pin_memory()
     h_q, h_k, h_v, h_do = bf(p.q), bf(p.k), bf(p.v), bf(p.dout)
     h_cu = torch.from_numpy(p.cu_seqlens).pin_memory()
     h_bi = torch.from_numpy(np.ascontiguousarray(p.block_idx)).pin_memory()
@@ -220,9 +222,9 @@ def run_ours(args, rank, world, local_rank, dist):
         return ctypes.cast(arr, ctypes.c_void_p), arr
 
     def step(fwd_ev=None, bwd_ev=None, q_=q, k_=k, v_=v, do_=do, cu_=cu, bi_=bi):
-        rc = lib.nsa_sel_attn_fwd_profiled(
+        rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream),
+            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream), f16_flag,
             fwd_ev, 4 if fwd_ev is not None else 0, ctypes.byref(n_fwd))
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
@@ -230,7 +232,7 @@ def run_ours(args, rank, world, local_rank, dist):
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(out), sp(lse), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq), sp(dk), sp(dv), sp(ws), ws_bytes,
-            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX, bwd_ev,
+            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX | f16_flag, bwd_ev,
             6 if bwd_ev is not None else 0, ctypes.byref(n_bwd))
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
@@ -240,15 +242,15 @@ def run_ours(args, rank, world, local_rank, dist):
         q_, k_, v_, do_, cu_, bi_ = ins
         o_, l_, dq_, dk_, dv_ = outs
         h = ctypes.c_void_p(strm.cuda_stream)
-        rc = lib.nsa_sel_attn_fwd_profiled(
+        rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(o_), sp(l_), sp(ws), ws_bytes, h, None, 0, None)
+            sp(o_), sp(l_), sp(ws), ws_bytes, h, f16_flag, None, 0, None)
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(o_), sp(l_), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq_), sp(dk_), sp(dv_), sp(ws), ws_bytes, h,
-            nsa.NSA_BWD_REUSE_INDEX, None, 0, None)
+            nsa.NSA_BWD_REUSE_INDEX | f16_flag, None, 0, None)
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
 
@@ -400,7 +402,7 @@ def run_ours(args, rank, world, local_rank, dist):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO; index rule init+local+random earlier)",
         "config": {"workload": args.workload, "total_tokens": T, "num_seqs": nseq, "hq": hq,
                    "hkv": hkv, "group": hq // hkv, "head_dim": d, "block_size": bs, "topk": topk,
@@ -485,6 +487,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=ni.HEADLINE, choices=sorted(ni.WORKLOADS))
+    ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16",
+                    help="element type of q, k, v, dO and the outputs (fp32 arithmetic)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=2048)
