@@ -346,13 +346,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss_lo_e(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
+                        mma_ss_e(tS, aq + oa, dq_k + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
     #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t oa = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t ob = (uint32_t)((ks >> 2) * kKHalf + (ks & 3) * 2);
-                        mma_bf16_ss_lo_e(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
+                        mma_ss_e(tdP, ad + oa, dq_v + ob, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
                     mma_commit_e(&S.sdp_full[s], elected);
                     return true;
@@ -367,15 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int ks = 0; ks < 8; ++ks) {   // K = 128 rows, 16 per step (2048 bytes)
                         const uint32_t off = (uint32_t)ks * 128u;
                         const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-                        mma_bf16_ss_lo_e(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc, elected);
-                        mma_bf16_ss_lo_e(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc, elected);
+                        mma_ss_e(tmem + kColDV, ad + off, dt_p + off, kIdescT, acc, elected);
+                        mma_ss_e(tmem + kColDK, aq + off, dt_ds + off, kIdescT, acc, elected);
                     }
                     mma_commit_e(&S.q_empty[stg], elected);   // the stage is free once dV / dK have read it
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)   // K = BS keys
-                        mma_bf16_ss_lo_e(tmem + s * kSlotCols,
-                                    dk_ds + (uint32_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
-                                    dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u, elected);
+                        mma_ss_e(tmem + s * kSlotCols,
+                                 dk_ds + (uint32_t)((ks >> 2) * kPChunk + (ks & 3) * 2),
+                                 dk_kmn + (uint32_t)ks * 128u, kIdescQ, ks > 0 ? 1u : 0u, elected);
                     mma_commit_e(&S.dq_full[s], elected);
                     mma_commit_e(&S.pds_empty, elected);
                     if (last) {

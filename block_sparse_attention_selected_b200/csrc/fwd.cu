@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t off = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t offk = (uint32_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
-                        mma_bf16_ss_lo_e(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u, elected);
+                        mma_ss_e(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u, elected);
                     }
                     mma_commit_e(&S.s_full[slot], elected);
                     mma_commit_e(&S.q_empty[stg], elected);
@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b0 = v_desc0 + (uint32_t)kvs * kKvStage;
     #pragma unroll
                     for (int ks = 0; ks < BS / 16; ++ks)    // 16 keys = 2048 bytes per step
-                        mma_bf16_ts_lo_e(tO, tS + (uint32_t)ks * 8u, b0 + (uint32_t)ks * 128u, kIdescO,
-                                         ks > 0 ? 1u : 0u, elected);
+                        mma_ts_e(tO, tS + (uint32_t)ks * 8u, b0 + (uint32_t)ks * 128u, kIdescO,
+                                 ks > 0 ? 1u : 0u, elected);
                     mma_commit_e(&S.o_full[ob], elected);
                     if (release_kv) mma_commit_e(&S.kv_empty[kvs], elected);
                     return true;

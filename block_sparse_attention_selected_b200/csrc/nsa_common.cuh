@@ -209,38 +209,17 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate (kind::f16).
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// The same from the low 32 bits of two SW128 descriptors whose stride byte offset
-// is 1024 (start address and LBO); the high word (SBO, descriptor version, swizzle
-// mode) is then a constant, which saves a register per descriptor in the issuer.
+// tcgen05.mma of kind::f16 (A and B both bf16 or both fp16, as the instruction
+// descriptor says; fp32 accumulate in TMEM), issued warp-uniformly: the issuing warp
+// runs its whole loop with every lane (so that descriptors and loop state stay
+// warp-uniform) and one elected lane executes the tcgen05 instructions.  A single
+// issuing lane inside a divergent branch was measured to lose most of its issue slots
+// to busy warps on the same SM sub-partition (about 150 instead of 50 cycles per
+// M=128, N=64 MMA).  Shared-memory operands come as the low 32 bits of SW128
+// descriptors whose stride byte offset is 1024 (start address and LBO); the high word
+// (SBO, descriptor version, swizzle mode) is then a constant, which saves a register
+// per descriptor in the issuer.
 constexpr uint32_t kSw128Sbo1024DescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-__device__ __forceinline__ void mma_bf16_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                               uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-        "mov.b64 da, {%1, %5};\n\t"
-        "mov.b64 db, {%2, %5};\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "r"(kSw128Sbo1024DescHi)
-        : "memory");
-}
-
-// Warp-uniform MMA issue.  The issuing warp runs its whole loop with every lane (so
-// that descriptors and loop state stay warp-uniform) and one elected lane executes the
-// tcgen05 instructions.  A single issuing lane inside a divergent branch was measured
-// to lose most of its issue slots to busy warps on the same SM sub-partition (about
-// 150 instead of 50 cycles per M=128, N=64 MMA).
 __device__ __forceinline__ uint32_t elect_one() {
     uint32_t e;
     asm volatile(
@@ -250,9 +229,9 @@ __device__ __forceinline__ uint32_t elect_one() {
         : "=r"(e));
     return e;
 }
-__device__ __forceinline__ void mma_bf16_ss_lo_e(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                                 uint32_t idesc, uint32_t accumulate,
-                                                 uint32_t elected) {
+// D[tmem] (+)= A[smem] * B[smem]^T
+__device__ __forceinline__ void mma_ss_e(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                         uint32_t idesc, uint32_t accumulate, uint32_t elected) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
         "setp.ne.b32 e, %5, 0;\n\t"
@@ -264,10 +243,10 @@ __device__ __forceinline__ void mma_bf16_ss_lo_e(uint32_t d_tmem, uint32_t a_lo,
         "r"(kSw128Sbo1024DescHi)
         : "memory");
 }
-// TS form (A from TMEM), B from the low word of an SBO-1024 SW128 descriptor.
-__device__ __forceinline__ void mma_bf16_ts_lo_e(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                                 uint32_t idesc, uint32_t accumulate,
-                                                 uint32_t elected) {
+// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M rows x K, two 16-bit values per
+// 32-bit column, row = TMEM lane) is read from tensor memory.
+__device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                         uint32_t idesc, uint32_t accumulate, uint32_t elected) {
     asm volatile(
         "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\t"
         "setp.ne.b32 e, %5, 0;\n\t"
@@ -278,6 +257,7 @@ __device__ __forceinline__ void mma_bf16_ts_lo_e(uint32_t d_tmem, uint32_t a_tme
         "r"(kSw128Sbo1024DescHi)
         : "memory");
 }
+// Arrive on an mbarrier once all tcgen05 ops the elected lane issued before have finished.
 __device__ __forceinline__ void mma_commit_e(uint64_t* bar, uint32_t elected) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
@@ -287,27 +267,6 @@ __device__ __forceinline__ void mma_commit_e(uint64_t* bar, uint32_t elected) {
         "r"(elected)
         : "memory");
 }
-
-// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M rows x K, two bf16 per 32-bit
-// column, row = TMEM lane) is read from tensor memory (kind::f16).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive on an mbarrier once all previously issued tcgen05 ops of this thread finish.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
 
 // Store 32 consecutive 32-bit columns of this thread's TMEM lane (32x32b shape) and wait
 // for the store: source registers of tcgen05.st may be read asynchronously, so the wait
@@ -414,10 +373,7 @@ __host__ __device__ constexpr uint32_t idesc_f16kind_f32(bool f16, int M, int N,
            | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
-    return idesc_f16kind_f32(false, M, N, a_mn_major, b_mn_major);
-}
+
 
 // Byte offset of the 16-byte chunk `c16` (0..7) of row `r` inside a K-major tile whose
 // rows are 128 bytes, stored as 8-row x 128-byte atoms with the 128-byte swizzle.
