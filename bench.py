@@ -174,6 +174,28 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------- our arm
 
+def rank_spec(workload: str, rank: int) -> dict:
+    """Problem of one rank: the workload's shapes, its own seed (independent problems)."""
+    spec = dict(ni.WORKLOADS[workload])
+    spec["seed"] = spec["seed"] + 1000 * rank
+    return spec
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's value (the job time of a weak-scaling step)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, step_flops: float, steps: int, elapsed_ms: float) -> float:
+    """Useful TFLOP/s of the whole job: every rank's steps over the slowest rank's time."""
+    return world * step_flops * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank, dist):
     import torch
     import block_sparse_attention_selected_b200 as nsa
@@ -184,8 +206,7 @@ def run_ours(args, rank, world, local_rank, dist):
     nsa_build.build()
     lib = nsa.load_library()
 
-    spec = dict(ni.WORKLOADS[args.workload])
-    spec["seed"] = spec["seed"] + 1000 * rank
+    spec = rank_spec(args.workload, rank)
     p = ni.make_problem(name=args.workload, head_dim=128, with_dout=True, **spec)
     fwd_flops, bwd_flops = useful_flops(p)
     step_flops = fwd_flops + bwd_flops
@@ -258,12 +279,6 @@ def run_ours(args, rank, world, local_rank, dist):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # warm-up
     for _ in range(args.warmup):
@@ -297,11 +312,11 @@ def run_ours(args, rank, world, local_rank, dist):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    elapsed_ms = max_over_ranks(t0.elapsed_time(t1))
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     if nsa.nsa_sel_check_status(ws) != 0:
         raise RuntimeError("device status error in the timed region")
     ms_step = elapsed_ms / K
-    value = world * step_flops * K / (elapsed_ms * 1e-3) / 1e12
+    value = job_tflops(world, step_flops, K, elapsed_ms)
 
     def avg(evs, a, b):
         return statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
@@ -387,8 +402,8 @@ def run_ours(args, rank, world, local_rank, dist):
         run_e2e(Ke, a, b)
         torch.cuda.synchronize()
         barrier()
-        e_ms = max_over_ranks(a.elapsed_time(b))
-        e2e = {"value": round(world * step_flops * Ke / (e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
+        e2e = {"value": round(job_tflops(world, step_flops, Ke, e_ms), 3), "unit": UNIT,
                "ms_per_step": round(e_ms / Ke, 3), "steps": Ke,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "overlap": "H2D of step k+1 and D2H of step k-1 run on their own streams "
