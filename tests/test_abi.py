@@ -95,6 +95,38 @@ def test_host_argument_errors(lib):
     assert lib.nsa_sel_check_status(None, None) == 1
 
 
+def test_option_flags_checked_on_the_host(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)           # never dereferenced: the flag check comes first
+    # forward: only NSA_F16 (2) is an option
+    rc = lib.nsa_sel_attn_fwd_ex(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
+                                 fake, fake, fake, 1 << 30, None, 1, None, 0, None)
+    assert rc == 1
+    rc = lib.nsa_sel_attn_fwd_ex(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
+                                 fake, fake, fake, 1 << 30, None, 4, None, 0, None)
+    assert rc == 1
+    # backward: NSA_BWD_REUSE_INDEX (1) and NSA_F16 (2)
+    rc = lib.nsa_sel_attn_bwd_ex(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 128,
+                                 fake, 8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None, 8,
+                                 None, 0, None)
+    assert rc == 1
+    # a valid flag still reaches the usual argument checks (here: head_dim 64)
+    rc = lib.nsa_sel_attn_bwd_ex(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 64,
+                                 fake, 8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None, 3,
+                                 None, 0, None)
+    assert rc == 2
+    assert nsa.NSA_BWD_REUSE_INDEX == 1 and nsa.NSA_F16 == 2
+
+
+def test_binding_rejects_other_element_types():
+    import torch
+    x = torch.zeros((4, 2, 128), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        nsa._elem_type(x)
+    assert nsa._elem_type(x.to(torch.float16))[1] == nsa.NSA_F16
+    assert nsa._elem_type(x.to(torch.bfloat16))[1] == 0
+
+
 def test_product_path_has_no_oracle_dependency():
     """The package and its sources never import, link or call the oracle."""
     pkg = os.path.join(ROOT, "block_sparse_attention_selected_b200")
