@@ -15,6 +15,9 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
 * ``bwd``            pinned: central finite differences, torch float64 autograd in
                      the dense-causal case, the identity D = <dO, O>.
 * ``bwd_dq`` / ``bwd_dkdv_keys``  pinned against ``bwd`` (itself pinned).
+* ``window`` (all four)  pinned: dense selection with a window against torch float64
+                     SDPA / autograd under an explicit band mask, W = 1 closed form,
+                     a window wider than every sequence changes nothing.
 * ``invert``         pinned: brute-force nested loops on tiny inputs, round trip,
                      sortedness, counts.
 """
@@ -56,14 +59,14 @@ def _load():
             L = ctypes.c_int64
             D = ctypes.c_double
             common = [P, P, P, P, I, I, I, I, P, I, I, D]
-            lib.nsa_oracle_fwd.argtypes = common[:] + [P, L, P, P, I]
+            lib.nsa_oracle_fwd.argtypes = common[:] + [P, L, P, P, L, I]
             lib.nsa_oracle_fwd.restype = I
-            lib.nsa_oracle_bwd.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, D, P, P, P, I]
+            lib.nsa_oracle_bwd.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, D, P, P, P, L, I]
             lib.nsa_oracle_bwd.restype = I
-            lib.nsa_oracle_bwd_dq.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, D, P, L, P, I]
+            lib.nsa_oracle_bwd_dq.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, D, P, L, P, L, I]
             lib.nsa_oracle_bwd_dq.restype = I
             lib.nsa_oracle_bwd_dkdv_keys.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, D,
-                                                     I, L, I, P, P, I]
+                                                     I, L, I, P, P, L, I]
             lib.nsa_oracle_bwd_dkdv_keys.restype = I
             lib.nsa_oracle_num_blocks.argtypes = [P, I, I]
             lib.nsa_oracle_num_blocks.restype = L
@@ -92,8 +95,11 @@ def _shape_args(q, k, cu, block_idx):
     return T, hq, hkv, d, topk, len(cu) - 1
 
 
-def fwd(q, k, v, cu_seqlens, block_idx, block_size, scale, tokens=None, nthreads=0):
-    """O [ntok, hq, d] float64 and LSE [ntok, hq] float64 for the listed tokens."""
+def fwd(q, k, v, cu_seqlens, block_idx, block_size, scale, tokens=None, nthreads=0, window=0):
+    """O [ntok, hq, d] float64 and LSE [ntok, hq] float64 for the listed tokens.
+
+    window > 0 restricts every query at local position i to keys j > i - window as well
+    (a sliding window of that many positions, the query's own included)."""
     lib = _load()
     q, k, v = _f32(q), _f32(k), _f32(v)
     cu, bi = _i32(cu_seqlens), _i32(block_idx)
@@ -104,14 +110,14 @@ def fwd(q, k, v, cu_seqlens, block_idx, block_size, scale, tokens=None, nthreads
     lse = np.empty((ntok, hq), dtype=np.float64)
     rc = lib.nsa_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), nseq, hq, hkv, d, _ptr(bi),
                             topk, block_size, float(scale), _ptr(toks), ntok, _ptr(out),
-                            _ptr(lse), int(nthreads))
+                            _ptr(lse), int(window), int(nthreads))
     if rc:
         raise RuntimeError(f"oracle fwd failed: {rc}")
     return out, lse
 
 
-def bwd(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, nthreads=0):
-    """Full backward: dQ [T, hq, d], dK, dV [T, hkv, d] float64."""
+def bwd(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, nthreads=0, window=0):
+    """Full backward: dQ [T, hq, d], dK, dV [T, hkv, d] float64 (window as in fwd)."""
     lib = _load()
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
     cu, bi = _i32(cu_seqlens), _i32(block_idx)
@@ -121,14 +127,15 @@ def bwd(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, nthreads=0):
     dv = np.empty((T, hkv, d), dtype=np.float64)
     rc = lib.nsa_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu), nseq, hq, hkv, d,
                             _ptr(bi), topk, block_size, float(scale), _ptr(dq), _ptr(dk),
-                            _ptr(dv), int(nthreads))
+                            _ptr(dv), int(window), int(nthreads))
     if rc:
         raise RuntimeError(f"oracle bwd failed: {rc}")
     return dq, dk, dv
 
 
-def bwd_dq(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, tokens, nthreads=0):
-    """dQ [ntok, hq, d] float64 for the listed tokens."""
+def bwd_dq(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, tokens, nthreads=0,
+           window=0):
+    """dQ [ntok, hq, d] float64 for the listed tokens (window as in fwd)."""
     lib = _load()
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
     cu, bi = _i32(cu_seqlens), _i32(block_idx)
@@ -137,15 +144,16 @@ def bwd_dq(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, tokens, nthr
     dq = np.empty((len(toks), hq, d), dtype=np.float64)
     rc = lib.nsa_oracle_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu), nseq, hq, hkv, d,
                                _ptr(bi), topk, block_size, float(scale), _ptr(toks), len(toks),
-                               _ptr(dq), int(nthreads))
+                               _ptr(dq), int(window), int(nthreads))
     if rc:
         raise RuntimeError(f"oracle bwd_dq failed: {rc}")
     return dq
 
 
 def bwd_dkdv_keys(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, g, key0, nkeys,
-                  nthreads=0):
-    """dK, dV [nkeys, d] float64 of KV head g for keys key0 .. key0+nkeys-1 (one sequence)."""
+                  nthreads=0, window=0):
+    """dK, dV [nkeys, d] float64 of KV head g for keys key0 .. key0+nkeys-1 (one sequence;
+    window as in fwd)."""
     lib = _load()
     q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
     cu, bi = _i32(cu_seqlens), _i32(block_idx)
@@ -154,7 +162,8 @@ def bwd_dkdv_keys(q, k, v, dout, cu_seqlens, block_idx, block_size, scale, g, ke
     dv = np.empty((nkeys, d), dtype=np.float64)
     rc = lib.nsa_oracle_bwd_dkdv_keys(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(cu), nseq, hq,
                                       hkv, d, _ptr(bi), topk, block_size, float(scale), int(g),
-                                      int(key0), int(nkeys), _ptr(dk), _ptr(dv), int(nthreads))
+                                      int(key0), int(nkeys), _ptr(dk), _ptr(dv), int(window),
+                                      int(nthreads))
     if rc:
         raise RuntimeError(f"oracle bwd_dkdv_keys failed: {rc}")
     return dk, dv

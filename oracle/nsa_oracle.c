@@ -15,6 +15,9 @@
  *
  *     Sel(t, g) = { b = block_idx[t, g, j] : 0 <= b < NB_s }  (a set; -1 pads)
  *     J(t, g)   = { j : floor(j / bs) in Sel(t, g), 0 <= j <= i }  (causal)
+ *                 and, with a sliding window W > 0, also j > i - W (the module's
+ *                 window_size of the project page's quick start: a query sees the W
+ *                 most recent positions, itself included)
  *     s_j       = scale * <q[t, h], k[c_s + j, g]>
  *     LSE       = log sum_{j in J} exp(s_j)   (computed as m + log sum exp(s_j - m))
  *     p_j       = exp(s_j - LSE)
@@ -57,6 +60,7 @@ typedef struct {
     int nseq, hq, hkv, d, topk, bs;
     const int32_t *bidx;
     double scale;
+    int64_t window;     /* 0: none; else keys j > i - window only */
 } problem_t;
 
 static int seq_of(const problem_t *P, int64_t t) {
@@ -81,7 +85,8 @@ static int64_t selected_keys(const problem_t *P, int64_t t, int g, unsigned char
         int32_t b = P->bidx[(t * P->hkv + g) * P->topk + j];
         if (b >= 0 && b < NB) blocksel[b] = 1;
     }
-    for (int64_t j = 0; j <= i; ++j) allowed[j] = blocksel[j / P->bs];
+    for (int64_t j = 0; j <= i; ++j)
+        allowed[j] = blocksel[j / P->bs] && (P->window <= 0 || j > i - P->window);
     *c_out = c;
     return i;
 }
@@ -128,7 +133,7 @@ static int check_problem(const problem_t *P) {
 
 #define MAKE_PROBLEM                                                                   \
     problem_t P = {q, k, v, cu_seqlens, nseq, hq, hkv, d, topk, block_size, block_idx, \
-                   scale};                                                             \
+                   scale, window};                                                     \
     if (check_problem(&P)) return ORACLE_ERR_ARG;
 
 static void set_threads(int nthreads) {
@@ -144,7 +149,7 @@ static void set_threads(int nthreads) {
 int nsa_oracle_fwd(const float *q, const float *k, const float *v, const int32_t *cu_seqlens,
                    int nseq, int hq, int hkv, int d, const int32_t *block_idx, int topk,
                    int block_size, double scale, const int64_t *tokens, int64_t ntok,
-                   double *out, double *lse, int nthreads) {
+                   double *out, double *lse, int64_t window, int nthreads) {
     MAKE_PROBLEM
     int64_t Lmax = max_len(&P);
     int64_t NBmax = (Lmax + block_size - 1) / block_size;
@@ -217,7 +222,7 @@ static double row_dp_and_D(const problem_t *P, const float *dout, int64_t t, int
 int nsa_oracle_bwd(const float *q, const float *k, const float *v, const float *dout,
                    const int32_t *cu_seqlens, int nseq, int hq, int hkv, int d,
                    const int32_t *block_idx, int topk, int block_size, double scale,
-                   double *dq, double *dk, double *dv, int nthreads) {
+                   double *dq, double *dk, double *dv, int64_t window, int nthreads) {
     MAKE_PROBLEM
     if (!dout) return ORACLE_ERR_ARG;
     int64_t T = cu_seqlens[nseq];
@@ -298,7 +303,8 @@ int nsa_oracle_bwd(const float *q, const float *k, const float *v, const float *
 int nsa_oracle_bwd_dq(const float *q, const float *k, const float *v, const float *dout,
                       const int32_t *cu_seqlens, int nseq, int hq, int hkv, int d,
                       const int32_t *block_idx, int topk, int block_size, double scale,
-                      const int64_t *tokens, int64_t ntok, double *dq, int nthreads) {
+                      const int64_t *tokens, int64_t ntok, double *dq, int64_t window,
+                      int nthreads) {
     MAKE_PROBLEM
     if (!dout || !tokens) return ORACLE_ERR_ARG;
     int64_t Lmax = max_len(&P);
@@ -353,7 +359,7 @@ int nsa_oracle_bwd_dkdv_keys(const float *q, const float *k, const float *v, con
                              const int32_t *cu_seqlens, int nseq, int hq, int hkv, int d,
                              const int32_t *block_idx, int topk, int block_size, double scale,
                              int g, int64_t key0, int nkeys, double *dk, double *dv,
-                             int nthreads) {
+                             int64_t window, int nthreads) {
     MAKE_PROBLEM
     if (!dout || g < 0 || g >= hkv || nkeys < 1) return ORACLE_ERR_ARG;
     int s = seq_of(&P, key0);

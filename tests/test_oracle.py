@@ -374,3 +374,87 @@ def test_inputs_recipe():
     x = np.array([1.0, 1.00390625, 1.005859375, -2.0e-3, 3.3], dtype=np.float32)
     r = ni.bf16_round(x)
     assert np.array_equal(r, torch.from_numpy(x).to(torch.bfloat16).float().numpy())
+
+
+# --------------------------------------------------------------------------- sliding window
+# window W > 0 keeps, of the selected keys, those with j > i - W (the W most recent
+# positions, the query's own included; the module's window_size in the project page's
+# quick start).
+
+def _band_sdpa_f64(q, k, v, dout, cu, scale, W):
+    """Dense causal attention restricted to a band of W positions, torch float64 with an
+    explicit boolean mask (forward, LSE and the autograd backward of sum(dO * O))."""
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    G = hq // hkv
+    qt = torch.from_numpy(q.astype(np.float64)).requires_grad_()
+    kt = torch.from_numpy(k.astype(np.float64)).requires_grad_()
+    vt = torch.from_numpy(v.astype(np.float64)).requires_grad_()
+    outs, lses, loss = [], [], 0
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        L = b - a
+        i = torch.arange(L)
+        mask = (i[None, :] <= i[:, None]) & (i[None, :] > i[:, None] - W)
+        qs = qt[a:b].permute(1, 0, 2)
+        ks = kt[a:b].repeat_interleave(G, 1).permute(1, 0, 2)
+        vs = vt[a:b].repeat_interleave(G, 1).permute(1, 0, 2)
+        o = torch.nn.functional.scaled_dot_product_attention(qs, ks, vs, attn_mask=mask, scale=scale)
+        sc = ((qs @ ks.transpose(1, 2)) * scale).masked_fill(~mask, float("-inf"))
+        outs.append(o.permute(1, 0, 2))
+        lses.append(torch.logsumexp(sc, dim=-1).permute(1, 0))
+        loss = loss + (o.permute(1, 0, 2) * torch.from_numpy(dout[a:b].astype(np.float64))).sum()
+    loss.backward()
+    return (torch.cat(outs).detach().numpy(), torch.cat(lses).detach().numpy(),
+            qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy())
+
+
+@pytest.mark.parametrize("W", [1, 5, 16, 23])
+def test_window_dense_selection_matches_band_sdpa(W):
+    lengths, hq, hkv, bs = [64, 37, 1], 4, 2, 16
+    cu = ni.cu_seqlens_from_lengths(lengths)
+    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=32, block_size=bs, topk=6, seed=61,
+                        block_idx=_all_blocks_idx(cu, hkv, bs, 6, np.random.default_rng(7)))
+    o, l = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, bs, p.scale, window=W)
+    dq, dk, dv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, bs, p.scale,
+                            window=W)
+    ro, rl, rdq, rdk, rdv = _band_sdpa_f64(p.q, p.k, p.v, p.dout, cu, p.scale, W)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, rl, rtol=0, atol=1e-12)
+    for a, b in ((dq, rdq), (dk, rdk), (dv, rdv)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-11)
+
+
+def test_window_closed_forms_and_invariance():
+    p = ni.make_problem([300, 90], hq=4, hkv=2, head_dim=32, block_size=16, topk=5, seed=62)
+    base = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, 16, p.scale)
+    wide = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, 16, p.scale, window=300)
+    assert np.array_equal(base[0], wide[0]) and np.array_equal(base[1], wide[1])
+    gb = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, 16, p.scale)
+    gw = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, 16, p.scale, window=300)
+    for a, b in zip(gb, gw):   # dK / dV sum over OpenMP threads: equal up to that order
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+    # W = 1: every query sees only itself (its own block is always selected)
+    o, l = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, 16, p.scale, window=1)
+    G = 2
+    for t in (0, 17, 299, 300, 389):
+        for h in range(4):
+            kk = p.k[t, h // G].astype(np.float64)
+            np.testing.assert_allclose(o[t, h], p.v[t, h // G].astype(np.float64), rtol=0, atol=1e-15)
+            assert l[t, h] == pytest.approx(p.scale * float(kk @ p.q[t, h].astype(np.float64)),
+                                            rel=0, abs=1e-12)
+
+
+def test_window_partial_entry_points_match_full():
+    p = ni.make_problem([200], hq=4, hkv=1, head_dim=32, block_size=16, topk=6, seed=63)
+    W = 40
+    dq, dk, dv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, 16, p.scale,
+                            window=W)
+    toks = np.array([0, 39, 40, 41, 150, 199])
+    np.testing.assert_allclose(
+        oracle.bwd_dq(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, 16, p.scale, toks,
+                      window=W), dq[toks], rtol=0, atol=1e-13)
+    k2, v2 = oracle.bwd_dkdv_keys(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, 16, p.scale,
+                                  0, 32, 48, window=W)
+    np.testing.assert_allclose(k2, dk[32:80, 0], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(v2, dv[32:80, 0], rtol=0, atol=1e-13)
