@@ -26,7 +26,7 @@
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers, contiguous, in the layouts stated.
- *    bf16 tensors and the workspace must be 16-byte aligned, int32/fp32 ones
+ *    16-bit tensors and the workspace must be 16-byte aligned, int32/fp32 ones
  *    4-byte aligned.
  *  - The caller owns every buffer, including the workspace; the library allocates
  *    nothing and keeps no state between calls.
@@ -37,7 +37,8 @@
  *    problems (a bounded wait that expired, malformed cu_seqlens) are recorded
  *    in the status block at the start of the workspace and read with
  *    nsa_sel_check_status.  No C++ exception crosses this interface.
- *  - Supported domain: bf16, head_dim == 128, block_size in {64, 128},
+ *  - Supported domain: bf16 (fp16 through the _ex calls' NSA_F16), head_dim == 128,
+ *    block_size in {64, 128},
  *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv a divisor of 128 (a 128-row tile
  *    holds whole query-head groups), total_tokens < 2^25.
  *    Anything else returns NSA_ERR_UNSUPPORTED.
