@@ -98,13 +98,14 @@ def _brute_fwd(q, k, v, M, scale):
 
 # --------------------------------------------------------------------------- forward pins
 
-@pytest.mark.parametrize("lengths,hq,hkv,bs", [([96], 4, 2, 16), ([40, 70, 1, 17], 2, 1, 16),
-                                              ([130], 8, 2, 32)])
-def test_fwd_dense_causal_equals_sdpa(lengths, hq, hkv, bs):
-    """topk covering every causal block reduces to dense causal attention."""
+@pytest.mark.parametrize("lengths,hq,hkv,bs,d", [([96], 4, 2, 16, 32), ([40, 70, 1, 17], 2, 1, 16, 32),
+                                                ([130], 8, 2, 32, 32), ([70], 2, 1, 32, 64),
+                                                ([70], 2, 2, 32, 128), ([45], 4, 1, 16, 256)])
+def test_fwd_dense_causal_equals_sdpa(lengths, hq, hkv, bs, d):
+    """topk covering every causal block reduces to dense causal attention (any head dim)."""
     cu = ni.cu_seqlens_from_lengths(lengths)
     nb = max((L + bs - 1) // bs for L in lengths)
-    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=32, block_size=bs, topk=nb + 1, seed=11,
+    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=d, block_size=bs, topk=nb + 1, seed=11,
                         block_idx=_all_blocks_idx(cu, hkv, bs, nb + 1, np.random.default_rng(3)))
     o, l = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, bs, p.scale)
     ro, rl = _sdpa_causal_f64(p.q, p.k, p.v, p.cu_seqlens, p.scale)
@@ -245,11 +246,12 @@ def test_bwd_finite_differences():
             assert abs(fd - an) <= 2e-6 * max(1.0, abs(an)), (name, fd, an)
 
 
-def test_bwd_dense_causal_matches_autograd():
+@pytest.mark.parametrize("d", [32, 64, 256])
+def test_bwd_dense_causal_matches_autograd(d):
     lengths, hq, hkv, bs = [64, 37], 4, 2, 16
     cu = ni.cu_seqlens_from_lengths(lengths)
     nb = 4
-    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=32, block_size=bs, topk=nb + 2, seed=12,
+    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=d, block_size=bs, topk=nb + 2, seed=12,
                         block_idx=_all_blocks_idx(cu, hkv, bs, nb + 2, np.random.default_rng(5)))
     dq, dk, dv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, bs, p.scale)
     G = hq // hkv
