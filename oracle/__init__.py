@@ -20,6 +20,10 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
                      a window wider than every sequence changes nothing.
 * ``invert``         pinned: brute-force nested loops on tiny inputs, round trip,
                      sortedness, counts.
+
+The block-selection step that produces ``block_idx`` (compression, compressed
+attention, block scores, top-k) is the numpy module ``oracle.selection``, pinned in
+``tests/test_selection_oracle.py``.
 """
 from __future__ import annotations
 
