@@ -129,14 +129,23 @@ def nsa_sel_attn_workspace_size(total_tokens, num_seqs, hq, hkv, head_dim, topk,
     return int(n)
 
 
+def _ws_key(dev: torch.device):
+    # one cached workspace per (device, stream): calls on different streams may overlap
+    # on the GPU and must not share scratch memory
+    return (dev, torch.cuda.current_stream(dev).cuda_stream)
+
+
 def get_workspace(nbytes: int, device) -> torch.Tensor:
-    """A cached uint8 device buffer of at least nbytes (grown on demand)."""
+    """A cached uint8 device buffer of at least nbytes (grown on demand) for the
+    device's current stream; it is allocated on that stream, so the caching allocator
+    orders its reuse after the calls that used it."""
     dev = torch.device(device)
-    ws = _ws_cache.get(dev)
+    key = _ws_key(dev)
+    ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
-        _ws_cache.pop(dev, None)
+        _ws_cache.pop(key, None)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-        _ws_cache[dev] = ws
+        _ws_cache[key] = ws
     return ws
 
 
@@ -290,9 +299,10 @@ def nsa_sel_validate_indices(cu_seqlens, block_idx, block_size, workspace=None):
 
 
 def nsa_sel_check_status(workspace=None, device=None) -> int:
-    """Device-side status of the last call that used this workspace (synchronises)."""
+    """Device-side status of the last call that used this workspace (synchronises); by
+    default the cached workspace of the device's current stream."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    ws = workspace if workspace is not None else _ws_cache.get(dev)
+    ws = workspace if workspace is not None else _ws_cache.get(_ws_key(dev))
     if ws is None:
         return NSA_OK
     return int(load_library().nsa_sel_check_status(_ptr(ws), _stream(ws.device)))

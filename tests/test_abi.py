@@ -135,3 +135,29 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.lower().replace("oracle_", ""), f
+
+
+def test_cached_workspace_is_per_stream(monkeypatch):
+    """Host logic of the binding's workspace cache, with the CUDA calls faked: one buffer
+    per (device, stream), grown on demand, reused on the same stream."""
+    import types
+    import torch
+    current = {"s": 11}
+    monkeypatch.setattr(torch.cuda, "current_stream",
+                        lambda dev=None: types.SimpleNamespace(cuda_stream=current["s"]))
+    real_empty = torch.empty
+    monkeypatch.setattr(torch, "empty", lambda n, dtype=None, device=None: real_empty(n, dtype=dtype))
+    nsa.release_workspaces()
+    dev = torch.device("cuda", 0)
+    a = nsa.get_workspace(100, dev)
+    assert nsa.get_workspace(50, dev) is a                  # same stream: reused
+    current["s"] = 22
+    b = nsa.get_workspace(50, dev)
+    assert b is not a                                       # another stream: its own buffer
+    current["s"] = 11
+    c = nsa.get_workspace(400, dev)
+    assert c is not a and c.numel() >= 400                  # grown on demand
+    assert nsa.get_workspace(10, dev) is c
+    current["s"] = 22
+    assert nsa.get_workspace(10, dev) is b
+    nsa.release_workspaces()
