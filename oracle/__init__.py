@@ -23,7 +23,8 @@ Parity status of each function (what pins it, see ``tests/test_oracle.py``):
 
 The block-selection step that produces ``block_idx`` (compression, compressed
 attention, block scores, top-k) is the numpy module ``oracle.selection``, pinned in
-``tests/test_selection_oracle.py``.
+``tests/test_selection_oracle.py``; threshold-pruned block attention (BSFA) is
+``oracle.bsfa``, pinned in ``tests/test_bsfa_oracle.py``.
 """
 from __future__ import annotations
 
