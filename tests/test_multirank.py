@@ -38,7 +38,8 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_weak_scaling_gloo():
     world, port = 2, _free_port()
-    with mp.Manager() as mgr:
+    # the manager process is spawned, not forked: the test process already runs threads
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         r = dict(out)
