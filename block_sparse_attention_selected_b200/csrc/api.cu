@@ -69,6 +69,8 @@ nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int b
     if ((long long)hkv * D->nwin * (D->nb_stride + 1) >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;
     D->fwd_tiles_cap = (nent + tpt - 1) / tpt +
                        std::min<long long>(nent, (long long)hkv * D->nwin * D->nb_stride);
+    // forward partial rows are addressed by 32-bit TMA row coordinates and row indices
+    if (D->fwd_tiles_cap * kTileRows >= (1ll << 31)) return NSA_ERR_UNSUPPORTED;
     return NSA_OK;
 }
 

@@ -59,6 +59,10 @@ def test_workspace_size_domain(lib):
     assert f(1024, 1, 6, 2, 128, 8, 64, 0) == 0         # group 3 does not divide 128
     assert f(1024, 1, 6, 4, 128, 8, 64, 0) == 0         # hq % hkv != 0
     assert f(1 << 25, 1, 4, 4, 128, 8, 64, 0) == 0      # too many tokens
+    # 2^22 tokens of 128 heads over one KV head, top-64: 2^35 forward partial rows,
+    # beyond 32-bit row coordinates (and any device memory)
+    assert f(1 << 22, 1, 128, 1, 128, 64, 64, 0) == 0
+    assert f(1 << 16, 1, 128, 1, 128, 64, 64, 0) > 0
 
 
 def test_host_argument_errors(lib):
