@@ -40,8 +40,10 @@
  *  - Supported domain: bf16 (fp16 through the _ex calls' NSA_F16), head_dim == 128,
  *    block_size in {64, 128},
  *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv a divisor of 128 (a 128-row tile
- *    holds whole query-head groups), total_tokens < 2^25.
- *    Anything else returns NSA_ERR_UNSUPPORTED.
+ *    holds whole query-head groups), total_tokens < 2^25, and (for 32-bit row
+ *    coordinates) total_tokens * hkv * topk < 2^31, total_tokens * hq < 2^31 and
+ *    fewer than 2^31 forward partial rows (about total_tokens * hq * topk; far
+ *    beyond any device memory).  Anything else returns NSA_ERR_UNSUPPORTED.
  */
 #ifndef NSA_SEL_H
 #define NSA_SEL_H
