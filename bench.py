@@ -245,7 +245,7 @@ def run_ours(args, rank, world, local_rank, dist):
     def step(fwd_ev=None, bwd_ev=None, q_=q, k_=k, v_=v, do_=do, cu_=cu, bi_=bi):
         rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream), f16_flag,
+            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream), f16_flag, 0,
             fwd_ev, 4 if fwd_ev is not None else 0, ctypes.byref(n_fwd))
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
@@ -253,7 +253,7 @@ def run_ours(args, rank, world, local_rank, dist):
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(out), sp(lse), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq), sp(dk), sp(dv), sp(ws), ws_bytes,
-            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX | f16_flag, bwd_ev,
+            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX | f16_flag, 0, bwd_ev,
             6 if bwd_ev is not None else 0, ctypes.byref(n_bwd))
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
@@ -265,13 +265,13 @@ def run_ours(args, rank, world, local_rank, dist):
         h = ctypes.c_void_p(strm.cuda_stream)
         rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(o_), sp(l_), sp(ws), ws_bytes, h, f16_flag, None, 0, None)
+            sp(o_), sp(l_), sp(ws), ws_bytes, h, f16_flag, 0, None, 0, None)
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(o_), sp(l_), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq_), sp(dk_), sp(dv_), sp(ws), ws_bytes, h,
-            nsa.NSA_BWD_REUSE_INDEX | f16_flag, None, 0, None)
+            nsa.NSA_BWD_REUSE_INDEX | f16_flag, 0, None, 0, None)
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
 
