@@ -384,22 +384,6 @@ def test_fp16_fwd_bwd_full_compare(name, spec, perturb):
 
 # ------------------------------------------------------------------ sliding window
 
-def _band_idx(p, W):
-    """block_idx of the sliding branch: the blocks qb, qb - 1, .. that the window of W
-    keys reaches (distinct, -1 padded), so that selection with the window is the band."""
-    cu = p.cu_seqlens.astype(np.int64)
-    T, hkv, topk = p.block_idx.shape
-    bi = np.full((T, hkv, topk), -1, dtype=np.int32)
-    for s in range(len(cu) - 1):
-        for t in range(int(cu[s]), int(cu[s + 1])):
-            qb = (t - int(cu[s])) // p.block_size
-            blocks = np.arange(qb, max(qb - (W + p.block_size - 1) // p.block_size, -1) - 1, -1)
-            blocks = blocks[blocks >= 0][:topk]
-            bi[t, :, :len(blocks)] = blocks
-    p.block_idx = bi
-    return p
-
-
 WINDOW_CASES = [
     # name, problem, window, perturb
     ("w512_g4_bs64_k16", dict(lengths=[1500, 40, 700], hq=8, hkv=2, block_size=64, topk=16, seed=61), 512, True),
@@ -440,7 +424,7 @@ def test_window_fwd_bwd_full_compare(name, spec, W, perturb):
 def test_window_sliding_branch_is_band_attention(bs, W):
     # the sliding branch: every block the window reaches selected -> banded causal attention
     p = ni.make_problem([2100, 333], hq=8, hkv=2, block_size=bs, topk=16, seed=65)
-    p = _band_idx(p, W)
+    p.block_idx = ni.band_block_idx(p.cu_seqlens, p.hkv, p.topk, bs, W)
     d = to_device(p)
     out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], bs, p.scale,
                                     window_size=W)
