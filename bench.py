@@ -44,8 +44,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ----------------------------------------------------------------------------- work
 
-def attended_keys(cu_seqlens, block_idx, block_size):
-    """Keys each (token, KV head) row attends after the causal mask (counting only)."""
+def attended_keys(cu_seqlens, block_idx, block_size, window=0):
+    """Keys each (token, KV head) row attends after the causal mask and, for window > 0,
+    the sliding window of that many keys (counting only)."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     T, hkv, topk = block_idx.shape
     out = np.zeros((T, hkv), dtype=np.int64)
@@ -60,14 +61,20 @@ def attended_keys(cu_seqlens, block_idx, block_size):
         first = np.ones_like(x, dtype=bool)
         first[:, :, 1:] = x[:, :, 1:] != x[:, :, :-1]
         keep = first & (x >= 0)
-        full = (keep & (x < qb)).sum(axis=2)
-        diag = (keep & (x == qb)).sum(axis=2)
-        out[a:b] = full * block_size + diag * ((i % block_size) + 1)[:, None]
+        if window <= 0:
+            full = (keep & (x < qb)).sum(axis=2)
+            diag = (keep & (x == qb)).sum(axis=2)
+            out[a:b] = full * block_size + diag * ((i % block_size) + 1)[:, None]
+        else:
+            ii = i[:, None, None]
+            lo = np.maximum(x * block_size, ii - window + 1)
+            hi = np.minimum((x + 1) * block_size - 1, ii)
+            out[a:b] = np.where(keep, np.maximum(hi - lo + 1, 0), 0).sum(axis=2)
     return out
 
 
-def useful_flops(p: ni.Problem):
-    keys = attended_keys(p.cu_seqlens, p.block_idx, p.block_size)
+def useful_flops(p: ni.Problem, window=0):
+    keys = attended_keys(p.cu_seqlens, p.block_idx, p.block_size, window)
     G = p.hq // p.hkv
     fwd = 4.0 * p.head_dim * float(keys.sum()) * G
     return fwd, 2.5 * fwd
@@ -208,7 +215,10 @@ def run_ours(args, rank, world, local_rank, dist):
 
     spec = rank_spec(args.workload, rank)
     p = ni.make_problem(name=args.workload, head_dim=128, with_dout=True, **spec)
-    fwd_flops, bwd_flops = useful_flops(p)
+    W = args.window
+    if W > 0:   # the sliding branch: every block the window reaches, then the window mask
+        p.block_idx = ni.band_block_idx(p.cu_seqlens, p.hkv, p.topk, p.block_size, W)
+    fwd_flops, bwd_flops = useful_flops(p, W)
     step_flops = fwd_flops + bwd_flops
     T, hq, hkv, d, topk, bs, nseq = p.T, p.hq, p.hkv, 128, p.topk, p.block_size, p.nseq
 
@@ -245,7 +255,7 @@ def run_ours(args, rank, world, local_rank, dist):
     def step(fwd_ev=None, bwd_ev=None, q_=q, k_=k, v_=v, do_=do, cu_=cu, bi_=bi):
         rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream), f16_flag,
+            sp(out), sp(lse), sp(ws), ws_bytes, ctypes.c_void_p(stream.cuda_stream), f16_flag, W,
             fwd_ev, 4 if fwd_ev is not None else 0, ctypes.byref(n_fwd))
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
@@ -253,7 +263,7 @@ def run_ours(args, rank, world, local_rank, dist):
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(out), sp(lse), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq), sp(dk), sp(dv), sp(ws), ws_bytes,
-            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX | f16_flag, bwd_ev,
+            ctypes.c_void_p(stream.cuda_stream), nsa.NSA_BWD_REUSE_INDEX | f16_flag, W, bwd_ev,
             6 if bwd_ev is not None else 0, ctypes.byref(n_bwd))
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
@@ -265,13 +275,13 @@ def run_ours(args, rank, world, local_rank, dist):
         h = ctypes.c_void_p(strm.cuda_stream)
         rc = lib.nsa_sel_attn_fwd_ex(
             sp(q_), sp(k_), sp(v_), sp(cu_), nseq, T, hq, hkv, d, sp(bi_), topk, bs, scale,
-            sp(o_), sp(l_), sp(ws), ws_bytes, h, f16_flag, None, 0, None)
+            sp(o_), sp(l_), sp(ws), ws_bytes, h, f16_flag, W, None, 0, None)
         if rc:
             raise RuntimeError(f"forward failed: {rc}")
         rc = lib.nsa_sel_attn_bwd_ex(
             sp(q_), sp(k_), sp(v_), sp(o_), sp(l_), sp(do_), sp(cu_), nseq, T, hq, hkv, d,
             sp(bi_), topk, bs, scale, sp(dq_), sp(dk_), sp(dv_), sp(ws), ws_bytes, h,
-            nsa.NSA_BWD_REUSE_INDEX | f16_flag, None, 0, None)
+            nsa.NSA_BWD_REUSE_INDEX | f16_flag, W, None, 0, None)
         if rc:
             raise RuntimeError(f"backward failed: {rc}")
 
@@ -411,16 +421,19 @@ def run_ours(args, rank, world, local_rank, dist):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, tokens=args.cpu_tokens)
+        cpu = cpu_baseline(args.workload, tokens=args.cpu_tokens, window=W)
 
     launches = K * (n_fwd.value + n_bwd.value)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
-        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO; index rule init+local+random earlier)",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO; index rule init+local+random earlier)"
+                if W == 0 else "synthetic (seeded N(0,1) bf16 Q/K/V/dO; sliding-branch index: "
+                               "every block the window reaches)",
         "config": {"workload": args.workload, "total_tokens": T, "num_seqs": nseq, "hq": hq,
                    "hkv": hkv, "group": hq // hkv, "head_dim": d, "block_size": bs, "topk": topk,
+                   "window_size": W,
                    "parallelism": f"independent problem per rank x{world}",
                    "l2": "inputs larger than L2 (Q 268 MB, partials 4.3 GB); no flush"},
         "fwd_ms": round(phase["fwd_ms"], 4), "bwd_ms": round(phase["bwd_ms"], 4),
@@ -441,26 +454,30 @@ def run_ours(args, rank, world, local_rank, dist):
 
 # ----------------------------------------------------------------- oracle baselines
 
-def oracle_sample(workload: str, tokens: int):
+def oracle_sample(workload: str, tokens: int, window: int = 0):
     spec = dict(ni.WORKLOADS[workload])
     spec["lengths"] = [min(tokens, sum(spec["lengths"]))]
-    return ni.make_problem(name=workload + f"_prefix{tokens}", head_dim=128, **spec)
+    p = ni.make_problem(name=workload + f"_prefix{tokens}", head_dim=128, **spec)
+    if window > 0:
+        p.block_idx = ni.band_block_idx(p.cu_seqlens, p.hkv, p.topk, p.block_size, window)
+    return p
 
 
-def time_oracle_step(p, nthreads):
+def time_oracle_step(p, nthreads, window=0):
     import oracle
     t = time.perf_counter()
-    oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale, nthreads=nthreads)
-    oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+    oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale, window=window,
                nthreads=nthreads)
+    oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+               window=window, nthreads=nthreads)
     return time.perf_counter() - t
 
 
-def cpu_baseline(workload: str, tokens: int):
+def cpu_baseline(workload: str, tokens: int, window: int = 0):
     cores = len(os.sched_getaffinity(0))
-    p = oracle_sample(workload, tokens)
-    f, b = useful_flops(p)
-    dt = time_oracle_step(p, cores)
+    p = oracle_sample(workload, tokens, window)
+    f, b = useful_flops(p, window)
+    dt = time_oracle_step(p, cores, window)
     return {"value": round((f + b) / dt / 1e12, 6), "unit": UNIT, "cores": cores,
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"first {p.T} tokens (all {p.hq} heads) of the workload, forward + full "
@@ -471,11 +488,11 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     cores = len(os.sched_getaffinity(0))
-    p = oracle_sample(args.workload, args.ref_tokens)
-    f, b = useful_flops(p)
+    p = oracle_sample(args.workload, args.ref_tokens, args.window)
+    f, b = useful_flops(p, args.window)
     for _ in range(args.warmup):
-        time_oracle_step(p, cores)
-    times = [time_oracle_step(p, cores) for _ in range(args.steps)]
+        time_oracle_step(p, cores, args.window)
+    times = [time_oracle_step(p, cores, args.window) for _ in range(args.steps)]
     total = sum(times)
     value = (f + b) * len(times) / total / 1e12
     sample = (f"first {p.T} tokens (all {p.hq} heads) of the workload per step, forward + full "
@@ -484,7 +501,8 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1000 * total / len(times), 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample_tokens": p.T},
+            "config": {"workload": args.workload, "sample_tokens": p.T,
+                       "window_size": args.window},
             "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
                              "value": round(value, 6), "unit": UNIT},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -504,6 +522,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=ni.HEADLINE, choices=sorted(ni.WORKLOADS))
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16",
                     help="element type of q, k, v, dO and the outputs (fp32 arithmetic)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window of this many keys (0: none); the index becomes the "
+                         "sliding branch's: every block the window reaches")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=2048)

@@ -62,9 +62,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_fwd_profiled.restype = I
             lib.nsa_sel_attn_bwd_profiled.argtypes = lib.nsa_sel_attn_bwd.argtypes + [P, I, IP]
             lib.nsa_sel_attn_bwd_profiled.restype = I
-            lib.nsa_sel_attn_fwd_ex.argtypes = lib.nsa_sel_attn_fwd.argtypes + [ctypes.c_uint, P, I, IP]
+            lib.nsa_sel_attn_fwd_ex.argtypes = lib.nsa_sel_attn_fwd.argtypes + [ctypes.c_uint, I, P, I, IP]
             lib.nsa_sel_attn_fwd_ex.restype = I
-            lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, P, I, IP]
+            lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, I, P, I, IP]
             lib.nsa_sel_attn_bwd_ex.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
@@ -174,11 +174,13 @@ def _elem_type(q):
 
 
 def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out=None, lse=None,
-                     workspace=None, with_lse=True):
+                     workspace=None, with_lse=True, window_size=0):
     """Forward selected attention; returns (out [T,hq,d], lse fp32 [hq,T]).
 
     q, k, v (and out) are all bf16 or all fp16.  with_lse=False: a forward with no
-    backward to follow; the LSE is not stored and None is returned in its place."""
+    backward to follow; the LSE is not stored and None is returned in its place.
+    window_size > 0: keys must also lie in the last window_size positions up to the
+    query's own (a sliding window on top of the selected blocks)."""
     dev = q.device
     et, flag = _elem_type(q)
     _need(q, "q", et, 3, dev)
@@ -202,13 +204,16 @@ def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out
     _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, _ptr(block_idx), topk,
         block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev), flag,
-        None, 0, None))
+        int(window_size), None, 0, None))
     return out, lse
 
 
 def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size, scale=None,
-                     dq=None, dk=None, dv=None, workspace=None, reuse_index=False):
+                     dq=None, dk=None, dv=None, workspace=None, reuse_index=False,
+                     window_size=0):
     """Backward; returns (dq, dk, dv) in the type of q (bf16 or fp16).
+
+    window_size: the forward's sliding window (0: none).
 
     reuse_index: `workspace` (sized for the backward) was given to the forward call for
     the same cu_seqlens / block_idx tensors and is reused untouched since; the backward
@@ -235,7 +240,7 @@ def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size,
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
         hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(ws), ws.numel(), _stream(dev), (NSA_BWD_REUSE_INDEX if reuse_index else 0) | flag,
-        None, 0, None))
+        int(window_size), None, 0, None))
     return dq, dk, dv
 
 
@@ -312,20 +317,22 @@ class SelectedAttention(torch.autograd.Function):
     """Autograd wrapper: forward saves LSE, backward returns dQ, dK, dV."""
 
     @staticmethod
-    def forward(ctx, q, k, v, cu_seqlens, block_idx, block_size, scale):
-        out, lse = nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale)
+    def forward(ctx, q, k, v, cu_seqlens, block_idx, block_size, scale, window_size=0):
+        out, lse = nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale,
+                                    window_size=window_size)
         ctx.save_for_backward(q, k, v, out, lse, cu_seqlens, block_idx)
-        ctx.block_size, ctx.scale = block_size, scale
+        ctx.block_size, ctx.scale, ctx.window_size = block_size, scale, window_size
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse, cu, bi = ctx.saved_tensors
         dq, dk, dv = nsa_sel_attn_bwd(q, k, v, out, lse, dout.contiguous(), cu, bi,
-                                      ctx.block_size, ctx.scale)
-        return dq, dk, dv, None, None, None, None
+                                      ctx.block_size, ctx.scale, window_size=ctx.window_size)
+        return dq, dk, dv, None, None, None, None, None
 
 
-def selected_attention(q, k, v, cu_seqlens, block_idx, block_size=64, scale=None):
+def selected_attention(q, k, v, cu_seqlens, block_idx, block_size=64, scale=None, window_size=0):
     return SelectedAttention.apply(q, k, v, cu_seqlens, block_idx, block_size,
-                                   float(q.shape[-1] ** -0.5 if scale is None else scale))
+                                   float(q.shape[-1] ** -0.5 if scale is None else scale),
+                                   int(window_size))

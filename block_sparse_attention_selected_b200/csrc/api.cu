@@ -180,7 +180,8 @@ struct Carved {
     Layout L;
 };
 
-Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const int32_t* bidx) {
+Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const int32_t* bidx,
+             int swin = 0) {
     Carved c{};
     uint8_t* b = static_cast<uint8_t*>(ws);
     c.base = b;
@@ -194,6 +195,7 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.bidx = bidx;
     p.topk = D.topk;
     p.bs = D.bs;
+    p.swin = swin;
     p.tokens_per_tile = kTileRows / D.G;
     p.chunk_tiles = kChunkTiles;
     p.nent = D.nent;
@@ -217,7 +219,7 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
                                  (unsigned long long)D.T, (unsigned long long)D.nseq,
                                  (unsigned long long)D.hkv, (unsigned long long)D.topk,
                                  (unsigned long long)D.bs, (unsigned long long)D.G,
-                                 (unsigned long long)kChunkTiles}) {
+                                 (unsigned long long)kChunkTiles, (unsigned long long)swin}) {
         h ^= x;
         h *= 1099511628211ull;
     }
@@ -293,7 +295,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
                       int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
                       const int32_t* block_idx, int topk, int block_size, float scale, void* out,
                       float* lse, void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
-                      void* const* events, int num_events, int* launches, bool f16) {
+                      void* const* events, int num_events, int* launches, bool f16, int swin) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, false, &D);
@@ -302,12 +304,12 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         !aligned(lse, 4))
         return NSA_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f) || swin < 0) return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
     if ((s = check_device(&num_sms)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     const Layout L = make_layout(D, false);
-    Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
+    Carved c = carve(D, L, workspace, cu_seqlens, block_idx, swin);
     const PhaseMarks pm{events, num_events, stream, launches};
     if (launches) *launches = 0;
     pm.mark(0);
@@ -343,6 +345,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.nseq = D.nseq; fp.T = D.T; fp.hq = D.hq; fp.hkv = D.hkv; fp.topk = D.topk; fp.bs = D.bs;
     fp.G = D.G;
     fp.f16 = f16 ? 1 : 0;
+    fp.swin = swin;
     fp.scale_log2 = scale * 1.4426950408889634f;
     fp.blkoff = c.inv.blkoff;
     fp.offsets = c.inv.offsets;
@@ -375,6 +378,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
     mp.G = D.G;
     mp.f16 = f16 ? 1 : 0;
+    mp.swin = swin;
     mp.bidx = block_idx;
     mp.posmap = posmap;
     mp.part_o = fp.part_o;
@@ -394,7 +398,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
                       int topk, int block_size, float scale, void* dq, void* dk, void* dv,
                       void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
                       void* const* events, int num_events, int* launches, bool reuse_index,
-                      bool f16) {
+                      bool f16, int swin) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, true, &D);
@@ -405,12 +409,12 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4))
         return NSA_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f) || swin < 0) return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
     if ((s = check_device(&num_sms)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     const Layout L = make_layout(D, true);
-    Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
+    Carved c = carve(D, L, workspace, cu_seqlens, block_idx, swin);
     const PhaseMarks pm{events, num_events, stream, launches};
     if (launches) *launches = 0;
     pm.mark(0);
@@ -450,6 +454,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.nseq = D.nseq; bp.T = D.T; bp.hq = D.hq; bp.hkv = D.hkv; bp.topk = D.topk; bp.bs = D.bs;
     bp.G = D.G;
     bp.f16 = f16 ? 1 : 0;
+    bp.swin = swin;
     bp.scale = scale;
     bp.scale_log2 = scale * 1.4426950408889634f;
     bp.blkoff = c.inv.blkoff;
@@ -493,7 +498,7 @@ nsa_status_t nsa_sel_attn_fwd(const void* q, const void* k, const void* v,
                               size_t workspace_bytes, nsa_stream_t stream) {
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, nullptr,
-                    0, nullptr, false);
+                    0, nullptr, false, 0);
 }
 
 nsa_status_t nsa_sel_attn_fwd_profiled(const void* q, const void* k, const void* v,
@@ -505,7 +510,7 @@ nsa_status_t nsa_sel_attn_fwd_profiled(const void* q, const void* k, const void*
                                        int* num_launches) {
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
-                    num_events, num_launches, false);
+                    num_events, num_launches, false, 0);
 }
 
 nsa_status_t nsa_sel_attn_fwd_ex(const void* q, const void* k, const void* v,
@@ -513,12 +518,12 @@ nsa_status_t nsa_sel_attn_fwd_ex(const void* q, const void* k, const void* v,
                                  int hkv, int head_dim, const int32_t* block_idx, int topk,
                                  int block_size, float scale, void* out, float* lse,
                                  void* workspace, size_t workspace_bytes, nsa_stream_t stream,
-                                 unsigned flags, void* const* events, int num_events,
-                                 int* num_launches) {
+                                 unsigned flags, int window_size, void* const* events,
+                                 int num_events, int* num_launches) {
     if (flags & ~(unsigned)NSA_F16) return NSA_ERR_INVALID_ARG;
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
-                    num_events, num_launches, (flags & NSA_F16) != 0);
+                    num_events, num_launches, (flags & NSA_F16) != 0, window_size);
 }
 
 nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const void* out,
@@ -529,7 +534,7 @@ nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const
                               size_t workspace_bytes, nsa_stream_t stream) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, nullptr, 0, nullptr, false, false);
+                    workspace_bytes, stream, nullptr, 0, nullptr, false, false, 0);
 }
 
 nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void* v,
@@ -542,7 +547,7 @@ nsa_status_t nsa_sel_attn_bwd_profiled(const void* q, const void* k, const void*
                                        int* num_launches) {
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
-                    workspace_bytes, stream, events, num_events, num_launches, false, false);
+                    workspace_bytes, stream, events, num_events, num_launches, false, false, 0);
 }
 
 nsa_status_t nsa_sel_attn_bwd_ex(const void* q, const void* k, const void* v, const void* out,
@@ -551,12 +556,13 @@ nsa_status_t nsa_sel_attn_bwd_ex(const void* q, const void* k, const void* v, co
                                  const int32_t* block_idx, int topk, int block_size, float scale,
                                  void* dq, void* dk, void* dv, void* workspace,
                                  size_t workspace_bytes, nsa_stream_t stream, unsigned flags,
-                                 void* const* events, int num_events, int* num_launches) {
+                                 int window_size, void* const* events, int num_events,
+                                 int* num_launches) {
     if (flags & ~(unsigned)(NSA_BWD_REUSE_INDEX | NSA_F16)) return NSA_ERR_INVALID_ARG;
     return bwd_impl(q, k, v, out, lse, dout, cu_seqlens, num_seqs, total_tokens, hq, hkv,
                     head_dim, block_idx, topk, block_size, scale, dq, dk, dv, workspace,
                     workspace_bytes, stream, events, num_events, num_launches,
-                    (flags & NSA_BWD_REUSE_INDEX) != 0, (flags & NSA_F16) != 0);
+                    (flags & NSA_BWD_REUSE_INDEX) != 0, (flags & NSA_F16) != 0, window_size);
 }
 
 nsa_status_t nsa_sel_invert_index(const int32_t* cu_seqlens, int num_seqs, int total_tokens,

@@ -6,7 +6,8 @@
 // (KV head, KV block) list.  Per tile (rows = gathered (token, head) pairs):
 //
 //   S  = Q K^T,  dP = dO V^T                    tcgen05.mma -> TMEM
-//   P  = exp(scale S - LSE) (causal on the diagonal block),  dS = P (dP - D)
+//   P  = exp(scale S - LSE) (causal on the diagonal block, and on the block where a
+//        sliding window starts),  dS = P (dP - D)
 //   dV^T += dO^T P,  dK^T += Q^T dS              accumulate in TMEM over the unit
 //   dQ_part = scale * dS K                       per (row, slot), bf16
 //
@@ -546,7 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int4 m = S.meta[stg][r];
                 const float lse2 = S.rlse[stg][r], delta = S.rdelta[stg][r];
                 mbar_arrive(&S.meta_empty[stg]);
-                const int my_lim = m.w;
+                const int my_lim = m.w;                   // keys my_lo .. my_lim visible
+                const int my_lo = p.swin > 0 ? my_lim - p.swin + 1 : 0;
                 const long long prow = m.x < 0 ? -1ll : ((long long)m.x * p.hq + m.y) * p.topk + m.z;
                 if (!(ok = wait(&S.sdp_full[s], (i / NTS) & 1, 61))) break;
                 tc_fence_after();
@@ -565,16 +567,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
                     const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
+                    auto p_ds = [&](const bool masked) {
 #pragma unroll
-                    for (int c = 0; c < kKeysWg; c += 2) {
-                        const int key = wg * kKeysWg + c;
-                        float2 x = fma2(make_float2(sv[c], sv[c + 1]), c2, nl2);
-                        x.x = key <= my_lim ? ex2_approx(x.x) : 0.f;
-                        x.y = key + 1 <= my_lim ? ex2_approx(x.y) : 0.f;
-                        const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
-                        pk[c / 2] = pack2<F16>(x.x, x.y);    // P, dS in the operands' type
-                        dk[c / 2] = pack2<F16>(ds.x, ds.y);
-                    }
+                        for (int c = 0; c < kKeysWg; c += 2) {
+                            const int key = wg * kKeysWg + c;
+                            float2 x = fma2(make_float2(sv[c], sv[c + 1]), c2, nl2);
+                            if (masked) {
+                                x.x = (key <= my_lim && key >= my_lo) ? ex2_approx(x.x) : 0.f;
+                                x.y = (key + 1 <= my_lim && key + 1 >= my_lo) ? ex2_approx(x.y) : 0.f;
+                            } else {
+                                x.x = ex2_approx(x.x);
+                                x.y = ex2_approx(x.y);
+                            }
+                            const float2 ds = mul2(x, add2(make_float2(dp[c], dp[c + 1]), nd2));
+                            pk[c / 2] = pack2<F16>(x.x, x.y);    // P, dS in the operands' type
+                            dk[c / 2] = pack2<F16>(ds.x, ds.y);
+                        }
+                    };
+                    // warps whose rows all see every key of this warpgroup's half skip the
+                    // mask (padding rows have my_lim = -1 and always take the masked form)
+                    if (__all_sync(0xffffffffu, my_lo <= wg * kKeysWg && my_lim >= (wg + 1) * kKeysWg - 1))
+                        p_ds(false);
+                    else
+                        p_ds(true);
                 }
                 tc_fence_before();
                 if (!(ok = wait(&S.pds_empty, (i & 1) ^ 1, 62))) break;

@@ -7,8 +7,9 @@
 // Attention" blog, second paragraph).  Per tile:
 //
 //   S   = Q K_B^T                  tcgen05.mma (Q, K from shared memory) -> TMEM
-//   P   = exp2(c S - c m), causal mask on the diagonal block, l = sum P; P is
-//         written as bf16 back into the S columns of TMEM
+//   P   = exp2(c S - c m), causal mask on the diagonal block (and, under a sliding
+//         window, on the block where the window starts), l = sum P; P is written as
+//         bf16 back into the S columns of TMEM
 //   O_B = P V_B                    tcgen05.mma with A = P read from TMEM
 //   partial: O_B * 2^-e / l as fp16, lse_B = m + log l.  e is the block's V
 //         exponent (k_vblock_exp): 0 unless max |V_B| > 2^14, so O_B / l, a convex
@@ -394,11 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             return (i < n && r < (d.z & 255)) ? __ldg(p.entries + d.y + r / p.G) : 0u;
         };
         auto ld_vexp = [&](const int4& d, int i) -> int { return i < n ? __ldg(p.vexp + d.w) : 0; };
-        // scores of keys past the causal limit -> -inf (diagonal tiles only)
-        auto mask64 = [&](float* v, int lim, int base) {
+        // scores of keys past the causal limit or before the sliding window -> -inf
+        // (diagonal and window-edge tiles only)
+        auto mask64 = [&](float* v, int lo, int lim, int base) {
 #pragma unroll
             for (int k = 0; k < 64; ++k)
-                if (base + k > lim) v[k] = -CUDART_INF_F;
+                if (base + k > lim || base + k < lo) v[k] = -CUDART_INF_F;
         };
         auto row_max64 = [&](const float* v) -> float {
             float a = -CUDART_INF_F, b = -CUDART_INF_F;
@@ -446,21 +448,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             vn = ld_vexp(dn, i + 2);
             const uint32_t ph = (i >> 1) & 1;
             const bool valid = r < (d.z & 255);
-            // keys 0 .. lim of the block are visible to this row (causal on the diagonal)
+            // keys lo .. lim of the block are visible to this row (causal on the diagonal,
+            // lo > 0 where the sliding window starts inside the block)
             const int lim = valid ? (int)(ent >> 6) - d.x : -1;
-            const bool nomask = __all_sync(0xffffffffu, !valid || lim >= BS - 1);
+            const int lo = p.swin > 0 ? lim - p.swin + 1 : 0;
+            const bool nomask = __all_sync(0xffffffffu, !valid || (lim >= BS - 1 && lo <= 0));
             if (!wait_w(&S.s_full[wg], ph, 38)) break;
             tc_fence_after();
             float sv[64];
             tmem_ld64_sync(tS, sv);
-            if (!nomask) mask64(sv, lim, 0);
+            if (!nomask) mask64(sv, lo, lim, 0);
             float mx = row_max64(sv);
             if constexpr (BS == 128) {
                 tmem_ld64_sync(tS + 64, sv);
-                if (!nomask) mask64(sv, lim, 64);
+                if (!nomask) mask64(sv, lo, lim, 64);
                 mx = fmaxf(mx, row_max64(sv));
             }
-            if (!valid) mx = 0.f;                      // every valid row has lim >= 0
+            if (!valid) mx = 0.f;                      // every valid row has lo <= lim
             const float mc = mx * c;
             float2 l2 = make_float2(0.f, 0.f);
             float l;
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c64 = 0; c64 < 2; ++c64) {    // scores of this 64-key chunk again
                     tmem_ld64_sync(tS + c64 * 64, sv);
-                    if (!nomask) mask64(sv, lim, c64 * 64);
+                    if (!nomask) mask64(sv, lo, lim, c64 * 64);
                     exp_chunk(sv, mc, l2);
                     pack_chunk(sv, 1.f, pk);
                     tmem_st32_sync(tS + c64 * 32, pk);

@@ -30,6 +30,7 @@ constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 struct SortArgs {
     const int32_t* cu;
     int nseq, T, hkv, topk, bs;
+    int swin;                // sliding window in keys, 0: none
     const int32_t* bidx;
     long long nent;
     int nbk_cap;
@@ -96,7 +97,8 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
 }
 
 // Bucket key of entry e (token-major, then KV head, then slot); kInvalidKey if the
-// entry selects nothing (padding, future or out-of-range block).
+// entry selects nothing (padding, future or out-of-range block, or a block that lies
+// wholly before the sliding window).
 __device__ __forceinline__ uint32_t entry_key(const SortArgs& a, long long e, uint32_t nbtot,
                                               uint32_t* val) {
     int j, g, t;
@@ -117,7 +119,7 @@ __device__ __forceinline__ uint32_t entry_key(const SortArgs& a, long long e, ui
     int s = seq_of_token(a.cu, a.nseq, t);
     int i = t - __ldg(a.cu + s);
     int qb = i >= 0 ? i / a.bs : -1;
-    if (!block_valid(b, qb)) return kInvalidKey;
+    if (!block_valid(b, qb, i, a.bs, a.swin)) return kInvalidKey;
     uint32_t key = (uint32_t)g * nbtot + (uint32_t)__ldg(a.blkoff + s) + (uint32_t)b;
     return key < (uint32_t)a.nbk_cap ? key : kInvalidKey;
 }
@@ -485,7 +487,7 @@ int invert_final_buf(const InvertPlan& p) {
 
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
     k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st, p.tag);
-    SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
+    SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.swin, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
     const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
     const uint32_t* kin = nullptr;
     const uint32_t* vin = nullptr;

@@ -48,15 +48,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     const int hoff = h - g * p.G;
     const unsigned nrows_part = (unsigned)p.st->ntiles_fwd * (unsigned)kTileRows;
     const int s = seq_of_token(p.cu, p.nseq, t);
-    const int qb = (t - __ldg(p.cu + s)) / p.bs;
+    const int i = t - __ldg(p.cu + s);
+    const int qb = i / p.bs;
     const size_t base = ((size_t)t * p.hkv + g) * p.topk;
     // level 1: validity and partial row of slots lane, lane + 32
     unsigned r0 = 0xFFFFFFFFu, r1 = 0xFFFFFFFFu;   // partial row, or none
-    if (lane < p.topk && block_valid(__ldg(p.bidx + base + lane), qb)) {
+    if (lane < p.topk && block_valid(__ldg(p.bidx + base + lane), qb, i, p.bs, p.swin)) {
         const unsigned r = (unsigned)__ldg(p.posmap + base + lane) * (unsigned)p.G + (unsigned)hoff;
         if (r < nrows_part) r0 = r;
     }
-    if (!kTopk32 && lane + 32 < p.topk && block_valid(__ldg(p.bidx + base + lane + 32), qb)) {
+    if (!kTopk32 && lane + 32 < p.topk && block_valid(__ldg(p.bidx + base + lane + 32), qb, i, p.bs, p.swin)) {
         const unsigned r = (unsigned)__ldg(p.posmap + base + lane + 32) * (unsigned)p.G + (unsigned)hoff;
         if (r < nrows_part) r1 = r;
     }
@@ -151,14 +152,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan 
     const int h = (int)(row - (long long)t * p.hq);
     const int g = h / p.G;
     const int s = seq_of_token(p.cu, p.nseq, t);
-    const int qb = (t - __ldg(p.cu + s)) / p.bs;
+    const int i = t - __ldg(p.cu + s);
+    const int qb = i / p.bs;
     const int32_t* bi = bidx + ((size_t)t * p.hkv + g) * p.topk;
     const uint2* pd = reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.part_dq) +
                                                      (size_t)row * p.topk * kHeadDim) + lane;
     const int b0 = lane < p.topk ? __ldg(bi + lane) : -1;
     const int b1 = lane + 32 < p.topk ? __ldg(bi + lane + 32) : -1;
-    const unsigned v0 = __ballot_sync(0xFFFFFFFFu, block_valid(b0, qb));
-    const unsigned v1 = __ballot_sync(0xFFFFFFFFu, block_valid(b1, qb));
+    const unsigned v0 = __ballot_sync(0xFFFFFFFFu, block_valid(b0, qb, i, p.bs, p.swin));
+    const unsigned v1 = __ballot_sync(0xFFFFFFFFu, block_valid(b1, qb, i, p.bs, p.swin));
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < p.topk; ++j) {
         const bool ok = j < 32 ? ((v0 >> j) & 1u) : ((v1 >> (j - 32)) & 1u);

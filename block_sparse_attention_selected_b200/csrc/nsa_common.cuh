@@ -411,8 +411,13 @@ __device__ __forceinline__ float2 unpack2(uint32_t u) {
     return F16 ? unpack_f16x2(u) : unpack_bf16x2(u);
 }
 
-// Entry validity shared by every kernel: a selected block b of a token at query block
-// qb contributes keys iff 0 <= b <= qb (-1 pads; future and out-of-range blocks drop).
-__device__ __forceinline__ bool block_valid(int b, int qb) { return b >= 0 && b <= qb; }
+// Entry validity shared by every kernel.  Slot value b of the token at local position
+// i (query block qb = i / bs) contributes keys iff 0 <= b <= qb (-1 pads; future and
+// out-of-range blocks drop) and, under a sliding window of swin > 0 keys, the block's
+// last key (b + 1) bs - 1 lies in the window (i - swin, i]; a valid entry therefore
+// always keeps at least one visible key.
+__device__ __forceinline__ bool block_valid(int b, int qb, int i, int bs, int swin) {
+    return b >= 0 && b <= qb && (swin <= 0 || i - (b + 1) * bs < swin - 1);
+}
 
 }  // namespace nsa

@@ -19,6 +19,7 @@ struct InvertPlan {
     const int32_t* bidx;     // [T, hkv, topk]
     int topk;
     int bs;
+    int swin;                // sliding window in keys (0: none); drops blocks before it
     int tokens_per_tile;     // 128 / G (query heads per KV head)
     int chunk_tiles;         // tiles per backward work unit
     long long nent;          // T * hkv * topk
@@ -78,6 +79,7 @@ struct FwdPlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
     int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
+    int swin;                // sliding window in keys (0: none)
     float scale_log2;        // scale * log2(e)
     const int32_t* blkoff;
     const int32_t* offsets;  // bucket offsets into entries
@@ -109,6 +111,7 @@ struct MergePlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
     int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
+    int swin;                // sliding window in keys (0: none)
     const int32_t* bidx;
     const int32_t* posmap;   // sorted position of each valid (t, g, j) entry
     const void* part_o;
@@ -128,6 +131,7 @@ struct BwdPlan {
     float* delta;            // [hq, T]  rowsum(dout * out)
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int swin;                // sliding window in keys (0: none)
     float scale, scale_log2;
     const int32_t* blkoff;
     const int32_t* offsets;

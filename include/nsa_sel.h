@@ -136,13 +136,22 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
 #define NSA_F16 2u
 /* The forward with options: flags = NSA_F16 makes q, k, v and out fp16 instead of bf16
  * (same layouts; the partials stay fp16 and all arithmetic fp32, as for bf16).  Other
- * flag bits return NSA_ERR_INVALID_ARG.  events / num_events / num_launches as in
- * nsa_sel_attn_fwd_profiled (null / 0 for none). */
+ * flag bits return NSA_ERR_INVALID_ARG.
+ *   window_size  0: no window.  W > 0: a sliding window of W keys as well: the token at
+ *       local position i attends key j only if j lies in a selected block, j <= i and
+ *       j > i - W (the window_size of the sliding branch in the quick start of the
+ *       "Relaxed-System-Lab/Flash-Sparse-Attention" project page; with block_idx
+ *       selecting the blocks qb - ceil(W / block_size) .. qb this is that branch).
+ *       Blocks wholly before the window contribute nothing; a row left with no key
+ *       gets out = 0, lse = -inf.  Negative values return NSA_ERR_INVALID_ARG.
+ * events / num_events / num_launches as in nsa_sel_attn_fwd_profiled (null / 0 for
+ * none). */
 NSA_API nsa_status_t nsa_sel_attn_fwd_ex(
     const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int num_seqs,
     int total_tokens, int hq, int hkv, int head_dim, const int32_t *block_idx, int topk,
     int block_size, float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
-    nsa_stream_t stream, unsigned flags, void *const *events, int num_events, int *num_launches);
+    nsa_stream_t stream, unsigned flags, int window_size, void *const *events, int num_events,
+    int *num_launches);
 
 /* The backward with options (flags, OR-ed):
  *   NSA_BWD_REUSE_INDEX  the workspace holds the block-index inversion that
@@ -156,7 +165,9 @@ NSA_API nsa_status_t nsa_sel_attn_fwd_ex(
  *       themselves are not compared.
  *   NSA_F16  q, k, v, out, dout, dq, dk, dv are fp16 instead of bf16 (the forward was
  *       called with NSA_F16 too).
- * Other flag bits return NSA_ERR_INVALID_ARG.  events / num_events / num_launches as in
+ * Other flag bits return NSA_ERR_INVALID_ARG.  window_size as in nsa_sel_attn_fwd_ex
+ * (the forward's value; a reused inversion made with another window_size is reported
+ * like other inputs).  events / num_events / num_launches as in
  * nsa_sel_attn_bwd_profiled (null / 0 for none).  Otherwise identical to
  * nsa_sel_attn_bwd. */
 NSA_API nsa_status_t nsa_sel_attn_bwd_ex(
@@ -164,7 +175,7 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_ex(
     const void *dout, const int32_t *cu_seqlens, int num_seqs, int total_tokens, int hq, int hkv,
     int head_dim, const int32_t *block_idx, int topk, int block_size, float scale, void *dq,
     void *dk, void *dv, void *workspace, size_t workspace_bytes, nsa_stream_t stream,
-    unsigned flags, void *const *events, int num_events, int *num_launches);
+    unsigned flags, int window_size, void *const *events, int num_events, int *num_launches);
 
 /* The block-index inversion on its own (the loop swap named in the file header):
  * for KV head g and global block B (blocks of earlier sequences first), the list of

@@ -130,6 +130,26 @@ def make_block_idx(cu_seqlens: np.ndarray, hkv: int, topk: int, block_size: int,
     return out
 
 
+def band_block_idx(cu_seqlens: np.ndarray, hkv: int, topk: int, block_size: int,
+                   window: int) -> np.ndarray:
+    """block_idx int32 [T, hkv, topk] of the sliding branch: for the token at local
+    position i (query block qb), the blocks qb, qb - 1, .., down to the block of key
+    i - window + 1 (at most ceil(window / block_size) + 1 blocks, never below 0), then
+    -1 pads; the same row for every KV head.  No random draws."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T = int(cu[-1])
+    nwb = (window + block_size - 1) // block_size + 1
+    if nwb > topk:
+        raise ValueError("topk is smaller than the number of blocks a window reaches")
+    out = np.full((T, hkv, topk), -1, dtype=np.int32)
+    for s in range(len(cu) - 1):
+        c0, c1 = int(cu[s]), int(cu[s + 1])
+        qb = np.arange(c1 - c0, dtype=np.int64) // block_size
+        blocks = qb[:, None] - np.arange(nwb, dtype=np.int64)[None, :]
+        out[c0:c1, :, :nwb] = np.where(blocks >= 0, blocks, -1)[:, None, :].astype(np.int32)
+    return out
+
+
 @dataclasses.dataclass
 class Problem:
     """One synthetic problem.  Float arrays are float32 holding bf16 values."""

@@ -104,21 +104,29 @@ def test_option_flags_checked_on_the_host(lib):
     fake = P(1 << 20)           # never dereferenced: the flag check comes first
     # forward: only NSA_F16 (2) is an option
     rc = lib.nsa_sel_attn_fwd_ex(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
-                                 fake, fake, fake, 1 << 30, None, 1, None, 0, None)
+                                 fake, fake, fake, 1 << 30, None, 1, 0, None, 0, None)
     assert rc == 1
     rc = lib.nsa_sel_attn_fwd_ex(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
-                                 fake, fake, fake, 1 << 30, None, 4, None, 0, None)
+                                 fake, fake, fake, 1 << 30, None, 4, 0, None, 0, None)
     assert rc == 1
     # backward: NSA_BWD_REUSE_INDEX (1) and NSA_F16 (2)
     rc = lib.nsa_sel_attn_bwd_ex(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 128,
                                  fake, 8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None, 8,
-                                 None, 0, None)
+                                 0, None, 0, None)
     assert rc == 1
     # a valid flag still reaches the usual argument checks (here: head_dim 64)
     rc = lib.nsa_sel_attn_bwd_ex(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 64,
                                  fake, 8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None, 3,
-                                 None, 0, None)
+                                 0, None, 0, None)
     assert rc == 2
+    # a negative sliding window is an argument error in both directions
+    rc = lib.nsa_sel_attn_fwd_ex(fake, fake, fake, fake, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,
+                                 fake, fake, fake, 1 << 30, None, 0, -1, None, 0, None)
+    assert rc == 1
+    rc = lib.nsa_sel_attn_bwd_ex(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 128,
+                                 fake, 8, 64, 0.1, fake, fake, fake, fake, 1 << 30, None, 0,
+                                 -5, None, 0, None)
+    assert rc == 1
     assert nsa.NSA_BWD_REUSE_INDEX == 1 and nsa.NSA_F16 == 2
 
 

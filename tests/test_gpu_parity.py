@@ -380,3 +380,86 @@ def test_fp16_fwd_bwd_full_compare(name, spec, perturb):
                                p.scale)
     e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
     assert max(e) <= TOL_GRAD, (name, e)
+
+
+# ------------------------------------------------------------------ sliding window
+
+WINDOW_CASES = [
+    # name, problem, window, perturb
+    ("w512_g4_bs64_k16", dict(lengths=[1500, 40, 700], hq=8, hkv=2, block_size=64, topk=16, seed=61), 512, True),
+    ("w100_g1_bs128_k8", dict(lengths=[1100, 1], hq=2, hkv=2, block_size=128, topk=8, seed=62), 100, True),
+    ("w1_g16_bs64_k5", dict(lengths=[700], hq=16, hkv=1, block_size=64, topk=5, seed=63), 1, False),
+    ("w70_g8_bs64_k12", dict(lengths=[900, 129], hq=8, hkv=1, block_size=64, topk=12, seed=64), 70, True),
+]
+
+
+@pytest.mark.parametrize("name,spec,W,perturb", WINDOW_CASES, ids=[c[0] for c in WINDOW_CASES])
+def test_window_fwd_bwd_full_compare(name, spec, W, perturb):
+    # selection and a sliding window of W keys; some rows keep no key (O = 0, LSE = -inf)
+    p = ni.make_problem(name=name, **spec)
+    if perturb:
+        p = _perturb(p, 8)
+    d = to_device(p)
+    out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], p.block_size,
+                                    p.scale, window_size=W)
+    dq, dk, dv = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"],
+                                      d["bidx"], p.block_size, p.scale, window_size=W)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+                              window=W)
+    o, l = f64(out), f64(lse).T
+    fin = np.isfinite(l_ref)
+    assert np.array_equal(np.isfinite(l), fin), name
+    assert not o[~fin].any(), name
+    eo, el = o_excess(o, o_ref), max_abs(l[fin], l_ref[fin])
+    assert eo <= TOL_O and el <= TOL_LSE, (name, eo, el)
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
+                               p.scale, window=W)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    assert max(e) <= TOL_GRAD, (name, e)
+
+
+@pytest.mark.parametrize("bs,W", [(64, 512), (128, 300)])
+def test_window_sliding_branch_is_band_attention(bs, W):
+    # the sliding branch: every block the window reaches selected -> banded causal attention
+    p = ni.make_problem([2100, 333], hq=8, hkv=2, block_size=bs, topk=16, seed=65)
+    p.block_idx = ni.band_block_idx(p.cu_seqlens, p.hkv, p.topk, bs, W)
+    d = to_device(p)
+    out, lse = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], bs, p.scale,
+                                    window_size=W)
+    dq, dk, dv = nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], out, lse, d["dout"], d["cu"],
+                                      d["bidx"], bs, p.scale, window_size=W)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    _check_fwd_window(p, out, lse, W)
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, bs, p.scale,
+                               window=W)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    assert max(e) <= TOL_GRAD, e
+
+
+def _check_fwd_window(p, out, lse, W):
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+                              window=W)
+    eo, el = o_excess(f64(out), o_ref), max_abs(f64(lse).T, l_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
+
+
+def test_window_wider_than_sequences_changes_nothing_and_tags_reuse():
+    p = ni.make_problem([1200, 300], hq=8, hkv=2, block_size=64, topk=16, seed=66)
+    d = to_device(p)
+    T, hq, hkv, topk = p.q.shape[0], p.q.shape[1], p.k.shape[1], p.block_idx.shape[2]
+    ref_o, ref_l = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], 64, p.scale)
+    nb = nsa.nsa_sel_attn_workspace_size(T, 2, hq, hkv, 128, topk, 64, True)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    o, l = nsa.nsa_sel_attn_fwd(d["q"], d["k"], d["v"], d["cu"], d["bidx"], 64, p.scale,
+                                workspace=ws, window_size=1 << 20)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status(ws) == 0
+    assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    # the inversion was made for window 1 << 20: a backward with another window refuses it
+    nsa.nsa_sel_attn_bwd(d["q"], d["k"], d["v"], o, l, d["dout"], d["cu"], d["bidx"], 64,
+                         p.scale, workspace=ws, reuse_index=True, window_size=512)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status(ws) == 1   # NSA_ERR_INVALID_ARG
