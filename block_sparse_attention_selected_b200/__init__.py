@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
                 6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
             "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_fwd_ex",
-            "nsa_sel_attn_bwd_ex",
+            "nsa_sel_attn_bwd_ex", "nsa_sel_compress_kv", "nsa_sel_select_topk",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
@@ -66,6 +66,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_fwd_ex.restype = I
             lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, P, I, IP]
             lib.nsa_sel_attn_bwd_ex.restype = I
+            lib.nsa_sel_compress_kv.argtypes = [P, P, P, I, I, I, I, I, I, ctypes.c_uint, P, P, P, P]
+            lib.nsa_sel_compress_kv.restype = I
+            lib.nsa_sel_select_topk.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, Z, P]
+            lib.nsa_sel_select_topk.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
             lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
@@ -296,6 +300,44 @@ def nsa_sel_validate_indices(cu_seqlens, block_idx, block_size, workspace=None):
     if code not in (0, 6):
         raise NsaError("nsa_sel_validate_indices", code)
     return int(a.value), int(b.value)
+
+
+def nsa_sel_compress_kv(k, v, cu_seqlens, kernel_size=32, kernel_stride=16):
+    """Mean-pooled compressed K and V of the selection step; returns (k_cmp, v_cmp,
+    cu_cmp): k_cmp / v_cmp [floor(T / stride), hkv, d] in the type of k (rows past
+    cu_cmp[-1] unused), cu_cmp int32 [nseq + 1]."""
+    dev = k.device
+    et, flag = _elem_type(k)
+    _need(k, "k", et, 3, dev)
+    _need(v, "v", et, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    T, hkv, d = k.shape
+    if v.shape != k.shape:
+        raise ValueError("inconsistent shapes")
+    nseq = cu_seqlens.numel() - 1
+    rows = max(T // kernel_stride, 1)
+    kc = torch.empty((rows, hkv, d), dtype=et, device=dev)
+    vc = torch.empty((rows, hkv, d), dtype=et, device=dev)
+    cu_cmp = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+    _check("nsa_sel_compress_kv", load_library().nsa_sel_compress_kv(
+        _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hkv, d, kernel_size, kernel_stride, flag,
+        _ptr(kc), _ptr(vc), _ptr(cu_cmp), _stream(dev)))
+    return kc, vc, cu_cmp
+
+
+def nsa_sel_select_topk(scores, cu_seqlens, block_size, topk, init_blocks=1, local_blocks=2,
+                        workspace=None):
+    """block_idx int32 [T, hkv, topk] from block scores fp32 [T, hkv, nb_stride]."""
+    dev = scores.device
+    _need(scores, "scores", torch.float32, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    T, hkv, nb = scores.shape
+    out = torch.empty((T, hkv, topk), dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else get_workspace(256, dev)
+    _check("nsa_sel_select_topk", load_library().nsa_sel_select_topk(
+        _ptr(scores), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, nb, block_size, topk,
+        init_blocks, local_blocks, _ptr(out), _ptr(ws), ws.numel(), _stream(dev)))
+    return out
 
 
 def nsa_sel_check_status(workspace=None, device=None) -> int:

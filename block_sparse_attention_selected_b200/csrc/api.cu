@@ -627,6 +627,56 @@ nsa_status_t nsa_sel_validate_indices(const int32_t* cu_seqlens, int num_seqs, i
     return (h.bad_range || h.bad_dup) ? NSA_ERR_BAD_INDEX : NSA_OK;
 }
 
+nsa_status_t nsa_sel_compress_kv(const void* k, const void* v, const int32_t* cu_seqlens,
+                                 int num_seqs, int total_tokens, int hkv, int head_dim,
+                                 int kernel_size, int kernel_stride, unsigned flags, void* k_cmp,
+                                 void* v_cmp, int32_t* cu_cmp, nsa_stream_t stream_) {
+    if (flags & ~(unsigned)NSA_F16) return NSA_ERR_INVALID_ARG;
+    if (total_tokens < 0 || num_seqs < 1 || hkv < 1 || kernel_stride < 1 ||
+        kernel_size < kernel_stride)
+        return NSA_ERR_INVALID_ARG;
+    if (head_dim != kHeadDim || kernel_size > 4096 || total_tokens >= (1 << 25))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !cu_cmp || (total_tokens >= kernel_stride && (!k || !v || !k_cmp || !v_cmp)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4) || !aligned(cu_cmp, 4) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(k_cmp, 16) || !aligned(v_cmp, 16))
+        return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    return cuda_status(launch_compress_kv(k, v, cu_seqlens, num_seqs, total_tokens, hkv, kernel_size,
+                                          kernel_stride, (flags & NSA_F16) ? 1 : 0, cu_cmp, k_cmp,
+                                          v_cmp, reinterpret_cast<cudaStream_t>(stream_)));
+}
+
+nsa_status_t nsa_sel_select_topk(const float* scores, const int32_t* cu_seqlens, int num_seqs,
+                                 int total_tokens, int hkv, int nb_stride, int block_size,
+                                 int topk, int init_blocks, int local_blocks, int32_t* block_idx,
+                                 void* workspace, size_t workspace_bytes, nsa_stream_t stream_) {
+    if (total_tokens < 0 || num_seqs < 1 || hkv < 1 || nb_stride < 1 || block_size < 1 ||
+        topk < 1 || init_blocks < 0 || local_blocks < 0)
+        return NSA_ERR_INVALID_ARG;
+    if (topk > kMaxTopk || nb_stride > 1024 || total_tokens >= (1 << 25) ||
+        (long long)total_tokens * hkv * nb_stride >= (1ll << 40))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !workspace || (total_tokens > 0 && (!scores || !block_idx)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4) || !aligned(scores, 4) || !aligned(block_idx, 4) ||
+        !aligned(workspace, 256))
+        return NSA_ERR_INVALID_ARG;
+    if (workspace_bytes < sizeof(DevStatus)) return NSA_ERR_WORKSPACE;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    return cuda_status(launch_select_topk(scores, cu_seqlens, num_seqs, total_tokens, hkv, nb_stride,
+                                          block_size, topk, init_blocks, local_blocks, block_idx,
+                                          st, stream));
+}
+
 nsa_status_t nsa_sel_check_status(const void* workspace, nsa_stream_t stream_) {
     if (!workspace || !aligned(workspace, 256)) return NSA_ERR_INVALID_ARG;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

@@ -153,6 +153,16 @@ cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq,
                                 cudaStream_t stream);
 cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStream_t stream);
 
+// Block-selection step (select.cu): cu_cmp[nseq + 1] and the mean-pooled compressed
+// K and V ([floor(T / stride) rows room, hkv, 128]); the top-k of the block scores
+// ([T, hkv, nb_stride] fp32) into block_idx [T, hkv, topk].
+cudaError_t launch_compress_kv(const void* k, const void* v, const int32_t* cu, int nseq, int T,
+                               int hkv, int ksize, int stride, int f16, int32_t* cu_cmp, void* kc,
+                               void* vc, cudaStream_t stream);
+cudaError_t launch_select_topk(const float* scores, const int32_t* cu, int nseq, int T, int hkv,
+                               int nb_stride, int bs, int topk, int init_blocks, int local_blocks,
+                               int32_t* bidx, DevStatus* st, cudaStream_t stream);
+
 cudaError_t launch_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
                             int topk, int bs, DevStatus* st, cudaStream_t stream);
 

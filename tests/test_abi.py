@@ -122,6 +122,27 @@ def test_option_flags_checked_on_the_host(lib):
     assert nsa.NSA_BWD_REUSE_INDEX == 1 and nsa.NSA_F16 == 2
 
 
+def test_selection_entry_points_check_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)           # never dereferenced: the checks come first
+    # compress: a kernel shorter than its stride, a head dim other than 128, a bad flag
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 128, 8, 16, 0, fake, fake, fake,
+                                   None) == 1
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 64, 32, 16, 0, fake, fake, fake,
+                                   None) == 2
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 128, 32, 16, 4, fake, fake, fake,
+                                   None) == 1
+    # top-k: topk 0, more than 64 slots, score rows over 1024 blocks, a short workspace
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 0, 1, 2, fake, fake, 1 << 20,
+                                   None) == 1
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 65, 1, 2, fake, fake, 1 << 20,
+                                   None) == 2
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 1025, 64, 16, 1, 2, fake, fake, 1 << 20,
+                                   None) == 2
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 16, 1, 2, fake, fake, 128,
+                                   None) == 3
+
+
 def test_binding_rejects_other_element_types():
     import torch
     x = torch.zeros((4, 2, 128), dtype=torch.float32)
