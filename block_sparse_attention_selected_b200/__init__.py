@@ -26,6 +26,7 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
             "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_fwd_ex",
             "nsa_sel_attn_bwd_ex", "nsa_sel_compress_kv", "nsa_sel_select_topk",
+            "nsa_sel_block_scores", "nsa_sel_block_scores_workspace_size",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
@@ -70,6 +71,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_compress_kv.restype = I
             lib.nsa_sel_select_topk.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, Z, P]
             lib.nsa_sel_select_topk.restype = I
+            lib.nsa_sel_block_scores_workspace_size.argtypes = [I]
+            lib.nsa_sel_block_scores_workspace_size.restype = Z
+            lib.nsa_sel_block_scores.argtypes = [P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, P, P, Z, P]
+            lib.nsa_sel_block_scores.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
             lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
@@ -323,6 +328,42 @@ def nsa_sel_compress_kv(k, v, cu_seqlens, kernel_size=32, kernel_stride=16):
         _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hkv, d, kernel_size, kernel_stride, flag,
         _ptr(kc), _ptr(vc), _ptr(cu_cmp), _stream(dev)))
     return kc, vc, cu_cmp
+
+
+def nsa_sel_block_scores(q, k_cmp, cu_seqlens, cu_cmp, block_size, nb_stride, scale=None,
+                         kernel_size=32, kernel_stride=16, workspace=None):
+    """Selection-block scores fp32 [T, hkv, nb_stride] from attention over the compressed
+    keys (entries past each row's own block are left uninitialised)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(k_cmp, "k_cmp", torch.bfloat16, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(cu_cmp, "cu_cmp", torch.int32, 1, dev)
+    T, hq, d = q.shape
+    rows, hkv, _ = k_cmp.shape
+    scale = float(d ** -0.5 if scale is None else scale)
+    nseq = cu_seqlens.numel() - 1
+    lib = load_library()
+    nbytes = int(lib.nsa_sel_block_scores_workspace_size(nseq))
+    ws = workspace if workspace is not None else get_workspace(nbytes, dev)
+    scores = torch.empty((T, hkv, nb_stride), dtype=torch.float32, device=dev)
+    _check("nsa_sel_block_scores", lib.nsa_sel_block_scores(
+        _ptr(q), _ptr(k_cmp), rows, _ptr(cu_seqlens), _ptr(cu_cmp), nseq, T, hq, hkv, d,
+        block_size, kernel_size, kernel_stride, scale, nb_stride, _ptr(scores), _ptr(ws),
+        ws.numel(), _stream(dev)))
+    return scores
+
+
+def nsa_sel_select_blocks(q, k, v, cu_seqlens, block_size=64, topk=16, init_blocks=1,
+                          local_blocks=2, max_seqlen=None, scale=None):
+    """The whole selection step on the GPU: compression, block scores, top-k; returns
+    block_idx int32 [T, hkv, topk].  max_seqlen (host int) sizes the score rows."""
+    T = q.shape[0]
+    L = int(max_seqlen) if max_seqlen is not None else T
+    nb_stride = max((L + block_size - 1) // block_size, 1)
+    kc, _, cu_cmp = nsa_sel_compress_kv(k, v, cu_seqlens)
+    sc = nsa_sel_block_scores(q, kc, cu_seqlens, cu_cmp, block_size, nb_stride, scale)
+    return nsa_sel_select_topk(sc, cu_seqlens, block_size, topk, init_blocks, local_blocks)
 
 
 def nsa_sel_select_topk(scores, cu_seqlens, block_size, topk, init_blocks=1, local_blocks=2,

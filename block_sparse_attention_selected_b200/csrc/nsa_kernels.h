@@ -159,6 +159,16 @@ cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStr
 cudaError_t launch_compress_kv(const void* k, const void* v, const int32_t* cu, int nseq, int T,
                                int hkv, int ksize, int stride, int f16, int32_t* cu_cmp, void* kc,
                                void* vc, cudaStream_t stream);
+// Block scores from attention over the compressed keys (kernel 32, stride 16):
+// scores [T, hkv, nb_stride] fp32; tile_off [nseq + 1] scratch; qmap over Q [T, hq, 128]
+// with box (64 columns, G heads, 128 / G tokens), kcmap over k_cmp [kc_rows, hkv, 128]
+// with box (64 columns, 1 head, 64 rows), both 128-byte swizzled.
+cudaError_t launch_cmp_scores(const void* q, const void* kc, long long kc_rows, const int32_t* cu,
+                              const int32_t* cu_cmp, int nseq, int T, int hq, int hkv,
+                              int nb_stride, int bs, float scale, float* scores,
+                              int32_t* tile_off, DevStatus* st, int num_sms,
+                              const CUtensorMap* qmap, const CUtensorMap* kcmap,
+                              cudaStream_t stream);
 cudaError_t launch_select_topk(const float* scores, const int32_t* cu, int nseq, int T, int hkv,
                                int nb_stride, int bs, int topk, int init_blocks, int local_blocks,
                                int32_t* bidx, DevStatus* st, cudaStream_t stream);

@@ -215,8 +215,8 @@ NSA_API nsa_status_t nsa_sel_validate_indices(const int32_t *cu_seqlens, int num
                                       long long *n_duplicates, void *workspace,
                                       size_t workspace_bytes, nsa_stream_t stream);
 
-/* Block-selection step, the stage that produces block_idx (kernels of its two ends;
- * the scoring by compressed attention in between is not part of this library yet).
+/* Block-selection step, the stage that produces block_idx: compression, block scores
+ * from attention over the compressed keys, top-k.
  * The quick start of the "Relaxed-System-Lab/Flash-Sparse-Attention" project page
  * sets kernel_size 32, kernel_stride 16, init_blocks 1, local_blocks 2; the pages
  * print no formula, so compressed keys / values are the means of the covered rows
@@ -238,6 +238,30 @@ NSA_API nsa_status_t nsa_sel_compress_kv(const void *k, const void *v, const int
                                          int kernel_size, int kernel_stride, unsigned flags,
                                          void *k_cmp, void *v_cmp, int32_t *cu_cmp,
                                          nsa_stream_t stream);
+
+/* nsa_sel_block_scores: the scores of the selection blocks from attention over the
+ * compressed keys (kernel_size 32, kernel_stride 16 only).  The token at local
+ * position i sees compressed block c when c * 16 + 31 <= i; its probabilities are the
+ * softmax of scale * q . k_cmp[c] over those blocks (none seen: all 0).  The score of
+ * selection block b for (token, KV head g) is the sum, over the G = hq / hkv query
+ * heads of g and over the compressed blocks whose span meets block b, of those
+ * probabilities.
+ *   q          bf16 [total_tokens, hq, head_dim], head_dim 128, G dividing 32
+ *   k_cmp      bf16 [k_cmp_rows, hkv, head_dim] and cu_cmp int32 [num_seqs + 1], as
+ *              nsa_sel_compress_kv wrote them (k_cmp_rows = its room)
+ *   scores     fp32 [total_tokens, hkv, nb_stride] (written for blocks
+ *              b < nb_stride up to the block of the row's own token; later entries of
+ *              a row are left as they were)
+ *   block_size 64 or 128; workspace of nsa_sel_block_scores_workspace_size(num_seqs)
+ *   bytes, 256-byte aligned (its status block is read by nsa_sel_check_status). */
+NSA_API size_t nsa_sel_block_scores_workspace_size(int num_seqs);
+NSA_API nsa_status_t nsa_sel_block_scores(const void *q, const void *k_cmp, int k_cmp_rows,
+                                          const int32_t *cu_seqlens, const int32_t *cu_cmp,
+                                          int num_seqs, int total_tokens, int hq, int hkv,
+                                          int head_dim, int block_size, int kernel_size,
+                                          int kernel_stride, float scale, int nb_stride,
+                                          float *scores, void *workspace, size_t workspace_bytes,
+                                          nsa_stream_t stream);
 
 /* nsa_sel_select_topk: block_idx row of (token at local position i, KV head g), with
  * qb = i / block_size: blocks 0 .. init_blocks - 1, then qb, qb - 1, .. (local_blocks

@@ -143,6 +143,23 @@ def test_selection_entry_points_check_arguments(lib):
                                    None) == 3
 
 
+def test_block_scores_entry_point_checks_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    F = ctypes.c_float
+    ws = lib.nsa_sel_block_scores_workspace_size(3)
+    assert ws >= 256 + 16 and lib.nsa_sel_block_scores_workspace_size(0) == 0
+    args = lambda hq, hkv, bs, ksz, kst, rows, wsb: (fake, fake, rows, fake, fake, 3, 256, hq, hkv,
+                                                     128, bs, ksz, kst, F(0.1), 8, fake, fake, wsb,
+                                                     None)
+    assert lib.nsa_sel_block_scores(*args(12, 4, 64, 32, 16, 16, ws)) == 2   # group 3
+    assert lib.nsa_sel_block_scores(*args(128, 2, 64, 32, 16, 16, ws)) == 2  # group 64 > 32
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 16, 16, 16, ws)) == 2    # other geometry
+    assert lib.nsa_sel_block_scores(*args(8, 2, 32, 32, 16, 16, ws)) == 2    # block 32
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 32, 16, 0, ws)) == 1     # no compressed rows
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 32, 16, 16, 100)) == 3   # short workspace
+
+
 def test_binding_rejects_other_element_types():
     import torch
     x = torch.zeros((4, 2, 128), dtype=torch.float32)

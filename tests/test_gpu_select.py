@@ -98,3 +98,68 @@ def test_select_topk_short_score_rows_reported():
                                   4, 1, 2)
     assert nsa.nsa_sel_check_status() == 1            # NSA_ERR_INVALID_ARG
     assert np.all(got[299].cpu().numpy() == -1)
+
+
+def _oracle_scores(p, hkv, bs):
+    """Oracle block scores from the oracle's own compressed keys rounded to bf16 (the
+    kernel's compressed keys are bf16)."""
+    kc, vc, cuc = sel.compress_kv(p.k, p.v, p.cu_seqlens, 32, 16)
+    kc = ni.bf16_round(kc.astype(np.float32)).astype(np.float64)
+    _, _, probs = sel.compressed_attention(p.q, kc, vc, p.cu_seqlens, cuc, p.scale, 32, 16)
+    return sel.block_scores(probs, p.cu_seqlens, hkv, bs, 32, 16)
+
+
+@pytest.mark.parametrize("lengths,hq,hkv,bs", [([1500, 40, 0, 700], 8, 2, 64),
+                                               ([2100], 4, 4, 128),
+                                               ([900, 1300], 16, 1, 64),
+                                               ([3000], 32, 1, 64)])
+def test_block_scores_match_oracle(lengths, hq, hkv, bs):
+    p = ni.make_problem(lengths, hq=hq, hkv=hkv, head_dim=128, block_size=bs, topk=4, seed=75,
+                        with_dout=False)
+    dev = torch.device("cuda", 0)
+    f = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
+    q, k, v = f(p.q), f(p.k), f(p.v)
+    cu = torch.from_numpy(p.cu_seqlens).to(dev)
+    kc, _, cu_cmp = nsa.nsa_sel_compress_kv(k, v, cu)
+    nb = max((L + bs - 1) // bs for L in lengths)
+    got = nsa.nsa_sel_block_scores(q, kc, cu, cu_cmp, bs, nb, p.scale).cpu().numpy()
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    want = _oracle_scores(p, hkv, bs)
+    G = hq // hkv
+    for s, ref in enumerate(want):
+        a = int(p.cu_seqlens[s])
+        for i in range(ref.shape[0]):
+            qb = i // bs
+            g_ = got[a + i, :, :qb + 1].astype(np.float64)
+            assert np.all(np.abs(g_ - ref[i, :, :qb + 1]) <= 1e-3 * G + 1e-3 * np.abs(ref[i, :, :qb + 1])), (s, i)
+
+
+def test_select_blocks_end_to_end():
+    # compression, scores and top-k on the GPU: forced slots exact; every other chosen
+    # block scores (by the oracle) within tolerance of the oracle's k-th best
+    bs, topk, hkv = 64, 8, 2
+    p = ni.make_problem([2500, 600], hq=8, hkv=hkv, head_dim=128, block_size=bs, topk=topk,
+                        seed=76, with_dout=False)
+    dev = torch.device("cuda", 0)
+    f = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
+    bi = nsa.nsa_sel_select_blocks(f(p.q), f(p.k), f(p.v), torch.from_numpy(p.cu_seqlens).to(dev),
+                                   bs, topk, 1, 2, max_seqlen=2500, scale=p.scale).cpu().numpy()
+    assert nsa.nsa_sel_check_status() == 0
+    ref = _oracle_scores(p, hkv, bs)
+    want = sel.select_topk(ref, p.cu_seqlens, topk, bs, 1, 2)
+    G = 4
+    for s in range(2):
+        a, L = int(p.cu_seqlens[s]), int(p.cu_seqlens[s + 1] - p.cu_seqlens[s])
+        for i in range(L):
+            qb = i // bs
+            nforced = min(3, qb + 1)
+            for g in range(hkv):
+                assert np.array_equal(bi[a + i, g, :nforced], want[a + i, g, :nforced])
+                row = [int(b) for b in bi[a + i, g] if b >= 0]
+                assert len(row) == len(set(row)) == min(topk, qb + 1)
+                rest = [int(b) for b in want[a + i, g, nforced:] if b >= 0]
+                if rest:
+                    kth = ref[s][i, g, rest[-1]]
+                    for b in row[nforced:]:
+                        assert ref[s][i, g, b] >= kth - 2e-3 * G, (s, i, g, b)
