@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
             "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_fwd_ex",
             "nsa_sel_attn_bwd_ex", "nsa_sel_compress_kv", "nsa_sel_select_topk",
-            "nsa_sel_block_scores", "nsa_sel_block_scores_workspace_size",
+            "nsa_sel_block_scores", "nsa_sel_block_scores_workspace_size", "nsa_sel_bsfa_fwd",
+            "nsa_sel_bsfa_workspace_size",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_block_scores_workspace_size.restype = Z
             lib.nsa_sel_block_scores.argtypes = [P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, P, P, Z, P]
             lib.nsa_sel_block_scores.restype = I
+            lib.nsa_sel_bsfa_workspace_size.argtypes = [I]
+            lib.nsa_sel_bsfa_workspace_size.restype = Z
+            lib.nsa_sel_bsfa_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, Z, P]
+            lib.nsa_sel_bsfa_fwd.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
             lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
@@ -364,6 +369,30 @@ def nsa_sel_select_blocks(q, k, v, cu_seqlens, block_size=64, topk=16, init_bloc
     kc, _, cu_cmp = nsa_sel_compress_kv(k, v, cu_seqlens)
     sc = nsa_sel_block_scores(q, kc, cu_seqlens, cu_cmp, block_size, nb_stride, scale)
     return nsa_sel_select_topk(sc, cu_seqlens, block_size, topk, init_blocks, local_blocks)
+
+
+def nsa_sel_bsfa_fwd(q, k, v, cu_seqlens, tau, scale=None, block_size=64, workspace=None):
+    """Threshold-pruned block attention; returns (out bf16 [T, hq, d], lse fp32 [hq, T]).
+    tau: fp32 [hq] thresholds on the device."""
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(tau, "tau", torch.float32, 1, dev)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if tau.numel() != hq:
+        raise ValueError("tau needs one threshold per query head")
+    scale = float(d ** -0.5 if scale is None else scale)
+    nseq = cu_seqlens.numel() - 1
+    lib = load_library()
+    ws = workspace if workspace is not None else get_workspace(int(lib.nsa_sel_bsfa_workspace_size(nseq)), dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    _check("nsa_sel_bsfa_fwd", lib.nsa_sel_bsfa_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, block_size, scale,
+        _ptr(tau), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
+    return out, lse
 
 
 def nsa_sel_select_topk(scores, cu_seqlens, block_size, topk, init_blocks=1, local_blocks=2,

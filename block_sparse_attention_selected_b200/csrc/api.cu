@@ -708,6 +708,43 @@ nsa_status_t nsa_sel_block_scores(const void* q, const void* k_cmp, int k_cmp_ro
                                          scores, tile_off, st, num_sms, &qmap, &kcmap, stream));
 }
 
+size_t nsa_sel_bsfa_workspace_size(int num_seqs) { return nsa_sel_block_scores_workspace_size(num_seqs); }
+
+nsa_status_t nsa_sel_bsfa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                          int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                          int block_size, float scale, const float* tau, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, nsa_stream_t stream_) {
+    if (total_tokens < 0 || num_seqs < 1 || hq < 1 || hkv < 1 || hq % hkv != 0)
+        return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (head_dim != kHeadDim || block_size != 64 || kTileRows % G != 0 ||
+        total_tokens >= (1 << 25) || (long long)total_tokens * hq >= (1ll << 31))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !workspace || (total_tokens > 0 && (!q || !k || !v || !tau || !out)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(cu_seqlens, 4) || !aligned(tau, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
+        return NSA_ERR_INVALID_ARG;
+    if (workspace_bytes < nsa_sel_bsfa_workspace_size(num_seqs)) return NSA_ERR_WORKSPACE;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    int32_t* tile_off = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                                   align256(sizeof(DevStatus)));
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) return NSA_OK;
+    CUtensorMap qmap, kmap, vmap;
+    if (!make_q_group_map(&qmap, q, total_tokens, hq, G) ||
+        !make_kv_map(&kmap, k, total_tokens, hkv, 64, false) ||
+        !make_kv_map(&vmap, v, total_tokens, hkv, 64, false))
+        return NSA_ERR_CUDA;
+    return cuda_status(launch_bsfa_fwd(cu_seqlens, num_seqs, total_tokens, hq, hkv, scale, tau, out,
+                                       lse, tile_off, st, num_sms, &qmap, &kmap, &vmap, stream));
+}
+
 nsa_status_t nsa_sel_select_topk(const float* scores, const int32_t* cu_seqlens, int num_seqs,
                                  int total_tokens, int hkv, int nb_stride, int block_size,
                                  int topk, int init_blocks, int local_blocks, int32_t* block_idx,

@@ -169,6 +169,13 @@ cudaError_t launch_cmp_scores(const void* q, const void* kc, long long kc_rows, 
                               int32_t* tile_off, DevStatus* st, int num_sms,
                               const CUtensorMap* qmap, const CUtensorMap* kcmap,
                               cudaStream_t stream);
+// Threshold-pruned block attention (bsfa.cu): out bf16 [T, hq, 128], lse [hq, T] (or
+// null); tau fp32 [hq]; qmap as for the block scores, kmap / vmap as for the forward.
+cudaError_t launch_bsfa_fwd(const int32_t* cu, int nseq, int T, int hq, int hkv, float scale,
+                            const float* tau, void* out, float* lse, int32_t* tile_off,
+                            DevStatus* st, int num_sms, const CUtensorMap* qmap,
+                            const CUtensorMap* kmap, const CUtensorMap* vmap,
+                            cudaStream_t stream);
 cudaError_t launch_select_topk(const float* scores, const int32_t* cu, int nseq, int T, int hkv,
                                int nb_stride, int bs, int topk, int init_blocks, int local_blocks,
                                int32_t* bidx, DevStatus* st, cudaStream_t stream);

@@ -280,6 +280,23 @@ NSA_API nsa_status_t nsa_sel_select_topk(const float *scores, const int32_t *cu_
                                          int local_blocks, int32_t *block_idx, void *workspace,
                                          size_t workspace_bytes, nsa_stream_t stream);
 
+/* Threshold-pruned block attention (BSFA; the "Block Sparse Flash Attention" news
+ * pages): every score is exact; key block b (64 keys of the token's sequence) is kept
+ * for row (token at local position i, query head h) iff
+ * max_{j in b, j <= i} scale * q . k_j >= tau[h]; the output is softmax attention
+ * over the keys of the kept blocks only (no kept block: out = 0, lse = -inf).
+ *   q bf16 [total_tokens, hq, 128]; k, v bf16 [total_tokens, hkv, 128]
+ *   tau   fp32 [hq] device array of thresholds (natural units of scale * q . k)
+ *   out   bf16 [total_tokens, hq, 128] (written); lse fp32 [hq, total_tokens] or null
+ *   block_size 64; hq / hkv must divide 128; workspace of
+ *   nsa_sel_bsfa_workspace_size(num_seqs) bytes, 256-byte aligned. */
+NSA_API size_t nsa_sel_bsfa_workspace_size(int num_seqs);
+NSA_API nsa_status_t nsa_sel_bsfa_fwd(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens, int num_seqs, int total_tokens,
+                                  int hq, int hkv, int head_dim, int block_size, float scale,
+                                  const float *tau, void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, nsa_stream_t stream);
+
 /* Synchronises `stream` and returns the device-side status of the last call that
  * used this workspace (NSA_OK, NSA_ERR_TIMEOUT or NSA_ERR_BAD_INDEX). */
 NSA_API nsa_status_t nsa_sel_check_status(const void *workspace, nsa_stream_t stream);

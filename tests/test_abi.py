@@ -160,6 +160,20 @@ def test_block_scores_entry_point_checks_arguments(lib):
     assert lib.nsa_sel_block_scores(*args(8, 2, 64, 32, 16, 16, 100)) == 3   # short workspace
 
 
+def test_bsfa_entry_point_checks_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    F = ctypes.c_float
+    ws = lib.nsa_sel_bsfa_workspace_size(2)
+    a = lambda hq, hkv, d, bs, wsb: (fake, fake, fake, fake, 2, 256, hq, hkv, d, bs, F(0.1), fake,
+                                     fake, fake, fake, wsb, None)
+    assert lib.nsa_sel_bsfa_fwd(*a(12, 4, 128, 64, ws)) == 2      # group 3
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 64, 64, ws)) == 2        # head dim 64
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 128, 128, ws)) == 2      # block 128
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 3, 128, 64, ws)) == 1       # hq % hkv
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 128, 64, 64)) == 3       # short workspace
+
+
 def test_binding_rejects_other_element_types():
     import torch
     x = torch.zeros((4, 2, 128), dtype=torch.float32)
