@@ -15,9 +15,11 @@
 //           blocks' keys update the row's running max and sum (its LSE);
 //   pass 2  S again; P = 2^(c S - lse) on the kept blocks (0 elsewhere), written as
 //           bf16 into the S columns of TMEM; O += P V (P read from TMEM).
-// Because pass 2 knows the final LSE, O is never rescaled.  This version computes
-// every block of the tile (pruned rows get P = 0); skipping a block that no row of
-// the tile keeps is the next step.
+// Because pass 2 knows the final LSE, O is never rescaled.  Pass 1 also marks, per
+// tile, the blocks that at least one row keeps (a bit mask in shared memory, one per
+// tile parity); pass 2 loads, multiplies and accumulates only those blocks (rows that
+// pruned a block of the mask get P = 0 there).  Tiles with more than kMaskBits blocks
+// (sequences beyond 131072 tokens) visit every block in pass 2.
 //
 //   warp 0       TMA producer: Q tile; K blocks (pass 1), K and V blocks (pass 2)
 //   warp 1       MMA issuer: S (8 x M128 N64 K16) into two TMEM slots, PV (4 x M128
@@ -36,6 +38,7 @@ constexpr int kBfThreads = 256;
 constexpr int kBfStages = 3;
 constexpr int kBfRows = 128;       // threads of the row warpgroup
 constexpr int kBfBS = 64;          // keys per block
+constexpr int kMaskBits = 2048;    // blocks a tile's keep mask covers
 
 struct alignas(1024) BsfaSmem {
     uint8_t q[2][kTileRows * 128];            // Q tile: [64-column half][row]
@@ -44,6 +47,8 @@ struct alignas(1024) BsfaSmem {
     uint64_t kv_full[kBfStages], kv_empty[kBfStages];
     uint64_t s_full[2], s_read[2], p_full[2], pv_done[2];
     uint64_t o_full, o_empty, drain;
+    uint64_t mask_ready;                      // the rows finished pass 1 of the tile
+    uint32_t keep[2][kMaskBits / 32];         // blocks kept by some row, per tile parity
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -95,6 +100,7 @@ __global__ void __launch_bounds__(kBfThreads, 1)
         }
         mbar_init(&S.o_full, 1);
         mbar_init(&S.o_empty, kBfRows);
+        mbar_init(&S.mask_ready, kBfRows);
         mbar_init(&S.drain, 1);
         fence_barrier_init();
     }
@@ -129,6 +135,21 @@ __global__ void __launch_bounds__(kBfThreads, 1)
         return t;
     };
     const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
+    // pass 2 visits the blocks kb >= from whose bit is set in the tile's mask (every
+    // block when the tile has more blocks than the mask covers); nkb when none is left
+    auto next_kept = [&](const Tile& t, int n, int from) -> int {
+        if (t.nkb > kMaskBits) return from;
+        const volatile uint32_t* km = S.keep[n & 1];
+        for (int w = from >> 5; w < (t.nkb + 31) >> 5; ++w) {
+            uint32_t bits = km[w];
+            if (w == (from >> 5)) bits &= ~0u << (from & 31);
+            if (bits) {
+                const int kb = w * 32 + __ffs(bits) - 1;
+                return kb < t.nkb ? kb : t.nkb;
+            }
+        }
+        return t.nkb;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------- TMA producer
@@ -148,8 +169,10 @@ __global__ void __launch_bounds__(kBfThreads, 1)
                 tma_load_3d(S.q[1], &qmap, &S.q_full, 64, t.g * p.G, tok0);
                 qpar = n & 1;
                 const int key0 = __ldg(p.cu + t.s);
-                for (int pass = 0; pass < 2 && ok; ++pass)
-                    for (int kb = 0; kb < t.nkb; ++kb, ++u) {
+                for (int pass = 0; pass < 2 && ok; ++pass) {
+                    if (pass == 1 && !(ok = wait(&S.mask_ready, n & 1, 136))) break;
+                    for (int kb = pass == 0 ? 0 : next_kept(t, n, 0); kb < t.nkb;
+                         kb = pass == 0 ? kb + 1 : next_kept(t, n, kb + 1), ++u) {
                         const int stg = u % kBfStages;
                         if (!(ok = wait(&S.kv_empty[stg], ((u / kBfStages) & 1) ^ 1, 121))) break;
                         const int row = key0 + kb * kBfBS;
@@ -162,6 +185,7 @@ __global__ void __launch_bounds__(kBfThreads, 1)
                         }
                         kvpar[stg] = (u / kBfStages) & 1;
                     }
+                }
             }
             if (*abort_flag) {   // let copies still in flight land before the CTA exits
                 if (qpar >= 0) mbar_wait(&S.q_full, qpar, st, 122);
@@ -215,8 +239,10 @@ __global__ void __launch_bounds__(kBfThreads, 1)
             if (!ok) break;
             // the previous tile's O has been read out before this tile's first PV
             if (!(ok = wait(&S.o_empty, (n & 1) ^ 1, 128))) break;
-            // pass 2: S(kb), then once the rows wrote P(kb), O += P(kb) V(kb)
-            for (int kb = 0; kb < t.nkb && ok; ++kb, ++u, ++j) {
+            // pass 2 over the kept blocks: S(kb), then once the rows wrote P(kb), O += P(kb) V(kb)
+            if (!(ok = wait(&S.mask_ready, n & 1, 134))) break;
+            bool first = true;
+            for (int kb = next_kept(t, n, 0); kb < t.nkb && ok; kb = next_kept(t, n, kb + 1), ++u, ++j) {
                 const int stg = u % kBfStages, slot = j & 1;
                 if (!(ok = wait(&S.kv_full[stg], (u / kBfStages) & 1, 129))) break;
                 if (!(ok = issue_s(j, stg))) break;
@@ -228,7 +254,8 @@ __global__ void __launch_bounds__(kBfThreads, 1)
 #pragma unroll
                 for (int ks = 0; ks < kBfBS / 16; ++ks)
                     mma_ts_e(tO, tS + (uint32_t)ks * 8u, b0 + (uint32_t)ks * 128u, kIdescO,
-                             (kb > 0 || ks > 0) ? 1u : 0u, elected);
+                             (!first || ks > 0) ? 1u : 0u, elected);
+                first = false;
                 mma_commit_e(&S.pv_done[slot], elected);
                 mma_commit_e(&S.kv_empty[stg], elected);
                 last_kind[slot] = 2;
@@ -255,8 +282,21 @@ __global__ void __launch_bounds__(kBfThreads, 1)
             const int head = t.g * p.G + h;
             const float tau2 = __ldg(p.tau + head) * 1.4426950408889634f;   // log2 units
             float m = -CUDART_INF_F, l = 0.f, lse2 = -CUDART_INF_F;
+            // this tile's keep mask starts empty (the producer and the issuer finished
+            // with the mask of tile n - 2 before this tile's first S could arrive)
+            if (r < kMaskBits / 32) S.keep[n & 1][r] = 0u;
+            if (kMaskBits / 32 > kBfRows)
+                for (int w = r + kBfRows; w < kMaskBits / 32; w += kBfRows) S.keep[n & 1][w] = 0u;
+            asm volatile("bar.sync 1, %0;" ::"n"(kBfRows) : "memory");
             for (int pass = 0; pass < 2 && ok; ++pass) {
-                for (int kb = 0; kb < t.nkb; ++kb, ++j) {
+                if (pass == 1) {
+                    // every row's bits are in the mask once all rows have arrived
+                    __threadfence_block();
+                    mbar_arrive(&S.mask_ready);
+                    if (!(ok = __all_sync(0xffffffffu, wait(&S.mask_ready, n & 1, 135)))) break;
+                }
+                for (int kb = pass == 0 ? 0 : next_kept(t, n, 0); kb < t.nkb;
+                     kb = pass == 0 ? kb + 1 : next_kept(t, n, kb + 1), ++j) {
                     const int slot = j & 1;
                     if (!(ok = __all_sync(0xffffffffu, wait(&S.s_full[slot], (j >> 1) & 1, 132)))) break;
                     tc_fence_after();
@@ -271,6 +311,8 @@ __global__ void __launch_bounds__(kBfThreads, 1)
                         bm = fmaxf(bm, sv[k]);
                     }
                     const bool kept = bm != -CUDART_INF_F && bm >= tau2;
+                    if (pass == 0 && t.nkb <= kMaskBits && __any_sync(0xffffffffu, kept) && lane == 0)
+                        atomicOr(&S.keep[n & 1][kb >> 5], 1u << (kb & 31));
                     if (pass == 0) {
                         tc_fence_before();
                         mbar_arrive(&S.s_read[slot]);
@@ -306,9 +348,15 @@ __global__ void __launch_bounds__(kBfThreads, 1)
             const uint32_t tO = tmem + kColO + lane_off;
             const int t_glob = __ldg(p.cu + t.s) + (valid ? i : 0);
             uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)t_glob * p.hq + head) * kHeadDim);
+            // a tile whose mask is empty issued no PV: its O columns are stale, O is 0
+            const bool any_pv = next_kept(t, n, 0) < t.nkb;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 tmem_ld64_sync(tO + (uint32_t)half * 64u, o);
+                if (!any_pv) {
+#pragma unroll
+                    for (int x = 0; x < 64; ++x) o[x] = 0.f;
+                }
                 if (valid) {
 #pragma unroll
                     for (int q8 = 0; q8 < 8; ++q8)
