@@ -452,6 +452,78 @@ def run_ours(args, rank, world, local_rank, dist):
     return line
 
 
+# ------------------------------------------------- the selection step and BSFA
+
+def run_next_path(args):
+    """One GPU, CUDA events: the block-selection step (compression, block scores,
+    top-k) or threshold-pruned block attention on the workload's shapes; one JSON line."""
+    import torch
+    import block_sparse_attention_selected_b200 as nsa
+    from block_sparse_attention_selected_b200 import build as nsa_build
+    nsa_build.build()
+    dev = torch.device("cuda", 0)
+    spec = dict(ni.WORKLOADS[args.workload])
+    p = ni.make_problem(name=args.workload, head_dim=128, with_dout=False, **spec)
+    bf = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
+    q, k, v = bf(p.q), bf(p.k), bf(p.v)
+    cu = torch.from_numpy(p.cu_seqlens).to(dev)
+    T, hq, hkv, bs, d = p.T, p.hq, p.hkv, p.block_size, 128
+    lens = np.diff(p.cu_seqlens.astype(np.int64))
+    i = np.concatenate([np.arange(L) for L in lens]) if T else np.zeros(0, np.int64)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    times = []
+    if args.path == "select":
+        nb = int(max((L + bs - 1) // bs for L in lens))
+        visible = np.where(i >= 31, (i - 31) // 16 + 1, 0)            # compressed keys seen
+        useful = 2.0 * d * float(visible.sum()) * hq                    # one Q Kc^T
+        issued = 2 * useful                                             # two passes
+        ws = nsa.get_workspace(int(nsa.load_library().nsa_sel_block_scores_workspace_size(p.nseq)), dev)
+
+        def step():
+            evs[0].record()
+            kc, _, cu_cmp = nsa.nsa_sel_compress_kv(k, v, cu)
+            evs[1].record()
+            sc = nsa.nsa_sel_block_scores(q, kc, cu, cu_cmp, bs, nb, p.scale, workspace=ws)
+            evs[2].record()
+            nsa.nsa_sel_select_topk(sc, cu, bs, p.topk, 1, 2, workspace=ws)
+            evs[3].record()
+        names = ("compress_ms", "scores_ms", "topk_ms")
+    else:
+        tau = torch.full((hq,), float(args.tau), dtype=torch.float32, device=dev)
+        causal = (i + 1).astype(np.float64)
+        useful = 2.0 * d * float(causal.sum()) * hq                     # exact scores (one pass)
+        issued = 3 * useful                                             # two S passes + PV on every block
+
+        def step():
+            evs[0].record()
+            nsa.nsa_sel_bsfa_fwd(q, k, v, cu, tau, p.scale)
+            evs[1].record()
+            evs[2].record()
+            evs[3].record()
+        names = ("bsfa_ms",)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        step()
+        torch.cuda.synchronize()
+        times.append([evs[a].elapsed_time(evs[a + 1]) for a in range(len(names))])
+    status = nsa.nsa_sel_check_status()
+    t = np.median(np.asarray(times), axis=0)
+    kernel_ms = float(t[1] if args.path == "select" else t[0])
+    line = {"metric": f"{args.path} step ms and TFLOP/s", "path": args.path,
+            "value": round(float(t.sum()), 4), "unit": "ms", "higher_is_better": False,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "status": int(status),
+            "config": {"workload": args.workload, "total_tokens": T, "hq": hq, "hkv": hkv,
+                       "block_size": bs, "topk": p.topk,
+                       **({"tau": float(args.tau)} if args.path == "bsfa" else {})},
+            "phases_ms": {n: round(float(x), 4) for n, x in zip(names, t)},
+            "useful_tflops": round(useful / (kernel_ms * 1e-3) / 1e12, 2),
+            "issued_tflops": round(issued / (kernel_ms * 1e-3) / 1e12, 2)}
+    print(json.dumps(line), flush=True)
+    return line
+
+
 # ----------------------------------------------------------------- oracle baselines
 
 def oracle_sample(workload: str, tokens: int, window: int = 0):
@@ -525,6 +597,10 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window of this many keys (0: none); the index becomes the "
                          "sliding branch's: every block the window reaches")
+    ap.add_argument("--path", choices=["attn", "select", "bsfa"], default="attn",
+                    help="attn: the selected attention step (the default line); select: the "
+                         "block-selection step; bsfa: threshold-pruned block attention")
+    ap.add_argument("--tau", type=float, default=2.0, help="BSFA threshold of every head")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=2048)
@@ -538,6 +614,10 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return 0
+    if args.path != "attn":
+        if rank == 0:
+            run_next_path(args)
         return 0
     dist = None
     if world > 1:

@@ -25,7 +25,9 @@ STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",
                 6: "NSA_ERR_BAD_INDEX", 7: "NSA_ERR_NO_DEVICE"}
 EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd",
             "nsa_sel_attn_fwd_profiled", "nsa_sel_attn_bwd_profiled", "nsa_sel_attn_fwd_ex",
-            "nsa_sel_attn_bwd_ex",
+            "nsa_sel_attn_bwd_ex", "nsa_sel_compress_kv", "nsa_sel_select_topk",
+            "nsa_sel_block_scores", "nsa_sel_block_scores_workspace_size", "nsa_sel_bsfa_fwd",
+            "nsa_sel_bsfa_workspace_size",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
@@ -66,6 +68,18 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_attn_fwd_ex.restype = I
             lib.nsa_sel_attn_bwd_ex.argtypes = lib.nsa_sel_attn_bwd.argtypes + [ctypes.c_uint, I, P, I, IP]
             lib.nsa_sel_attn_bwd_ex.restype = I
+            lib.nsa_sel_compress_kv.argtypes = [P, P, P, I, I, I, I, I, I, ctypes.c_uint, P, P, P, P]
+            lib.nsa_sel_compress_kv.restype = I
+            lib.nsa_sel_select_topk.argtypes = [P, P, I, I, I, I, I, I, I, I, P, P, Z, P]
+            lib.nsa_sel_select_topk.restype = I
+            lib.nsa_sel_block_scores_workspace_size.argtypes = [I]
+            lib.nsa_sel_block_scores_workspace_size.restype = Z
+            lib.nsa_sel_block_scores.argtypes = [P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, P, P, Z, P]
+            lib.nsa_sel_block_scores.restype = I
+            lib.nsa_sel_bsfa_workspace_size.argtypes = [I]
+            lib.nsa_sel_bsfa_workspace_size.restype = Z
+            lib.nsa_sel_bsfa_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P, P, Z, P]
+            lib.nsa_sel_bsfa_fwd.restype = I
             lib.nsa_sel_invert_index.argtypes = [P, I, I, I, P, I, I, P, P, P, P, Z, P]
             lib.nsa_sel_invert_index.restype = I
             lib.nsa_sel_invert_index_noalloc.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
@@ -301,6 +315,104 @@ def nsa_sel_validate_indices(cu_seqlens, block_idx, block_size, workspace=None):
     if code not in (0, 6):
         raise NsaError("nsa_sel_validate_indices", code)
     return int(a.value), int(b.value)
+
+
+def nsa_sel_compress_kv(k, v, cu_seqlens, kernel_size=32, kernel_stride=16):
+    """Mean-pooled compressed K and V of the selection step; returns (k_cmp, v_cmp,
+    cu_cmp): k_cmp / v_cmp [floor(T / stride), hkv, d] in the type of k (rows past
+    cu_cmp[-1] unused), cu_cmp int32 [nseq + 1]."""
+    dev = k.device
+    et, flag = _elem_type(k)
+    _need(k, "k", et, 3, dev)
+    _need(v, "v", et, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    T, hkv, d = k.shape
+    if v.shape != k.shape:
+        raise ValueError("inconsistent shapes")
+    nseq = cu_seqlens.numel() - 1
+    rows = max(T // kernel_stride, 1)
+    kc = torch.empty((rows, hkv, d), dtype=et, device=dev)
+    vc = torch.empty((rows, hkv, d), dtype=et, device=dev)
+    cu_cmp = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
+    _check("nsa_sel_compress_kv", load_library().nsa_sel_compress_kv(
+        _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hkv, d, kernel_size, kernel_stride, flag,
+        _ptr(kc), _ptr(vc), _ptr(cu_cmp), _stream(dev)))
+    return kc, vc, cu_cmp
+
+
+def nsa_sel_block_scores(q, k_cmp, cu_seqlens, cu_cmp, block_size, nb_stride, scale=None,
+                         kernel_size=32, kernel_stride=16, workspace=None):
+    """Selection-block scores fp32 [T, hkv, nb_stride] from attention over the compressed
+    keys (entries past each row's own block are left uninitialised)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, 3, dev)
+    _need(k_cmp, "k_cmp", torch.bfloat16, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(cu_cmp, "cu_cmp", torch.int32, 1, dev)
+    T, hq, d = q.shape
+    rows, hkv, _ = k_cmp.shape
+    scale = float(d ** -0.5 if scale is None else scale)
+    nseq = cu_seqlens.numel() - 1
+    lib = load_library()
+    nbytes = int(lib.nsa_sel_block_scores_workspace_size(nseq))
+    ws = workspace if workspace is not None else get_workspace(nbytes, dev)
+    scores = torch.empty((T, hkv, nb_stride), dtype=torch.float32, device=dev)
+    _check("nsa_sel_block_scores", lib.nsa_sel_block_scores(
+        _ptr(q), _ptr(k_cmp), rows, _ptr(cu_seqlens), _ptr(cu_cmp), nseq, T, hq, hkv, d,
+        block_size, kernel_size, kernel_stride, scale, nb_stride, _ptr(scores), _ptr(ws),
+        ws.numel(), _stream(dev)))
+    return scores
+
+
+def nsa_sel_select_blocks(q, k, v, cu_seqlens, block_size=64, topk=16, init_blocks=1,
+                          local_blocks=2, max_seqlen=None, scale=None):
+    """The whole selection step on the GPU: compression, block scores, top-k; returns
+    block_idx int32 [T, hkv, topk].  max_seqlen (host int) sizes the score rows."""
+    T = q.shape[0]
+    L = int(max_seqlen) if max_seqlen is not None else T
+    nb_stride = max((L + block_size - 1) // block_size, 1)
+    kc, _, cu_cmp = nsa_sel_compress_kv(k, v, cu_seqlens)
+    sc = nsa_sel_block_scores(q, kc, cu_seqlens, cu_cmp, block_size, nb_stride, scale)
+    return nsa_sel_select_topk(sc, cu_seqlens, block_size, topk, init_blocks, local_blocks)
+
+
+def nsa_sel_bsfa_fwd(q, k, v, cu_seqlens, tau, scale=None, block_size=64, workspace=None):
+    """Threshold-pruned block attention; returns (out bf16 [T, hq, d], lse fp32 [hq, T]).
+    tau: fp32 [hq] thresholds on the device."""
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    _need(tau, "tau", torch.float32, 1, dev)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    if tau.numel() != hq:
+        raise ValueError("tau needs one threshold per query head")
+    scale = float(d ** -0.5 if scale is None else scale)
+    nseq = cu_seqlens.numel() - 1
+    lib = load_library()
+    ws = workspace if workspace is not None else get_workspace(int(lib.nsa_sel_bsfa_workspace_size(nseq)), dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
+    _check("nsa_sel_bsfa_fwd", lib.nsa_sel_bsfa_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, block_size, scale,
+        _ptr(tau), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
+    return out, lse
+
+
+def nsa_sel_select_topk(scores, cu_seqlens, block_size, topk, init_blocks=1, local_blocks=2,
+                        workspace=None):
+    """block_idx int32 [T, hkv, topk] from block scores fp32 [T, hkv, nb_stride]."""
+    dev = scores.device
+    _need(scores, "scores", torch.float32, 3, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1, dev)
+    T, hkv, nb = scores.shape
+    out = torch.empty((T, hkv, topk), dtype=torch.int32, device=dev)
+    ws = workspace if workspace is not None else get_workspace(256, dev)
+    _check("nsa_sel_select_topk", load_library().nsa_sel_select_topk(
+        _ptr(scores), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, nb, block_size, topk,
+        init_blocks, local_blocks, _ptr(out), _ptr(ws), ws.numel(), _stream(dev)))
+    return out
 
 
 def nsa_sel_check_status(workspace=None, device=None) -> int:

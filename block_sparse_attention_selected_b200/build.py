@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnsa_sel.so")
-SOURCES = ["api.cu", "invert.cu", "fwd.cu", "merge.cu", "bwd.cu"]
+SOURCES = ["api.cu", "invert.cu", "fwd.cu", "merge.cu", "bwd.cu", "select.cu", "bsfa.cu"]
 HEADERS = ["nsa_common.cuh", "nsa_kernels.h"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -158,6 +158,21 @@ bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs, boo
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a bf16 Q [T, hq, 128]; box = (64 columns, G heads, 128 / G tokens):
+// one 128-row tile of G heads of consecutive tokens, rows token-major, 128-byte swizzle.
+bool make_q_group_map(CUtensorMap* map, const void* base, int T, int hq, int G) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)hq, (cuuint64_t)(T > 0 ? T : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)hq * kHeadDim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kTileRows / G)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, box_rows),
 // 128-byte swizzle: the epilogue's TMA stores of 8-row groups and of whole warps.
 bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows) {
@@ -631,6 +646,136 @@ nsa_status_t nsa_sel_validate_indices(const int32_t* cu_seqlens, int num_seqs, i
     if (n_out_of_range) *n_out_of_range = h.bad_range;
     if (n_duplicates) *n_duplicates = h.bad_dup;
     return (h.bad_range || h.bad_dup) ? NSA_ERR_BAD_INDEX : NSA_OK;
+}
+
+nsa_status_t nsa_sel_compress_kv(const void* k, const void* v, const int32_t* cu_seqlens,
+                                 int num_seqs, int total_tokens, int hkv, int head_dim,
+                                 int kernel_size, int kernel_stride, unsigned flags, void* k_cmp,
+                                 void* v_cmp, int32_t* cu_cmp, nsa_stream_t stream_) {
+    if (flags & ~(unsigned)NSA_F16) return NSA_ERR_INVALID_ARG;
+    if (total_tokens < 0 || num_seqs < 1 || hkv < 1 || kernel_stride < 1 ||
+        kernel_size < kernel_stride)
+        return NSA_ERR_INVALID_ARG;
+    if (head_dim != kHeadDim || kernel_size > 4096 || total_tokens >= (1 << 25))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !cu_cmp || (total_tokens >= kernel_stride && (!k || !v || !k_cmp || !v_cmp)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4) || !aligned(cu_cmp, 4) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(k_cmp, 16) || !aligned(v_cmp, 16))
+        return NSA_ERR_INVALID_ARG;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    return cuda_status(launch_compress_kv(k, v, cu_seqlens, num_seqs, total_tokens, hkv, kernel_size,
+                                          kernel_stride, (flags & NSA_F16) ? 1 : 0, cu_cmp, k_cmp,
+                                          v_cmp, reinterpret_cast<cudaStream_t>(stream_)));
+}
+
+size_t nsa_sel_block_scores_workspace_size(int num_seqs) {
+    return num_seqs < 1 ? 0 : align256(sizeof(DevStatus)) + align256(sizeof(int32_t) * ((size_t)num_seqs + 1));
+}
+
+nsa_status_t nsa_sel_block_scores(const void* q, const void* k_cmp, int k_cmp_rows,
+                                  const int32_t* cu_seqlens, const int32_t* cu_cmp, int num_seqs,
+                                  int total_tokens, int hq, int hkv, int head_dim, int block_size,
+                                  int kernel_size, int kernel_stride, float scale, int nb_stride,
+                                  float* scores, void* workspace, size_t workspace_bytes,
+                                  nsa_stream_t stream_) {
+    if (total_tokens < 0 || num_seqs < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 ||
+        nb_stride < 1 || k_cmp_rows < 1)
+        return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (head_dim != kHeadDim || kernel_size != 32 || kernel_stride != 16 ||
+        (block_size != 64 && block_size != 128) || G > 32 || 32 % G != 0 ||
+        total_tokens >= (1 << 25) || (long long)total_tokens * hkv * nb_stride >= (1ll << 40))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !cu_cmp || !workspace || !k_cmp || (total_tokens > 0 && (!q || !scores)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cmp, 16) || !aligned(cu_seqlens, 4) || !aligned(cu_cmp, 4) ||
+        !aligned(scores, 4) || !aligned(workspace, 256))
+        return NSA_ERR_INVALID_ARG;
+    if (workspace_bytes < nsa_sel_block_scores_workspace_size(num_seqs)) return NSA_ERR_WORKSPACE;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    int32_t* tile_off = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                                   align256(sizeof(DevStatus)));
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) return NSA_OK;
+    CUtensorMap qmap, kcmap;
+    if (!make_q_group_map(&qmap, q, total_tokens, hq, G) ||
+        !make_kv_map(&kcmap, k_cmp, k_cmp_rows, hkv, 64, false))
+        return NSA_ERR_CUDA;
+    return cuda_status(launch_cmp_scores(q, k_cmp, k_cmp_rows, cu_seqlens, cu_cmp, num_seqs,
+                                         total_tokens, hq, hkv, nb_stride, block_size, scale,
+                                         scores, tile_off, st, num_sms, &qmap, &kcmap, stream));
+}
+
+size_t nsa_sel_bsfa_workspace_size(int num_seqs) { return nsa_sel_block_scores_workspace_size(num_seqs); }
+
+nsa_status_t nsa_sel_bsfa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                          int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
+                          int block_size, float scale, const float* tau, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, nsa_stream_t stream_) {
+    if (total_tokens < 0 || num_seqs < 1 || hq < 1 || hkv < 1 || hq % hkv != 0)
+        return NSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !(scale < 1e30f)) return NSA_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (head_dim != kHeadDim || block_size != 64 || kTileRows % G != 0 ||
+        total_tokens >= (1 << 25) || (long long)total_tokens * hq >= (1ll << 31))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !workspace || (total_tokens > 0 && (!q || !k || !v || !tau || !out)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(cu_seqlens, 4) || !aligned(tau, 4) || !aligned(lse, 4) || !aligned(workspace, 256))
+        return NSA_ERR_INVALID_ARG;
+    if (workspace_bytes < nsa_sel_bsfa_workspace_size(num_seqs)) return NSA_ERR_WORKSPACE;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    int32_t* tile_off = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                                   align256(sizeof(DevStatus)));
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (total_tokens == 0) return NSA_OK;
+    CUtensorMap qmap, kmap, vmap;
+    if (!make_q_group_map(&qmap, q, total_tokens, hq, G) ||
+        !make_kv_map(&kmap, k, total_tokens, hkv, 64, false) ||
+        !make_kv_map(&vmap, v, total_tokens, hkv, 64, false))
+        return NSA_ERR_CUDA;
+    return cuda_status(launch_bsfa_fwd(cu_seqlens, num_seqs, total_tokens, hq, hkv, scale, tau, out,
+                                       lse, tile_off, st, num_sms, &qmap, &kmap, &vmap, stream));
+}
+
+nsa_status_t nsa_sel_select_topk(const float* scores, const int32_t* cu_seqlens, int num_seqs,
+                                 int total_tokens, int hkv, int nb_stride, int block_size,
+                                 int topk, int init_blocks, int local_blocks, int32_t* block_idx,
+                                 void* workspace, size_t workspace_bytes, nsa_stream_t stream_) {
+    if (total_tokens < 0 || num_seqs < 1 || hkv < 1 || nb_stride < 1 || block_size < 1 ||
+        topk < 1 || init_blocks < 0 || local_blocks < 0)
+        return NSA_ERR_INVALID_ARG;
+    if (topk > kMaxTopk || nb_stride > 1024 || total_tokens >= (1 << 25) ||
+        (long long)total_tokens * hkv * nb_stride >= (1ll << 40))
+        return NSA_ERR_UNSUPPORTED;
+    if (!cu_seqlens || !workspace || (total_tokens > 0 && (!scores || !block_idx)))
+        return NSA_ERR_INVALID_ARG;
+    if (!aligned(cu_seqlens, 4) || !aligned(scores, 4) || !aligned(block_idx, 4) ||
+        !aligned(workspace, 256))
+        return NSA_ERR_INVALID_ARG;
+    if (workspace_bytes < sizeof(DevStatus)) return NSA_ERR_WORKSPACE;
+    int num_sms = 0;
+    nsa_status_t s = check_device(&num_sms);
+    if (s != NSA_OK) return s;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    DevStatus* st = static_cast<DevStatus*>(workspace);
+    if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    return cuda_status(launch_select_topk(scores, cu_seqlens, num_seqs, total_tokens, hkv, nb_stride,
+                                          block_size, topk, init_blocks, local_blocks, block_idx,
+                                          st, stream));
 }
 
 nsa_status_t nsa_sel_check_status(const void* workspace, nsa_stream_t stream_) {

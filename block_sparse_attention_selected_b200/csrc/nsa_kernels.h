@@ -157,6 +157,33 @@ cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq,
                                 cudaStream_t stream);
 cudaError_t launch_bwd_dkdv_reduce(const BwdPlan& p, void* dk, void* dv, cudaStream_t stream);
 
+// Block-selection step (select.cu): cu_cmp[nseq + 1] and the mean-pooled compressed
+// K and V ([floor(T / stride) rows room, hkv, 128]); the top-k of the block scores
+// ([T, hkv, nb_stride] fp32) into block_idx [T, hkv, topk].
+cudaError_t launch_compress_kv(const void* k, const void* v, const int32_t* cu, int nseq, int T,
+                               int hkv, int ksize, int stride, int f16, int32_t* cu_cmp, void* kc,
+                               void* vc, cudaStream_t stream);
+// Block scores from attention over the compressed keys (kernel 32, stride 16):
+// scores [T, hkv, nb_stride] fp32; tile_off [nseq + 1] scratch; qmap over Q [T, hq, 128]
+// with box (64 columns, G heads, 128 / G tokens), kcmap over k_cmp [kc_rows, hkv, 128]
+// with box (64 columns, 1 head, 64 rows), both 128-byte swizzled.
+cudaError_t launch_cmp_scores(const void* q, const void* kc, long long kc_rows, const int32_t* cu,
+                              const int32_t* cu_cmp, int nseq, int T, int hq, int hkv,
+                              int nb_stride, int bs, float scale, float* scores,
+                              int32_t* tile_off, DevStatus* st, int num_sms,
+                              const CUtensorMap* qmap, const CUtensorMap* kcmap,
+                              cudaStream_t stream);
+// Threshold-pruned block attention (bsfa.cu): out bf16 [T, hq, 128], lse [hq, T] (or
+// null); tau fp32 [hq]; qmap as for the block scores, kmap / vmap as for the forward.
+cudaError_t launch_bsfa_fwd(const int32_t* cu, int nseq, int T, int hq, int hkv, float scale,
+                            const float* tau, void* out, float* lse, int32_t* tile_off,
+                            DevStatus* st, int num_sms, const CUtensorMap* qmap,
+                            const CUtensorMap* kmap, const CUtensorMap* vmap,
+                            cudaStream_t stream);
+cudaError_t launch_select_topk(const float* scores, const int32_t* cu, int nseq, int T, int hkv,
+                               int nb_stride, int bs, int topk, int init_blocks, int local_blocks,
+                               int32_t* bidx, DevStatus* st, cudaStream_t stream);
+
 cudaError_t launch_validate(const int32_t* cu, int nseq, int T, int hkv, const int32_t* bidx,
                             int topk, int bs, DevStatus* st, cudaStream_t stream);
 

@@ -226,6 +226,88 @@ NSA_API nsa_status_t nsa_sel_validate_indices(const int32_t *cu_seqlens, int num
                                       long long *n_duplicates, void *workspace,
                                       size_t workspace_bytes, nsa_stream_t stream);
 
+/* Block-selection step, the stage that produces block_idx: compression, block scores
+ * from attention over the compressed keys, top-k.
+ * The quick start of the "Relaxed-System-Lab/Flash-Sparse-Attention" project page
+ * sets kernel_size 32, kernel_stride 16, init_blocks 1, local_blocks 2; the pages
+ * print no formula, so compressed keys / values are the means of the covered rows
+ * and the top-k breaks score ties toward the lower block.
+ *
+ * nsa_sel_compress_kv: for each sequence s (length L_s), compressed block c covers
+ * its tokens [c * kernel_stride, c * kernel_stride + kernel_size); there are
+ * floor((L_s - kernel_size) / kernel_stride) + 1 of them (0 if L_s < kernel_size).
+ *   k, v      bf16 (fp16 with flags = NSA_F16) [total_tokens, hkv, head_dim]
+ *   k_cmp, v_cmp  same type, [floor(total_tokens / kernel_stride), hkv, head_dim] room;
+ *             block c of sequence s at row cu_cmp[s] + c (written): the mean of the
+ *             covered rows, accumulated in fp32
+ *   cu_cmp    int32 [num_seqs + 1] (written on the device): exclusive prefix sums of
+ *             the per-sequence block counts
+ * Requires kernel_stride <= kernel_size <= 4096 and head_dim 128; other flag bits
+ * return NSA_ERR_INVALID_ARG. */
+NSA_API nsa_status_t nsa_sel_compress_kv(const void *k, const void *v, const int32_t *cu_seqlens,
+                                         int num_seqs, int total_tokens, int hkv, int head_dim,
+                                         int kernel_size, int kernel_stride, unsigned flags,
+                                         void *k_cmp, void *v_cmp, int32_t *cu_cmp,
+                                         nsa_stream_t stream);
+
+/* nsa_sel_block_scores: the scores of the selection blocks from attention over the
+ * compressed keys (kernel_size 32, kernel_stride 16 only).  The token at local
+ * position i sees compressed block c when c * 16 + 31 <= i; its probabilities are the
+ * softmax of scale * q . k_cmp[c] over those blocks (none seen: all 0).  The score of
+ * selection block b for (token, KV head g) is the sum, over the G = hq / hkv query
+ * heads of g and over the compressed blocks whose span meets block b, of those
+ * probabilities.
+ *   q          bf16 [total_tokens, hq, head_dim], head_dim 128, G dividing 32
+ *   k_cmp      bf16 [k_cmp_rows, hkv, head_dim] and cu_cmp int32 [num_seqs + 1], as
+ *              nsa_sel_compress_kv wrote them (k_cmp_rows = its room)
+ *   scores     fp32 [total_tokens, hkv, nb_stride] (written for blocks
+ *              b < nb_stride up to the block of the row's own token; later entries of
+ *              a row are left as they were)
+ *   block_size 64 or 128; workspace of nsa_sel_block_scores_workspace_size(num_seqs)
+ *   bytes, 256-byte aligned (its status block is read by nsa_sel_check_status). */
+NSA_API size_t nsa_sel_block_scores_workspace_size(int num_seqs);
+NSA_API nsa_status_t nsa_sel_block_scores(const void *q, const void *k_cmp, int k_cmp_rows,
+                                          const int32_t *cu_seqlens, const int32_t *cu_cmp,
+                                          int num_seqs, int total_tokens, int hq, int hkv,
+                                          int head_dim, int block_size, int kernel_size,
+                                          int kernel_stride, float scale, int nb_stride,
+                                          float *scores, void *workspace, size_t workspace_bytes,
+                                          nsa_stream_t stream);
+
+/* nsa_sel_select_topk: block_idx row of (token at local position i, KV head g), with
+ * qb = i / block_size: blocks 0 .. init_blocks - 1, then qb, qb - 1, .. (local_blocks
+ * of them), each within [0, qb] and listed once, then the other blocks b <= qb in
+ * descending scores[t, g, b] (ties: the lower block first), at most topk in all, the
+ * rest -1.
+ *   scores     fp32 [total_tokens, hkv, nb_stride], finite; nb_stride >= the largest
+ *              qb + 1 (a row whose qb does not fit records NSA_ERR_INVALID_ARG in the
+ *              status block and is written as -1), nb_stride <= 1024
+ *   block_idx  int32 [total_tokens, hkv, topk] (written), 1 <= topk <= 64
+ *   workspace  at least 256 bytes, 256-byte aligned: its status block is cleared and
+ *              then read by nsa_sel_check_status. */
+NSA_API nsa_status_t nsa_sel_select_topk(const float *scores, const int32_t *cu_seqlens,
+                                         int num_seqs, int total_tokens, int hkv, int nb_stride,
+                                         int block_size, int topk, int init_blocks,
+                                         int local_blocks, int32_t *block_idx, void *workspace,
+                                         size_t workspace_bytes, nsa_stream_t stream);
+
+/* Threshold-pruned block attention (BSFA; the "Block Sparse Flash Attention" news
+ * pages): every score is exact; key block b (64 keys of the token's sequence) is kept
+ * for row (token at local position i, query head h) iff
+ * max_{j in b, j <= i} scale * q . k_j >= tau[h]; the output is softmax attention
+ * over the keys of the kept blocks only (no kept block: out = 0, lse = -inf).
+ *   q bf16 [total_tokens, hq, 128]; k, v bf16 [total_tokens, hkv, 128]
+ *   tau   fp32 [hq] device array of thresholds (natural units of scale * q . k)
+ *   out   bf16 [total_tokens, hq, 128] (written); lse fp32 [hq, total_tokens] or null
+ *   block_size 64; hq / hkv must divide 128; workspace of
+ *   nsa_sel_bsfa_workspace_size(num_seqs) bytes, 256-byte aligned. */
+NSA_API size_t nsa_sel_bsfa_workspace_size(int num_seqs);
+NSA_API nsa_status_t nsa_sel_bsfa_fwd(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens, int num_seqs, int total_tokens,
+                                  int hq, int hkv, int head_dim, int block_size, float scale,
+                                  const float *tau, void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, nsa_stream_t stream);
+
 /* Synchronises `stream` and returns the device-side status of the last call that
  * used this workspace (NSA_OK, NSA_ERR_TIMEOUT or NSA_ERR_BAD_INDEX). */
 NSA_API nsa_status_t nsa_sel_check_status(const void *workspace, nsa_stream_t stream);

@@ -130,6 +130,58 @@ def test_option_flags_checked_on_the_host(lib):
     assert nsa.NSA_BWD_REUSE_INDEX == 1 and nsa.NSA_F16 == 2
 
 
+def test_selection_entry_points_check_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)           # never dereferenced: the checks come first
+    # compress: a kernel shorter than its stride, a head dim other than 128, a bad flag
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 128, 8, 16, 0, fake, fake, fake,
+                                   None) == 1
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 64, 32, 16, 0, fake, fake, fake,
+                                   None) == 2
+    assert lib.nsa_sel_compress_kv(fake, fake, fake, 1, 64, 2, 128, 32, 16, 4, fake, fake, fake,
+                                   None) == 1
+    # top-k: topk 0, more than 64 slots, score rows over 1024 blocks, a short workspace
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 0, 1, 2, fake, fake, 1 << 20,
+                                   None) == 1
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 65, 1, 2, fake, fake, 1 << 20,
+                                   None) == 2
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 1025, 64, 16, 1, 2, fake, fake, 1 << 20,
+                                   None) == 2
+    assert lib.nsa_sel_select_topk(fake, fake, 1, 64, 2, 8, 64, 16, 1, 2, fake, fake, 128,
+                                   None) == 3
+
+
+def test_block_scores_entry_point_checks_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    F = ctypes.c_float
+    ws = lib.nsa_sel_block_scores_workspace_size(3)
+    assert ws >= 256 + 16 and lib.nsa_sel_block_scores_workspace_size(0) == 0
+    args = lambda hq, hkv, bs, ksz, kst, rows, wsb: (fake, fake, rows, fake, fake, 3, 256, hq, hkv,
+                                                     128, bs, ksz, kst, F(0.1), 8, fake, fake, wsb,
+                                                     None)
+    assert lib.nsa_sel_block_scores(*args(12, 4, 64, 32, 16, 16, ws)) == 2   # group 3
+    assert lib.nsa_sel_block_scores(*args(128, 2, 64, 32, 16, 16, ws)) == 2  # group 64 > 32
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 16, 16, 16, ws)) == 2    # other geometry
+    assert lib.nsa_sel_block_scores(*args(8, 2, 32, 32, 16, 16, ws)) == 2    # block 32
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 32, 16, 0, ws)) == 1     # no compressed rows
+    assert lib.nsa_sel_block_scores(*args(8, 2, 64, 32, 16, 16, 100)) == 3   # short workspace
+
+
+def test_bsfa_entry_point_checks_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    F = ctypes.c_float
+    ws = lib.nsa_sel_bsfa_workspace_size(2)
+    a = lambda hq, hkv, d, bs, wsb: (fake, fake, fake, fake, 2, 256, hq, hkv, d, bs, F(0.1), fake,
+                                     fake, fake, fake, wsb, None)
+    assert lib.nsa_sel_bsfa_fwd(*a(12, 4, 128, 64, ws)) == 2      # group 3
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 64, 64, ws)) == 2        # head dim 64
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 128, 128, ws)) == 2      # block 128
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 3, 128, 64, ws)) == 1       # hq % hkv
+    assert lib.nsa_sel_bsfa_fwd(*a(8, 2, 128, 64, 64)) == 3       # short workspace
+
+
 def test_binding_rejects_other_element_types():
     import torch
     x = torch.zeros((4, 2, 128), dtype=torch.float32)
