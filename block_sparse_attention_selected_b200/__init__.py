@@ -215,10 +215,11 @@ def nsa_sel_attn_fwd(q, k, v, cu_seqlens, block_idx, block_size, scale=None, out
         _need(lse, "lse", torch.float32, 2, dev)
     nbytes = nsa_sel_attn_workspace_size(T, nseq, hq, hkv, d, topk, block_size, False)
     ws = workspace if workspace is not None else get_workspace(nbytes, dev)
-    _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd_ex(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, _ptr(block_idx), topk,
-        block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev), flag,
-        int(window_size), None, 0, None))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_attn_fwd", load_library().nsa_sel_attn_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, _ptr(block_idx), topk,
+            block_size, scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev), flag,
+            int(window_size), None, 0, None))
     return out, lse
 
 
@@ -250,11 +251,12 @@ def nsa_sel_attn_bwd(q, k, v, out, lse, dout, cu_seqlens, block_idx, block_size,
     if reuse_index and workspace is None:
         raise ValueError("reuse_index needs the workspace the forward used")
     ws = workspace if workspace is not None else get_workspace(nbytes, dev)
-    _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd_ex(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
-        hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(ws), ws.numel(), _stream(dev), (NSA_BWD_REUSE_INDEX if reuse_index else 0) | flag,
-        int(window_size), None, 0, None))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_attn_bwd", load_library().nsa_sel_attn_bwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(cu_seqlens), nseq, T,
+            hq, hkv, d, _ptr(block_idx), topk, block_size, scale, _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(ws), ws.numel(), _stream(dev), (NSA_BWD_REUSE_INDEX if reuse_index else 0) | flag,
+            int(window_size), None, 0, None))
     return dq, dk, dv
 
 
@@ -270,9 +272,10 @@ def nsa_sel_invert_index(cu_seqlens, block_idx, block_size, workspace=None):
     offsets = torch.empty(hkv * (T // block_size + nseq) + 1, dtype=torch.int32, device=dev)
     entries = torch.empty(max(T * hkv * topk, 1), dtype=torch.int32, device=dev)
     counts = torch.zeros(2, dtype=torch.int32, device=dev)
-    _check("nsa_sel_invert_index", load_library().nsa_sel_invert_index(
-        _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
-        _ptr(entries), _ptr(counts), _ptr(ws), ws.numel(), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_invert_index", load_library().nsa_sel_invert_index(
+            _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
+            _ptr(entries), _ptr(counts), _ptr(ws), ws.numel(), _stream(dev)))
     nb, n = (int(x) for x in counts.tolist())
     return offsets[:hkv * nb + 1], entries[:n]
 
@@ -294,9 +297,10 @@ def nsa_sel_invert_index_noalloc(cu_seqlens, block_idx, block_size):
     offsets = torch.empty(hkv * (T // block_size + nseq) + 1, dtype=torch.int32, device=dev)
     entries = torch.empty(max(T * hkv * topk, 1), dtype=torch.int32, device=dev)
     counts = torch.zeros(2, dtype=torch.int32, device=dev)
-    _check("nsa_sel_invert_index_noalloc", load_library().nsa_sel_invert_index_noalloc(
-        _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
-        _ptr(entries), _ptr(counts), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_invert_index_noalloc", load_library().nsa_sel_invert_index_noalloc(
+            _ptr(cu_seqlens), nseq, T, hkv, _ptr(block_idx), topk, block_size, _ptr(offsets),
+            _ptr(entries), _ptr(counts), _stream(dev)))
     nb, n = (int(x) for x in counts.tolist())
     return offsets[:hkv * nb + 1], entries[:n]
 
@@ -309,9 +313,10 @@ def nsa_sel_validate_indices(cu_seqlens, block_idx, block_size, workspace=None):
     T, hkv, topk = block_idx.shape
     ws = workspace if workspace is not None else get_workspace(256, dev)
     a, b = ctypes.c_longlong(0), ctypes.c_longlong(0)
-    code = load_library().nsa_sel_validate_indices(
-        _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, _ptr(block_idx), topk, block_size,
-        ctypes.byref(a), ctypes.byref(b), _ptr(ws), ws.numel(), _stream(dev))
+    with torch.cuda.device(dev):
+        code = load_library().nsa_sel_validate_indices(
+            _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, _ptr(block_idx), topk, block_size,
+            ctypes.byref(a), ctypes.byref(b), _ptr(ws), ws.numel(), _stream(dev))
     if code not in (0, 6):
         raise NsaError("nsa_sel_validate_indices", code)
     return int(a.value), int(b.value)
@@ -334,9 +339,10 @@ def nsa_sel_compress_kv(k, v, cu_seqlens, kernel_size=32, kernel_stride=16):
     kc = torch.empty((rows, hkv, d), dtype=et, device=dev)
     vc = torch.empty((rows, hkv, d), dtype=et, device=dev)
     cu_cmp = torch.empty(nseq + 1, dtype=torch.int32, device=dev)
-    _check("nsa_sel_compress_kv", load_library().nsa_sel_compress_kv(
-        _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hkv, d, kernel_size, kernel_stride, flag,
-        _ptr(kc), _ptr(vc), _ptr(cu_cmp), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_compress_kv", load_library().nsa_sel_compress_kv(
+            _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hkv, d, kernel_size, kernel_stride, flag,
+            _ptr(kc), _ptr(vc), _ptr(cu_cmp), _stream(dev)))
     return kc, vc, cu_cmp
 
 
@@ -357,10 +363,11 @@ def nsa_sel_block_scores(q, k_cmp, cu_seqlens, cu_cmp, block_size, nb_stride, sc
     nbytes = int(lib.nsa_sel_block_scores_workspace_size(nseq))
     ws = workspace if workspace is not None else get_workspace(nbytes, dev)
     scores = torch.empty((T, hkv, nb_stride), dtype=torch.float32, device=dev)
-    _check("nsa_sel_block_scores", lib.nsa_sel_block_scores(
-        _ptr(q), _ptr(k_cmp), rows, _ptr(cu_seqlens), _ptr(cu_cmp), nseq, T, hq, hkv, d,
-        block_size, kernel_size, kernel_stride, scale, nb_stride, _ptr(scores), _ptr(ws),
-        ws.numel(), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_block_scores", lib.nsa_sel_block_scores(
+            _ptr(q), _ptr(k_cmp), rows, _ptr(cu_seqlens), _ptr(cu_cmp), nseq, T, hq, hkv, d,
+            block_size, kernel_size, kernel_stride, scale, nb_stride, _ptr(scores), _ptr(ws),
+            ws.numel(), _stream(dev)))
     return scores
 
 
@@ -394,9 +401,10 @@ def nsa_sel_bsfa_fwd(q, k, v, cu_seqlens, tau, scale=None, block_size=64, worksp
     ws = workspace if workspace is not None else get_workspace(int(lib.nsa_sel_bsfa_workspace_size(nseq)), dev)
     out = torch.empty_like(q)
     lse = torch.empty((hq, T), dtype=torch.float32, device=dev)
-    _check("nsa_sel_bsfa_fwd", lib.nsa_sel_bsfa_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, block_size, scale,
-        _ptr(tau), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_bsfa_fwd", lib.nsa_sel_bsfa_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, hq, hkv, d, block_size, scale,
+            _ptr(tau), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(dev)))
     return out, lse
 
 
@@ -409,9 +417,10 @@ def nsa_sel_select_topk(scores, cu_seqlens, block_size, topk, init_blocks=1, loc
     T, hkv, nb = scores.shape
     out = torch.empty((T, hkv, topk), dtype=torch.int32, device=dev)
     ws = workspace if workspace is not None else get_workspace(256, dev)
-    _check("nsa_sel_select_topk", load_library().nsa_sel_select_topk(
-        _ptr(scores), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, nb, block_size, topk,
-        init_blocks, local_blocks, _ptr(out), _ptr(ws), ws.numel(), _stream(dev)))
+    with torch.cuda.device(dev):
+        _check("nsa_sel_select_topk", load_library().nsa_sel_select_topk(
+            _ptr(scores), _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, hkv, nb, block_size, topk,
+            init_blocks, local_blocks, _ptr(out), _ptr(ws), ws.numel(), _stream(dev)))
     return out
 
 
@@ -422,7 +431,8 @@ def nsa_sel_check_status(workspace=None, device=None) -> int:
     ws = workspace if workspace is not None else _ws_cache.get(_ws_key(dev))
     if ws is None:
         return NSA_OK
-    return int(load_library().nsa_sel_check_status(_ptr(ws), _stream(ws.device)))
+    with torch.cuda.device(ws.device):
+        return int(load_library().nsa_sel_check_status(_ptr(ws), _stream(ws.device)))
 
 
 class SelectedAttention(torch.autograd.Function):

@@ -34,6 +34,7 @@ struct Dims {
 
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
+    size_t inv_end;   // end of the regions the index inversion (InvertPlan) uses
     size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket, uorder;
     size_t total;
@@ -89,6 +90,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.offsets = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.tile_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.chunk_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
+    L.inv_end = o;   // everything the inversion alone touches lies below this offset
     const size_t wrows = (size_t)D.hkv * D.nwin;
     L.win_rng = take(sizeof(int2) * wrows * (size_t)D.nb_stride);
     L.wtile_off = take(sizeof(int32_t) * wrows * ((size_t)D.nb_stride + 1));
@@ -115,9 +117,18 @@ Layout make_layout(const Dims& D, bool bwd) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-nsa_status_t check_device(int* num_sms) {
+// The current device must be an sm_100 part, and `stream` (when it is not one of the
+// default-stream handles) must belong to it: the launches, the scratch of the
+// no-allocation entry point and the SM count are all taken from the current device.
+nsa_status_t check_device(int* num_sms, nsa_stream_t stream_) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_NO_DEVICE;
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (stream != nullptr && stream != cudaStreamLegacy && stream != cudaStreamPerThread) {
+        int sdev = -1;
+        if (cudaStreamGetDevice(stream, &sdev) != cudaSuccess) return NSA_ERR_INVALID_ARG;
+        if (sdev != dev) return NSA_ERR_INVALID_ARG;
+    }
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
@@ -321,7 +332,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
         return NSA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !(scale < 1e30f) || swin < 0) return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
-    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    if ((s = check_device(&num_sms, stream_)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     const Layout L = make_layout(D, false);
     Carved c = carve(D, L, workspace, cu_seqlens, block_idx, swin);
@@ -426,7 +437,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
         return NSA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || !(scale < 1e30f) || swin < 0) return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
-    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    if ((s = check_device(&num_sms, stream_)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     const Layout L = make_layout(D, true);
     Carved c = carve(D, L, workspace, cu_seqlens, block_idx, swin);
@@ -593,7 +604,7 @@ nsa_status_t nsa_sel_invert_index(const int32_t* cu_seqlens, int num_seqs, int t
         !aligned(counts, 4))
         return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
-    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    if ((s = check_device(&num_sms, stream_)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     const Layout L = make_layout(D, false);
     Carved c = carve(D, L, workspace, cu_seqlens, block_idx);
@@ -632,7 +643,7 @@ nsa_status_t nsa_sel_validate_indices(const int32_t* cu_seqlens, int num_seqs, i
         return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
     nsa_status_t s;
-    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    if ((s = check_device(&num_sms, stream_)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* st = static_cast<DevStatus*>(workspace);
     if (cudaMemsetAsync(st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
@@ -664,7 +675,7 @@ nsa_status_t nsa_sel_compress_kv(const void* k, const void* v, const int32_t* cu
         !aligned(k_cmp, 16) || !aligned(v_cmp, 16))
         return NSA_ERR_INVALID_ARG;
     int num_sms = 0;
-    nsa_status_t s = check_device(&num_sms);
+    nsa_status_t s = check_device(&num_sms, stream_);
     if (s != NSA_OK) return s;
     return cuda_status(launch_compress_kv(k, v, cu_seqlens, num_seqs, total_tokens, hkv, kernel_size,
                                           kernel_stride, (flags & NSA_F16) ? 1 : 0, cu_cmp, k_cmp,
@@ -697,7 +708,7 @@ nsa_status_t nsa_sel_block_scores(const void* q, const void* k_cmp, int k_cmp_ro
         return NSA_ERR_INVALID_ARG;
     if (workspace_bytes < nsa_sel_block_scores_workspace_size(num_seqs)) return NSA_ERR_WORKSPACE;
     int num_sms = 0;
-    nsa_status_t s = check_device(&num_sms);
+    nsa_status_t s = check_device(&num_sms, stream_);
     if (s != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* st = static_cast<DevStatus*>(workspace);
@@ -734,7 +745,7 @@ nsa_status_t nsa_sel_bsfa_fwd(const void* q, const void* k, const void* v, const
         return NSA_ERR_INVALID_ARG;
     if (workspace_bytes < nsa_sel_bsfa_workspace_size(num_seqs)) return NSA_ERR_WORKSPACE;
     int num_sms = 0;
-    nsa_status_t s = check_device(&num_sms);
+    nsa_status_t s = check_device(&num_sms, stream_);
     if (s != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* st = static_cast<DevStatus*>(workspace);
@@ -768,7 +779,7 @@ nsa_status_t nsa_sel_select_topk(const float* scores, const int32_t* cu_seqlens,
         return NSA_ERR_INVALID_ARG;
     if (workspace_bytes < sizeof(DevStatus)) return NSA_ERR_WORKSPACE;
     int num_sms = 0;
-    nsa_status_t s = check_device(&num_sms);
+    nsa_status_t s = check_device(&num_sms, stream_);
     if (s != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     DevStatus* st = static_cast<DevStatus*>(workspace);
@@ -816,20 +827,59 @@ __device__ __align__(256) unsigned char g_invert_scratch[kInvertScratchBytes];
 
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_address[kMaxScratchDevices] = {};
+struct ScratchSlot {
+    unsigned long long ctx_id;   // the context the address was resolved in (0: none yet)
+    void* ptr;
+};
+ScratchSlot g_scratch[kMaxScratchDevices] = {};
 
-// Device address of this device's scratch array (resolved once per device).
+// Driver-API context identity (through the runtime's entry-point query, so that the
+// library links no driver library): a device's primary context that was torn down and
+// created again gets a new id, and the module (with its array) is loaded anew.
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+bool current_context_id(unsigned long long* id) {
+    static std::once_flag once;
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    std::call_once(once, [] {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<PfnCtxGetCurrent>(a);
+            get_id = reinterpret_cast<PfnCtxGetId>(b);
+        }
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the current device's scratch array.  It is resolved with
+// cudaGetSymbolAddress once per device and context, and looked up again only if that
+// context was replaced (or its identity cannot be read).
 nsa_status_t scratch_for_current_device(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return NSA_ERR_NO_DEVICE;
     if (dev < 0 || dev >= kMaxScratchDevices) return NSA_ERR_UNSUPPORTED;
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id) && id != 0;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_address[dev]) {
+    ScratchSlot& slot = g_scratch[dev];
+    if (!have_id || slot.ctx_id != id || !slot.ptr) {
+        // first use on this device (or in a new context): the lookup also makes the
+        // device's primary context current if nothing did before
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_invert_scratch) != cudaSuccess || !ptr) return NSA_ERR_CUDA;
-        g_scratch_address[dev] = ptr;
+        unsigned long long id2 = 0;
+        slot.ptr = ptr;
+        slot.ctx_id = (current_context_id(&id2) && id2 != 0) ? id2 : 0;
     }
-    *out = g_scratch_address[dev];
+    *out = slot.ptr;
     return NSA_OK;
 }
 
@@ -854,9 +904,9 @@ nsa_status_t nsa_sel_invert_index_noalloc(const int32_t* cu_seqlens, int num_seq
         !aligned(entries, 4) || !aligned(counts, 4))
         return NSA_ERR_INVALID_ARG;
     const Layout L = make_layout(D, false);
-    if (L.win_rng > kInvertScratchBytes) return NSA_ERR_WORKSPACE;   // too large for the array
+    if (L.inv_end > kInvertScratchBytes) return NSA_ERR_WORKSPACE;   // too large for the array
     int num_sms = 0;
-    if ((s = check_device(&num_sms)) != NSA_OK) return s;
+    if ((s = check_device(&num_sms, stream_)) != NSA_OK) return s;
     void* scratch = nullptr;
     if ((s = scratch_for_current_device(&scratch)) != NSA_OK) return s;
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

@@ -7,7 +7,7 @@ import torch
 import nsa_inputs as ni
 
 # Tolerances for the bf16 path against the fp64 oracle.
-TOL_O = 1e-2        # max |O_gpu - O_ref| beyond the bf16 quantisation of O_ref itself
+TOL_O = 1e-2        # max |O_gpu - O_ref| (beyond half a bf16 ulp of O_ref where |O_ref| >= 2)
 TOL_LSE = 1e-3      # max |LSE_gpu - LSE_ref|
 TOL_GRAD = 2e-2     # ||g_gpu - g_ref||_F / ||g_ref||_F for dQ, dK, dV
 
@@ -59,12 +59,39 @@ def bf16_half_ulp(x):
     return np.where(x > 0, np.exp2(e - 8), 0.0)
 
 
-def o_excess(o_gpu, o_ref):
-    """max over elements of |O_gpu - O_ref| - half_ulp_bf16(O_ref): the kernel's error
-    beyond the unavoidable rounding of the exact answer to the bf16 output format."""
+# Below this magnitude of the exact answer a correctly rounded bf16 O is within 1e-2
+# (half an ulp is at most 2^-8 = 0.0039 there), so the plain bound applies; from 2 up
+# the rounding alone approaches or exceeds the budget (half an ulp is 0.0078 in
+# [2, 4) and 0.0156 from 4 on) and the error beyond that rounding is gated instead.
+O_PLAIN_BELOW = 2.0
+
+# worst values seen in this process, printed at the end of the pytest run
+O_RECORD = {"raw": 0.0, "gate": 0.0, "n": 0}
+
+
+def o_errors(o_gpu, o_ref):
+    """(raw, gate): raw = max |O_gpu - O_ref| over every element; gate = the larger of
+    max |O_gpu - O_ref| over elements with |O_ref| < 2 and max (|O_gpu - O_ref| -
+    half_ulp_bf16(O_ref)) over elements with |O_ref| >= 2.  The parity bound is
+    gate <= 1e-2."""
     a = np.asarray(o_gpu, dtype=np.float64)
     b = np.asarray(o_ref, dtype=np.float64)
-    return float((np.abs(a - b) - bf16_half_ulp(b)).max()) if a.size else 0.0
+    if a.size == 0:
+        return 0.0, 0.0
+    d = np.abs(a - b)
+    small = np.abs(b) < O_PLAIN_BELOW
+    raw = float(d.max())
+    gate = max(float(d[small].max(initial=0.0)),
+               float((d[~small] - bf16_half_ulp(b[~small])).max(initial=0.0)))
+    O_RECORD["raw"] = max(O_RECORD["raw"], raw)
+    O_RECORD["gate"] = max(O_RECORD["gate"], gate)
+    O_RECORD["n"] += a.size
+    return raw, gate
+
+
+def o_gate(o_gpu, o_ref):
+    """The gated O error (see o_errors)."""
+    return o_errors(o_gpu, o_ref)[1]
 
 
 def rel_fro(a, b):

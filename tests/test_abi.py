@@ -225,3 +225,36 @@ def test_cached_workspace_is_per_stream(monkeypatch):
     current["s"] = 22
     assert nsa.get_workspace(10, dev) is b
     nsa.release_workspaces()
+
+
+def test_binding_makes_the_tensors_device_current():
+    """Every call into the library runs with the tensors' device current: the C side
+    launches on, and takes the no-allocation scratch of, the current device, and
+    rejects a stream of another device."""
+    import ast
+    import inspect
+    tree = ast.parse(inspect.getsource(nsa))
+    calls = 0
+
+    def guarded(node, parents):
+        for p in parents:
+            if isinstance(p, ast.With) and any(
+                    isinstance(it.context_expr, ast.Call) and
+                    ast.unparse(it.context_expr.func) == "torch.cuda.device" for it in p.items):
+                return True
+        return False
+
+    def visit(node, parents):
+        nonlocal calls
+        if isinstance(node, ast.Call) and isinstance(node.func, ast.Attribute) and \
+                node.func.attr.startswith("nsa_sel_") and \
+                not node.func.attr.endswith(("_size", "_max_bytes", "_string")):
+            base = ast.unparse(node.func.value)
+            if base in ("lib", "load_library()"):
+                calls += 1
+                assert guarded(node, parents), f"{node.func.attr} at line {node.lineno}"
+        for ch in ast.iter_child_nodes(node):
+            visit(ch, parents + [node])
+
+    visit(tree, [])
+    assert calls >= 10

@@ -7,7 +7,7 @@ import torch
 
 import block_sparse_attention_selected_b200 as nsa
 import nsa_inputs as ni
-from gpu_util import TOL_LSE, TOL_O, f64, o_excess
+from gpu_util import TOL_LSE, TOL_O, f64, o_gate
 from oracle import bsfa
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +48,7 @@ def test_bsfa_matches_oracle(lengths, hq, hkv, taus):
     ro, rl, _ = bsfa.bsfa_fwd(p.q, p.k, p.v, p.cu_seqlens, 64, p.scale, tau)
     keep = ~_near_threshold_rows(p, tau)
     o, l = f64(out), f64(lse).T
-    assert o_excess(o[keep], ro[keep]) <= TOL_O
+    assert o_gate(o[keep], ro[keep]) <= TOL_O
     fin = keep & np.isfinite(rl)
     assert np.array_equal(np.isneginf(l[keep]), np.isneginf(rl[keep]))
     assert np.abs(l[fin] - rl[fin]).max(initial=0.0) <= TOL_LSE

@@ -1,13 +1,13 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
-Small problems are compared element by element over every output; the workloads
-at their full sizes are compared on stratified token / block samples that the
-oracle computes one by one.  Tolerances: |O - O_ref| <= 1e-2 beyond half a bf16 ulp
-of O_ref (the rounding of the exact answer to the bf16 output), <= 1e-3 on fp32 LSE,
-relative Frobenius <= 2e-2 on dQ, dK, dV; the inversion is bit-exact.
+Small problems are compared element by element over every output; so are the
+headline forward and the training shape's forward and backward at their full sizes;
+the other full-size workloads are compared on stratified token samples that the
+oracle computes one by one.  Tolerances: |O - O_ref| <= 1e-2 on every element whose
+exact value has |O_ref| < 2, and beyond half a bf16 ulp of O_ref (the rounding of the
+exact answer to the bf16 output) where |O_ref| >= 2; <= 1e-3 on fp32 LSE; relative
+Frobenius <= 2e-2 on dQ, dK, dV; the inversion is bit-exact.
 """
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -15,8 +15,8 @@ import torch
 import block_sparse_attention_selected_b200 as nsa
 import nsa_inputs as ni
 import oracle
-from gpu_util import (TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, o_excess, rel_fro, sample_tokens,
-                      to_device)
+from gpu_util import (TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, o_errors, o_gate, rel_fro,
+                      sample_tokens, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,8 +62,8 @@ def _check_fwd(p, out, lse, tokens=None):
                               tokens=tokens)
     o = f64(out) if tokens is None else f64(out[torch.from_numpy(tokens).cuda()])
     l = f64(lse).T if tokens is None else f64(lse[:, torch.from_numpy(tokens).cuda()]).T
-    eo, el = o_excess(o, o_ref), max_abs(l, l_ref)
-    assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el, max_abs(o, o_ref))
+    (raw, eo), el = o_errors(o, o_ref), max_abs(l, l_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, (p.name, "gated", eo, "raw", raw, "lse", el)
     return eo, el
 
 
@@ -138,14 +138,13 @@ def test_fwd_small_full_compare(name, spec, perturb):
     _check_fwd(p, out, lse)
 
 
-# Every (group, block) pair of the T=65536 sweep at topk 16, plus the topk ends; all
-# 30 points with NSA_FULL_SWEEP=1.
-_SWEEP = [(g, bs, 16) for g in (1, 2, 4, 8, 16) for bs in (64, 128)] + \
-    [(4, 64, 8), (4, 64, 32), (1, 64, 8), (16, 128, 32)]
-if os.environ.get("NSA_FULL_SWEEP") == "1":
-    _SWEEP = list(ni.SWEEP_POINTS)
+# Every point of the T=65536 sweep (group 1-16, block 64 / 128, topk 8 / 16 / 32).
 FWD_FULL = ["fwd_t32k_hq32_g4_k16", "varlen_64k_32k_g1_k16", "train_t32k_hq64_g8_k16"] + \
-    [f"sweep_t64k_g{g}_bs{bs}_k{k}" for g, bs, k in _SWEEP]
+    [f"sweep_t64k_g{g}_bs{bs}_k{k}" for g, bs, k in ni.SWEEP_POINTS]
+# Compared on every output element (the oracle needs up to ~30 s for each on 16 cores);
+# the other sweep points on stratified token samples.
+FWD_FULL_EVERY_ELEMENT = {ni.HEADLINE, "fwd_t32k_hq32_g4_k16", "varlen_64k_32k_g1_k16",
+                          "train_t32k_hq64_g8_k16"}
 
 
 @pytest.mark.parametrize("bs", [64, 128])
@@ -161,19 +160,21 @@ def test_fwd_large_v_uses_block_exponent(bs):
     # O scales exactly with V (a power of two), LSE does not change: compare O / 2^15
     # with the standard tolerance (bf16 rounding is invariant under that scaling)
     o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale)
-    eo = o_excess(f64(out) / 32768.0, o_ref / 32768.0)
+    eo = o_gate(f64(out) / 32768.0, o_ref / 32768.0)
     el = max_abs(f64(lse).T, l_ref)
     assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
 
 
 @pytest.mark.parametrize("wl", FWD_FULL)
-def test_fwd_full_size_sampled(wl):
+def test_fwd_full_size(wl):
     p = ni.workload(wl, with_dout=False)
     _, out, lse = _fwd(p)
-    toks = sample_tokens(p.cu_seqlens, p.block_size, n_random=96, seed=1)
-    _check_fwd(p, out, lse, tokens=toks)
-    # properties that hold everywhere: finite outputs, LSE >= the LSE of the
-    # structural blocks alone is not checkable cheaply, but finiteness is
+    if wl in FWD_FULL_EVERY_ELEMENT:
+        _check_fwd(p, out, lse)
+    else:
+        toks = sample_tokens(p.cu_seqlens, p.block_size, n_random=96, seed=1)
+        _check_fwd(p, out, lse, tokens=toks)
+    # properties that hold on every element at any size: finite outputs
     assert torch.isfinite(out.float()).all()
     assert torch.isfinite(lse).all()
 
@@ -282,14 +283,21 @@ def test_bwd_medium_multi_unit():
                                               (0, 8128, 64)])
 
 
-def test_bwd_full_size_training_shape_sampled():
+def test_bwd_full_size_training_shape():
+    """The training shape (T = 32768, 64 query heads, 8 KV heads, topk 16): dQ, dK and dV
+    compared with the oracle over the whole tensors (about 100 s of oracle time on 16
+    cores), block 0 -- selected by every token -- included."""
     p = ni.workload("train_t32k_hq64_g8_k16")
     d, out, lse = _fwd(p)
     dq, dk, dv = _bwd(p, d, out, lse)
     assert torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all()
     assert torch.isfinite(dv.float()).all()
-    _check_bwd_sampled(p, dq, dk, dv, blocks=[(3, 64 * 300, 64), (7, 32768 - 64, 64),
-                                              (0, 64 * 20, 64)], n_random=24)
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
+                               p.scale)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    # block 0 of every KV head on its own (the most-reduced keys)
+    e0 = max(rel_fro(f64(dk[:64]), rdk[:64]), rel_fro(f64(dv[:64]), rdv[:64]))
+    assert max(e) <= TOL_GRAD and e0 <= TOL_GRAD, (e, e0)
 
 
 def test_bwd_deterministic():
@@ -412,7 +420,7 @@ def test_window_fwd_bwd_full_compare(name, spec, W, perturb):
     fin = np.isfinite(l_ref)
     assert np.array_equal(np.isfinite(l), fin), name
     assert not o[~fin].any(), name
-    eo, el = o_excess(o, o_ref), max_abs(l[fin], l_ref[fin])
+    eo, el = o_gate(o, o_ref), max_abs(l[fin], l_ref[fin])
     assert eo <= TOL_O and el <= TOL_LSE, (name, eo, el)
     rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
                                p.scale, window=W)
@@ -442,7 +450,7 @@ def test_window_sliding_branch_is_band_attention(bs, W):
 def _check_fwd_window(p, out, lse, W):
     o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
                               window=W)
-    eo, el = o_excess(f64(out), o_ref), max_abs(f64(lse).T, l_ref)
+    eo, el = o_gate(f64(out), o_ref), max_abs(f64(lse).T, l_ref)
     assert eo <= TOL_O and el <= TOL_LSE, (p.name, eo, el)
 
 
