@@ -17,7 +17,9 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libnsa_sel.so")
+# NSA_SEL_LIBRARY=checks loads the bounds-checking build (libnsa_sel_checks.so) instead
+LIB_PATH = os.path.join(_HERE, "libnsa_sel_checks.so" if os.environ.get("NSA_SEL_LIBRARY") == "checks"
+                        else "libnsa_sel.so")
 
 NSA_OK = 0
 STATUS_NAMES = {0: "NSA_OK", 1: "NSA_ERR_INVALID_ARG", 2: "NSA_ERR_UNSUPPORTED",

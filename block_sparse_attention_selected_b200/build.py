@@ -13,7 +13,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnsa_sel.so")
-SOURCES = ["api.cu", "invert.cu", "fwd.cu", "merge.cu", "bwd.cu", "select.cu", "bsfa.cu"]
+# the bounds-checking build (-DNSA_SEL_CHECKS): same ABI, every gathered row and K/V
+# block coordinate checked before its copy (nsa_common.cuh)
+LIB_CHECKS = os.path.join(HERE, "libnsa_sel_checks.so")
+SOURCES = ["api.cu", "invert.cu", "fwd.cu", "dense.cu", "merge.cu", "bwd.cu", "select.cu",
+           "bsfa.cu"]
 HEADERS = ["nsa_common.cuh", "nsa_kernels.h"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -28,26 +32,28 @@ def _nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "nsa_sel.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+def build(force: bool = False, verbose: bool = False, checks: bool = False) -> str:
+    """Builds libnsa_sel.so (checks=True: the bounds-checking libnsa_sel_checks.so)."""
+    lib = LIB_CHECKS if checks else LIB
+    if not force and not _stale(lib):
+        return lib
+    objdir = os.path.join(HERE, "_build_checks" if checks else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     procs = []
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c",
-               os.path.join(CSRC, src), "-o", obj]
+        cmd = [_nvcc(), *NVCC_FLAGS, *(["-DNSA_SEL_CHECKS"] if checks else []), "-I",
+               os.path.join(ROOT, "include"), "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), file=sys.stderr)
@@ -62,12 +68,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for {failed}")
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     subprocess.check_call([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
                            "-o", tmp, *objs])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                checks="--checks" in sys.argv))

@@ -33,7 +33,8 @@ struct Dims {
 };
 
 struct Layout {
-    size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
+    size_t status, blkoff, dtile_off, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off,
+        chunk_off;
     size_t inv_end;   // end of the regions the index inversion (InvertPlan) uses
     size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket, uorder;
@@ -81,6 +82,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
     L.status = take(sizeof(DevStatus));
     L.blkoff = take(sizeof(int32_t) * (D.nseq + 1));
+    L.dtile_off = take(sizeof(int32_t) * (D.nseq + 1));
     L.keys0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.keys1 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.vals0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
@@ -171,14 +173,15 @@ bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs, boo
 
 // Tensor map over a bf16 Q [T, hq, 128]; box = (64 columns, G heads, 128 / G tokens):
 // one 128-row tile of G heads of consecutive tokens, rows token-major, 128-byte swizzle.
-bool make_q_group_map(CUtensorMap* map, const void* base, int T, int hq, int G) {
+bool make_q_group_map(CUtensorMap* map, const void* base, int T, int hq, int G, bool f16 = false) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)hq, (cuuint64_t)(T > 0 ? T : 1)};
     cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)hq * kHeadDim * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kTileRows / G)};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     3, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -229,6 +232,7 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.key_bits = D.key_bits;
     p.sort_tiles = D.sort_tiles;
     p.blkoff = reinterpret_cast<int32_t*>(b + L.blkoff);
+    p.dtile_off = reinterpret_cast<int32_t*>(b + L.dtile_off);
     p.keys[0] = reinterpret_cast<uint32_t*>(b + L.keys0);
     p.keys[1] = reinterpret_cast<uint32_t*>(b + L.keys1);
     p.vals[0] = reinterpret_cast<uint32_t*>(b + L.vals0);
@@ -321,7 +325,8 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
                       int num_seqs, int total_tokens, int hq, int hkv, int head_dim,
                       const int32_t* block_idx, int topk, int block_size, float scale, void* out,
                       float* lse, void* workspace, size_t workspace_bytes, nsa_stream_t stream_,
-                      void* const* events, int num_events, int* launches, bool f16, int swin) {
+                      void* const* events, int num_events, int* launches, bool f16, int swin,
+                      bool test_short_waits = false, bool test_skip_arrive = false) {
     Dims D;
     nsa_status_t s = check_common(cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim,
                                   block_idx, topk, block_size, workspace, workspace_bytes, false, &D);
@@ -340,6 +345,9 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if (launches) *launches = 0;
     pm.mark(0);
     if (cudaMemsetAsync(c.st, 0, sizeof(DevStatus), stream) != cudaSuccess) return NSA_ERR_CUDA;
+    if (test_short_waits &&   // low four bytes 0x01 each: a budget of 0x01010101 cycles
+        cudaMemsetAsync(&c.st->wait_budget, 0x01, 4, stream) != cudaSuccess)
+        return NSA_ERR_CUDA;
     if (total_tokens == 0) {
         for (int i = 1; i < 4; ++i) pm.mark(i);
         return NSA_OK;
@@ -388,6 +396,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.part_meta = reinterpret_cast<float2*>(c.base + L.part_lse);
     fp.st = c.st;
     fp.num_sms = num_sms;
+    fp.test_skip_arrive = test_skip_arrive ? 1 : 0;
     int32_t* vexp = reinterpret_cast<int32_t*>(c.base + L.vexp);
     fp.vexp = vexp;
     if ((s = cuda_status(launch_vblock_exp(fp, v, D.nb_stride, vexp, stream))) != NSA_OK) return s;
@@ -399,20 +408,26 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     pm.add(2);
     pm.mark(2);
 
-    MergePlan mp{};
-    mp.cu = cu_seqlens;
-    mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
-    mp.G = D.G;
-    mp.f16 = f16 ? 1 : 0;
-    mp.swin = swin;
-    mp.bidx = block_idx;
-    mp.posmap = posmap;
-    mp.part_o = fp.part_o;
-    mp.part_meta = fp.part_meta;
-    mp.out = out;
-    mp.lse = lse;
-    mp.st = c.st;
-    if ((s = cuda_status(launch_merge(mp, stream))) != NSA_OK) return s;
+    DensePlan dp{};
+    dp.cu = cu_seqlens;
+    dp.nseq = D.nseq; dp.T = D.T; dp.hq = D.hq; dp.hkv = D.hkv; dp.topk = D.topk; dp.bs = D.bs;
+    dp.G = D.G;
+    dp.tpt = kTileRows / D.G;
+    dp.f16 = f16 ? 1 : 0;
+    dp.swin = swin;
+    dp.scale_log2 = fp.scale_log2;
+    dp.bidx = block_idx;
+    dp.dtile_off = c.inv.dtile_off;
+    dp.posmap = posmap;
+    dp.part_o = fp.part_o;
+    dp.part_meta = fp.part_meta;
+    dp.out = out;
+    dp.lse = lse;
+    dp.st = c.st;
+    dp.num_sms = num_sms;
+    CUtensorMap qmap;
+    if (!make_q_group_map(&qmap, q, D.T, D.hq, D.G, f16)) return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_fwd_dense(dp, &qmap, &kmap, &vmap, stream))) != NSA_OK) return s;
     pm.add(1);
     pm.mark(3);
     return NSA_OK;
@@ -546,10 +561,12 @@ nsa_status_t nsa_sel_attn_fwd_ex(const void* q, const void* k, const void* v,
                                  void* workspace, size_t workspace_bytes, nsa_stream_t stream,
                                  unsigned flags, int window_size, void* const* events,
                                  int num_events, int* num_launches) {
-    if (flags & ~(unsigned)NSA_F16) return NSA_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(NSA_F16 | NSA_TEST_SHORT_WAITS | NSA_TEST_SKIP_ARRIVE))
+        return NSA_ERR_INVALID_ARG;
     return fwd_impl(q, k, v, cu_seqlens, num_seqs, total_tokens, hq, hkv, head_dim, block_idx,
                     topk, block_size, scale, out, lse, workspace, workspace_bytes, stream, events,
-                    num_events, num_launches, (flags & NSA_F16) != 0, window_size);
+                    num_events, num_launches, (flags & NSA_F16) != 0, window_size,
+                    (flags & NSA_TEST_SHORT_WAITS) != 0, (flags & NSA_TEST_SKIP_ARRIVE) != 0);
 }
 
 nsa_status_t nsa_sel_attn_bwd(const void* q, const void* k, const void* v, const void* out,

@@ -225,6 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     long long offA = -1;
                     float lA = 0.f, dA = 0.f;
                     int4 mA = make_int4(-1, 0, 0, -1);
+                    if (kChecks) {   // the gathered row must lie inside q and dout
+                        const bool row_in = ea == 0xFFFFFFFFu ||
+                                            ((int)(ea >> 6) < p.T && (int)(ea & 63u) < p.topk && g < p.hkv);
+                        if (!__all_sync(0xffffffffu, check_ok(row_in, st, 142, i))) {
+                            *abort_flag = 1;
+                            stopped = true;
+                            break;
+                        }
+                    }
                     if (ea != 0xFFFFFFFFu) {
                         mA = make_int4((int)(ea >> 6), g * p.G + rA % p.G, (int)(ea & 63u), (int)(ea >> 6) - d.x);
                         offA = ((long long)mA.x * p.hq + mA.y) * (kHeadDim * 2);
@@ -291,6 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     u0 = u1; b0 = b1; u1 = ld_unit(k + 2); b1 = ld_bucket(k + 2);
                     if (b == prev) continue;
                     prev = b;
+                    if (!check_ok(d.x >= 0 && d.x < p.T && (d.w >> 8) < p.hkv, st, 143, k)) {
+                        *abort_flag = 1;
+                        break;
+                    }
                     if (!wait(&S.kv_empty, (loads & 1) ^ 1, 52)) break;
                     const int g = d.w >> 8;
                     mbar_arrive_expect_tx(&S.kv_full, 4u * BS * 128u);
@@ -400,6 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // last of unit << 1 | first of unit (registers, no local-memory array)
                 int pend0 = 0, pend1 = 0;
                 long long idle_since = clock64();
+                const long long wait_budget =
+                    st->wait_budget > 0 ? st->wait_budget : kWaitBudgetCycles;
                 while (ok && (fk < nk || ri < fi)) {
                     bool go_r = false, go_s = false;
                     const int pend = (ri & 1) ? pend1 : pend0;
@@ -438,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         idle_since = clock64();
                     } else if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
                         ok = false;
-                    } else if (__shfl_sync(0xffffffffu, clock64() - idle_since > kWaitBudgetCycles, 0)) {
+                    } else if (__shfl_sync(0xffffffffu, clock64() - idle_since > wait_budget, 0)) {
                         if (lane == 0) record_error(st, NSA_ERR_TIMEOUT, 56, blockIdx.x);
                         *abort_flag = 1;
                         ok = false;

@@ -223,6 +223,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return reinterpret_cast<unsigned long long>(
                     qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (kHeadDim * 2));
             };
+            // test-only fault injection (NSA_TEST_SKIP_ARRIVE): loader 0 of CTA 0 withholds
+            // its arrival on the first tile's Q barrier; its copies still complete, and no
+            // MMA reads the stage, so the MMA issuer's bounded wait expires with nothing
+            // in flight behind it
+            auto skip_arrive = [&](int tile) {
+                return p.test_skip_arrive && blockIdx.x == 0 && w == 0 && tile == 0;
+            };
             int4 d0 = ld_desc(0), d1 = ld_desc(1);
             uint32_t ea = ld_ent(d0, rA);
             int published = 0, issued = 0;
@@ -231,6 +238,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < n; ++i) {
                 const int4 d = d0;
                 const unsigned long long addrA = row_addr(d, rA, ea);
+                if (kChecks) {   // the gathered row must lie inside q
+                    const bool row_in = !(lane < nr_w && rA < (d.z & 255)) ||
+                                        ((int)(ea >> 6) < p.T && (int)(ea & 63u) < p.topk &&
+                                         (d.z >> 8) < p.hkv);
+                    if (!__all_sync(0xffffffffu, check_ok(row_in, st, 140, i))) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                }
                 d0 = d1;
                 d1 = ld_desc(i + 2);
                 ea = ld_ent(d0, rA);           // next tile's entries, used one iteration later
@@ -252,14 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (i > 0) {
                     cp_async_wait_one_pending();
                     fence_async_smem();
-                    mbar_arrive(&S.q_full[(i - 1) % kNQ]);
+                    if (!skip_arrive(i - 1)) mbar_arrive(&S.q_full[(i - 1) % kNQ]);
                     published = i;
                 }
             }
             cp_async_wait_all();   // nothing may still be in flight when the CTA exits
             if (issued == n && published == n - 1 && n > 0) {
                 fence_async_smem();
-                mbar_arrive(&S.q_full[(n - 1) % kNQ]);
+                if (!skip_arrive(n - 1)) mbar_arrive(&S.q_full[(n - 1) % kNQ]);
             }
         } else if (warp == kTmaWarp) {
             // ------------------------------------------------------------- K/V producer
@@ -276,6 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     d0 = d1; d1 = d2; d2 = ld_desc(i + 3);
                     if (d.w == prev) continue;
                     prev = d.w;
+                    if (!check_ok(d.x >= 0 && d.x < p.T && (d.z >> 8) < p.hkv, st, 141, i)) {
+                        *abort_flag = 1;
+                        break;
+                    }
                     const int stg = uses % NKV;
                     if (!wait(&S.kv_empty[stg], ((uses / NKV) & 1) ^ 1, 32)) break;
                     const int g = d.z >> 8;

@@ -35,7 +35,8 @@ struct DevStatus {
     int ntiles_fwd;    // number of forward tiles in window order
     int pad0;
     unsigned long long index_tag;   // identifies the inputs of the inversion held here
-    int pad[48];
+    long long wait_budget;          // cycles a bounded wait may spin (0: kWaitBudgetCycles)
+    int pad[46];
 };
 static_assert(sizeof(DevStatus) == 256, "status block is 256 bytes");
 
@@ -46,6 +47,23 @@ __device__ __forceinline__ void record_error(DevStatus* st, int code, int where,
         st->aux0 = a0;
         st->aux1 = a1;
     }
+}
+
+// Bounds-checking build (compiled with -DNSA_SEL_CHECKS, libnsa_sel_checks.so): every
+// gathered row and every K/V block coordinate taken from the index inversion is checked
+// before its copy is issued.  A failed check records NSA_ERR_BAD_INDEX (with the
+// kernel's location tag) in the status block and the CTA stops early, like an expired
+// wait: the copy is not issued and nothing traps.
+#ifdef NSA_SEL_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+
+__device__ __forceinline__ bool check_ok(bool cond, DevStatus* st, int where, int a0 = 0) {
+    if (!kChecks || cond) return true;
+    record_error(st, NSA_ERR_BAD_INDEX, where, a0, (int)blockIdx.x);
+    return false;
 }
 
 // ------------------------------------------------------------------ small utilities
@@ -115,19 +133,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  About one second of SM clock
-// at most; on expiry records NSA_ERR_TIMEOUT and returns false.
+// Bounded wait for the phase with the given parity.  By default about one second of
+// SM clock at most (the call's status block may set a shorter budget: the test-only
+// NSA_TEST_SHORT_WAITS option); on expiry records NSA_ERR_TIMEOUT and returns false.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DevStatus* st,
                                           int where) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
+    const long long set = st->wait_budget;
+    const long long budget = set > 0 ? set : kWaitBudgetCycles;
     // a compact loop: this function is inlined at every wait of the warp-specialised
     // kernels, whose code must stay small enough for the instruction caches
 #pragma unroll 1
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - start > kWaitBudgetCycles) {
+        if (clock64() - start > budget) {
             record_error(st, NSA_ERR_TIMEOUT, where, blockIdx.x);
             return false;
         }

@@ -35,6 +35,8 @@ struct InvertPlan {
     int32_t* offsets;        // [nbk_cap + 1]
     int32_t* tile_off;       // [nbk_cap + 1]
     int32_t* chunk_off;      // [nbk_cap + 1]
+    int32_t* dtile_off;      // [nseq + 1]: forward dense tiles (of tokens_per_tile tokens)
+                             // of the sequences before s (k_seq_blocks)
     DevStatus* st;
     unsigned long long tag;  // written to st->index_tag by the inversion
     // result: the sorted values live in vals[final_buf]
@@ -97,6 +99,7 @@ struct FwdPlan {
     const int32_t* vexp;     // [hkv * NB]: exponent e of each (g, B) block's V
     DevStatus* st;
     int num_sms;
+    int test_skip_arrive;    // test-only fault injection (NSA_TEST_SKIP_ARRIVE), 0 normally
 };
 
 // vexp[g * NB + B] = 0, or the exponent that brings max |V_B| under 2^15
@@ -107,21 +110,30 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream);
 
-struct MergePlan {
+// The forward's query-major pass over the init and local blocks, with the merge of
+// the KV-major partials folded in (dense.cu).
+struct DensePlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
-    int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
+    int tpt;                 // tokens per dense tile: 128 / G
+    int f16;                 // 1: q, k, v, out are fp16; 0: bf16
     int swin;                // sliding window in keys (0: none)
+    float scale_log2;        // scale * log2(e)
     const int32_t* bidx;
-    const int32_t* posmap;   // sorted position of each valid (t, g, j) entry
+    const int32_t* dtile_off;   // [nseq + 1] dense tiles before sequence s
+    const int32_t* posmap;   // partial position of each KV-major (t, g, j) entry
     const void* part_o;
     const float2* part_meta;
     void* out;
-    float* lse;
-    const DevStatus* st;
+    float* lse;              // may be null (no LSE stored)
+    DevStatus* st;
+    int num_sms;
 };
 
-cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream);
+// qmap: Q [T, hq, 128] with boxes of 64 columns x G heads x 128 / G tokens (128B swizzle);
+// kmap / vmap as for the tile kernel
+cudaError_t launch_fwd_dense(const DensePlan& p, const CUtensorMap* qmap, const CUtensorMap* kmap,
+                             const CUtensorMap* vmap, cudaStream_t stream);
 
 struct BwdPlan {
     const void* q;

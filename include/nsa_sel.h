@@ -134,9 +134,21 @@ NSA_API nsa_status_t nsa_sel_attn_bwd_profiled(
 /* Option flags of the _ex calls below (OR-ed). */
 #define NSA_BWD_REUSE_INDEX 1u
 #define NSA_F16 2u
+/* Test-only options of nsa_sel_attn_fwd_ex, for the failure-detection tests (no
+ * counterpart in the pages).  NSA_TEST_SHORT_WAITS limits every bounded wait of the
+ * call's kernels to 0x01010101 SM cycles (about 8.6 ms at 1.965 GHz) instead of about
+ * one second.  NSA_TEST_SKIP_ARRIVE makes one Q loader warp of the first CTA of the
+ * tile kernel withhold its arrival on the first tile's Q barrier (its copies still
+ * complete and nothing reads the stage), so that the MMA issuer's wait expires: the
+ * call then records NSA_ERR_TIMEOUT in the status block, every CTA drains its own
+ * copies and tensor-core work and frees its tensor memory, the later kernels of the
+ * call leave out and lse untouched, and the device stays usable. */
+#define NSA_TEST_SHORT_WAITS 0x100u
+#define NSA_TEST_SKIP_ARRIVE 0x200u
 /* The forward with options: flags = NSA_F16 makes q, k, v and out fp16 instead of bf16
- * (same layouts; the partials stay fp16 and all arithmetic fp32, as for bf16).  Other
- * flag bits return NSA_ERR_INVALID_ARG.
+ * (same layouts; the partials stay fp16 and all arithmetic fp32, as for bf16);
+ * NSA_TEST_SHORT_WAITS and NSA_TEST_SKIP_ARRIVE as above.  Other flag bits return
+ * NSA_ERR_INVALID_ARG.
  *   window_size  0: no window.  W > 0: a sliding window of W keys as well: the token at
  *       local position i attends key j only if j lies in a selected block, j <= i and
  *       j > i - W (the window_size of the sliding branch in the quick start of the

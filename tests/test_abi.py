@@ -258,3 +258,14 @@ def test_binding_makes_the_tensors_device_current():
 
     visit(tree, [])
     assert calls >= 10
+
+
+def test_test_only_flags_are_forward_only(lib):
+    """The fault-injection options exist for the forward's failure-detection test only;
+    the backward rejects them on the host, before any device work."""
+    rc = lib.nsa_sel_attn_bwd_ex(*([None] * 7), 1, 0, 1, 1, 128, None, 1, 64, ctypes.c_float(0.1),
+                                 None, None, None, None, 0, None, 0x200, 0, None, 0, None)
+    assert rc == 1   # NSA_ERR_INVALID_ARG
+    rc = lib.nsa_sel_attn_fwd_ex(*([None] * 4), 1, 0, 1, 1, 128, None, 1, 64, ctypes.c_float(0.1),
+                                 None, None, None, 0, None, 0x400, 0, None, 0, None)
+    assert rc == 1   # an unknown bit
