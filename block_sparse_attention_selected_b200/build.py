@@ -16,8 +16,7 @@ LIB = os.path.join(HERE, "libnsa_sel.so")
 # the bounds-checking build (-DNSA_SEL_CHECKS): same ABI, every gathered row and K/V
 # block coordinate checked before its copy (nsa_common.cuh)
 LIB_CHECKS = os.path.join(HERE, "libnsa_sel_checks.so")
-SOURCES = ["api.cu", "invert.cu", "fwd.cu", "dense.cu", "merge.cu", "bwd.cu", "select.cu",
-           "bsfa.cu"]
+SOURCES = ["api.cu", "invert.cu", "fwd.cu", "merge.cu", "bwd.cu", "select.cu", "bsfa.cu"]
 HEADERS = ["nsa_common.cuh", "nsa_kernels.h"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

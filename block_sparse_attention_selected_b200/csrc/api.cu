@@ -33,8 +33,7 @@ struct Dims {
 };
 
 struct Layout {
-    size_t status, blkoff, dtile_off, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off,
-        chunk_off;
+    size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
     size_t inv_end;   // end of the regions the index inversion (InvertPlan) uses
     size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket, uorder;
@@ -82,7 +81,6 @@ Layout make_layout(const Dims& D, bool bwd) {
     auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
     L.status = take(sizeof(DevStatus));
     L.blkoff = take(sizeof(int32_t) * (D.nseq + 1));
-    L.dtile_off = take(sizeof(int32_t) * (D.nseq + 1));
     L.keys0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.keys1 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
     L.vals0 = take(sizeof(uint32_t) * (size_t)std::max<long long>(D.nent, 1));
@@ -232,7 +230,6 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.key_bits = D.key_bits;
     p.sort_tiles = D.sort_tiles;
     p.blkoff = reinterpret_cast<int32_t*>(b + L.blkoff);
-    p.dtile_off = reinterpret_cast<int32_t*>(b + L.dtile_off);
     p.keys[0] = reinterpret_cast<uint32_t*>(b + L.keys0);
     p.keys[1] = reinterpret_cast<uint32_t*>(b + L.keys1);
     p.vals[0] = reinterpret_cast<uint32_t*>(b + L.vals0);
@@ -408,26 +405,20 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     pm.add(2);
     pm.mark(2);
 
-    DensePlan dp{};
-    dp.cu = cu_seqlens;
-    dp.nseq = D.nseq; dp.T = D.T; dp.hq = D.hq; dp.hkv = D.hkv; dp.topk = D.topk; dp.bs = D.bs;
-    dp.G = D.G;
-    dp.tpt = kTileRows / D.G;
-    dp.f16 = f16 ? 1 : 0;
-    dp.swin = swin;
-    dp.scale_log2 = fp.scale_log2;
-    dp.bidx = block_idx;
-    dp.dtile_off = c.inv.dtile_off;
-    dp.posmap = posmap;
-    dp.part_o = fp.part_o;
-    dp.part_meta = fp.part_meta;
-    dp.out = out;
-    dp.lse = lse;
-    dp.st = c.st;
-    dp.num_sms = num_sms;
-    CUtensorMap qmap;
-    if (!make_q_group_map(&qmap, q, D.T, D.hq, D.G, f16)) return NSA_ERR_CUDA;
-    if ((s = cuda_status(launch_fwd_dense(dp, &qmap, &kmap, &vmap, stream))) != NSA_OK) return s;
+    MergePlan mp{};
+    mp.cu = cu_seqlens;
+    mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
+    mp.G = D.G;
+    mp.f16 = f16 ? 1 : 0;
+    mp.swin = swin;
+    mp.bidx = block_idx;
+    mp.posmap = posmap;
+    mp.part_o = fp.part_o;
+    mp.part_meta = fp.part_meta;
+    mp.out = out;
+    mp.lse = lse;
+    mp.st = c.st;
+    if ((s = cuda_status(launch_merge(mp, stream))) != NSA_OK) return s;
     pm.add(1);
     pm.mark(3);
     return NSA_OK;

@@ -62,33 +62,26 @@ __device__ __forceinline__ unsigned long long block_incl_scan_u64(unsigned long 
     return r;
 }
 
-// 1. blkoff[s] = sum_{s' < s} ceil(L_s' / bs) and dtile_off[s] = sum_{s' < s}
-//    ceil(L_s' / tpt) (the forward's dense tiles); checks cu_seqlens.
+// 1. blkoff[s] = sum_{s' < s} ceil(L_s' / bs); checks cu_seqlens.
 __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq, int T, int bs,
-                                                     int tpt, int32_t* blkoff, int32_t* dtile_off,
-                                                     DevStatus* st, unsigned long long tag) {
+                                                     int32_t* blkoff, DevStatus* st,
+                                                     unsigned long long tag) {
     __shared__ unsigned long long warp_tot[32];
     __shared__ unsigned long long round_total;
     __shared__ int bad;
     if (threadIdx.x == 0) bad = (cu[0] != 0 || cu[nseq] != T) ? 1 : 0;
     __syncthreads();
-    unsigned long long carry = 0;   // (dense tiles << 32) | blocks
+    unsigned long long carry = 0;
     for (int base = 0; base < nseq; base += blockDim.x) {
         int s = base + threadIdx.x;
-        unsigned long long x = 0;
+        unsigned long long nb = 0;
         if (s < nseq) {
             int L = cu[s + 1] - cu[s];
             if (L < 0) bad = 1;
-            if (L > 0)
-                x = ((unsigned long long)((L + tpt - 1) / tpt) << 32) |
-                    (unsigned long long)((L + bs - 1) / bs);
+            nb = L > 0 ? (unsigned long long)((L + bs - 1) / bs) : 0ull;
         }
-        unsigned long long incl = block_incl_scan_u64(x, warp_tot);
-        if (s < nseq) {
-            const unsigned long long ex = carry + incl - x;
-            blkoff[s] = (int32_t)(ex & 0xFFFFFFFFull);
-            dtile_off[s] = (int32_t)(ex >> 32);
-        }
+        unsigned long long incl = block_incl_scan_u64(nb, warp_tot);
+        if (s < nseq) blkoff[s] = (int32_t)(carry + incl - nb);
         // total of this round = inclusive value of the last thread
         if (threadIdx.x == blockDim.x - 1) round_total = incl;
         __syncthreads();
@@ -96,9 +89,8 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        blkoff[nseq] = (int32_t)(carry & 0xFFFFFFFFull);
-        dtile_off[nseq] = (int32_t)(carry >> 32);
-        st->nblocks_total = (int)(carry & 0xFFFFFFFFull);
+        blkoff[nseq] = (int32_t)carry;
+        st->nblocks_total = (int)carry;
         st->index_tag = tag;
         if (bad) record_error(st, NSA_ERR_BAD_INDEX, 1);
     }
@@ -314,12 +306,7 @@ __device__ __forceinline__ int lower_bound_u32(const uint32_t* a, int lo, int hi
     return lo;
 }
 
-//    Only the entries of the KV-major kernel are split: the (g, B) list minus its
-//    prefix of tokens in the query blocks b and b + 1 (b = B's block within its
-//    sequence), for which B is an init or local block, and minus the whole list for
-//    b = 0; those entries belong to the dense pass (dense.cu).
 __global__ void k_window_split(const uint32_t* entries, const int32_t* offsets, const DevStatus* st,
-                               const int32_t* cu, const int32_t* blkoff, int nseq, int T, int bs,
                                int hkv, int nwin, int wtok, int nb_stride, int2* win_rng) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const int nbtot = st->nblocks_total;
@@ -329,22 +316,12 @@ __global__ void k_window_split(const uint32_t* entries, const int32_t* offsets, 
     const long long r = idx / nbtot;          // (g * nwin + w)
     const int w = (int)(r % nwin);
     const int g = (int)(r / nwin);
-    int lo = offsets[g * nbtot + B];
-    const int hi = offsets[g * nbtot + B + 1];
-    const int s = upper_index(blkoff, nseq, B);
-    const int b = B - blkoff[s];
-    if (b == 0) {
-        lo = hi;
-    } else {   // first token past the query blocks b and b + 1, as an entry value
-        const long long tok = min((long long)cu[s] + (long long)(b + 2) * bs, (long long)T);
-        lo = lower_bound_u32(entries, lo, hi, (uint32_t)(tok * 64));
-    }
+    const int lo = offsets[g * nbtot + B], hi = offsets[g * nbtot + B + 1];
     const uint32_t v0 = (uint32_t)w * (uint32_t)wtok * 64u;
     const uint32_t v1 = (uint32_t)(w + 1) * (uint32_t)wtok * 64u;
     const int a = lower_bound_u32(entries, lo, hi, v0);
-    const int e = (w + 1 == nwin) ? hi : lower_bound_u32(entries, a, hi, v1);
-    const int a2 = max(a, lo);
-    win_rng[r * nb_stride + B] = make_int2(a2, max(e - a2, 0));
+    const int b = (w + 1 == nwin) ? hi : lower_bound_u32(entries, a, hi, v1);
+    win_rng[r * nb_stride + B] = make_int2(a, b - a);
 }
 
 // 6. Per (g, w) row: exclusive scan over B of ceil(count / tpt) tiles, and the row's
@@ -529,8 +506,7 @@ int invert_final_buf(const InvertPlan& p) {
 }
 
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
-    k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.tokens_per_tile, p.blkoff,
-                                         p.dtile_off, p.st, p.tag);
+    k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st, p.tag);
     SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.swin, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
     const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
     const uint32_t* kin = nullptr;
@@ -566,8 +542,7 @@ cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaSt
     const int nrows = p.hkv * w.nwin;
     const long long n = (long long)nrows * w.nb_stride;      // upper bound (device NB <= stride)
     k_window_split<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
-        p.vals[p.final_buf], p.offsets, p.st, p.cu, p.blkoff, p.nseq, p.T, p.bs, p.hkv, w.nwin,
-        w.wtok, w.nb_stride, w.win_rng);
+        p.vals[p.final_buf], p.offsets, p.st, p.hkv, w.nwin, w.wtok, w.nb_stride, w.win_rng);
     k_window_tiles<<<nrows, 1024, 0, stream>>>(w.win_rng, p.st, w.nb_stride, p.tokens_per_tile,
                                                w.tile_off, w.row_tiles);
     k_row_offsets<<<1, 1024, 0, stream>>>(w.row_tiles, nrows, w.row_off, p.st);

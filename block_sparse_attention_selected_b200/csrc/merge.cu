@@ -1,6 +1,10 @@
-// merge.cu -- the memory-bound passes around the backward's tensor-core kernel (the
-// forward's merge is folded into dense.cu).
+// merge.cu -- the memory-bound passes around the tensor-core kernels.
 //
+//  k_merge         forward: per (token, query head) the log-sum-exp merge of the
+//                  per-block partials, O = sum_j e^{lse_j - LSE} o_j and
+//                  LSE = log sum_j e^{lse_j}; one warp per row, no atomics (the
+//                  reduction / online-softmax kernels of the key-features table on
+//                  the "Relaxed-System-Lab/Flash-Sparse-Attention" project page).
 //  k_bwd_delta     backward preprocess D = rowsum(dO * O) (fp32, [hq, T]).
 //  k_dq_merge      backward: dQ = sum over the row's slots of the dQ partials.
 //  k_dkdv_reduce   backward: dK, dV of every key = sum over the backward work
@@ -14,6 +18,97 @@ namespace nsa {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ float warp_max(float x) {
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    return x;
+}
+
+// One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: a slot whose
+// block is valid has its partial at row posmap * G + head offset of the forward tiles.
+// The block numbers and positions come in one round of requests, then every valid
+// slot's partial row (4 columns per lane) and each lane's (lse_j, exponent_j) in a
+// second: the row costs two dependent memory latencies.
+template <int kS, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk); fp16 output
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge(const MergePlan p) {
+    constexpr bool kTopk32 = kS <= 32;
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    if (row >= (long long)p.T * p.hq) return;
+    // after a recorded device error (malformed cu_seqlens, an expired wait) the
+    // position map and partials are incomplete: leave the outputs untouched
+    if (*reinterpret_cast<const volatile int*>(&p.st->code) != 0) return;
+    const int t = (int)(row / p.hq);
+    const int h = (int)(row - (long long)t * p.hq);
+    const int g = h / p.G;
+    const int hoff = h - g * p.G;
+    const unsigned nrows_part = (unsigned)p.st->ntiles_fwd * (unsigned)kTileRows;
+    const int s = seq_of_token(p.cu, p.nseq, t);
+    const int i = t - __ldg(p.cu + s);
+    const int qb = i / p.bs;
+    const size_t base = ((size_t)t * p.hkv + g) * p.topk;
+    // level 1: block number and position of slots lane, lane + 32, loaded together (the
+    // position is read whether or not the slot turns out to be a KV-major one: it is
+    // always in bounds, and the row then costs two memory latencies instead of three)
+    auto slot_row = [&](int b, int pos) -> unsigned {
+        if (!block_valid(b, qb, i, p.bs, p.swin)) return 0xFFFFFFFFu;
+        const unsigned r = (unsigned)pos * (unsigned)p.G + (unsigned)hoff;
+        return r < nrows_part ? r : 0xFFFFFFFFu;
+    };
+    int b0 = -1, b1 = -1, pos0 = 0, pos1 = 0;
+    if (lane < p.topk) {
+        b0 = __ldg(p.bidx + base + lane);
+        pos0 = __ldg(p.posmap + base + lane);
+    }
+    if (!kTopk32 && lane + 32 < p.topk) {
+        b1 = __ldg(p.bidx + base + lane + 32);
+        pos1 = __ldg(p.posmap + base + lane + 32);
+    }
+    const unsigned r0 = slot_row(b0, pos0);
+    const unsigned r1 = kTopk32 ? 0xFFFFFFFFu : slot_row(b1, pos1);
+    // level 2: the (lse, exponent) of this lane's slots and every valid partial row
+    float2 m0 = make_float2(-CUDART_INF_F, 0.f), m1 = m0;
+    if (r0 != 0xFFFFFFFFu) m0 = __ldg(p.part_meta + r0);
+    if (r1 != 0xFFFFFFFFu) m1 = __ldg(p.part_meta + r1);
+    const uint2* po = reinterpret_cast<const uint2*>(p.part_o) + lane;
+    const int nslot = min(p.topk, kS);
+    uint2 u[kS];
+#pragma unroll
+    for (int j = 0; j < kS; ++j) {
+        const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
+        u[j] = (j < nslot && rj != 0xFFFFFFFFu) ? __ldg(po + (size_t)rj * (kHeadDim / 4))
+                                                : make_uint2(0u, 0u);
+    }
+    const float M = warp_max(fmaxf(m0.x, m1.x));
+    uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                           (size_t)row * kHeadDim) + lane;
+    if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
+        *outp = make_uint2(0u, 0u);
+        if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
+        return;
+    }
+    const float w0 = m0.x == -CUDART_INF_F ? 0.f : __expf(m0.x - M);
+    const float w1 = m1.x == -CUDART_INF_F ? 0.f : __expf(m1.x - M);
+    const float Lam = warp_sum(w0 + w1);
+    const float s0 = ldexpf(w0, (int)m0.y), s1 = ldexpf(w1, (int)m1.y);   // weight x 2^e
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kS; ++j) {
+        const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
+        const float2 a = unpack_f16x2(u[j].x), b = unpack_f16x2(u[j].y);
+        acc[0] = fmaf(wj, a.x, acc[0]);
+        acc[1] = fmaf(wj, a.y, acc[1]);
+        acc[2] = fmaf(wj, b.x, acc[2]);
+        acc[3] = fmaf(wj, b.y, acc[3]);
+    }
+    const float inv = 1.f / Lam;
+    *outp = make_uint2(pack2<F16>(acc[0] * inv, acc[1] * inv), pack2<F16>(acc[2] * inv, acc[3] * inv));
+    if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
+}
 
 // Eight rows per warp, half a warp per row and 16-byte loads: four rows' loads of O and
 // dO are in flight per lane before the first reduction.
@@ -126,6 +221,22 @@ inline unsigned blocks_for(long long rows) {
 }
 
 }  // namespace
+
+cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
+    const unsigned nb = blocks_for((long long)p.T * p.hq);
+    const unsigned nt = kWarpsPerBlock * 32;
+    if (p.topk <= 16) {
+        if (p.f16) k_merge<16, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<16, 0><<<nb, nt, 0, stream>>>(p);
+    } else if (p.topk <= 32) {
+        if (p.f16) k_merge<32, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<32, 0><<<nb, nt, 0, stream>>>(p);
+    } else {
+        if (p.f16) k_merge<64, 1><<<nb, nt, 0, stream>>>(p);
+        else k_merge<64, 0><<<nb, nt, 0, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
                                   int f16, cudaStream_t stream) {

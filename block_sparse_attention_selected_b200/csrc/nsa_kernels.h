@@ -35,8 +35,6 @@ struct InvertPlan {
     int32_t* offsets;        // [nbk_cap + 1]
     int32_t* tile_off;       // [nbk_cap + 1]
     int32_t* chunk_off;      // [nbk_cap + 1]
-    int32_t* dtile_off;      // [nseq + 1]: forward dense tiles (of tokens_per_tile tokens)
-                             // of the sequences before s (k_seq_blocks)
     DevStatus* st;
     unsigned long long tag;  // written to st->index_tag by the inversion
     // result: the sorted values live in vals[final_buf]
@@ -110,30 +108,22 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream);
 
-// The forward's query-major pass over the init and local blocks, with the merge of
-// the KV-major partials folded in (dense.cu).
-struct DensePlan {
+struct MergePlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
-    int tpt;                 // tokens per dense tile: 128 / G
-    int f16;                 // 1: q, k, v, out are fp16; 0: bf16
+    int f16;                 // 1: out is fp16; 0: bf16
     int swin;                // sliding window in keys (0: none)
-    float scale_log2;        // scale * log2(e)
     const int32_t* bidx;
-    const int32_t* dtile_off;   // [nseq + 1] dense tiles before sequence s
-    const int32_t* posmap;   // partial position of each KV-major (t, g, j) entry
-    const void* part_o;
+    const int32_t* posmap;   // tile position of each KV-major (t, g, j) entry
+    const void* part_o;      // KV-major partials
     const float2* part_meta;
     void* out;
-    float* lse;              // may be null (no LSE stored)
-    DevStatus* st;
-    int num_sms;
+    float* lse;              // may be null
+    const DevStatus* st;
 };
 
-// qmap: Q [T, hq, 128] with boxes of 64 columns x G heads x 128 / G tokens (128B swizzle);
-// kmap / vmap as for the tile kernel
-cudaError_t launch_fwd_dense(const DensePlan& p, const CUtensorMap* qmap, const CUtensorMap* kmap,
-                             const CUtensorMap* vmap, cudaStream_t stream);
+// O and LSE of every row from its KV-major partials
+cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream);
 
 struct BwdPlan {
     const void* q;
