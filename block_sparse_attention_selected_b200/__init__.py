@@ -32,6 +32,7 @@ EXPORTED = ["nsa_sel_attn_workspace_size", "nsa_sel_attn_fwd", "nsa_sel_attn_bwd
             "nsa_sel_bsfa_workspace_size",
             "nsa_sel_invert_index",
             "nsa_sel_invert_index_noalloc", "nsa_sel_invert_index_noalloc_max_bytes",
+            "nsa_sel_invert_index_scratch_bytes",
             "nsa_sel_validate_indices", "nsa_sel_check_status", "nsa_sel_status_string"]
 
 _lib = None
@@ -88,6 +89,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             lib.nsa_sel_invert_index_noalloc.restype = I
             lib.nsa_sel_invert_index_noalloc_max_bytes.argtypes = []
             lib.nsa_sel_invert_index_noalloc_max_bytes.restype = Z
+            lib.nsa_sel_invert_index_scratch_bytes.argtypes = [I, I, I, I, I]
+            lib.nsa_sel_invert_index_scratch_bytes.restype = Z
             lib.nsa_sel_validate_indices.argtypes = [P, I, I, I, P, I, I, P, P, P, Z, P]
             lib.nsa_sel_validate_indices.restype = I
             lib.nsa_sel_check_status.argtypes = [P, P]

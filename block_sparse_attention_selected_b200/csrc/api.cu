@@ -897,6 +897,15 @@ extern "C" {
 
 size_t nsa_sel_invert_index_noalloc_max_bytes(void) { return kInvertScratchBytes; }
 
+size_t nsa_sel_invert_index_scratch_bytes(int total_tokens, int num_seqs, int hkv, int topk,
+                                          int block_size) {
+    Dims D;
+    // hq = hkv (group 1) fixes the tile geometry; it does not change the inversion.
+    if (check_dims(total_tokens, num_seqs, hkv, hkv, kHeadDim, topk, block_size, &D) != NSA_OK)
+        return 0;
+    return make_layout(D, false).inv_end;
+}
+
 nsa_status_t nsa_sel_invert_index_noalloc(const int32_t* cu_seqlens, int num_seqs,
                                           int total_tokens, int hkv, const int32_t* block_idx,
                                           int topk, int block_size, int32_t* offsets,

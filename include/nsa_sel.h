@@ -204,6 +204,15 @@ NSA_API nsa_status_t nsa_sel_invert_index(const int32_t *cu_seqlens, int num_seq
                                   int32_t *offsets, int32_t *entries, int32_t *counts,
                                   void *workspace, size_t workspace_bytes, nsa_stream_t stream);
 
+/* Bytes of scratch the block-index inversion needs for these sizes (0 when they are
+ * outside the supported domain): 256-byte-aligned regions of about 16.25 bytes per
+ * (token, KV head, slot) entry (two key and two value buffers of the radix sort and
+ * its digit histograms) plus 12 bytes per (KV head, block) and 4 per sequence.
+ * nsa_sel_invert_index_noalloc accepts exactly the sizes for which this is at most
+ * nsa_sel_invert_index_noalloc_max_bytes().  Host only; no device work. */
+NSA_API size_t nsa_sel_invert_index_scratch_bytes(int total_tokens, int num_seqs, int hkv,
+                                                  int topk, int block_size);
+
 /* The block-index inversion above, for callers that cannot allocate device memory
  * (for example a plug-in whose host framework owns all device memory and offers no
  * allocation hook, or a loop where cudaMalloc's possible device synchronisation is
@@ -211,14 +220,15 @@ NSA_API nsa_status_t nsa_sel_invert_index(const int32_t *cu_seqlens, int num_seq
  *   Arguments and outputs are those of nsa_sel_invert_index, without the workspace:
  *   the scratch is a fixed array in the library's device data, of
  *   nsa_sel_invert_index_noalloc_max_bytes() bytes (64 MiB) per device, held until
- *   the process exits.  Problems whose inversion scratch would not fit return
- *   NSA_ERR_WORKSPACE before any device work (about 17 bytes per (token, KV head,
- *   slot) entry: T * hkv * topk up to roughly 3.5 million).
- *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
- *   All calls share the array and it keeps the last call's contents; each call
- *   clears what it reads before writing it, but calls whose work overlaps on the GPU
- *   (other streams, other host threads) race: serialise them. */
+ *   the process exits.  Problems whose inversion scratch
+ *   (nsa_sel_invert_index_scratch_bytes; at topk 16 and block 64 roughly
+ *   T * hkv <= 250,000) would not fit return NSA_ERR_WORKSPACE before any device work.
+ *   The first call on a device (and the first after the device's context was
+ *   replaced) looks up the array's device address with that device current; make
+ *   that first call before any stream capture.
+ *   All calls share the array and it keeps the last call's contents; everything a
+ *   call reads from it is first written by the same call, but calls whose work
+ *   overlaps on the GPU (other streams, other host threads) race: serialise them. */
 NSA_API nsa_status_t nsa_sel_invert_index_noalloc(const int32_t *cu_seqlens, int num_seqs,
                                                   int total_tokens, int hkv,
                                                   const int32_t *block_idx, int topk,

@@ -269,3 +269,27 @@ def test_test_only_flags_are_forward_only(lib):
     rc = lib.nsa_sel_attn_fwd_ex(*([None] * 4), 1, 0, 1, 1, 128, None, 1, 64, ctypes.c_float(0.1),
                                  None, None, None, 0, None, 0x400, 0, None, 0, None)
     assert rc == 1   # an unknown bit
+
+
+def test_noalloc_size_boundary(lib):
+    """The no-allocation inversion takes exactly the sizes whose scratch (as reported by
+    nsa_sel_invert_index_scratch_bytes) fits its fixed array: the largest such size
+    passes the size check (and then, without a GPU, stops at the device check), the
+    next one is refused with NSA_ERR_WORKSPACE before any device work."""
+    limit = lib.nsa_sel_invert_index_noalloc_max_bytes()
+    need = lib.nsa_sel_invert_index_scratch_bytes
+    assert need(1000, 1, 4, 16, 64) > 1000 * 4 * 16 * 16
+    assert need(1000, 1, 4, 16, 32) == 0                 # block 32: outside the domain
+    lo, hi = 1, 1 << 22
+    while lo < hi:                                       # largest T that fits
+        mid = (lo + hi + 1) // 2
+        if need(mid, 1, 4, 16, 64) <= limit:
+            lo = mid
+        else:
+            hi = mid - 1
+    P = ctypes.c_void_p
+    fake = P(1 << 20)          # never dereferenced
+    call = lambda T: lib.nsa_sel_invert_index_noalloc(fake, 1, T, 4, fake, 16, 64, fake, fake,
+                                                      fake, None)
+    assert call(lo + 1) == 3                             # NSA_ERR_WORKSPACE
+    assert call(lo) != 3                                 # past the size check

@@ -26,7 +26,9 @@ def _case(lengths, hkv, topk, bs, seed):
 
 def test_noalloc_inversion_matches_workspace_inversion_twice():
     # two calls in a row with different problems: the second must not see the
-    # first call's leftovers in the shared scratch array
+    # first call's leftovers in the shared scratch array; each result equals the
+    # workspace inversion's and, bit for bit, the oracle's
+    import oracle
     for lengths, hkv, topk, bs, seed in (([3000, 777, 1], 4, 16, 64, 41), ([5000], 2, 8, 128, 42)):
         cu, bi, bs = _case(lengths, hkv, topk, bs, seed)
         ref_off, ref_ent = nsa.nsa_sel_invert_index(cu, bi, bs)
@@ -34,6 +36,23 @@ def test_noalloc_inversion_matches_workspace_inversion_twice():
         torch.cuda.synchronize()
         assert torch.equal(off, ref_off)
         assert torch.equal(ent, ref_ent)
+        o_off, o_ent = oracle.invert(cu.cpu().numpy(), bi.cpu().numpy(), bs)
+        assert np.array_equal(off.cpu().numpy(), o_off)
+        assert np.array_equal(ent.cpu().numpy(), o_ent)
+
+
+def test_noalloc_inversion_of_nothing():
+    # no tokens: empty lists, and the next call is unaffected
+    cu = torch.zeros(2, dtype=torch.int32, device="cuda")
+    bi = torch.empty((0, 2, 8), dtype=torch.int32, device="cuda")
+    off, ent = nsa.nsa_sel_invert_index_noalloc(cu, bi, 64)
+    torch.cuda.synchronize()
+    assert ent.numel() == 0 and bool((off == 0).all())
+    cu, bi, bs = _case([700], 2, 8, 64, 43)
+    off, ent = nsa.nsa_sel_invert_index_noalloc(cu, bi, bs)
+    ref_off, ref_ent = nsa.nsa_sel_invert_index(cu, bi, bs)
+    torch.cuda.synchronize()
+    assert torch.equal(off, ref_off) and torch.equal(ent, ref_ent)
 
 
 def test_noalloc_rejects_sizes_beyond_the_array():
