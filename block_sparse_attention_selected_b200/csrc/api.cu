@@ -40,11 +40,16 @@ struct Layout {
     size_t total;
 };
 
-nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int bs, Dims* D) {
+// Head dimensions: 64, 128 and 256 in the forward (256 with block 64: its Q and K / V
+// tiles fill the shared memory); 128 in the backward (bwd = true).
+nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int bs, Dims* D,
+                        bool bwd = false) {
     if (T < 0 || nseq < 1 || hq < 1 || hkv < 1 || d < 1 || topk < 1 || bs < 1)
         return NSA_ERR_INVALID_ARG;
     if (hq % hkv != 0) return NSA_ERR_INVALID_ARG;
-    if (d != kHeadDim || (bs != 64 && bs != 128) || topk > kMaxTopk) return NSA_ERR_UNSUPPORTED;
+    if ((bs != 64 && bs != 128) || topk > kMaxTopk) return NSA_ERR_UNSUPPORTED;
+    if (d != 64 && d != kHeadDim && d != 256) return NSA_ERR_UNSUPPORTED;
+    if ((d == 256 && bs != 64) || (bwd && d != kHeadDim)) return NSA_ERR_UNSUPPORTED;
     const int G = hq / hkv;
     if (G > kMaxGroup || kTileRows % G != 0) return NSA_ERR_UNSUPPORTED;
     if (T >= (1 << 25)) return NSA_ERR_UNSUPPORTED;
@@ -102,7 +107,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     // forward: one 128-row slot per tile; backward: one row per (token, head, slot)
     const size_t rows = std::max((size_t)D.T * D.hq * D.topk,
                                  (size_t)std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows);
-    L.part_o = take(rows * kHeadDim * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
+    L.part_o = take(rows * (size_t)D.d * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
     if (bwd) {
         L.delta = take(sizeof(float) * (size_t)D.hq * D.T);
@@ -155,11 +160,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // Tensor map over a bf16 [T, hkv, 128] tensor; box = (64 columns, 1 head, bs keys),
 // 128-byte swizzle (the layout the tensor-core descriptors expect).
-bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs, bool f16) {
+bool make_kv_map(CUtensorMap* map, const void* base, int T, int hkv, int bs, bool f16,
+                 int d = kHeadDim) {
     auto enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)hkv, (cuuint64_t)(T > 0 ? T : 1)};
-    cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)hkv * kHeadDim * 2};
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)(T > 0 ? T : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)bs};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -187,11 +193,11 @@ bool make_q_group_map(CUtensorMap* map, const void* base, int T, int hq, int G, 
 
 // Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, box_rows),
 // 128-byte swizzle: the epilogue's TMA stores of 8-row groups and of whole warps.
-bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows) {
+bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows, int d = kHeadDim) {
     auto enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
     cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr,
@@ -261,7 +267,7 @@ nsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA
 nsa_status_t check_common(const int32_t* cu, int nseq, int T, int hq, int hkv, int d,
                           const int32_t* bidx, int topk, int bs, void* ws, size_t ws_bytes,
                           bool bwd, Dims* D) {
-    nsa_status_t s = check_dims(T, nseq, hq, hkv, d, topk, bs, D);
+    nsa_status_t s = check_dims(T, nseq, hq, hkv, d, topk, bs, D, bwd);
     if (s != NSA_OK) return s;
     if (!cu || !ws || (T > 0 && !bidx)) return NSA_ERR_INVALID_ARG;
     if (!aligned(cu, 4) || !aligned(bidx, 4) || !aligned(ws, 256)) return NSA_ERR_INVALID_ARG;
@@ -276,7 +282,8 @@ extern "C" {
 size_t nsa_sel_attn_workspace_size(int total_tokens, int num_seqs, int hq, int hkv, int head_dim,
                                    int topk, int block_size, int for_bwd) {
     Dims D;
-    if (check_dims(total_tokens, num_seqs, hq, hkv, head_dim, topk, block_size, &D) != NSA_OK)
+    if (check_dims(total_tokens, num_seqs, hq, hkv, head_dim, topk, block_size, &D, for_bwd != 0) !=
+        NSA_OK)
         return 0;
     return make_layout(D, for_bwd != 0).total;
 }
@@ -351,7 +358,8 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     }
 
     CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16))
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16, D.d) ||
+        !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16, D.d))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
     WindowPlan wp{};
@@ -375,6 +383,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.cu = cu_seqlens;
     fp.nseq = D.nseq; fp.T = D.T; fp.hq = D.hq; fp.hkv = D.hkv; fp.topk = D.topk; fp.bs = D.bs;
     fp.G = D.G;
+    fp.d = D.d;
     fp.f16 = f16 ? 1 : 0;
     fp.swin = swin;
     fp.scale_log2 = scale * 1.4426950408889634f;
@@ -399,7 +408,8 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if ((s = cuda_status(launch_vblock_exp(fp, v, D.nb_stride, vexp, stream))) != NSA_OK) return s;
     CUtensorMap omap[2];
     const long long prow = std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows;
-    if (!make_part_map(&omap[0], fp.part_o, prow, 8) || !make_part_map(&omap[1], fp.part_o, prow, 32))
+    if (!make_part_map(&omap[0], fp.part_o, prow, 8, D.d) ||
+        !make_part_map(&omap[1], fp.part_o, prow, 32, D.d))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_fwd_tiles(fp, &kmap, &vmap, omap, stream))) != NSA_OK) return s;
     pm.add(2);
@@ -409,6 +419,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     mp.cu = cu_seqlens;
     mp.nseq = D.nseq; mp.T = D.T; mp.hq = D.hq; mp.hkv = D.hkv; mp.topk = D.topk; mp.bs = D.bs;
     mp.G = D.G;
+    mp.d = D.d;
     mp.f16 = f16 ? 1 : 0;
     mp.swin = swin;
     mp.bidx = block_idx;

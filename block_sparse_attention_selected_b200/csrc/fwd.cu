@@ -71,18 +71,27 @@ __device__ __forceinline__ void reg_alloc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 constexpr int kWgThreads = 128;
-constexpr int kNQ = 3;         // Q stages; S(i) completing frees stage i % kNQ (q_empty)
 constexpr int kChunk = 4;      // consecutive tiles per scheduling chunk
+// Per head dimension D = 64 NH (NH 64-column halves):
+//   kNQ   Q stages (S(i) completing frees stage i % kNQ: q_empty); two for D = 256,
+//         whose 64 KB Q tiles leave room for one K / V stage only
+//   kNSt  epilogue staging halves per warp (reused every kNSt halves)
+template <int NH>
+struct FwdCfg {
+    static constexpr int kNQ = NH == 4 ? 2 : 3;
+    static constexpr int kNSt = NH == 4 ? 1 : 2;
+};
 // Row-scale buffers: softmax(i + kNSc) may run once PV(i + kNSc - 2) is issued, which
 // waits for the epilogue of tile i + kNSc - 2 - NO; kNSc >= NO + 2 keeps it behind the
 // epilogue's read of sc[i % kNSc].
 constexpr int kNSc = 8;
 
-template <int BS, int NKV>
+template <int BS, int NKV, int NH>
 struct alignas(1024) FwdSmem {
-    uint8_t q[kNQ][2][kTileRows * 128];       // Q tile per stage: [64-column half][row]
-    uint8_t kv[NKV][2][2][BS * 128];          // [stage][K, V][64-column half][key]
-    uint8_t stage[4][2][32 * 128];            // epilogue staging: [warp][64-column half]
+    static constexpr int kNQ = FwdCfg<NH>::kNQ;
+    uint8_t q[kNQ][NH][kTileRows * 128];      // Q tile per stage: [64-column half][row]
+    uint8_t kv[NKV][2][NH][BS * 128];         // [stage][K, V][64-column half][key]
+    uint8_t stage[4][FwdCfg<NH>::kNSt][32 * 128];   // epilogue staging: [warp][half buffer]
     float sc[kNSc][kTileRows];                // row scale 2^-e / l of tile i in sc[i % kNSc]
     uint64_t q_full[kNQ], q_empty[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
@@ -95,9 +104,9 @@ struct alignas(1024) FwdSmem {
     int ntiles;
 };
 
-template <int BS, int NKV>
+template <int BS, int NKV, int NH>
 constexpr size_t fwd_smem_bytes() {
-    return sizeof(FwdSmem<BS, NKV>) + 1024;
+    return sizeof(FwdSmem<BS, NKV, NH>) + 1024;
 }
 
 __device__ __forceinline__ void cp_async_wait_one_pending() {
@@ -119,23 +128,25 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
-template <int BS, int NKV, int F16>
+template <int BS, int NKV, int NH, int F16>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fwd_tiles(const FwdPlan p, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap8,
                 const __grid_constant__ CUtensorMap omap32) {
+    constexpr int kNQ = FwdCfg<NH>::kNQ, kNSt = FwdCfg<NH>::kNSt;
+    constexpr int D = 64 * NH;                // head dimension
     extern __shared__ uint8_t smem_raw[];
-    FwdSmem<BS, NKV>& S = *reinterpret_cast<FwdSmem<BS, NKV>*>(
+    FwdSmem<BS, NKV, NH>& S = *reinterpret_cast<FwdSmem<BS, NKV, NH>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     DevStatus* st = p.st;
     // TMEM columns: S of slot s (and P, bf16, in its first BS/2 columns) at s * BS;
-    // O accumulator buffer b at 2 * BS + b * 128.
-    constexpr int NO = BS == 64 ? 3 : 2;
+    // O accumulator buffer b at 2 * BS + b * D.
+    constexpr int NO = NH == 4 ? 1 : ((BS == 64 || NH == 1) ? 3 : 2);
     constexpr int kColO = 2 * BS;
-    static_assert(kColO + NO * kHeadDim <= 512, "TMEM budget");
+    static_assert(kColO + NO * D <= 512, "TMEM budget");
 
     if (tid == 0) {
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto row_addr = [&](const int4& d, int r, uint32_t ent) -> unsigned long long {
                 const int g = d.z >> 8;
                 return reinterpret_cast<unsigned long long>(
-                    qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (kHeadDim * 2));
+                    qb + ((size_t)(ent >> 6) * p.hq + g * p.G + r % p.G) * (D * 2));
             };
             // test-only fault injection (NSA_TEST_SKIP_ARRIVE): loader 0 of CTA 0 withholds
             // its arrival on the first tile's Q barrier; its copies still complete, and no
@@ -233,7 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int4 d0 = ld_desc(0), d1 = ld_desc(1);
             uint32_t ea = ld_ent(d0, rA);
             int published = 0, issued = 0;
-            const int c = lane & 15;
+            // a row is 2 D bytes = kCpr 16-byte chunks; one warp instruction copies kRpi rows
+            constexpr int kCpr = 8 * NH, kRpi = 32 / kCpr;
+            const int c = lane % kCpr;
             const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
             for (int i = 0; i < n; ++i) {
                 const int4 d = d0;
@@ -256,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_w(&S.q_empty[stg], ((i / kNQ) & 1) ^ 1, 30)) break;
                 const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c;
     #pragma unroll 4
-                for (int k = 0; k < (kRowsPerLoader + 1) / 2; ++k) {
-                    const int rw = 2 * k + (lane >> 4);          // row within the loader's rows
+                for (int k = 0; k < (kRowsPerLoader + kRpi - 1) / kRpi; ++k) {
+                    const int rw = kRpi * k + lane / kCpr;       // row within the loader's rows
                     const unsigned long long a = __shfl_sync(0xffffffffu, addrA, rw & 31) + c * 16;
                     const int row = kRowsPerLoader * w + rw;
                     if (rw < nr_w && row < nrows)
@@ -299,11 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int stg = uses % NKV;
                     if (!wait(&S.kv_empty[stg], ((uses / NKV) & 1) ^ 1, 32)) break;
                     const int g = d.z >> 8;
-                    mbar_arrive_expect_tx(&S.kv_full[stg], 4u * BS * 128u);
-                    tma_load_3d(S.kv[stg][0][0], &kmap, &S.kv_full[stg], 0, g, d.x);
-                    tma_load_3d(S.kv[stg][0][1], &kmap, &S.kv_full[stg], 64, g, d.x);
-                    tma_load_3d(S.kv[stg][1][0], &vmap, &S.kv_full[stg], 0, g, d.x);
-                    tma_load_3d(S.kv[stg][1][1], &vmap, &S.kv_full[stg], 64, g, d.x);
+                    mbar_arrive_expect_tx(&S.kv_full[stg], 2u * NH * BS * 128u);
+    #pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        tma_load_3d(S.kv[stg][0][h], &kmap, &S.kv_full[stg], 64 * h, g, d.x);
+                        tma_load_3d(S.kv[stg][1][h], &vmap, &S.kv_full[stg], 64 * h, g, d.x);
+                    }
                     last_parity[stg] = (uses / NKV) & 1;
                     loaded[stg] = true;
                     ++uses;
@@ -319,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 const uint32_t elected = elect_one();
                 constexpr uint32_t kIdescS = idesc_f16kind_f32(F16, 128, BS, false, false);
-                constexpr uint32_t kIdescO = idesc_f16kind_f32(F16, 128, 128, false, true);
+                constexpr uint32_t kIdescO = idesc_f16kind_f32(F16, 128, D, false, true);
                 int kv_uses = 0, prev_bucket = -1, cur = 0;
                 int kvs_of[2] = {0, 0};
                 // S(i) = Q K^T into slot i & 1.  The slot's previous S / P (tile i - 2) was
@@ -356,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a0 = q_desc0 + (uint32_t)stg * kQStage;
                     const uint32_t b0 = k_desc0 + (uint32_t)cur * kKvStage;
     #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
+                    for (int ks = 0; ks < 4 * NH; ++ks) {     // K = D, 16 per step
                         const uint32_t off = (uint32_t)((ks >> 2) * kQHalf + (ks & 3) * 2);
                         const uint32_t offk = (uint32_t)((ks >> 2) * kKvHalf + (ks & 3) * 2);
                         mma_ss_e(tS, a0 + off, b0 + offk, kIdescS, ks > 0 ? 1u : 0u, elected);
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!wait(&S.p_full[slot], (i >> 1) & 1, 36)) return false;
                     if (!wait(&S.o_free[ob], ((i / NO) & 1) ^ 1, 34)) return false;
                     tc_fence_after();
-                    const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * kHeadDim;
+                    const uint32_t tS = tmem + slot * BS, tO = tmem + kColO + ob * D;
                     const int kvs = kvs_of[slot];
                     const uint32_t b0 = v_desc0 + (uint32_t)kvs * kKvStage;
     #pragma unroll
@@ -541,19 +555,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int valid = min(32, max(0, (d.z & 255) - quad * 32));
             const int nbox = (valid + 7) >> 3;
             const int prow0 = tile_of(i) * kTileRows + quad * 32;   // warp's first row
-            const uint32_t tO = tmem + kColO + ob * kHeadDim + lane_off;
+            const uint32_t tO = tmem + kColO + ob * D + lane_off;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < NH; ++h) {
                 float x[64];
                 tmem_ld64_sync(tO + h * 64, x);
-                if (h == 1) {                 // the buffer's O has been read: release it
+                if (h == NH - 1) {            // the buffer's O has been read: release it
                     tc_fence_before();
                     mbar_arrive(&S.o_free[ob]);
                 }
-                // the TMA store that last read this staging half (tile i - 1) is done
-                if (lane == 0) bulk_wait_read<1>();
+                // the TMA store that last read this staging buffer is done
+                if (lane == 0) bulk_wait_read<kNSt - 1>();
                 __syncwarp();
-                const uint32_t sb = smem_u32(S.stage[ew][h]);
+                const uint32_t sb = smem_u32(S.stage[ew][h % kNSt]);
 #pragma unroll
                 for (int pc = 0; pc < 8; ++pc) {
                     const float* y = x + pc * 8;
@@ -571,10 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0 && nbox > 0) {
                     if (nbox == 4) {
-                        tma_store_2d(&omap32, S.stage[ew][h], h * 64, prow0);
+                        tma_store_2d(&omap32, S.stage[ew][h % kNSt], h * 64, prow0);
                     } else {
                         for (int b = 0; b < nbox; ++b)
-                            tma_store_2d(&omap8, S.stage[ew][h] + b * 1024, h * 64, prow0 + b * 8);
+                            tma_store_2d(&omap8, S.stage[ew][h % kNSt] + b * 1024, h * 64, prow0 + b * 8);
                     }
                     bulk_commit();
                 }
@@ -592,13 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Per (KV head g, global block B): e = 0 unless max |V_B| > 2^14, then the exponent
-// that brings it under 2^15 (fp16 partials of O / l stay finite).  One block of 128
+// that brings it under 2^15 (fp16 partials of O / l stay finite).  One block of d
 // threads per (B, g), thread = column.
-__global__ void __launch_bounds__(128) k_vblock_exp(const __nv_bfloat16* v, const int32_t* cu,
-                                                    int nseq, int hkv, int bs,
+__global__ void __launch_bounds__(256) k_vblock_exp(const __nv_bfloat16* v, const int32_t* cu,
+                                                    int nseq, int hkv, int d, int bs,
                                                     const int32_t* blkoff, const DevStatus* st,
                                                     int32_t* vexp) {
-    __shared__ float wmax[4];
+    __shared__ float wmax[8];
     const int B = blockIdx.x, g = blockIdx.y;
     const int nbtot = st->nblocks_total;
     if (st->code != 0 || B >= nbtot) return;
@@ -607,12 +621,13 @@ __global__ void __launch_bounds__(128) k_vblock_exp(const __nv_bfloat16* v, cons
     const int kend = min(key0 + bs, __ldg(cu + s + 1));
     float m = 0.f;
     for (int key = key0; key < kend; ++key)
-        m = fmaxf(m, fabsf(__bfloat162float(v[((size_t)key * hkv + g) * kHeadDim + threadIdx.x])));
+        m = fmaxf(m, fabsf(__bfloat162float(v[((size_t)key * hkv + g) * d + threadIdx.x])));
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        m = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+        m = fmaxf(m, wmax[0]);
         vexp[g * nbtot + B] = m > 16384.f ? min(ilogbf(m) - 14, 120) : 0;
     }
 }
@@ -624,30 +639,49 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
     if (p.T > 0 && nb_stride > 0) {
         if (p.f16)   // |V| <= 65504 already fits the fp16 partials: every exponent is 0
             return cudaMemsetAsync(vexp, 0, sizeof(int32_t) * (size_t)p.hkv * nb_stride, stream);
-        k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), 128, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(v), p.cu, p.nseq, p.hkv, p.bs, p.blkoff, p.st, vexp);
+        k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), (unsigned)p.d, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(v), p.cu, p.nseq, p.hkv, p.d, p.bs, p.blkoff, p.st,
+            vexp);
     }
     return cudaGetLastError();
 }
 
-template <int BS, int NKV, int F16>
+template <int BS, int NKV, int NH, int F16>
 static void launch_fwd_variant(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                                const CUtensorMap* omap, cudaStream_t stream) {
-    constexpr size_t smem = fwd_smem_bytes<BS, NKV>();
-    cudaFuncSetAttribute(k_fwd_tiles<BS, NKV, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    constexpr size_t smem = fwd_smem_bytes<BS, NKV, NH>();
+    static_assert(smem <= 232448, "shared memory per CTA");
+    cudaFuncSetAttribute(k_fwd_tiles<BS, NKV, NH, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    k_fwd_tiles<BS, NKV, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0],
-                                                                      omap[1]);
+    k_fwd_tiles<BS, NKV, NH, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, omap[0],
+                                                                          omap[1]);
+}
+
+template <int NH, int F16>
+static void launch_fwd_nh(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                          const CUtensorMap* omap, cudaStream_t stream) {
+    if (p.bs == 64) launch_fwd_variant<64, NH == 4 ? 1 : 2, NH, F16>(p, kmap, vmap, omap, stream);
+    else if constexpr (NH != 4) launch_fwd_variant<128, 1, NH, F16>(p, kmap, vmap, omap, stream);
 }
 
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream) {
-    if (p.bs == 64) {
-        if (p.f16) launch_fwd_variant<64, 2, 1>(p, kmap, vmap, omap, stream);
-        else launch_fwd_variant<64, 2, 0>(p, kmap, vmap, omap, stream);
-    } else {
-        if (p.f16) launch_fwd_variant<128, 1, 1>(p, kmap, vmap, omap, stream);
-        else launch_fwd_variant<128, 1, 0>(p, kmap, vmap, omap, stream);
+    if (p.d == 256 && p.bs != 64) return cudaErrorInvalidValue;   // no shared memory for it
+    switch (p.d) {
+        case 64:
+            if (p.f16) launch_fwd_nh<1, 1>(p, kmap, vmap, omap, stream);
+            else launch_fwd_nh<1, 0>(p, kmap, vmap, omap, stream);
+            break;
+        case 128:
+            if (p.f16) launch_fwd_nh<2, 1>(p, kmap, vmap, omap, stream);
+            else launch_fwd_nh<2, 0>(p, kmap, vmap, omap, stream);
+            break;
+        case 256:
+            if (p.f16) launch_fwd_nh<4, 1>(p, kmap, vmap, omap, stream);
+            else launch_fwd_nh<4, 0>(p, kmap, vmap, omap, stream);
+            break;
+        default:
+            return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

@@ -28,14 +28,39 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// The 2 NH fp16 values of a partial row (d = 64 NH) that one lane owns: lane l holds
+// columns [2 NH l, 2 NH l + 2 NH).
+template <int NH> struct LaneVec;
+template <> struct LaneVec<1> { uint32_t w[1]; };
+template <> struct LaneVec<2> { uint32_t w[2]; };
+template <> struct LaneVec<4> { uint32_t w[4]; };
+
+template <int NH>
+__device__ __forceinline__ LaneVec<NH> ld_lane(const uint8_t* row_base, int lane) {
+    LaneVec<NH> v;
+    if constexpr (NH == 1) {
+        v.w[0] = __ldg(reinterpret_cast<const uint32_t*>(row_base) + lane);
+    } else if constexpr (NH == 2) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(row_base) + lane);
+        v.w[0] = u.x; v.w[1] = u.y;
+    } else {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row_base) + lane);
+        v.w[0] = u.x; v.w[1] = u.y; v.w[2] = u.z; v.w[3] = u.w;
+    }
+    return v;
+}
+
 // One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: a slot whose
 // block is valid has its partial at row posmap * G + head offset of the forward tiles.
-// The block numbers and positions come in one round of requests, then every valid
-// slot's partial row (4 columns per lane) and each lane's (lse_j, exponent_j) in a
-// second: the row costs two dependent memory latencies.
-template <int kS, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk); fp16 output
+// The block numbers and positions come in one round of requests, then the valid slots'
+// (lse_j, exponent_j) and partial rows (2 NH columns per lane) in a second: the row
+// costs two dependent memory latencies for up to 16 slots (larger topk: one more
+// round per further 16 slots).
+template <int kS, int NH, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk)
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge(const MergePlan p) {
     constexpr bool kTopk32 = kS <= 32;
+    constexpr int kChunk = 16;        // partial rows in flight per round
+    constexpr size_t kRowBytes = (size_t)128 * NH;
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hq) return;
@@ -52,8 +77,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     const int qb = i / p.bs;
     const size_t base = ((size_t)t * p.hkv + g) * p.topk;
     // level 1: block number and position of slots lane, lane + 32, loaded together (the
-    // position is read whether or not the slot turns out to be a KV-major one: it is
-    // always in bounds, and the row then costs two memory latencies instead of three)
+    // position is read whether or not the slot is valid: it is always in bounds)
     auto slot_row = [&](int b, int pos) -> unsigned {
         if (!block_valid(b, qb, i, p.bs, p.swin)) return 0xFFFFFFFFu;
         const unsigned r = (unsigned)pos * (unsigned)p.G + (unsigned)hoff;
@@ -70,24 +94,37 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     }
     const unsigned r0 = slot_row(b0, pos0);
     const unsigned r1 = kTopk32 ? 0xFFFFFFFFu : slot_row(b1, pos1);
-    // level 2: the (lse, exponent) of this lane's slots and every valid partial row
+    // level 2: the (lse, exponent) of this lane's slots and the first kChunk partial rows
     float2 m0 = make_float2(-CUDART_INF_F, 0.f), m1 = m0;
     if (r0 != 0xFFFFFFFFu) m0 = __ldg(p.part_meta + r0);
     if (r1 != 0xFFFFFFFFu) m1 = __ldg(p.part_meta + r1);
-    const uint2* po = reinterpret_cast<const uint2*>(p.part_o) + lane;
+    const uint8_t* po = static_cast<const uint8_t*>(p.part_o);
     const int nslot = min(p.topk, kS);
-    uint2 u[kS];
-#pragma unroll
-    for (int j = 0; j < kS; ++j) {
+    auto ld_slot = [&](int j) -> LaneVec<NH> {
         const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
-        u[j] = (j < nslot && rj != 0xFFFFFFFFu) ? __ldg(po + (size_t)rj * (kHeadDim / 4))
-                                                : make_uint2(0u, 0u);
-    }
+        LaneVec<NH> z;
+#pragma unroll
+        for (int q = 0; q < NH; ++q) z.w[q] = 0u;
+        return (j < nslot && rj != 0xFFFFFFFFu) ? ld_lane<NH>(po + (size_t)rj * kRowBytes, lane) : z;
+    };
+    LaneVec<NH> u[kChunk];
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) u[j] = ld_slot(j);
     const float M = warp_max(fmaxf(m0.x, m1.x));
-    uint2* outp = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                           (size_t)row * kHeadDim) + lane;
+    uint8_t* outb = static_cast<uint8_t*>(p.out) + (size_t)row * kRowBytes;
+    auto store = [&](const float* a) {
+        uint32_t w[NH];
+#pragma unroll
+        for (int q = 0; q < NH; ++q) w[q] = pack2<F16>(a[2 * q], a[2 * q + 1]);
+        if constexpr (NH == 1) reinterpret_cast<uint32_t*>(outb)[lane] = w[0];
+        else if constexpr (NH == 2) reinterpret_cast<uint2*>(outb)[lane] = make_uint2(w[0], w[1]);
+        else reinterpret_cast<uint4*>(outb)[lane] = make_uint4(w[0], w[1], w[2], w[3]);
+    };
     if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
-        *outp = make_uint2(0u, 0u);
+        float zero[2 * NH];
+#pragma unroll
+        for (int q = 0; q < 2 * NH; ++q) zero[q] = 0.f;
+        store(zero);
         if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
         return;
     }
@@ -95,18 +132,31 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     const float w1 = m1.x == -CUDART_INF_F ? 0.f : __expf(m1.x - M);
     const float Lam = warp_sum(w0 + w1);
     const float s0 = ldexpf(w0, (int)m0.y), s1 = ldexpf(w1, (int)m1.y);   // weight x 2^e
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[2 * NH];
 #pragma unroll
-    for (int j = 0; j < kS; ++j) {
+    for (int q = 0; q < 2 * NH; ++q) acc[q] = 0.f;
+    auto add = [&](const LaneVec<NH>& v, int j) {
         const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
-        const float2 a = unpack_f16x2(u[j].x), b = unpack_f16x2(u[j].y);
-        acc[0] = fmaf(wj, a.x, acc[0]);
-        acc[1] = fmaf(wj, a.y, acc[1]);
-        acc[2] = fmaf(wj, b.x, acc[2]);
-        acc[3] = fmaf(wj, b.y, acc[3]);
+#pragma unroll
+        for (int q = 0; q < NH; ++q) {
+            const float2 a = unpack_f16x2(v.w[q]);
+            acc[2 * q] = fmaf(wj, a.x, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(wj, a.y, acc[2 * q + 1]);
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) add(u[j], j);
+#pragma unroll
+    for (int j0 = kChunk; j0 < kS; j0 += kChunk) {   // topk > 16: further rounds
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) u[j] = ld_slot(j0 + j);
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) add(u[j], j0 + j);
     }
     const float inv = 1.f / Lam;
-    *outp = make_uint2(pack2<F16>(acc[0] * inv, acc[1] * inv), pack2<F16>(acc[2] * inv, acc[3] * inv));
+#pragma unroll
+    for (int q = 0; q < 2 * NH; ++q) acc[q] *= inv;
+    store(acc);
     if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
 }
 
@@ -222,18 +272,21 @@ inline unsigned blocks_for(long long rows) {
 
 }  // namespace
 
+template <int NH, int F16>
+static void launch_merge_nh(const MergePlan& p, unsigned nb, cudaStream_t stream) {
+    const unsigned nt = kWarpsPerBlock * 32;
+    if (p.topk <= 16) k_merge<16, NH, F16><<<nb, nt, 0, stream>>>(p);
+    else if (p.topk <= 32) k_merge<32, NH, F16><<<nb, nt, 0, stream>>>(p);
+    else k_merge<64, NH, F16><<<nb, nt, 0, stream>>>(p);
+}
+
 cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
     const unsigned nb = blocks_for((long long)p.T * p.hq);
-    const unsigned nt = kWarpsPerBlock * 32;
-    if (p.topk <= 16) {
-        if (p.f16) k_merge<16, 1><<<nb, nt, 0, stream>>>(p);
-        else k_merge<16, 0><<<nb, nt, 0, stream>>>(p);
-    } else if (p.topk <= 32) {
-        if (p.f16) k_merge<32, 1><<<nb, nt, 0, stream>>>(p);
-        else k_merge<32, 0><<<nb, nt, 0, stream>>>(p);
-    } else {
-        if (p.f16) k_merge<64, 1><<<nb, nt, 0, stream>>>(p);
-        else k_merge<64, 0><<<nb, nt, 0, stream>>>(p);
+    switch (p.d) {
+        case 64: if (p.f16) launch_merge_nh<1, 1>(p, nb, stream); else launch_merge_nh<1, 0>(p, nb, stream); break;
+        case 128: if (p.f16) launch_merge_nh<2, 1>(p, nb, stream); else launch_merge_nh<2, 0>(p, nb, stream); break;
+        case 256: if (p.f16) launch_merge_nh<4, 1>(p, nb, stream); else launch_merge_nh<4, 0>(p, nb, stream); break;
+        default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
 }

@@ -78,6 +78,7 @@ struct FwdPlan {
     const void* q;
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int d;                   // head dimension: 64, 128 or 256 (256 with block 64 only)
     int f16;                 // 1: q, k, v, out (dout, dq, dk, dv) are fp16; 0: bf16
     int swin;                // sliding window in keys (0: none)
     float scale_log2;        // scale * log2(e)
@@ -92,7 +93,7 @@ struct FwdPlan {
     const int32_t* wtile_off;
     const int32_t* row_off;
     const int4* tile_desc;
-    void* part_o;            // fp16 [tiles * 128, 128]: O_B / l_B * 2^-e, row tile * 128 + r
+    void* part_o;            // fp16 [tiles * 128, d]: O_B / l_B * 2^-e, row tile * 128 + r
     float2* part_meta;       // [tiles * 128]: (lse_B, e)
     const int32_t* vexp;     // [hkv * NB]: exponent e of each (g, B) block's V
     DevStatus* st;
@@ -111,6 +112,7 @@ cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CU
 struct MergePlan {
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int d;                   // head dimension: 64, 128 or 256
     int f16;                 // 1: out is fp16; 0: bf16
     int swin;                // sliding window in keys (0: none)
     const int32_t* bidx;

@@ -51,7 +51,13 @@ def test_workspace_size_domain(lib):
     assert ws(65536, 1, 16, 4, 128, 16, 64, True) > base
     assert ws(0, 1, 4, 4, 128, 8, 64, False) > 0
     f = lib.nsa_sel_attn_workspace_size
-    assert f(1024, 1, 4, 4, 64, 8, 64, 0) == 0          # head_dim 64 not supported
+    assert f(1024, 1, 4, 4, 64, 8, 64, 0) > 0           # head_dim 64: forward
+    assert f(1024, 1, 4, 4, 64, 8, 64, 1) == 0          # ... but no backward
+    assert f(1024, 1, 4, 4, 256, 8, 64, 0) > 0          # head_dim 256 with block 64: forward
+    assert f(1024, 1, 4, 4, 256, 8, 128, 0) == 0        # ... not with block 128
+    assert f(1024, 1, 4, 4, 256, 8, 64, 1) == 0         # ... and no backward
+    assert f(1024, 1, 4, 4, 96, 8, 64, 0) == 0          # head_dim 96 not supported
+    assert f(1024, 1, 4, 4, 64, 8, 64, 0) < f(1024, 1, 4, 4, 256, 8, 64, 0)   # partial rows of 2 d bytes
     assert f(1024, 1, 4, 4, 128, 8, 32, 0) == 0         # block 32 not supported
     assert f(1024, 1, 4, 4, 128, 65, 64, 0) == 0        # topk > 64
     assert f(1024, 1, 64, 2, 128, 8, 64, 0) > 0         # group 32 fills a tile with 4 tokens
@@ -68,9 +74,16 @@ def test_workspace_size_domain(lib):
 def test_host_argument_errors(lib):
     P = ctypes.c_void_p
     fake = P(1 << 20)           # never dereferenced: checks fail first
-    # unsupported head_dim
-    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 64, fake, 8, 64, 0.1,
+    # unsupported head_dim (96; and 256 with block 128)
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 96, fake, 8, 64, 0.1,
                               fake, fake, fake, 1 << 30, None)
+    assert rc == 2
+    rc = lib.nsa_sel_attn_fwd(fake, fake, fake, fake, 1, 64, 4, 4, 256, fake, 8, 128, 0.1,
+                              fake, fake, fake, 1 << 30, None)
+    assert rc == 2
+    # head_dim 64 in the backward
+    rc = lib.nsa_sel_attn_bwd(fake, fake, fake, fake, fake, fake, fake, 1, 64, 4, 4, 64, fake, 8,
+                              64, 0.1, fake, fake, fake, fake, 1 << 30, None)
     assert rc == 2
     # null cu_seqlens
     rc = lib.nsa_sel_attn_fwd(fake, fake, fake, None, 1, 64, 4, 4, 128, fake, 8, 64, 0.1,

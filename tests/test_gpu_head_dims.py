@@ -1,0 +1,89 @@
+"""Head dimensions 64 and 256 in the forward (the project page's Limitations: one head
+dimension for Q, K and V, at most 256), against the fp64 oracle element by element.
+The backward takes head dimension 128 only and refuses the others on the host."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_selected_b200 as nsa
+import nsa_inputs as ni
+import oracle
+from gpu_util import TOL_LSE, TOL_O, f64, max_abs, o_errors, to_device
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, problem, window, perturbed
+    ("d64_g1_bs64_k16", dict(lengths=[1500, 37, 1, 600], hq=2, hkv=2, block_size=64, topk=16, seed=101), 0, True),
+    ("d64_g4_bs128_k8", dict(lengths=[2000, 129], hq=8, hkv=2, block_size=128, topk=8, seed=102), 0, True),
+    ("d64_g16_bs64_k64", dict(lengths=[1800], hq=16, hkv=1, block_size=64, topk=64, seed=103), 0, False),
+    ("d64_g8_bs64_k12_w100", dict(lengths=[900, 129], hq=8, hkv=1, block_size=64, topk=12, seed=104), 100, True),
+    ("d256_g1_bs64_k16", dict(lengths=[1500, 40, 1], hq=2, hkv=2, block_size=64, topk=16, seed=105), 0, True),
+    ("d256_g4_bs64_k8", dict(lengths=[2500, 64, 63], hq=8, hkv=2, block_size=64, topk=8, seed=106), 0, True),
+    ("d256_g32_bs64_k32", dict(lengths=[700, 77], hq=64, hkv=2, block_size=64, topk=32, seed=107), 0, False),
+]
+
+
+def _perturb(p, seed):
+    rng = np.random.default_rng(seed)
+    bi = p.block_idx
+    idx = np.argsort(rng.random(bi.shape), axis=2)
+    p.block_idx = np.ascontiguousarray(np.take_along_axis(bi, idx, axis=2))
+    return p
+
+
+@pytest.mark.parametrize("name,spec,W,perturb", CASES, ids=[c[0] for c in CASES])
+def test_fwd_head_dim_full_compare(name, spec, W, perturb):
+    d = 64 if name.startswith("d64") else 256
+    p = ni.make_problem(name=name, head_dim=d, with_dout=False, **spec)
+    if perturb:
+        p = _perturb(p, 9)
+    t = to_device(p)
+    out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], p.block_size,
+                                    p.scale, window_size=W)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    assert out.shape == (p.T, p.hq, d)
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, p.block_size, p.scale,
+                              window=W)
+    o, l = f64(out), f64(lse).T
+    fin = np.isfinite(l_ref)
+    assert np.array_equal(np.isfinite(l), fin), name
+    (raw, eo), el = o_errors(o, o_ref), max_abs(l[fin], l_ref[fin])
+    assert eo <= TOL_O and el <= TOL_LSE, (name, "gated", eo, "raw", raw, "lse", el)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_fwd_head_dim_fp16_and_large_v(d):
+    # fp16 tensors, and V scaled by 2^15 in bf16 (the per-block V exponent of the fp16
+    # partials, with one thread per column of the head dimension)
+    p = ni.make_problem([1300, 200], hq=8, hkv=2, head_dim=d, block_size=64, topk=8, seed=108,
+                        with_dout=False, name=f"d{d}_f16")
+    for a in ("q", "k", "v"):
+        setattr(p, a, getattr(p, a).astype(np.float16).astype(np.float32))
+    t = to_device(p, dtype=torch.float16)
+    out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, p.scale)
+    torch.cuda.synchronize()
+    assert out.dtype == torch.float16 and nsa.nsa_sel_check_status() == 0
+    o_ref, l_ref = oracle.fwd(p.q, p.k, p.v, p.cu_seqlens, p.block_idx, 64, p.scale)
+    assert o_errors(f64(out), o_ref)[1] <= TOL_O and max_abs(f64(lse).T, l_ref) <= TOL_LSE
+    q = ni.make_problem([1300, 200], hq=8, hkv=2, head_dim=d, block_size=64, topk=8, seed=109,
+                        with_dout=False, name=f"d{d}_large_v")
+    q.v = (q.v * 32768.0).astype(q.v.dtype)
+    t = to_device(q)
+    out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, q.scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    o_ref, l_ref = oracle.fwd(q.q, q.k, q.v, q.cu_seqlens, q.block_idx, 64, q.scale)
+    assert o_errors(f64(out) / 32768.0, o_ref / 32768.0)[1] <= TOL_O
+    assert max_abs(f64(lse).T, l_ref) <= TOL_LSE
+
+
+def test_bwd_head_dim_other_than_128_is_refused():
+    p = ni.make_problem([300], hq=4, hkv=2, head_dim=64, block_size=64, topk=4, seed=110)
+    t = to_device(p)
+    out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, p.scale)
+    with pytest.raises(nsa.NsaError) as e:
+        nsa.nsa_sel_attn_bwd(t["q"], t["k"], t["v"], out, lse, t["dout"], t["cu"], t["bidx"], 64,
+                             p.scale)
+    assert e.value.code == 2   # NSA_ERR_UNSUPPORTED
