@@ -96,7 +96,8 @@ struct alignas(1024) FwdSmem {
     uint64_t q_full[kNQ], q_empty[kNQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
     uint64_t s_full[2], p_full[2];
-    uint64_t o_full[3], o_free[3];            // O accumulator buffers (BS == 64: 3, else 2)
+    uint64_t o_full[3], o_free[3];            // O accumulator buffers (1 to 3 of them)
+    uint64_t pv_done[2];                      // PV of S slot s done (one O buffer only)
     uint64_t l_full[kNSc];                    // sc[i % kNSc] written
     uint64_t drain;
     uint32_t tmem_base;
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S.o_full[i], 1);
             mbar_init(&S.o_free[i], kWgThreads);
         }
+        for (int i = 0; i < 2; ++i) mbar_init(&S.pv_done[i], 1);
         for (int i = 0; i < kNSc; ++i) mbar_init(&S.l_full[i], kWgThreads);
         for (int i = 0; i < NKV; ++i) {
             mbar_init(&S.kv_full[i], 1);
@@ -361,10 +363,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int slot = i & 1, stg = i % kNQ;
                     kvs_of[slot] = cur;
                     if (!wait(&S.q_full[stg], (i / kNQ) & 1, 35)) return false;
-                    // S(i) overwrites the TMEM slot from which PV(i - 2), the last MMA issued
-                    // before it, reads P(i - 2) as its A operand: S(i) waits until PV(i - 2)
-                    // has completed, so that no write of it can overtake those reads.
-                    if (i >= 2 && !wait(&S.o_full[(i - 2) % NO], ((i - 2) / NO) & 1, 42)) return false;
+                    // S(i) overwrites the TMEM slot from which PV(i - 2) reads P(i - 2) as its
+                    // A operand: S(i) waits until PV(i - 2) has completed, so that no write of
+                    // it can overtake those reads.  With two or three O buffers PV(i - 1) and
+                    // PV(i - 2) arrive on different o_full barriers; with one, PV(i - 1) may
+                    // already be done when S(i) comes after it, and waiting on the shared
+                    // barrier's parity would alias, so each S slot has its own pv_done.
+                    if constexpr (NO == 1) {
+                        if (i >= 2 && !wait(&S.pv_done[slot], ((i >> 1) - 1) & 1, 42)) return false;
+                    } else {
+                        if (i >= 2 && !wait(&S.o_full[(i - 2) % NO], ((i - 2) / NO) & 1, 42)) return false;
+                    }
                     tc_fence_after();
                     const uint32_t tS = tmem + slot * BS;
                     const uint32_t a0 = q_desc0 + (uint32_t)stg * kQStage;
@@ -394,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_ts_e(tO, tS + (uint32_t)ks * 8u, b0 + (uint32_t)ks * 128u, kIdescO,
                                  ks > 0 ? 1u : 0u, elected);
                     mma_commit_e(&S.o_full[ob], elected);
+                    if constexpr (NO == 1) mma_commit_e(&S.pv_done[slot], elected);
                     if (release_kv) mma_commit_e(&S.kv_empty[kvs], elected);
                     return true;
                 };

@@ -133,18 +133,14 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_hist(SortArgs a, const ui
     __syncthreads();
     const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
     const long long base = (long long)blockIdx.x * kSortTile;
-    // every key of the thread first (independent loads in flight together), then the
-    // shared-memory counts
-    uint32_t key[kItems];
-#pragma unroll
     for (int it = 0; it < kItems; ++it) {
-        const long long e = base + it * kSortThreads + threadIdx.x;
-        uint32_t v;
-        key[it] = e < a.nent ? (kFirst ? entry_key(a, e, nbtot, &v) : __ldg(keys_in + e)) : 0u;
+        long long e = base + it * kSortThreads + threadIdx.x;
+        if (e < a.nent) {
+            uint32_t v;
+            uint32_t key = kFirst ? entry_key(a, e, nbtot, &v) : keys_in[e];
+            atomicAdd(&h[(key >> shift) & 255u], 1u);
+        }
     }
-#pragma unroll
-    for (int it = 0; it < kItems; ++it)
-        if (base + it * kSortThreads + threadIdx.x < a.nent) atomicAdd(&h[(key[it] >> shift) & 255u], 1u);
     __syncthreads();
     hist[(size_t)threadIdx.x * gridDim.x + blockIdx.x] = h[threadIdx.x];
 }
@@ -202,22 +198,15 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const
     const int nvalid = (int)min((long long)kSortTile, a.nent - tile0);
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t key[kItems], val[kItems], rank[kItems];
-    // every entry of the lane first (independent loads in flight together), then the
-    // warp-ordered ranks
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {
-        const long long e = base + it * 32 + lane;
-        key[it] = 0u;
-        val[it] = 0u;
+        long long e = base + it * 32 + lane;
+        uint32_t d = 256u;   // sentinel for entries past the end
         if (e < a.nent) {
-            key[it] = kFirst ? entry_key(a, e, nbtot, &val[it]) : __ldg(keys_in + e);
-            if (!kFirst) val[it] = __ldg(vals_in + e);
+            key[it] = kFirst ? entry_key(a, e, nbtot, &val[it]) : keys_in[e];
+            if (!kFirst) val[it] = vals_in[e];
+            d = (key[it] >> shift) & 255u;
         }
-    }
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const long long e = base + it * 32 + lane;
-        const uint32_t d = e < a.nent ? (key[it] >> shift) & 255u : 256u;   // 256: past the end
         uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
         uint32_t before = __popc(peers & lt_mask);
         if (d < 256u) rank[it] = whist[w][d] + before;

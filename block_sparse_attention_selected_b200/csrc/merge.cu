@@ -28,39 +28,36 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// The 2 NH fp16 values of a partial row (d = 64 NH) that one lane owns: lane l holds
-// columns [2 NH l, 2 NH l + 2 NH).
-template <int NH> struct LaneVec;
-template <> struct LaneVec<1> { uint32_t w[1]; };
-template <> struct LaneVec<2> { uint32_t w[2]; };
-template <> struct LaneVec<4> { uint32_t w[4]; };
+// The 2 NH fp16 values of a partial or output row (d = 64 NH) that one lane owns: lane
+// l holds columns [2 NH l, 2 NH l + 2 NH), loaded and stored as one vector.
+template <int NH> struct LaneVecT;
+template <> struct LaneVecT<1> { using type = uint32_t; };
+template <> struct LaneVecT<2> { using type = uint2; };
+template <> struct LaneVecT<4> { using type = uint4; };
 
-template <int NH>
-__device__ __forceinline__ LaneVec<NH> ld_lane(const uint8_t* row_base, int lane) {
-    LaneVec<NH> v;
-    if constexpr (NH == 1) {
-        v.w[0] = __ldg(reinterpret_cast<const uint32_t*>(row_base) + lane);
-    } else if constexpr (NH == 2) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(row_base) + lane);
-        v.w[0] = u.x; v.w[1] = u.y;
-    } else {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row_base) + lane);
-        v.w[0] = u.x; v.w[1] = u.y; v.w[2] = u.z; v.w[3] = u.w;
-    }
-    return v;
+template <typename V> __device__ __forceinline__ uint32_t vget(const V& v, int q);
+template <> __device__ __forceinline__ uint32_t vget<uint32_t>(const uint32_t& v, int) { return v; }
+template <> __device__ __forceinline__ uint32_t vget<uint2>(const uint2& v, int q) { return q ? v.y : v.x; }
+template <> __device__ __forceinline__ uint32_t vget<uint4>(const uint4& v, int q) {
+    return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
+template <typename V> __device__ __forceinline__ V vzero();
+template <> __device__ __forceinline__ uint32_t vzero<uint32_t>() { return 0u; }
+template <> __device__ __forceinline__ uint2 vzero<uint2>() { return make_uint2(0u, 0u); }
+template <> __device__ __forceinline__ uint4 vzero<uint4>() { return make_uint4(0u, 0u, 0u, 0u); }
 
 // One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: a slot whose
 // block is valid has its partial at row posmap * G + head offset of the forward tiles.
 // The block numbers and positions come in one round of requests, then the valid slots'
 // (lse_j, exponent_j) and partial rows (2 NH columns per lane) in a second: the row
-// costs two dependent memory latencies for up to 16 slots (larger topk: one more
-// round per further 16 slots).
+// costs two dependent memory latencies (d = 256 with topk > 16: further rounds of 16
+// partial rows, so that the loads in flight fit the registers).
 template <int kS, int NH, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk)
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge(const MergePlan p) {
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? (NH == 4 ? 2 : 5) : 1)
+    k_merge(const MergePlan p) {
+    using V = typename LaneVecT<NH>::type;
     constexpr bool kTopk32 = kS <= 32;
-    constexpr int kChunk = 16;        // partial rows in flight per round
-    constexpr size_t kRowBytes = (size_t)128 * NH;
+    constexpr int kChunk = (NH == 4 && kS > 16) ? 16 : kS;   // partial rows in flight per round
     const int lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
     if (row >= (long long)p.T * p.hq) return;
@@ -94,37 +91,22 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     }
     const unsigned r0 = slot_row(b0, pos0);
     const unsigned r1 = kTopk32 ? 0xFFFFFFFFu : slot_row(b1, pos1);
-    // level 2: the (lse, exponent) of this lane's slots and the first kChunk partial rows
+    // level 2: the (lse, exponent) of this lane's slots and every valid partial row
     float2 m0 = make_float2(-CUDART_INF_F, 0.f), m1 = m0;
     if (r0 != 0xFFFFFFFFu) m0 = __ldg(p.part_meta + r0);
     if (r1 != 0xFFFFFFFFu) m1 = __ldg(p.part_meta + r1);
-    const uint8_t* po = static_cast<const uint8_t*>(p.part_o);
+    const V* po = reinterpret_cast<const V*>(p.part_o) + lane;
     const int nslot = min(p.topk, kS);
-    auto ld_slot = [&](int j) -> LaneVec<NH> {
+    V u[kChunk];
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) {
         const unsigned rj = __shfl_sync(0xFFFFFFFFu, j < 32 ? r0 : r1, j & 31);
-        LaneVec<NH> z;
-#pragma unroll
-        for (int q = 0; q < NH; ++q) z.w[q] = 0u;
-        return (j < nslot && rj != 0xFFFFFFFFu) ? ld_lane<NH>(po + (size_t)rj * kRowBytes, lane) : z;
-    };
-    LaneVec<NH> u[kChunk];
-#pragma unroll
-    for (int j = 0; j < kChunk; ++j) u[j] = ld_slot(j);
+        u[j] = (j < nslot && rj != 0xFFFFFFFFu) ? __ldg(po + (size_t)rj * 32) : vzero<V>();
+    }
     const float M = warp_max(fmaxf(m0.x, m1.x));
-    uint8_t* outb = static_cast<uint8_t*>(p.out) + (size_t)row * kRowBytes;
-    auto store = [&](const float* a) {
-        uint32_t w[NH];
-#pragma unroll
-        for (int q = 0; q < NH; ++q) w[q] = pack2<F16>(a[2 * q], a[2 * q + 1]);
-        if constexpr (NH == 1) reinterpret_cast<uint32_t*>(outb)[lane] = w[0];
-        else if constexpr (NH == 2) reinterpret_cast<uint2*>(outb)[lane] = make_uint2(w[0], w[1]);
-        else reinterpret_cast<uint4*>(outb)[lane] = make_uint4(w[0], w[1], w[2], w[3]);
-    };
+    V* outp = reinterpret_cast<V*>(p.out) + (size_t)row * 32 + lane;
     if (M == -CUDART_INF_F) {          // nothing selected: O = 0, LSE = -inf
-        float zero[2 * NH];
-#pragma unroll
-        for (int q = 0; q < 2 * NH; ++q) zero[q] = 0.f;
-        store(zero);
+        *outp = vzero<V>();
         if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = -CUDART_INF_F;
         return;
     }
@@ -135,11 +117,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
     float acc[2 * NH];
 #pragma unroll
     for (int q = 0; q < 2 * NH; ++q) acc[q] = 0.f;
-    auto add = [&](const LaneVec<NH>& v, int j) {
+    auto add = [&](const V& v, int j) {
         const float wj = __shfl_sync(0xFFFFFFFFu, j < 32 ? s0 : s1, j & 31);
 #pragma unroll
         for (int q = 0; q < NH; ++q) {
-            const float2 a = unpack_f16x2(v.w[q]);
+            const float2 a = unpack_f16x2(vget<V>(v, q));
             acc[2 * q] = fmaf(wj, a.x, acc[2 * q]);
             acc[2 * q + 1] = fmaf(wj, a.y, acc[2 * q + 1]);
         }
@@ -147,16 +129,22 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? 5 : 1) k_merge
 #pragma unroll
     for (int j = 0; j < kChunk; ++j) add(u[j], j);
 #pragma unroll
-    for (int j0 = kChunk; j0 < kS; j0 += kChunk) {   // topk > 16: further rounds
+    for (int j0 = kChunk; j0 < kS; j0 += kChunk) {    // d = 256, topk > 16: further rounds
 #pragma unroll
-        for (int j = 0; j < kChunk; ++j) u[j] = ld_slot(j0 + j);
+        for (int j = 0; j < kChunk; ++j) {
+            const unsigned rj = __shfl_sync(0xFFFFFFFFu, j0 + j < 32 ? r0 : r1, (j0 + j) & 31);
+            u[j] = (j0 + j < nslot && rj != 0xFFFFFFFFu) ? __ldg(po + (size_t)rj * 32) : vzero<V>();
+        }
 #pragma unroll
         for (int j = 0; j < kChunk; ++j) add(u[j], j0 + j);
     }
     const float inv = 1.f / Lam;
+    uint32_t w[NH];
 #pragma unroll
-    for (int q = 0; q < 2 * NH; ++q) acc[q] *= inv;
-    store(acc);
+    for (int q = 0; q < NH; ++q) w[q] = pack2<F16>(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+    if constexpr (NH == 1) *outp = w[0];
+    else if constexpr (NH == 2) *outp = make_uint2(w[0], w[1]);
+    else *outp = make_uint4(w[0], w[1], w[2], w[3]);
     if (lane == 0 && p.lse) p.lse[(size_t)h * p.T + t] = M + __logf(Lam);
 }
 
