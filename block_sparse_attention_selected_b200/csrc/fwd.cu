@@ -11,9 +11,11 @@
 //         window, on the block where the window starts), l = sum P; P is written as
 //         bf16 back into the S columns of TMEM
 //   O_B = P V_B                    tcgen05.mma with A = P read from TMEM
-//   partial: O_B * 2^-e / l as fp16, lse_B = m + log l.  e is the block's V
-//         exponent (k_vblock_exp): 0 unless max |V_B| > 2^14, so O_B / l, a convex
-//         combination of V_B's rows, always fits fp16 after the 2^-e.
+//   partial: O_B * 2^-e / lr as fp16 (lr the sum of the rounded P values O_B used),
+//         lse_B = m + log l (l the fp32 sum), and the factor f that brings the stored
+//         row back to the block's convex combination of V_B's rows.  e is the block's V
+//         exponent (k_vblock_exp): 0 unless max |V_B| > 2^14, so the convex combination
+//         always fits fp16 after the 2^-e.
 //
 // A tile covers the consecutive entries [e0, e0 + ntok) of the sorted index list
 // (invert.cu), so its partial rows (entry * G + head offset) are one contiguous
@@ -468,13 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 v[2 * k2 + 1] = x.y;
             }
         };
-        // 64 values times s as packed bf16 pairs
-        auto pack_chunk = [&](const float* v, float s, uint32_t* pk) {
+        // 64 values times s as packed bf16 pairs; ls += the packed (rounded) values, the
+        // weights the P V product will actually use
+        auto pack_chunk = [&](const float* v, float s, uint32_t* pk, float2& ls) {
             const float2 s2 = make_float2(s, s);
 #pragma unroll
             for (int k2 = 0; k2 < 32; ++k2) {
                 const float2 x = mul2(make_float2(v[2 * k2], v[2 * k2 + 1]), s2);
                 pk[k2] = pack2<F16>(x.x, x.y);   // P in the type of V (one MMA, one type)
+                ls = add2(ls, unpack2<F16>(pk[k2]));
             }
         };
         // descriptors two tiles ahead, entries and exponents one tile ahead, so that no
@@ -510,35 +514,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!valid) mx = 0.f;                      // every valid row has lo <= lim
             const float mc = mx * c;
-            float2 l2 = make_float2(0.f, 0.f);
-            float l;
+            // l (fp32 sum of P) gives the block's LSE; the partial O is normalised by lr,
+            // the sum of the rounded P values the product uses, so that its weights sum to
+            // one exactly (a plain 1 / l would leave a bias of up to 2^-9 |V| on rows
+            // where one key dominates).
+            float2 l2 = make_float2(0.f, 0.f), lr2 = make_float2(0.f, 0.f);
+            float l, f;                                // f: partial O x f = the block's O
             uint32_t pk[32];
             if constexpr (BS == 64) {
                 // P pre-scaled by 2^-e / l: the epilogue only converts O
                 exp_chunk(sv, mc, l2);
                 l = l2.x + l2.y;
-                pack_chunk(sv, valid ? ldexpf(1.f / l, -ve) : 0.f, pk);
+                pack_chunk(sv, valid ? ldexpf(1.f / l, -ve) : 0.f, pk, lr2);
                 tmem_st32_sync(tS, pk);
+                f = 1.f / (lr2.x + lr2.y);
             } else {
 #pragma unroll
                 for (int c64 = 0; c64 < 2; ++c64) {    // scores of this 64-key chunk again
                     tmem_ld64_sync(tS + c64 * 64, sv);
                     if (!nomask) mask64(sv, lo, lim, c64 * 64);
                     exp_chunk(sv, mc, l2);
-                    pack_chunk(sv, 1.f, pk);
+                    pack_chunk(sv, 1.f, pk, lr2);
                     tmem_st32_sync(tS + c64 * 32, pk);
                 }
                 l = l2.x + l2.y;
+                f = ldexpf(1.f, ve);
             }
             tc_fence_before();
             mbar_arrive(&S.p_full[wg]);
-            if constexpr (BS != 64) {                  // the epilogue applies 2^-e / l
-                S.sc[i % kNSc][r] = valid ? ldexpf(1.f / l, -ve) : 0.f;
+            if constexpr (BS != 64) {                  // the epilogue applies 2^-e / lr
+                S.sc[i % kNSc][r] = valid ? ldexpf(1.f / (lr2.x + lr2.y), -ve) : 0.f;
                 mbar_arrive(&S.l_full[i % kNSc]);
             }
             if (valid)
                 p.part_meta[(size_t)tile_of(i) * kTileRows + r] =
-                    make_float2((mc + __log2f(l)) * kLn2, (float)ve);
+                    make_float2((mc + __log2f(l)) * kLn2, f);
         }
     } else {
         // ----------------------------------------------------------------- epilogue
@@ -574,10 +584,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     mbar_arrive(&S.o_free[ob]);
                 }
-                // the TMA store that last read this staging buffer is done
+                // staging buffers in turn over the halves of consecutive tiles; the TMA
+                // store that last read this one (kNSt halves ago) is done
+                const int hb = (i * NH + h) % kNSt;
                 if (lane == 0) bulk_wait_read<kNSt - 1>();
                 __syncwarp();
-                const uint32_t sb = smem_u32(S.stage[ew][h % kNSt]);
+                const uint32_t sb = smem_u32(S.stage[ew][hb]);
 #pragma unroll
                 for (int pc = 0; pc < 8; ++pc) {
                     const float* y = x + pc * 8;
@@ -595,10 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0 && nbox > 0) {
                     if (nbox == 4) {
-                        tma_store_2d(&omap32, S.stage[ew][h % kNSt], h * 64, prow0);
+                        tma_store_2d(&omap32, S.stage[ew][hb], h * 64, prow0);
                     } else {
                         for (int b = 0; b < nbox; ++b)
-                            tma_store_2d(&omap8, S.stage[ew][h % kNSt] + b * 1024, h * 64, prow0 + b * 8);
+                            tma_store_2d(&omap8, S.stage[ew][hb] + b * 1024, h * 64, prow0 + b * 8);
                     }
                     bulk_commit();
                 }

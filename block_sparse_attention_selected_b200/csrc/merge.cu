@@ -49,7 +49,7 @@ template <> __device__ __forceinline__ uint4 vzero<uint4>() { return make_uint4(
 // One warp per (token, query head) row.  Lane j (and j + 32) owns slot j: a slot whose
 // block is valid has its partial at row posmap * G + head offset of the forward tiles.
 // The block numbers and positions come in one round of requests, then the valid slots'
-// (lse_j, exponent_j) and partial rows (2 NH columns per lane) in a second: the row
+// (lse_j, factor_j) and partial rows (2 NH columns per lane) in a second: the row
 // costs two dependent memory latencies (d = 256 with topk > 16: further rounds of 16
 // partial rows, so that the loads in flight fit the registers).
 template <int kS, int NH, int F16>   // slots held by the warp: 16, 32 or 64 (>= topk)
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? (NH == 4 ? 2 :
     }
     const unsigned r0 = slot_row(b0, pos0);
     const unsigned r1 = kTopk32 ? 0xFFFFFFFFu : slot_row(b1, pos1);
-    // level 2: the (lse, exponent) of this lane's slots and every valid partial row
+    // level 2: the (lse, factor) of this lane's slots and every valid partial row
     float2 m0 = make_float2(-CUDART_INF_F, 0.f), m1 = m0;
     if (r0 != 0xFFFFFFFFu) m0 = __ldg(p.part_meta + r0);
     if (r1 != 0xFFFFFFFFu) m1 = __ldg(p.part_meta + r1);
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? (NH == 4 ? 2 :
     const float w0 = m0.x == -CUDART_INF_F ? 0.f : __expf(m0.x - M);
     const float w1 = m1.x == -CUDART_INF_F ? 0.f : __expf(m1.x - M);
     const float Lam = warp_sum(w0 + w1);
-    const float s0 = ldexpf(w0, (int)m0.y), s1 = ldexpf(w1, (int)m1.y);   // weight x 2^e
+    const float s0 = w0 * m0.y, s1 = w1 * m1.y;   // weight x the partial's factor
     float acc[2 * NH];
 #pragma unroll
     for (int q = 0; q < 2 * NH; ++q) acc[q] = 0.f;

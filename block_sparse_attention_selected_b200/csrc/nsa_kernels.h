@@ -93,8 +93,8 @@ struct FwdPlan {
     const int32_t* wtile_off;
     const int32_t* row_off;
     const int4* tile_desc;
-    void* part_o;            // fp16 [tiles * 128, d]: O_B / l_B * 2^-e, row tile * 128 + r
-    float2* part_meta;       // [tiles * 128]: (lse_B, e)
+    void* part_o;            // fp16 [tiles * 128, d]: the block's O over f, row tile * 128 + r
+    float2* part_meta;       // [tiles * 128]: (lse_B, f)
     const int32_t* vexp;     // [hkv * NB]: exponent e of each (g, B) block's V
     DevStatus* st;
     int num_sms;

@@ -87,3 +87,19 @@ def test_bwd_head_dim_other_than_128_is_refused():
         nsa.nsa_sel_attn_bwd(t["q"], t["k"], t["v"], out, lse, t["dout"], t["cu"], t["bidx"], 64,
                              p.scale)
     assert e.value.code == 2   # NSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_fwd_head_dim_repeat_calls_bitwise_identical(d):
+    # many back-to-back calls must reproduce the first bit for bit (a hand-off hazard in
+    # the pipeline -- a staging buffer reused before its store has read it, a barrier
+    # parity that aliases -- shows as an occasional difference)
+    p = ni.make_problem([8192], hq=16, hkv=4, head_dim=d, block_size=64, topk=16, seed=111,
+                        with_dout=False)
+    t = to_device(p)
+    o0, l0 = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, p.scale)
+    for _ in range(40):
+        o, l = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, p.scale)
+        assert torch.equal(o, o0) and torch.equal(l, l0)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
