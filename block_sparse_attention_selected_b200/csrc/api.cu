@@ -35,7 +35,7 @@ struct Dims {
 struct Layout {
     size_t status, blkoff, keys0, keys1, vals0, vals1, hist, digit_tot, offsets, tile_off, chunk_off;
     size_t inv_end;   // end of the regions the index inversion (InvertPlan) uses
-    size_t win_rng, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
+    size_t wstart, wtile_off, row_tiles, row_off, tile_desc, posmap, vexp;
     size_t part_o, part_lse, delta, part_dkdv, udesc, ubucket, uorder;
     size_t total;
 };
@@ -97,7 +97,7 @@ Layout make_layout(const Dims& D, bool bwd) {
     L.chunk_off = take(sizeof(int32_t) * ((size_t)D.nbk_cap + 1));
     L.inv_end = o;   // everything the inversion alone touches lies below this offset
     const size_t wrows = (size_t)D.hkv * D.nwin;
-    L.win_rng = take(sizeof(int2) * wrows * (size_t)D.nb_stride);
+    L.wstart = take(sizeof(int32_t) * (wrows * (size_t)D.nb_stride + 1));
     L.wtile_off = take(sizeof(int32_t) * wrows * ((size_t)D.nb_stride + 1));
     L.row_tiles = take(sizeof(int32_t) * wrows);
     L.row_off = take(sizeof(int32_t) * (wrows + 1));
@@ -245,6 +245,9 @@ Carved carve(const Dims& D, const Layout& L, void* ws, const int32_t* cu, const 
     p.offsets = reinterpret_cast<int32_t*>(b + L.offsets);
     p.tile_off = reinterpret_cast<int32_t*>(b + L.tile_off);
     p.chunk_off = reinterpret_cast<int32_t*>(b + L.chunk_off);
+    p.wstart = nullptr;   // set by the forward, which needs the window runs
+    p.nwin = 1;
+    p.wtok = 1;
     p.st = c.st;
     // identity of the inversion's inputs: the index arrays and every size it depends on
     unsigned long long h = 1469598103934665603ull;
@@ -361,12 +364,14 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16, D.d) ||
         !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16, D.d))
         return NSA_ERR_CUDA;
+    c.inv.wstart = reinterpret_cast<int32_t*>(c.base + L.wstart);
+    c.inv.nwin = D.nwin;
+    c.inv.wtok = D.wtok;
     if ((s = cuda_status(launch_invert(c.inv, stream))) != NSA_OK) return s;
     WindowPlan wp{};
     wp.nwin = D.nwin;
     wp.wtok = D.wtok;
     wp.nb_stride = D.nb_stride;
-    wp.win_rng = reinterpret_cast<int2*>(c.base + L.win_rng);
     wp.tile_off = reinterpret_cast<int32_t*>(c.base + L.wtile_off);
     wp.row_tiles = reinterpret_cast<int32_t*>(c.base + L.row_tiles);
     wp.row_off = reinterpret_cast<int32_t*>(c.base + L.row_off);
@@ -375,7 +380,7 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     if ((s = cuda_status(launch_window_split(c.inv, wp, stream))) != NSA_OK) return s;
     int32_t* posmap = reinterpret_cast<int32_t*>(c.base + L.posmap);
     if ((s = cuda_status(launch_posmap(c.inv, wp, posmap, stream))) != NSA_OK) return s;
-    pm.add(invert_launches(D) + 5);
+    pm.add(invert_launches(D) + 4);
     pm.mark(1);
 
     FwdPlan fp{};
@@ -394,7 +399,6 @@ nsa_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t
     fp.nbk_cap = D.nbk_cap;
     fp.nwin = wp.nwin;
     fp.nb_stride = wp.nb_stride;
-    fp.win_rng = wp.win_rng;
     fp.wtile_off = wp.tile_off;
     fp.row_off = wp.row_off;
     fp.tile_desc = wp.tile_desc;

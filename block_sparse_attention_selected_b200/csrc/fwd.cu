@@ -628,8 +628,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Per (KV head g, global block B): e = 0 unless max |V_B| > 2^14, then the exponent
-// that brings it under 2^15 (fp16 partials of O / l stay finite).  One block of d
-// threads per (B, g), thread = column.
+// that brings it under 2^15 (fp16 partials of O / l stay finite).  One CTA of 256
+// threads per (B, g) reads the block as 16-byte chunks: d / 8 threads per key row,
+// 256 / (d / 8) rows per pass, the loads of four passes in flight together.
 __global__ void __launch_bounds__(256) k_vblock_exp(const __nv_bfloat16* v, const int32_t* cu,
                                                     int nseq, int hkv, int d, int bs,
                                                     const int32_t* blkoff, const DevStatus* st,
@@ -641,9 +642,22 @@ __global__ void __launch_bounds__(256) k_vblock_exp(const __nv_bfloat16* v, cons
     const int s = upper_index(blkoff, nseq, B);
     const int key0 = __ldg(cu + s) + (B - __ldg(blkoff + s)) * bs;
     const int kend = min(key0 + bs, __ldg(cu + s + 1));
+    const int cpr = d >> 3;                       // 16-byte chunks per key row
+    const int rpp = (int)blockDim.x / cpr;        // key rows per pass
+    const int r = (int)threadIdx.x / cpr, c = (int)threadIdx.x - r * cpr;
+    const uint4* base = reinterpret_cast<const uint4*>(v + (size_t)g * d) + c;
+    const size_t row_stride = (size_t)hkv * d / 8;   // in 16-byte chunks
     float m = 0.f;
-    for (int key = key0; key < kend; ++key)
-        m = fmaxf(m, fabsf(__bfloat162float(v[((size_t)key * hkv + g) * d + threadIdx.x])));
+#pragma unroll 4
+    for (int key = key0 + r; key < kend; key += rpp) {
+        const uint4 x = __ldg(base + (size_t)key * row_stride);
+        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[k2]));
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
     __syncthreads();
@@ -661,7 +675,7 @@ cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, in
     if (p.T > 0 && nb_stride > 0) {
         if (p.f16)   // |V| <= 65504 already fits the fp16 partials: every exponent is 0
             return cudaMemsetAsync(vexp, 0, sizeof(int32_t) * (size_t)p.hkv * nb_stride, stream);
-        k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), (unsigned)p.d, 0, stream>>>(
+        k_vblock_exp<<<dim3((unsigned)nb_stride, (unsigned)p.hkv), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(v), p.cu, p.nseq, p.hkv, p.d, p.bs, p.blkoff, p.st,
             vexp);
     }

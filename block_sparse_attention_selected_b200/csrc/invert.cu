@@ -12,9 +12,11 @@
 //
 // Steps (all on the caller's stream, no host synchronisation):
 //   1. k_seq_blocks      global block offset of every sequence, cu_seqlens check
-//   2. per 8-bit digit:  k_sort_hist -> k_scan_digits -> k_sort_scatter (LSD radix,
-//                        stable: warp-ordered ranks with __match_any_sync)
-//   3. k_bucket_offsets  CSR offsets from the sorted keys
+//   2. per digit (at most 8 bits, the key's bits split evenly over the passes):
+//                        k_sort_hist -> k_scan_digits -> k_sort_scatter (LSD radix,
+//                        stable: warp-ordered ranks from per-bit ballots)
+//   3. k_run_offsets     CSR offsets from the sorted keys (and, for the forward, the
+//                        start of every (bucket, token window) run)
 //   4. k_tile_offsets    per-bucket 128-row tile and backward-chunk prefix sums
 #include "nsa_common.cuh"
 #include "nsa_kernels.h"
@@ -30,6 +32,7 @@ constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 struct SortArgs {
     const int32_t* cu;
     int nseq, T, hkv, topk, bs;
+    int bs_log2;             // block sizes are powers of two
     int swin;                // sliding window in keys, 0: none
     const int32_t* bidx;
     long long nent;
@@ -90,56 +93,93 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
     }
     if (threadIdx.x == 0) {
         blkoff[nseq] = (int32_t)carry;
-        st->nblocks_total = (int)carry;
+        // invalid cu_seqlens: no blocks, so no later table outgrows its T / bs + nseq rows
+        st->nblocks_total = bad ? 0 : (int)carry;
         st->index_tag = tag;
         if (bad) record_error(st, NSA_ERR_BAD_INDEX, 1);
     }
 }
 
-// Bucket key of entry e (token-major, then KV head, then slot); kInvalidKey if the
-// entry selects nothing (padding, future or out-of-range block, or a block that lies
-// wholly before the sliding window).
-__device__ __forceinline__ uint32_t entry_key(const SortArgs& a, long long e, uint32_t nbtot,
-                                              uint32_t* val) {
-    int j, g, t;
-    if (a.nent <= 0x7FFFFFFFll) {   // 32-bit division (the 64-bit one is far longer)
-        const uint32_t e32 = (uint32_t)e, tk = (uint32_t)a.topk, hk = (uint32_t)a.hkv;
-        const uint32_t r = e32 / tk;
-        j = (int)(e32 - r * tk);
-        t = (int)(r / hk);
-        g = (int)(r - (uint32_t)t * hk);
-    } else {
-        j = (int)(e % a.topk);
-        const long long r = e / a.topk;
-        g = (int)(r % a.hkv);
-        t = (int)(r / a.hkv);
+// Position of entry e = (t * hkv + g) * topk + j (token-major, then KV head, then
+// slot) in its row, and the sequence that holds its token.  A thread walks its entries
+// with a fixed stride, so the position advances by a precomputed (dt, dg, dj) with one
+// carry per level and the sequence by a forward scan of cu_seqlens: no division and
+// no search per entry.
+struct EntryCursor {
+    int t, g, j;             // token, KV head, slot
+    int s, seq0, seq1, blk;  // sequence of t, its token range [seq0, seq1), global block offset
+    int dt, dg, dj;          // the stride, decomposed like an entry index
+
+    __device__ __forceinline__ void init(const SortArgs& a, long long e, int stride) {
+        const long long rowk = (long long)a.hkv * a.topk;
+        t = (int)(e / rowk);
+        const int r = (int)(e - (long long)t * rowk);
+        g = r / a.topk;
+        j = r - g * a.topk;
+        dt = stride / (int)rowk;
+        const int rs = stride - dt * (int)rowk;
+        dg = rs / a.topk;
+        dj = rs - dg * a.topk;
+        s = t < a.T ? seq_of_token(a.cu, a.nseq, t) : a.nseq - 1;
+        seq0 = __ldg(a.cu + s);
+        seq1 = __ldg(a.cu + s + 1);
+        blk = __ldg(a.blkoff + s);
     }
-    *val = (uint32_t)t * 64u + (uint32_t)j;
-    int b = __ldg(a.bidx + e);
-    int s = seq_of_token(a.cu, a.nseq, t);
-    int i = t - __ldg(a.cu + s);
-    int qb = i >= 0 ? i / a.bs : -1;
-    if (!block_valid(b, qb, i, a.bs, a.swin)) return kInvalidKey;
-    uint32_t key = (uint32_t)g * nbtot + (uint32_t)__ldg(a.blkoff + s) + (uint32_t)b;
-    return key < (uint32_t)a.nbk_cap ? key : kInvalidKey;
-}
+    __device__ __forceinline__ void advance(const SortArgs& a) {
+        j += dj;
+        int c = j >= a.topk;
+        j -= c ? a.topk : 0;
+        g += dg + c;
+        c = g >= a.hkv;
+        g -= c ? a.hkv : 0;
+        t += dt + c;
+    }
+    // the bucket key g * NB + global block of block b (kInvalidKey if it selects
+    // nothing: padding, a future or out-of-range block, or a block wholly before the
+    // sliding window); t must be < T
+    __device__ __forceinline__ uint32_t key(const SortArgs& a, int b, uint32_t nbtot) {
+        while (t >= seq1 && s + 1 < a.nseq) {
+            ++s;
+            seq0 = seq1;
+            seq1 = __ldg(a.cu + s + 1);
+            blk = __ldg(a.blkoff + s);
+        }
+        const int i = t - seq0;
+        const int qb = i >> a.bs_log2;
+        if (!block_valid(b, qb, i, a.bs, a.swin)) return kInvalidKey;
+        const uint32_t k = (uint32_t)g * nbtot + (uint32_t)blk + (uint32_t)b;
+        return k < (uint32_t)a.nbk_cap ? k : kInvalidKey;
+    }
+    __device__ __forceinline__ uint32_t val() const { return (uint32_t)t * 64u + (uint32_t)j; }
+};
 
 // 2a. per-tile digit histogram, stored digit-major: hist[d * ntiles + tile].
 template <bool kFirst>
 __global__ void __launch_bounds__(kSortThreads) k_sort_hist(SortArgs a, const uint32_t* keys_in,
-                                                           int shift, uint32_t* hist) {
+                                                           int shift, uint32_t mask, uint32_t* hist) {
     __shared__ uint32_t h[256];
     h[threadIdx.x] = 0;
+    const long long base = (long long)blockIdx.x * kSortTile + threadIdx.x;
+    const int nitems = a.nent > base ? (int)min((long long)kItems, (a.nent - base + kSortThreads - 1) / kSortThreads) : 0;
+    const uint32_t* src = (kFirst ? reinterpret_cast<const uint32_t*>(a.bidx) : keys_in) + base;
+    // every load of the thread first (independent loads in flight together)
+    uint32_t x[kItems];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) x[it] = it < nitems ? __ldg(src + it * kSortThreads) : 0u;
     __syncthreads();
-    const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
-    const long long base = (long long)blockIdx.x * kSortTile;
-    for (int it = 0; it < kItems; ++it) {
-        long long e = base + it * kSortThreads + threadIdx.x;
-        if (e < a.nent) {
-            uint32_t v;
-            uint32_t key = kFirst ? entry_key(a, e, nbtot, &v) : keys_in[e];
-            atomicAdd(&h[(key >> shift) & 255u], 1u);
+    if (kFirst) {
+        const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
+        EntryCursor c;
+        c.init(a, base, kSortThreads);
+#pragma unroll
+        for (int it = 0; it < kItems; ++it) {
+            if (it < nitems) atomicAdd(&h[(c.key(a, (int)x[it], nbtot) >> shift) & mask], 1u);
+            c.advance(a);
         }
+    } else {
+#pragma unroll
+        for (int it = 0; it < kItems; ++it)
+            if (it < nitems) atomicAdd(&h[(x[it] >> shift) & mask], 1u);
     }
     __syncthreads();
     hist[(size_t)threadIdx.x * gridDim.x + blockIdx.x] = h[threadIdx.x];
@@ -166,15 +206,16 @@ __global__ void __launch_bounds__(1024) k_scan_digits(uint32_t* hist, int ntiles
     if (threadIdx.x == blockDim.x - 1) digit_tot[blockIdx.x] = (uint32_t)incl;
 }
 
-// 2c. stable scatter of one tile by the digit at `shift`.  Entries are ranked within
-//     the tile (warp-ordered ranks with __match_any_sync, then the warps in order), put
+// 2c. stable scatter of one tile by the digit (key >> shift) & mask.  Entries are ranked within
+//     the tile (warp-ordered ranks from one ballot per digit bit, then the warps in order), put
 //     into shared memory in the tile's digit order, and written out from there: thread
 //     k stores the tile's k-th entry of that order, so each digit's run of the tile
 //     goes to consecutive global addresses (coalesced) instead of one scattered word
 //     per entry.
 template <bool kFirst>
-__global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const uint32_t* keys_in,
+__global__ void __launch_bounds__(kSortThreads, 3) k_sort_scatter(SortArgs a, const uint32_t* keys_in,
                                                               const uint32_t* vals_in, int shift,
+                                                              uint32_t mask,
                                                               const uint32_t* hist_scan,
                                                               const uint32_t* digit_tot,
                                                               uint32_t* keys_out,
@@ -183,8 +224,20 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const
     __shared__ uint32_t tile_base[256];      // global start of each digit's run of this tile
     __shared__ uint32_t local_start[256];    // start of each digit's run within the tile
     __shared__ unsigned long long warp_tot[32];
-    __shared__ uint2 stage[kSortTile];       // (key, value) in the tile's digit order
+    __shared__ uint32_t stage_k[kSortTile];  // keys in the tile's digit order
+    __shared__ uint32_t stage_v[kSortTile];  // their values
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const long long tile0 = (long long)blockIdx.x * kSortTile;
+    const long long base = tile0 + (long long)w * (kItems * 32) + lane;
+    const int nvalid = (int)min((long long)kSortTile, a.nent - tile0);
+    const int nitems = a.nent > base ? (int)min((long long)kItems, (a.nent - base + 31) / 32) : 0;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint32_t* src = (kFirst ? reinterpret_cast<const uint32_t*>(a.bidx) : keys_in) + base;
+    // every key of the lane first (independent loads in flight together, and in flight
+    // during the prologue), then the warp-ordered ranks
+    uint32_t key[kItems], pos[kItems];
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) key[it] = it < nitems ? __ldg(src + it * 32) : 0u;
     for (int i = tid; i < kSortWarps * 256; i += kSortThreads) (&whist[0][0])[i] = 0;
     {   // start of digit tid in the output = totals of smaller digits + earlier tiles
         const uint32_t tot = digit_tot[tid];
@@ -192,24 +245,30 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const
         tile_base[tid] = (uint32_t)(incl - tot) + hist_scan[(size_t)tid * gridDim.x + blockIdx.x];
     }
     __syncthreads();
-    const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
-    const long long tile0 = (long long)blockIdx.x * kSortTile;
-    const long long base = tile0 + (long long)w * (kItems * 32);
-    const int nvalid = (int)min((long long)kSortTile, a.nent - tile0);
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t key[kItems], val[kItems], rank[kItems];
+    if (kFirst) {
+        const uint32_t nbtot = (uint32_t)a.st->nblocks_total;
+        EntryCursor c;
+        c.init(a, base, 32);
+#pragma unroll
+        for (int it = 0; it < kItems; ++it) {
+            if (it < nitems) key[it] = c.key(a, (int)key[it], nbtot);
+            c.advance(a);
+        }
+    }
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {
-        long long e = base + it * 32 + lane;
-        uint32_t d = 256u;   // sentinel for entries past the end
-        if (e < a.nent) {
-            key[it] = kFirst ? entry_key(a, e, nbtot, &val[it]) : keys_in[e];
-            if (!kFirst) val[it] = vals_in[e];
-            d = (key[it] >> shift) & 255u;
+        const uint32_t d = it < nitems ? (key[it] >> shift) & mask : 256u;   // 256: past the end
+        // lanes with the same digit: a ballot per digit bit (cheaper than match.any)
+        uint32_t peers = __ballot_sync(0xFFFFFFFFu, d < 256u);
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            if ((mask >> b) == 0u) break;
+            const uint32_t bit = (d >> b) & 1u;
+            const uint32_t ones = __ballot_sync(0xFFFFFFFFu, bit);
+            peers &= bit ? ones : ~ones;
         }
-        uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
-        uint32_t before = __popc(peers & lt_mask);
-        if (d < 256u) rank[it] = whist[w][d] + before;
+        const uint32_t before = __popc(peers & lt_mask);
+        if (d < 256u) pos[it] = whist[w][d] + before;
         __syncwarp();
         if (d < 256u && before == 0) whist[w][d] += __popc(peers);
         __syncwarp();
@@ -219,41 +278,100 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_scatter(SortArgs a, const
         // start within the tile (a scan over the digits)
         uint32_t run = 0;
         for (int ww = 0; ww < kSortWarps; ++ww) {
-            uint32_t c = whist[ww][tid];
+            uint32_t cnt = whist[ww][tid];
             whist[ww][tid] = run;
-            run += c;
+            run += cnt;
         }
         const unsigned long long incl = block_incl_scan_u64(run, warp_tot);
         local_start[tid] = (uint32_t)(incl - run);
     }
     __syncthreads();
+    // the keys into their staging slots, then the values (loaded together)
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {
-        long long e = base + it * 32 + lane;
-        if (e < a.nent) {
-            uint32_t d = (key[it] >> shift) & 255u;
-            stage[local_start[d] + whist[w][d] + rank[it]] = make_uint2(key[it], val[it]);
+        if (it < nitems) {
+            const uint32_t d = (key[it] >> shift) & mask;
+            pos[it] += local_start[d] + whist[w][d];
+            stage_k[pos[it]] = key[it];
         }
+    }
+    if (kFirst) {
+        EntryCursor c;
+        c.init(a, base, 32);
+#pragma unroll
+        for (int it = 0; it < kItems; ++it) {
+            if (it < nitems) stage_v[pos[it]] = c.val();
+            c.advance(a);
+        }
+    } else {
+        const uint32_t* vsrc = vals_in + base;
+#pragma unroll
+        for (int it = 0; it < kItems; ++it) key[it] = it < nitems ? __ldg(vsrc + it * 32) : 0u;
+#pragma unroll
+        for (int it = 0; it < kItems; ++it)
+            if (it < nitems) stage_v[pos[it]] = key[it];
     }
     __syncthreads();
     for (int k = tid; k < nvalid; k += kSortThreads) {
-        const uint2 kv = stage[k];
-        const uint32_t d = (kv.x >> shift) & 255u;
-        const uint32_t pos = tile_base[d] + (uint32_t)k - local_start[d];
-        keys_out[pos] = kv.x;
-        vals_out[pos] = kv.y;
+        const uint32_t kk = stage_k[k];
+        const uint32_t d = (kk >> shift) & mask;
+        const uint32_t at = tile_base[d] + (uint32_t)k - local_start[d];
+        keys_out[at] = kk;
+        vals_out[at] = stage_v[k];
     }
 }
 
-// 3. offsets[B] = number of sorted keys below B, for B in [0, hkv * NB].
-__global__ void k_bucket_offsets(const uint32_t* keys, long long nent, const DevStatus* st,
-                                 int hkv, int32_t* offsets) {
-    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i > nent) return;
-    const long long nbk = (long long)hkv * st->nblocks_total;
-    long long prev = i == 0 ? -1 : min((long long)keys[i - 1], nbk);
-    long long cur = i == nent ? nbk : min((long long)keys[i], nbk);
-    for (long long B = prev + 1; B <= cur; ++B) offsets[B] = (int32_t)i;
+// 3. Run offsets of the sorted list.  offsets[B] = number of sorted keys below B, for
+//    B in [0, hkv * NB].  With a window table (the forward), also the start of every
+//    (bucket, token window) run: entries are sorted by bucket and, within a bucket, by
+//    token, so the composite c = bucket * nwin + window of the token is ascending too,
+//    and wstart[c] = number of entries whose composite is below c, for c in
+//    [0, hkv * NB * nwin].  Entries of invalid key sort last and count as c = the end.
+__device__ __forceinline__ int run_code(uint32_t key, uint32_t val, int nbk, int nwin, uint32_t wtok) {
+    const int k = (int)min(key, (uint32_t)nbk);
+    if (k == nbk || nwin == 1) return k * nwin;
+    return k * nwin + min((int)((val >> 6) / wtok), nwin - 1);
+}
+
+// Four consecutive entries per thread (one 16-byte load of keys and of values).
+__global__ void k_run_offsets(const uint32_t* keys, const uint32_t* vals, long long nent,
+                              const DevStatus* st, int hkv, int nwin, int wtok, int32_t* offsets,
+                              int32_t* wstart) {
+    const long long i0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (i0 > nent) return;
+    const int nbk = hkv * st->nblocks_total;
+    const int cend = nbk * nwin;   // code of the end (and of invalid keys)
+    const bool wins = nwin > 1;
+    uint32_t k[5], v[5];           // entries i0 - 1 .. i0 + 3
+    if (i0 + 4 <= nent) {
+        const uint4 kk = __ldg(reinterpret_cast<const uint4*>(keys + i0));
+        k[1] = kk.x; k[2] = kk.y; k[3] = kk.z; k[4] = kk.w;
+        if (wins) {
+            const uint4 vv = __ldg(reinterpret_cast<const uint4*>(vals + i0));
+            v[1] = vv.x; v[2] = vv.y; v[3] = vv.z; v[4] = vv.w;
+        }
+    } else {
+#pragma unroll
+        for (int q = 1; q < 5; ++q) {
+            k[q] = i0 + q - 1 < nent ? __ldg(keys + i0 + q - 1) : 0u;
+            v[q] = wins && i0 + q - 1 < nent ? __ldg(vals + i0 + q - 1) : 0u;
+        }
+    }
+    k[0] = i0 > 0 ? __ldg(keys + i0 - 1) : 0u;
+    v[0] = wins && i0 > 0 ? __ldg(vals + i0 - 1) : 0u;
+    int prev = i0 > 0 ? run_code(k[0], v[0], nbk, nwin, (uint32_t)wtok) : -1;
+#pragma unroll
+    for (int q = 1; q < 5; ++q) {
+        const long long i = i0 + q - 1;
+        if (i > nent) break;
+        const int cur = i < nent ? run_code(k[q], v[q], nbk, nwin, (uint32_t)wtok) : cend;
+        for (int c = prev + 1; c <= cur; ++c) {
+            if (wstart) wstart[c] = (int32_t)i;
+            if (!wins) offsets[c] = (int32_t)i;
+            else if (c % nwin == 0) offsets[c / nwin] = (int32_t)i;
+        }
+        prev = cur;
+    }
 }
 
 // 4. tile and chunk prefix sums per bucket; totals into the status block.
@@ -268,10 +386,10 @@ __global__ void __launch_bounds__(1024) k_tile_offsets(const int32_t* offsets, D
         long long B = base + threadIdx.x;
         unsigned long long x = 0;
         if (B < nbk) {
-            long long cnt = offsets[B + 1] - offsets[B];
-            unsigned long long nt = (unsigned long long)((cnt + tpt - 1) / tpt);
-            unsigned long long nc = (nt + chunk_tiles - 1) / chunk_tiles;
-            x = (nc << 32) | nt;
+            const uint32_t cnt = (uint32_t)(offsets[B + 1] - offsets[B]);
+            const uint32_t nt = (cnt + (uint32_t)tpt - 1u) / (uint32_t)tpt;
+            const uint32_t nc = (nt + (uint32_t)chunk_tiles - 1u) / (uint32_t)chunk_tiles;
+            x = ((unsigned long long)nc << 32) | nt;
         }
         unsigned long long incl = block_incl_scan_u64(x, warp_tot);
         unsigned long long ex = carry + incl - x;
@@ -293,52 +411,32 @@ __global__ void __launch_bounds__(1024) k_tile_offsets(const int32_t* offsets, D
     }
 }
 
-// 5. Window split for the forward's tile order.  Tokens are cut into windows of
-//    `wtok` (packed) tokens; for every (g, window w, global block B) the sub-range of
-//    the (g, B) list whose tokens lie in w (the list is sorted by token, so it is a
-//    contiguous run found by binary search on the entry value token * 64 + slot).
-//    win_rng[(g * nwin + w) * nb_stride + B] = (first entry, count).
-__device__ __forceinline__ int lower_bound_u32(const uint32_t* a, int lo, int hi, uint32_t x) {
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(a + mid) < x) lo = mid + 1; else hi = mid;
-    }
-    return lo;
-}
-
-__global__ void k_window_split(const uint32_t* entries, const int32_t* offsets, const DevStatus* st,
-                               int hkv, int nwin, int wtok, int nb_stride, int2* win_rng) {
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const int nbtot = st->nblocks_total;
-    const long long n = (long long)hkv * nwin * nbtot;
-    if (idx >= n) return;
-    const int B = (int)(idx % nbtot);
-    const long long r = idx / nbtot;          // (g * nwin + w)
-    const int w = (int)(r % nwin);
-    const int g = (int)(r / nwin);
-    const int lo = offsets[g * nbtot + B], hi = offsets[g * nbtot + B + 1];
-    const uint32_t v0 = (uint32_t)w * (uint32_t)wtok * 64u;
-    const uint32_t v1 = (uint32_t)(w + 1) * (uint32_t)wtok * 64u;
-    const int a = lower_bound_u32(entries, lo, hi, v0);
-    const int b = (w + 1 == nwin) ? hi : lower_bound_u32(entries, a, hi, v1);
-    win_rng[r * nb_stride + B] = make_int2(a, b - a);
+// 5. Window runs for the forward's tile order.  Tokens are cut into windows of `wtok`
+//    (packed) tokens; the run of the (g, B) list whose tokens lie in window w is
+//    [wstart[c], wstart[c + 1]) with c = (g * NB + B) * nwin + w (k_run_offsets).
+__device__ __forceinline__ int2 window_run(const int32_t* wstart, int nbtot, int nwin, int g,
+                                           int w, int B) {
+    const size_t c = ((size_t)g * nbtot + B) * nwin + w;
+    const int a = __ldg(wstart + c);
+    return make_int2(a, __ldg(wstart + c + 1) - a);
 }
 
 // 6. Per (g, w) row: exclusive scan over B of ceil(count / tpt) tiles, and the row's
 //    total.  One block per row.
-__global__ void __launch_bounds__(1024) k_window_tiles(const int2* win_rng, const DevStatus* st,
-                                                       int nb_stride, int tpt, int32_t* tile_off,
-                                                       int32_t* row_tiles) {
+__global__ void __launch_bounds__(1024) k_window_tiles(const int32_t* wstart, const DevStatus* st,
+                                                       int nwin, int nb_stride, int tpt,
+                                                       int32_t* tile_off, int32_t* row_tiles) {
     __shared__ unsigned long long warp_tot[32];
     __shared__ unsigned long long round_total;
     const int nbtot = st->nblocks_total;
-    const int2* rng = win_rng + (size_t)blockIdx.x * nb_stride;
+    const int g = blockIdx.x / nwin, w = blockIdx.x - g * nwin;
     int32_t* out = tile_off + (size_t)blockIdx.x * (nb_stride + 1);
     unsigned long long carry = 0;
     for (int base = 0; base < nbtot; base += blockDim.x) {
         const int B = base + threadIdx.x;
         unsigned long long x = 0;
-        if (B < nbtot) x = (unsigned long long)((rng[B].y + tpt - 1) / tpt);
+        if (B < nbtot)
+            x = (unsigned long long)((window_run(wstart, nbtot, nwin, g, w, B).y + tpt - 1) / tpt);
         const unsigned long long incl = block_incl_scan_u64(x, warp_tot);
         if (B < nbtot) out[B] = (int32_t)(carry + incl - x);
         if (threadIdx.x == blockDim.x - 1) round_total = incl;
@@ -378,7 +476,7 @@ __global__ void __launch_bounds__(1024) k_row_offsets(const int32_t* row_tiles, 
 //    geometry with one load instead of three dependent binary searches:
 //    (first key of the block, first entry, nrows | g << 8, g * NB + B).
 __global__ void k_tile_desc(const DevStatus* st, const int32_t* row_off, const int32_t* tile_off,
-                            const int2* win_rng, const int32_t* blkoff, const int32_t* cu,
+                            const int32_t* wstart, const int32_t* blkoff, const int32_t* cu,
                             int nseq, int hkv, int nwin, int nb_stride, int G, int bs,
                             int4* desc) {
     const int tile = blockIdx.x * blockDim.x + threadIdx.x;
@@ -388,9 +486,9 @@ __global__ void k_tile_desc(const DevStatus* st, const int32_t* row_off, const i
     const int tr = tile - row_off[row];
     const int32_t* toff = tile_off + (size_t)row * (nb_stride + 1);
     const int B = upper_index(toff, nbtot, tr);
-    const int2 rng = win_rng[(size_t)row * nb_stride + B];
     const int tpt = kTileRows / G;
     const int g = row / nwin;
+    const int2 rng = window_run(wstart, nbtot, nwin, g, row - g * nwin, B);
     const int s = upper_index(blkoff, nseq, B);
     const int key0 = cu[s] + (B - blkoff[s]) * bs;
     const int e0 = rng.x + (tr - toff[B]) * tpt;
@@ -507,32 +605,48 @@ int invert_final_buf(const InvertPlan& p) {
 
 cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
     k_seq_blocks<<<1, 1024, 0, stream>>>(p.cu, p.nseq, p.T, p.bs, p.blkoff, p.st, p.tag);
-    SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, p.swin, p.bidx, p.nent, p.nbk_cap, p.blkoff, p.st};
+    int bs_log2 = 0;
+    while ((2 << bs_log2) <= p.bs) ++bs_log2;   // p.bs is a power of two (64 or 128)
+    SortArgs a{p.cu, p.nseq, p.T, p.hkv, p.topk, p.bs, bs_log2, p.swin, p.bidx, p.nent,
+               p.nbk_cap, p.blkoff, p.st};
+    // digits of at most 8 bits, split evenly over the passes (13 bits: 7 + 6), so that
+    // every pass scatters runs of similar length
     const int passes = p.key_bits <= 8 ? 1 : (p.key_bits + 7) / 8;
     const uint32_t* kin = nullptr;
     const uint32_t* vin = nullptr;
+    int shift = 0;
+    // the scatter's 42 KB of static shared memory: ask for the largest carveout so that
+    // three CTAs fit on an SM
+    cudaFuncSetAttribute(k_sort_scatter<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    cudaFuncSetAttribute(k_sort_scatter<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     for (int pass = 0; pass < passes; ++pass) {
-        const int shift = 8 * pass;
+        const int bits = p.key_bits / passes + (pass < p.key_bits % passes ? 1 : 0);
+        const uint32_t mask = (1u << bits) - 1u;
         uint32_t* kout = p.keys[pass & 1];
         uint32_t* vout = p.vals[pass & 1];
         if (pass == 0)
-            k_sort_hist<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, nullptr, shift, p.hist);
+            k_sort_hist<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, nullptr, shift, mask, p.hist);
         else
-            k_sort_hist<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, shift, p.hist);
+            k_sort_hist<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(a, kin, shift, mask, p.hist);
         k_scan_digits<<<256, 1024, 0, stream>>>(p.hist, p.sort_tiles, p.digit_tot);
         if (pass == 0)
             k_sort_scatter<true><<<p.sort_tiles, kSortThreads, 0, stream>>>(
-                a, nullptr, nullptr, shift, p.hist, p.digit_tot, kout, vout);
+                a, nullptr, nullptr, shift, mask, p.hist, p.digit_tot, kout, vout);
         else
             k_sort_scatter<false><<<p.sort_tiles, kSortThreads, 0, stream>>>(
-                a, kin, vin, shift, p.hist, p.digit_tot, kout, vout);
+                a, kin, vin, shift, mask, p.hist, p.digit_tot, kout, vout);
         kin = kout;
         vin = vout;
+        shift += bits;
     }
     p.final_buf = invert_final_buf(p);
     const long long n1 = p.nent + 1;
-    k_bucket_offsets<<<(unsigned)((n1 + 255) / 256), 256, 0, stream>>>(p.keys[p.final_buf], p.nent,
-                                                                      p.st, p.hkv, p.offsets);
+    const long long nthr = (n1 + 3) / 4;
+    k_run_offsets<<<(unsigned)((nthr + 255) / 256), 256, 0, stream>>>(
+        p.keys[p.final_buf], p.vals[p.final_buf], p.nent, p.st, p.hkv, p.wstart ? p.nwin : 1,
+        p.wtok, p.offsets, p.wstart);
     k_tile_offsets<<<1, 1024, 0, stream>>>(p.offsets, p.st, p.hkv, p.tokens_per_tile,
                                            p.chunk_tiles, p.tile_off, p.chunk_off);
     return cudaGetLastError();
@@ -540,14 +654,12 @@ cudaError_t launch_invert(InvertPlan& p, cudaStream_t stream) {
 
 cudaError_t launch_window_split(const InvertPlan& p, const WindowPlan& w, cudaStream_t stream) {
     const int nrows = p.hkv * w.nwin;
-    const long long n = (long long)nrows * w.nb_stride;      // upper bound (device NB <= stride)
-    k_window_split<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
-        p.vals[p.final_buf], p.offsets, p.st, p.hkv, w.nwin, w.wtok, w.nb_stride, w.win_rng);
-    k_window_tiles<<<nrows, 1024, 0, stream>>>(w.win_rng, p.st, w.nb_stride, p.tokens_per_tile,
-                                               w.tile_off, w.row_tiles);
+    if (!p.wstart || p.nwin != w.nwin || p.wtok != w.wtok) return cudaErrorInvalidValue;
+    k_window_tiles<<<nrows, 1024, 0, stream>>>(p.wstart, p.st, w.nwin, w.nb_stride,
+                                               p.tokens_per_tile, w.tile_off, w.row_tiles);
     k_row_offsets<<<1, 1024, 0, stream>>>(w.row_tiles, nrows, w.row_off, p.st);
     k_tile_desc<<<(unsigned)((w.tiles_cap + 255) / 256), 256, 0, stream>>>(
-        p.st, w.row_off, w.tile_off, w.win_rng, p.blkoff, p.cu, p.nseq, p.hkv, w.nwin, w.nb_stride,
+        p.st, w.row_off, w.tile_off, p.wstart, p.blkoff, p.cu, p.nseq, p.hkv, w.nwin, w.nb_stride,
         kTileRows / p.tokens_per_tile, p.bs, w.tile_desc);
     return cudaGetLastError();
 }

@@ -35,6 +35,10 @@ struct InvertPlan {
     int32_t* offsets;        // [nbk_cap + 1]
     int32_t* tile_off;       // [nbk_cap + 1]
     int32_t* chunk_off;      // [nbk_cap + 1]
+    // forward only (null otherwise): the start of every (bucket, token window) run,
+    // [hkv * NB * nwin + 1], windows of wtok tokens
+    int32_t* wstart;
+    int nwin, wtok;
     DevStatus* st;
     unsigned long long tag;  // written to st->index_tag by the inversion
     // result: the sorted values live in vals[final_buf]
@@ -51,7 +55,6 @@ struct WindowPlan {
     int nwin;                // number of token windows
     int wtok;                // tokens per window
     int nb_stride;           // row stride of the tables: T / bs + nseq >= NB
-    int2* win_rng;           // [hkv * nwin * nb_stride]: (first entry, count)
     int32_t* tile_off;       // [hkv * nwin * (nb_stride + 1)]: tile offsets within a row
     int32_t* row_tiles;      // [hkv * nwin]
     int32_t* row_off;        // [hkv * nwin + 1]
@@ -89,7 +92,6 @@ struct FwdPlan {
     int nbk_cap;
     // window order of the tiles (see WindowPlan)
     int nwin, nb_stride;
-    const int2* win_rng;
     const int32_t* wtile_off;
     const int32_t* row_off;
     const int4* tile_desc;
