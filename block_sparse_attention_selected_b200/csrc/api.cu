@@ -191,6 +191,22 @@ bool make_q_group_map(CUtensorMap* map, const void* base, int T, int hq, int G, 
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a bf16 / fp16 [rows, d] tensor (Q or dO viewed as [T * hq, d]); box =
+// (64 columns, 1 row), 128-byte swizzle: the gather4 loads of the tile kernels.
+bool make_row_map(CUtensorMap* map, const void* base, long long rows, bool f16, int d = kHeadDim) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, box_rows),
 // 128-byte swizzle: the epilogue's TMA stores of 8-row groups and of whole warps.
 bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows, int d = kHeadDim) {
@@ -522,7 +538,11 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
         return s;
     pm.add(1);
     pm.mark(2);
-    if ((s = cuda_status(launch_bwd_tiles(bp, &kmap, &vmap, stream))) != NSA_OK) return s;
+    CUtensorMap qmap, domap;
+    if (!make_row_map(&qmap, q, (long long)D.T * D.hq, f16) ||
+        !make_row_map(&domap, dout, (long long)D.T * D.hq, f16))
+        return NSA_ERR_CUDA;
+    if ((s = cuda_status(launch_bwd_tiles(bp, &kmap, &vmap, &qmap, &domap, stream))) != NSA_OK) return s;
     pm.add(1);
     pm.mark(3);
     if ((s = cuda_status(launch_bwd_dq_merge(bp, block_idx, dq, stream))) != NSA_OK) return s;

@@ -18,8 +18,8 @@
 // One persistent CTA per SM takes units (largest first, dealt in snake order); it is
 // warp-specialised:
 //
-//   warps 0-3, 14, 15  loaders: row metadata, cp.async gather of the Q and dO rows (NQ
-//                      stages; rows past the list are zero, so they add nothing to dV / dK)
+//   warps 0-3          loaders: row metadata, TMA gather4 of the Q and dO rows (NQ
+//                      stages; rows past the list read as zero, so they add nothing to dV / dK)
 //   warp 12            TMA producer: K_B and V_B of each unit
 //   warp 13            MMA issuer (one thread): S/dP may run one tile ahead of the
 //                      dV/dK/dQ products; it issues whichever of the two is ready first
@@ -36,18 +36,18 @@ namespace nsa {
 namespace {
 
 // Warp roles (four warpgroups; warp % 4 = TMEM lane quadrant):
-//   warpgroup 0 (warps 0-3)      Q / dO loaders 0-3
+//   warpgroup 0 (warps 0-3)      Q / dO loaders, one tile row per lane
 //   warpgroups 1, 2 (4-11)       P / dS and the epilogues, half of the columns each
-//   warpgroup 3 (12-15)          TMA producer (12), MMA issuer (13), loaders 4-5 (14, 15)
-// A cp.async gather's throughput grows with the number of issuing warps, and a tile
-// needs 64 KB of gathered Q and dO rows, so six warps load.  setmaxnreg rebalances
-// the launch's 128 registers per thread: warpgroups 0 and 3 take 64, the P / dS
-// warpgroups 192 (2 x 128 x 64 + 2 x 128 x 192 = 512 x 128).
+//   warpgroup 3 (12-15)          TMA producer (12), MMA issuer (13); 14, 15 idle
+// The 64 KB of Q and dO rows a tile needs arrive by TMA gather4 (four arbitrary rows of
+// one 64-column half per instruction), issued by every fourth loader lane.  setmaxnreg
+// rebalances the launch's 128 registers per thread: warpgroups 0 and 3 take 64, the
+// P / dS warpgroups 192 (2 x 128 x 64 + 2 x 128 x 192 = 512 x 128).
 constexpr int kThreads = 512;
-constexpr int kLoaderWarps = 6;
+constexpr int kLoaderWarps = 4;
 constexpr int kLoaderThreads = kLoaderWarps * 32;
-constexpr int kRowsPerLoader = (kTileRows + kLoaderWarps - 1) / kLoaderWarps;   // 22
-static_assert(kRowsPerLoader <= 32, "one row per loader lane");
+static_assert(kLoaderThreads == kTileRows, "one row per loader lane");
+constexpr int kGatherLanes = kTileRows / 4;   // lanes that issue a tile's gathers
 constexpr int kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kRegsLow = 64, kRegsWg = 192;
 constexpr int kWgThreads = 128;
@@ -106,7 +106,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <int BS, int NQ, int NSLOT, int F16>
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_tiles(const BwdPlan p, const __grid_constant__ CUtensorMap kmap,
-                const __grid_constant__ CUtensorMap vmap) {
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap,
+                const __grid_constant__ CUtensorMap domap) {
     extern __shared__ uint8_t smem_raw[];
     BwdSmem<BS, NQ, NSLOT>& S = *reinterpret_cast<BwdSmem<BS, NQ, NSLOT>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
         S.nunits = *reinterpret_cast<volatile int*>(&st->nchunks);
         for (int i = 0; i < NQ; ++i) {
-            mbar_init(&S.q_full[i], kLoaderThreads);
+            mbar_init(&S.q_full[i], kGatherLanes);
             mbar_init(&S.q_empty[i], 1);
             mbar_init(&S.meta_full[i], kLoaderThreads);
             mbar_init(&S.meta_empty[i], 2 * kWgThreads);
@@ -177,37 +178,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     static_assert(kColDK + BS <= 512, "TMEM budget");
 
     const int wgrp = warp >> 2;
-    const int li = wgrp == 0 ? warp : warp >= 14 ? warp - 10 : -1;
+    const int li = wgrp == 0 ? warp : -1;
 
     if (wgrp == 0 || wgrp == 3) {
         reg_dealloc<kRegsLow>();
         if (li >= 0) {
             // ------------------------------------------------------------------ loaders
-            // Loader w fills tile rows [R w, min(R w + R, 128)), R = kRowsPerLoader; lane l
-            // owns row R w + l: it writes the row's metadata, LSE (times log2 e) and D into
-            // shared memory for the P / dS warps and computes its Q / dO source address.  In
-            // copy step k the loader moves rows R w + 2k and R w + 2k + 1 (lane l: 16-byte
-            // chunk l % 16 of row R w + 2k + l / 16, a 512-byte coalesced read); rows past
-            // the list are zeroed, so that they add nothing to dV and dK.  Tile i - 1's copies are published
-            // (wait, fence, arrive on q_full) once tile i's row data is requested, before the
-            // loader waits for tile i's metadata slot and stage: that stage is released by the
-            // products of tile i - 2, which may wait for S / dP of tile i - 1, so publishing
-            // after that wait could close a cycle.
+            // Loader w fills tile rows [32 w, 32 w + 32); lane l owns row 32 w + l: it
+            // writes the row's metadata, LSE (times log2 e) and D into shared memory for the
+            // P / dS warps and contributes the row's coordinate in the [T hq, 128] view of
+            // Q and dO.  Lanes 4j then gather rows 32 w + 4j .. 32 w + 4j + 3: one gather4
+            // per 64-column half and tensor, 2 KB per lane, armed on q_full with their byte
+            // count.  A row past the list takes the out-of-range coordinate T hq and reads
+            // as zero, so it adds nothing to dV and dK.
             const int w = li;
-            const int nr_w = min(kRowsPerLoader, kTileRows - kRowsPerLoader * w);   // rows of this loader
-            const uint8_t* qb = static_cast<const uint8_t*>(p.q);
-            const uint8_t* db = static_cast<const uint8_t*>(p.dout);
             const float kLog2e = 1.4426950408889634f;
             int4 u0 = ld_unit(0), u1 = ld_unit(1), u2 = ld_unit(2);
-            auto ld_ent = [&](int e0, int ehi, int r) -> uint32_t {
-                return (lane < nr_w && e0 + r / p.G < ehi) ? __ldg(p.entries + e0 + r / p.G) : 0xFFFFFFFFu;
+            const int rA = 32 * w + lane;
+            auto ld_ent = [&](int e0, int ehi) -> uint32_t {
+                return e0 + rA / p.G < ehi ? __ldg(p.entries + e0 + rA / p.G) : 0xFFFFFFFFu;
             };
-            const int rA = kRowsPerLoader * w + lane;
             uint32_t entA = 0xFFFFFFFFu;
-            if (nk > 0) entA = ld_ent(u0.y, u0.z, rA);
-            const int c = lane & 15;
-            const uint32_t dst_c = (uint32_t)(c >> 3) * (kTileRows * 128);
-            int i = 0, issued = 0, published = 0;
+            if (nk > 0) entA = ld_ent(u0.y, u0.z);
+            if (lane == 0) {
+                prefetch_tmap(&qmap);
+                prefetch_tmap(&domap);
+            }
+            const int oob_row = p.T * p.hq;
+            int i = 0, issued = 0;
             bool stopped = false;
             for (int k = 0; k < nk && !stopped; ++k) {
                 const int4 d = u0;
@@ -219,10 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph_empty = ((i / NQ) & 1) ^ 1;
                     const uint32_t ea = entA;
                     // index entries of the next tile (this unit's or the next unit's first)
-                    if (tt + 1 < ntl) entA = ld_ent(e0 + tpt, d.z, rA);
-                    else if (k + 1 < nk) entA = ld_ent(u0.y, u0.z, rA);
-                    // this lane's row: metadata, LSE, D, source offset (-1: past the list)
-                    long long offA = -1;
+                    if (tt + 1 < ntl) entA = ld_ent(e0 + tpt, d.z);
+                    else if (k + 1 < nk) entA = ld_ent(u0.y, u0.z);
+                    // this lane's row: metadata, LSE, D, row coordinate
+                    int rowc = oob_row;
                     float lA = 0.f, dA = 0.f;
                     int4 mA = make_int4(-1, 0, 0, -1);
                     if (kChecks) {   // the gathered row must lie inside q and dout
@@ -236,55 +234,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (ea != 0xFFFFFFFFu) {
                         mA = make_int4((int)(ea >> 6), g * p.G + rA % p.G, (int)(ea & 63u), (int)(ea >> 6) - d.x);
-                        offA = ((long long)mA.x * p.hq + mA.y) * (kHeadDim * 2);
+                        rowc = mA.x * p.hq + mA.y;
                         lA = __ldg(p.lse + (size_t)mA.y * p.T + mA.x) * kLog2e;
                         dA = __ldg(p.delta + (size_t)mA.y * p.T + mA.x);
-                    }
-                    if (i > 0) {                       // publish tile i - 1 (the loads above land meanwhile)
-                        cp_async_wait_all();
-                        fence_async_smem();
-                        mbar_arrive(&S.q_full[(i - 1) % NQ]);
-                        published = i;
                     }
                     if (!__all_sync(0xffffffffu, wait(&S.meta_empty[stg], ph_empty, 50))) {
                         stopped = true;
                         break;
                     }
-                    if (lane < nr_w) {
-                        S.meta[stg][rA] = mA;
-                        S.rlse[stg][rA] = lA;
-                        S.rdelta[stg][rA] = dA;
-                    }
+                    S.meta[stg][rA] = mA;
+                    S.rlse[stg][rA] = lA;
+                    S.rdelta[stg][rA] = dA;
                     mbar_arrive(&S.meta_full[stg]);
                     if (!__all_sync(0xffffffffu, wait(&S.q_empty[stg], ph_empty, 51))) {
                         stopped = true;
                         break;
                     }
-                    // gather Q and dO
-                    const uint32_t q0 = smem_u32(S.q[stg][0]) + dst_c, d0 = smem_u32(S.dout[stg][0]) + dst_c;
-    #pragma unroll 1
-                    for (int kk = 0; kk < (kRowsPerLoader + 1) / 2; ++kk) {
-                        const int rw = 2 * kk + (lane >> 4);          // row within the loader's rows
-                        const long long off = __shfl_sync(0xffffffffu, offA, rw & 31);
-                        if (rw >= nr_w) continue;
-                        const uint32_t so = sw128_offset(kRowsPerLoader * w + rw, c & 7);
-                        if (off >= 0) {
-                            cp_async_16(q0 + so, qb + off + c * 16);
-                            cp_async_16(d0 + so, db + off + c * 16);
-                        } else {
-                            st_shared_v4(q0 + so, 0u, 0u, 0u, 0u);
-                            st_shared_v4(d0 + so, 0u, 0u, 0u, 0u);
-                        }
+                    // gather Q and dO (the stage's previous readers, the products of tile
+                    // i - NQ, completed before q_empty)
+                    const int r1 = __shfl_down_sync(0xffffffffu, rowc, 1);
+                    const int r2 = __shfl_down_sync(0xffffffffu, rowc, 2);
+                    const int r3 = __shfl_down_sync(0xffffffffu, rowc, 3);
+                    if ((lane & 3) == 0) {
+                        const uint32_t ro = (uint32_t)rA * 128u;
+                        mbar_arrive_expect_tx(&S.q_full[stg], 4u * 4u * 128u);
+                        tma_gather4(S.q[stg][0] + ro, &qmap, &S.q_full[stg], 0, rowc, r1, r2, r3);
+                        tma_gather4(S.q[stg][1] + ro, &qmap, &S.q_full[stg], 64, rowc, r1, r2, r3);
+                        tma_gather4(S.dout[stg][0] + ro, &domap, &S.q_full[stg], 0, rowc, r1, r2, r3);
+                        tma_gather4(S.dout[stg][1] + ro, &domap, &S.q_full[stg], 64, rowc, r1, r2, r3);
                     }
-                    cp_async_commit();
                     issued = i + 1;
                 }
             }
-            cp_async_wait_all();   // nothing may still be in flight when the CTA exits
-            if (!stopped && issued > 0 && published == issued - 1) {
-                fence_async_smem();
-                mbar_arrive(&S.q_full[(issued - 1) % NQ]);
-            }
+            // nothing may still be in flight when the CTA exits: after an abort, wait
+            // (bounded) until the last gathered stage has landed
+            if (*abort_flag && issued > 0)
+                mbar_wait(&S.q_full[(issued - 1) % NQ], ((issued - 1) / NQ) & 1, st, 53);
         } else if (warp == kTmaWarp) {
             // ------------------------------------------------------------- K/V producer
             if (lane == 0) {
@@ -643,21 +628,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BS, int NQ, int NSLOT, int F16>
 static void launch_bwd_variant(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                               const CUtensorMap* qmap, const CUtensorMap* domap,
                                cudaStream_t stream) {
     constexpr size_t smem = bwd_smem_bytes<BS, NQ, NSLOT>();
     cudaFuncSetAttribute(k_bwd_tiles<BS, NQ, NSLOT, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    k_bwd_tiles<BS, NQ, NSLOT, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap);
+    k_bwd_tiles<BS, NQ, NSLOT, F16><<<p.num_sms, kThreads, smem, stream>>>(p, *kmap, *vmap, *qmap,
+                                                                          *domap);
 }
 
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                             const CUtensorMap* qmap, const CUtensorMap* domap,
                              cudaStream_t stream) {
     if (p.bs == 64) {
-        if (p.f16) launch_bwd_variant<64, 2, 2, 1>(p, kmap, vmap, stream);
-        else launch_bwd_variant<64, 2, 2, 0>(p, kmap, vmap, stream);
+        if (p.f16) launch_bwd_variant<64, 2, 2, 1>(p, kmap, vmap, qmap, domap, stream);
+        else launch_bwd_variant<64, 2, 2, 0>(p, kmap, vmap, qmap, domap, stream);
     } else {
-        if (p.f16) launch_bwd_variant<128, 1, 1, 1>(p, kmap, vmap, stream);
-        else launch_bwd_variant<128, 1, 1, 0>(p, kmap, vmap, stream);
+        if (p.f16) launch_bwd_variant<128, 1, 1, 1>(p, kmap, vmap, qmap, domap, stream);
+        else launch_bwd_variant<128, 1, 1, 0>(p, kmap, vmap, qmap, domap, stream);
     }
     return cudaGetLastError();
 }

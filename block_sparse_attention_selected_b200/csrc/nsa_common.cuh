@@ -167,6 +167,20 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four rows of a 2D tensor map (box: 64 columns x 1 row) at arbitrary row coordinates
+// r0..r3, column c0, into four consecutive 128-byte rows of shared memory, with the
+// map's swizzle applied from the destination address (so a 4-row group may start at any
+// 512-byte offset of a 128B-swizzled tile).  Rows outside the tensor read as zero.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1),
+        "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // TMA tile store shared -> global (bulk-group completion); x must be a multiple of 16
 // bytes, neither coordinate negative.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0,

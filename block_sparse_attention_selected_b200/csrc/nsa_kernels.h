@@ -157,7 +157,10 @@ struct BwdPlan {
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
                                   int f16, cudaStream_t stream);
+// qmap / domap: 2D maps over Q and dO viewed as [T * hq, 128], box 64 columns x 1 row,
+// 128-byte swizzle (the tile kernel's gather4 loads)
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
+                             const CUtensorMap* qmap, const CUtensorMap* domap,
                              cudaStream_t stream);
 cudaError_t launch_bwd_dq_merge(const BwdPlan& p, const int32_t* bidx, void* dq,
                                 cudaStream_t stream);
