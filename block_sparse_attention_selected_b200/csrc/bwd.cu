@@ -267,9 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // nothing may still be in flight when the CTA exits: after an abort, wait
-            // (bounded) until the last gathered stage has landed
-            if (*abort_flag && issued > 0)
-                mbar_wait(&S.q_full[(issued - 1) % NQ], ((issued - 1) / NQ) & 1, st, 53);
+            // (bounded) for the last gathers into every stage
+            if (*abort_flag)
+                for (int j = issued - 1; j >= 0 && j >= issued - NQ; --j)
+                    mbar_wait(&S.q_full[j % NQ], (j / NQ) & 1, st, 53);
         } else if (warp == kTmaWarp) {
             // ------------------------------------------------------------- K/V producer
             if (lane == 0) {

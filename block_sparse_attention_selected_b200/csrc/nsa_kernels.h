@@ -106,7 +106,7 @@ struct FwdPlan {
 // vexp[g * NB + B] = 0, or the exponent that brings max |V_B| under 2^15
 cudaError_t launch_vblock_exp(const FwdPlan& p, const void* v, int nb_stride, int32_t* vexp,
                               cudaStream_t stream);
-// omap[0], omap[1]: tensor maps over part_o (fp16 [tiles_cap * 128, 128], 128B swizzle)
+// omap[0], omap[1]: tensor maps over part_o (fp16 [tiles_cap * 128, d], 128B swizzle)
 // with boxes of 64 columns x 8 rows and 64 columns x 32 rows
 cudaError_t launch_fwd_tiles(const FwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,
                              const CUtensorMap* omap, cudaStream_t stream);
