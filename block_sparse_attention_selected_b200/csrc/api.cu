@@ -49,7 +49,9 @@ nsa_status_t check_dims(int T, int nseq, int hq, int hkv, int d, int topk, int b
     if (hq % hkv != 0) return NSA_ERR_INVALID_ARG;
     if ((bs != 64 && bs != 128) || topk > kMaxTopk) return NSA_ERR_UNSUPPORTED;
     if (d != 64 && d != kHeadDim && d != 256) return NSA_ERR_UNSUPPORTED;
-    if ((d == 256 && bs != 64) || (bwd && d != kHeadDim)) return NSA_ERR_UNSUPPORTED;
+    // the backward runs d = 64 as d = 128 with the upper half read as zeros; d = 256 has no
+    // shared memory for its Q / dO stages
+    if ((d == 256 && bs != 64) || (bwd && d == 256)) return NSA_ERR_UNSUPPORTED;
     const int G = hq / hkv;
     if (G > kMaxGroup || kTileRows % G != 0) return NSA_ERR_UNSUPPORTED;
     if (T >= (1 << 25)) return NSA_ERR_UNSUPPORTED;
@@ -107,7 +109,8 @@ Layout make_layout(const Dims& D, bool bwd) {
     // forward: one 128-row slot per tile; backward: one row per (token, head, slot)
     const size_t rows = std::max((size_t)D.T * D.hq * D.topk,
                                  (size_t)std::max<long long>(D.fwd_tiles_cap, 1) * kTileRows);
-    L.part_o = take(rows * (size_t)D.d * 2);   // fp16 partial O (forward) / bf16 dQ (backward)
+    // fp16 partial O (forward, d columns) / bf16 dQ (backward, 128 columns)
+    L.part_o = take(rows * (size_t)(bwd ? std::max(D.d, kHeadDim) : D.d) * 2);
     L.part_lse = take(rows * sizeof(float2));  // (lse, exponent) per partial
     if (bwd) {
         L.delta = take(sizeof(float) * (size_t)D.hq * D.T);
@@ -490,7 +493,10 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     }
 
     CUtensorMap kmap, vmap;
-    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16) || !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16))
+    // d = 64: the maps cover the d columns, and the kernel's loads of columns 64..127 lie
+    // outside them and read as zeros
+    if (!make_kv_map(&kmap, k, D.T, D.hkv, D.bs, f16, D.d) ||
+        !make_kv_map(&vmap, v, D.T, D.hkv, D.bs, f16, D.d))
         return NSA_ERR_CUDA;
     if (reuse_index) {
         c.inv.final_buf = invert_final_buf(c.inv);
@@ -516,6 +522,7 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.cu = cu_seqlens;
     bp.nseq = D.nseq; bp.T = D.T; bp.hq = D.hq; bp.hkv = D.hkv; bp.topk = D.topk; bp.bs = D.bs;
     bp.G = D.G;
+    bp.d = D.d;
     bp.f16 = f16 ? 1 : 0;
     bp.swin = swin;
     bp.scale = scale;
@@ -534,13 +541,13 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
     bp.part_dkdv = reinterpret_cast<float*>(c.base + L.part_dkdv);
     bp.st = c.st;
     bp.num_sms = num_sms;
-    if ((s = cuda_status(launch_bwd_preprocess(out, dout, bp.delta, D.T, D.hq, bp.f16, stream))) != NSA_OK)
+    if ((s = cuda_status(launch_bwd_preprocess(out, dout, bp.delta, D.T, D.hq, D.d, bp.f16, stream))) != NSA_OK)
         return s;
     pm.add(1);
     pm.mark(2);
     CUtensorMap qmap, domap;
-    if (!make_row_map(&qmap, q, (long long)D.T * D.hq, f16) ||
-        !make_row_map(&domap, dout, (long long)D.T * D.hq, f16))
+    if (!make_row_map(&qmap, q, (long long)D.T * D.hq, f16, D.d) ||
+        !make_row_map(&domap, dout, (long long)D.T * D.hq, f16, D.d))
         return NSA_ERR_CUDA;
     if ((s = cuda_status(launch_bwd_tiles(bp, &kmap, &vmap, &qmap, &domap, stream))) != NSA_OK) return s;
     pm.add(1);

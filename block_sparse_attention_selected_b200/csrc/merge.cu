@@ -149,29 +149,32 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kS == 16 ? (NH == 4 ? 2 :
 }
 
 // Eight rows per warp, half a warp per row and 16-byte loads: four rows' loads of O and
-// dO are in flight per lane before the first reduction.
+// dO are in flight per lane before the first reduction (d = 64: the row's 8 chunks on
+// lanes 0-7 of the half warp).
 constexpr int kDeltaRowsPerWarp = 8;
 template <int F16>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_bwd_delta(const void* out, const void* dout,
-                                                                  float* delta, int T, int hq) {
+                                                                  float* delta, int T, int hq,
+                                                                  int d) {
     const int lane = threadIdx.x & 31, half = lane >> 4, c = lane & 15;
     const long long nrows = (long long)T * hq;
     const long long row0 =
         ((long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * kDeltaRowsPerWarp;
-    uint4 o[kDeltaRowsPerWarp / 2], d[kDeltaRowsPerWarp / 2];
+    const int cpr = d >> 3;   // 16-byte chunks per row
+    uint4 o[kDeltaRowsPerWarp / 2], dv[kDeltaRowsPerWarp / 2];
 #pragma unroll
     for (int it = 0; it < kDeltaRowsPerWarp / 2; ++it) {
         const long long row = row0 + 2 * it + half;
-        o[it] = d[it] = make_uint4(0u, 0u, 0u, 0u);
-        if (row < nrows) {
-            o[it] = __ldg(reinterpret_cast<const uint4*>(out) + row * (kHeadDim / 8) + c);
-            d[it] = __ldg(reinterpret_cast<const uint4*>(dout) + row * (kHeadDim / 8) + c);
+        o[it] = dv[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (row < nrows && c < cpr) {
+            o[it] = __ldg(reinterpret_cast<const uint4*>(out) + row * cpr + c);
+            dv[it] = __ldg(reinterpret_cast<const uint4*>(dout) + row * cpr + c);
         }
     }
 #pragma unroll
     for (int it = 0; it < kDeltaRowsPerWarp / 2; ++it) {
         const uint32_t ow[4] = {o[it].x, o[it].y, o[it].z, o[it].w};
-        const uint32_t dw[4] = {d[it].x, d[it].y, d[it].z, d[it].w};
+        const uint32_t dw[4] = {dv[it].x, dv[it].y, dv[it].z, dv[it].w};
         float x = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -219,8 +222,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dq_merge(const BwdPlan 
         acc[2] += b.x;
         acc[3] += b.y;
     }
-    uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dq) + (size_t)row * kHeadDim) + lane;
-    *o = make_uint2(pack2<F16>(acc[0], acc[1]), pack2<F16>(acc[2], acc[3]));
+    // d = 64: the partials' columns 64..127 are zero and not stored
+    if (lane * 4 < p.d) {
+        uint2* o = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dq) + (size_t)row * p.d) + lane;
+        *o = make_uint2(pack2<F16>(acc[0], acc[1]), pack2<F16>(acc[2], acc[3]));
+    }
 }
 
 // One warp per (key token, KV head); each lane owns 4 of the 128 columns.
@@ -248,8 +254,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_dkdv_reduce(const BwdPl
         av.x += x.x; av.y += x.y; av.z += x.z; av.w += x.w;
         ak.x += y.x; ak.y += y.y; ak.z += y.z; ak.w += y.w;
     }
-    uint2* ov = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dv) + (size_t)row * kHeadDim) + lane;
-    uint2* ok = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dk) + (size_t)row * kHeadDim) + lane;
+    if (lane * 4 >= p.d) return;   // d = 64: the partials' columns 64..127 are zero
+    uint2* ov = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dv) + (size_t)row * p.d) + lane;
+    uint2* ok = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dk) + (size_t)row * p.d) + lane;
     *ov = make_uint2(pack2<F16>(av.x, av.y), pack2<F16>(av.z, av.w));
     *ok = make_uint2(pack2<F16>(ak.x, ak.y), pack2<F16>(ak.z, ak.w));
 }
@@ -280,13 +287,13 @@ cudaError_t launch_merge(const MergePlan& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
-                                  int f16, cudaStream_t stream) {
+                                  int d, int f16, cudaStream_t stream) {
     const long long rows = (long long)T * hq;
     const long long per_block = (long long)kWarpsPerBlock * kDeltaRowsPerWarp;
     const unsigned nb = (unsigned)((rows + per_block - 1) / per_block);
     if (rows > 0) {
-        if (f16) k_bwd_delta<1><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
-        else k_bwd_delta<0><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq);
+        if (f16) k_bwd_delta<1><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq, d);
+        else k_bwd_delta<0><<<nb, kWarpsPerBlock * 32, 0, stream>>>(out, dout, delta, T, hq, d);
     }
     return cudaGetLastError();
 }

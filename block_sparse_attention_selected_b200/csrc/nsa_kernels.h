@@ -137,6 +137,8 @@ struct BwdPlan {
     float* delta;            // [hq, T]  rowsum(dout * out)
     const int32_t* cu;
     int nseq, T, hq, hkv, topk, bs, G;
+    int d;                   // head dimension of q, k, v, dout, dq, dk, dv (64 or 128); the
+                             // tile kernel and its partials work at 128 columns
     int swin;                // sliding window in keys (0: none)
     float scale, scale_log2;
     const int32_t* blkoff;
@@ -156,7 +158,7 @@ struct BwdPlan {
 };
 
 cudaError_t launch_bwd_preprocess(const void* out, const void* dout, float* delta, int T, int hq,
-                                  int f16, cudaStream_t stream);
+                                  int d, int f16, cudaStream_t stream);
 // qmap / domap: 2D maps over Q and dO viewed as [T * hq, 128], box 64 columns x 1 row,
 // 128-byte swizzle (the tile kernel's gather4 loads)
 cudaError_t launch_bwd_tiles(const BwdPlan& p, const CUtensorMap* kmap, const CUtensorMap* vmap,

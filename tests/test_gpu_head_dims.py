@@ -1,6 +1,7 @@
-"""Head dimensions 64 and 256 in the forward (the project page's Limitations: one head
-dimension for Q, K and V, at most 256), against the fp64 oracle element by element.
-The backward takes head dimension 128 only and refuses the others on the host."""
+"""Head dimensions 64 and 256 (the project page's Limitations: one head dimension for Q,
+K and V, at most 256), against the fp64 oracle element by element.  The forward takes
+64, 128 and 256; the backward 64 and 128 (64 runs the 128-column pipeline with the upper
+half read as zeros) and refuses 256 on the host."""
 import numpy as np
 import pytest
 import torch
@@ -8,7 +9,7 @@ import torch
 import block_sparse_attention_selected_b200 as nsa
 import nsa_inputs as ni
 import oracle
-from gpu_util import TOL_LSE, TOL_O, f64, max_abs, o_errors, to_device
+from gpu_util import TOL_GRAD, TOL_LSE, TOL_O, f64, max_abs, o_errors, rel_fro, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -79,14 +80,43 @@ def test_fwd_head_dim_fp16_and_large_v(d):
     assert max_abs(f64(lse).T, l_ref) <= TOL_LSE
 
 
-def test_bwd_head_dim_other_than_128_is_refused():
-    p = ni.make_problem([300], hq=4, hkv=2, head_dim=64, block_size=64, topk=4, seed=110)
+def test_bwd_head_dim_256_is_refused():
+    p = ni.make_problem([300], hq=4, hkv=2, head_dim=256, block_size=64, topk=4, seed=110)
     t = to_device(p)
     out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], 64, p.scale)
     with pytest.raises(nsa.NsaError) as e:
         nsa.nsa_sel_attn_bwd(t["q"], t["k"], t["v"], out, lse, t["dout"], t["cu"], t["bidx"], 64,
                              p.scale)
     assert e.value.code == 2   # NSA_ERR_UNSUPPORTED
+
+
+BWD64 = [
+    # name, problem, window, perturbed, dtype
+    ("bwd_d64_g1_bs64_k16", dict(lengths=[1500, 37, 1, 600], hq=2, hkv=2, block_size=64, topk=16, seed=121), 0, True, torch.bfloat16),
+    ("bwd_d64_g4_bs128_k8", dict(lengths=[2000, 129], hq=8, hkv=2, block_size=128, topk=8, seed=122), 0, True, torch.bfloat16),
+    ("bwd_d64_g16_bs64_k64", dict(lengths=[1800], hq=16, hkv=1, block_size=64, topk=64, seed=123), 0, False, torch.bfloat16),
+    ("bwd_d64_g8_bs64_k12_w100", dict(lengths=[900, 129], hq=8, hkv=1, block_size=64, topk=12, seed=124), 100, True, torch.bfloat16),
+    ("bwd_d64_g4_bs64_k16_fp16", dict(lengths=[1200, 300], hq=8, hkv=2, block_size=64, topk=16, seed=125), 0, True, torch.float16),
+]
+
+
+@pytest.mark.parametrize("name,spec,W,perturb,dtype", BWD64, ids=[c[0] for c in BWD64])
+def test_bwd_head_dim_64_full_compare(name, spec, W, perturb, dtype):
+    p = ni.make_problem(name=name, head_dim=64, **spec)
+    if perturb:
+        p = _perturb(p, 8)
+    t = to_device(p, dtype=dtype)
+    out, lse = nsa.nsa_sel_attn_fwd(t["q"], t["k"], t["v"], t["cu"], t["bidx"], p.block_size,
+                                    p.scale, window_size=W)
+    dq, dk, dv = nsa.nsa_sel_attn_bwd(t["q"], t["k"], t["v"], out, lse, t["dout"], t["cu"],
+                                      t["bidx"], p.block_size, p.scale, window_size=W)
+    torch.cuda.synchronize()
+    assert nsa.nsa_sel_check_status() == 0
+    assert dq.shape == t["q"].shape and dk.shape == t["k"].shape and dv.shape == t["v"].shape
+    rdq, rdk, rdv = oracle.bwd(p.q, p.k, p.v, p.dout, p.cu_seqlens, p.block_idx, p.block_size,
+                               p.scale, window=W)
+    e = (rel_fro(f64(dq), rdq), rel_fro(f64(dk), rdk), rel_fro(f64(dv), rdv))
+    assert max(e) <= TOL_GRAD, (name, e)
 
 
 @pytest.mark.parametrize("d", [64, 256])
