@@ -74,6 +74,10 @@ INV_CASES = [
     ("varlen_ragged", dict(lengths=[700, 37, 1, 515], hq=2, hkv=2, block_size=64, topk=16, seed=3), True),
     ("bs128_k64", dict(lengths=[3000, 129], hq=4, hkv=1, block_size=128, topk=64, seed=5), True),
     ("empty_seq", dict(lengths=[0, 300, 0, 65], hq=3, hkv=3, block_size=64, topk=5, seed=6), True),
+    # many short sequences, empty ones among them: a sort thread's entries cross several
+    # sequence boundaries
+    ("many_seqs", dict(lengths=[int(x) for x in np.random.default_rng(7).integers(0, 90, 160)],
+                       hq=4, hkv=2, block_size=64, topk=3, seed=7), True),
 ]
 
 
