@@ -210,6 +210,24 @@ bool make_row_map(CUtensorMap* map, const void* base, long long rows, bool f16, 
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a bf16 / fp16 [T, hq, d] tensor as (d columns, hq heads, T tokens);
+// box = (64 columns, G heads, 1 token), 128-byte swizzle: one token's G rows of a KV
+// group (G >= 8: whole 1 KB swizzle atoms).
+bool make_token_map(CUtensorMap* map, const void* base, int T, int hq, int G, bool f16,
+                    int d = kHeadDim) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hq, (cuuint64_t)(T > 0 ? T : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hq * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Tensor map over the forward partials, fp16 [rows, 128]; box = (64 columns, box_rows),
 // 128-byte swizzle: the epilogue's TMA stores of 8-row groups and of whole warps.
 bool make_part_map(CUtensorMap* map, void* base, long long rows, int box_rows, int d = kHeadDim) {
@@ -545,10 +563,17 @@ nsa_status_t bwd_impl(const void* q, const void* k, const void* v, const void* o
         return s;
     pm.add(1);
     pm.mark(2);
+    // G >= 8: 3D maps (columns, heads, tokens) with a box of one token's G heads, whole
+    // swizzle atoms; otherwise 2D row maps for the four-row gathers
     CUtensorMap qmap, domap;
-    if (!make_row_map(&qmap, q, (long long)D.T * D.hq, f16, D.d) ||
-        !make_row_map(&domap, dout, (long long)D.T * D.hq, f16, D.d))
+    if (D.G >= 8) {
+        if (!make_token_map(&qmap, q, D.T, D.hq, D.G, f16, D.d) ||
+            !make_token_map(&domap, dout, D.T, D.hq, D.G, f16, D.d))
+            return NSA_ERR_CUDA;
+    } else if (!make_row_map(&qmap, q, (long long)D.T * D.hq, f16, D.d) ||
+               !make_row_map(&domap, dout, (long long)D.T * D.hq, f16, D.d)) {
         return NSA_ERR_CUDA;
+    }
     if ((s = cuda_status(launch_bwd_tiles(bp, &kmap, &vmap, &qmap, &domap, stream))) != NSA_OK) return s;
     pm.add(1);
     pm.mark(3);

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.abort_flag = (*reinterpret_cast<volatile int*>(&st->code) != 0);
         S.nunits = *reinterpret_cast<volatile int*>(&st->nchunks);
         for (int i = 0; i < NQ; ++i) {
-            mbar_init(&S.q_full[i], kGatherLanes);
+            // gathering lanes: every fourth (gather4), or one per token for G >= 8
+            mbar_init(&S.q_full[i], p.G >= 8 ? kTileRows / p.G : kGatherLanes);
             mbar_init(&S.q_empty[i], 1);
             mbar_init(&S.meta_full[i], kLoaderThreads);
             mbar_init(&S.meta_empty[i], 2 * kWgThreads);
@@ -255,7 +256,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int r1 = __shfl_down_sync(0xffffffffu, rowc, 1);
                     const int r2 = __shfl_down_sync(0xffffffffu, rowc, 2);
                     const int r3 = __shfl_down_sync(0xffffffffu, rowc, 3);
-                    if ((lane & 3) == 0) {
+                    if (p.G >= 8) {
+                        // the G rows of a token are adjacent in Q and dO and fill whole
+                        // 1 KB swizzle atoms of the tile: one tiled box per token, half and
+                        // tensor (the maps are 3D here: columns, heads, tokens), issued by
+                        // the token's first lane; a token past the list reads as zero
+                        if (rA % p.G == 0) {
+                            const uint32_t ro = (uint32_t)rA * 128u;
+                            const int tok = ea != 0xFFFFFFFFu ? mA.x : p.T;
+                            mbar_arrive_expect_tx(&S.q_full[stg], 4u * (uint32_t)p.G * 128u);
+                            tma_load_3d(S.q[stg][0] + ro, &qmap, &S.q_full[stg], 0, g * p.G, tok);
+                            tma_load_3d(S.q[stg][1] + ro, &qmap, &S.q_full[stg], 64, g * p.G, tok);
+                            tma_load_3d(S.dout[stg][0] + ro, &domap, &S.q_full[stg], 0, g * p.G, tok);
+                            tma_load_3d(S.dout[stg][1] + ro, &domap, &S.q_full[stg], 64, g * p.G, tok);
+                        }
+                    } else if ((lane & 3) == 0) {
                         const uint32_t ro = (uint32_t)rA * 128u;
                         mbar_arrive_expect_tx(&S.q_full[stg], 4u * 4u * 128u);
                         tma_gather4(S.q[stg][0] + ro, &qmap, &S.q_full[stg], 0, rowc, r1, r2, r3);
