@@ -37,8 +37,10 @@
  *    problems (a bounded wait that expired, malformed cu_seqlens) are recorded
  *    in the status block at the start of the workspace and read with
  *    nsa_sel_check_status.  No C++ exception crosses this interface.
- *  - Supported domain: bf16 (fp16 through the _ex calls' NSA_F16), head_dim == 128,
- *    block_size in {64, 128},
+ *  - Supported domain: bf16 (fp16 through the _ex calls' NSA_F16); head_dim 64, 128
+ *    or 256 in the forward (256 with block_size 64 only: its Q stages fill the shared
+ *    memory), 64 or 128 in the backward (64 runs the 128-column backward with columns
+ *    64..127 read as zeros); block_size in {64, 128},
  *    1 <= topk <= 64, hq % hkv == 0 with hq / hkv a divisor of 128 (a 128-row tile
  *    holds whole query-head groups), total_tokens < 2^25, and (for 32-bit row
  *    coordinates) total_tokens * hkv * topk < 2^31, total_tokens * hq < 2^31 and
