@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(1024) k_seq_blocks(const int32_t* cu, int nseq
         }
         unsigned long long incl = block_incl_scan_u64(nb, warp_tot);
         if (s < nseq) blkoff[s] = (int32_t)(carry + incl - nb);
-        // total of this round = inclusive value of the last thread
+        // total of this pass of the loop = inclusive value of the last thread
         if (threadIdx.x == blockDim.x - 1) round_total = incl;
         __syncthreads();
         carry += round_total;
