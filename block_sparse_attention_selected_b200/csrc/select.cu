@@ -13,7 +13,8 @@
 //   k_compress_kv   one warp per (compressed block, KV head): mean of kernel_size rows
 //                   of K and of V (lane = four columns, 256-byte coalesced rows)
 //   k_select_topk   one warp per (token, KV head): forced blocks, then repeated warp
-//                   arg-max over the remaining causal blocks' scores held in registers
+//                   arg-max (two redux operations) over the remaining causal blocks'
+//                   scores held in registers
 #include <math_constants.h>
 
 #include "nsa_common.cuh"
@@ -103,6 +104,13 @@ __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
     return a > b || (a == b && ia < ib);
 }
 
+// Unsigned key with the order of the float (a -0 counts as +0, as the float compare
+// does); finite scores and +-inf map above 0.
+__device__ __forceinline__ uint32_t order_key(float x) {
+    const uint32_t u = __float_as_uint(x + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // J = candidate blocks per lane (nb_stride <= 32 J)
 template <int J>
 __global__ void __launch_bounds__(kSelWarps * 32) k_select_topk(const float* scores,
@@ -170,14 +178,11 @@ __global__ void __launch_bounds__(kSelWarps * 32) k_select_topk(const float* sco
         else if (j >= nforced + nrest) out[j] = -1;
     }
     for (int n = 0; n < nrest; ++n) {
-        float wv = bv;
-        int wb = bb;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
-            const int ob = __shfl_xor_sync(0xffffffffu, wb, o);
-            if (better(ov, ob, wv, wb)) { wv = ov; wb = ob; }
-        }
+        // the warp's best: the highest score (one redux over the order keys), then the
+        // lowest block among the lanes holding it (a second redux)
+        const uint32_t key = bv == -CUDART_INF_F ? 0u : order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int wb = __reduce_min_sync(0xffffffffu, key == kmax ? bb : 0x7fffffff);
         if (lane == 0) out[nforced + n] = wb;
         if ((wb & 31) == lane) {                    // the winner drops it and rescans
 #pragma unroll
